@@ -1,0 +1,207 @@
+/*
+ * MapFlow hot-path oracle: a plain, slow, double-precision CPU statement of what
+ * block-sparse attention-map compression and fused map retrieval compute.
+ *
+ * TEST INFRASTRUCTURE ONLY.  The tests, the package's smoke check and the
+ * benchmark's CPU-baseline leg may load it; the library never does.  It shares
+ * no code, header, table or helper with the CUDA path.
+ *
+ * Sources (MapFlow pages: "MapFlow开源:大模型换班,Prefill为何能快20%?",
+ * aitest123.com, section "存不下、读得慢?三个工程优化手段", and its English
+ * rendering on roboind.com, section "When it comes to real savings in reuse"):
+ *   1. block-sparse compression: the map is cut into regular 2-D blocks and
+ *      the important ones are chosen by cumulative attention probability;
+ *      block statistics are computed first, then the blocks to keep are chosen
+ *      (subsection 1 "只存重要的:块稀疏压缩").
+ *   2. fused retrieval: read the sparse blocks, form the linear combination of
+ *      sender heads into receiver heads, multiply by the receiver's own V and
+ *      accumulate (subsection 3 "算得省的:融合内核执行"); the receiver keeps its
+ *      own Value ("不传 KV Cache,改传注意力关系"); heads are mapped by learned
+ *      linear-combination weights (same section, "头映射").
+ *
+ * Readings taken where the pages are silent:
+ *   - selection is per query block on the head-summed mass, one index set for
+ *     all heads; the diagonal block is always kept and counts toward tau;
+ *   - the other key blocks are walked in (mass descending, index ascending)
+ *     order; the walk keeps the fewest blocks whose running sum S reaches
+ *     tau * total, where total is the sum of all the row's masses taken in the
+ *     same walk order (so at tau = 1 the walk stops where S stops growing);
+ *   - entries with j > i, i >= L or j >= L are 0 in the stored blocks and do not
+ *     count toward any mass;
+ *   - kept blocks are stored raw (no renormalisation), col_idx ascending;
+ *   - receiver head r reads KV head g(r) = floor(r * h_kv / h_r).
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* dtype codes: 0 = float32, 1 = bfloat16 (stored as its upper 16 bits). */
+static double value_at(const void* p, int dtype, int64_t idx) {
+  if (dtype == 0) return (double)((const float*)p)[idx];
+  uint32_t bits = (uint32_t)((const uint16_t*)p)[idx] << 16;
+  float f;
+  memcpy(&f, &bits, sizeof f);
+  return (double)f;
+}
+
+/*
+ * Block statistics of one query-block row (compression, step 1).
+ * slab: the rows [qb*B, qb*B + B) of every sender head; element (s, ii, j) at
+ * s*head_stride + ii*row_stride + j.  mass[kb] for kb = 0..qb.
+ */
+void mfo_row_masses(const void* slab, int dtype, int h_s, int B, int64_t head_stride,
+                    int64_t row_stride, int qb, int L, double* mass) {
+  for (int kb = 0; kb <= qb; ++kb) {
+    double m = 0.0;
+    for (int s = 0; s < h_s; ++s)
+      for (int ii = 0; ii < B; ++ii) {
+        const int i = qb * B + ii;
+        if (i >= L) break;
+        for (int jj = 0; jj < B; ++jj) {
+          const int j = kb * B + jj;
+          if (j >= L || j > i) continue;
+          m += value_at(slab, dtype, s * head_stride + ii * row_stride + j);
+        }
+      }
+    mass[kb] = m;
+  }
+}
+
+/* walk order of a row: the diagonal first, then kb < qb by (mass desc, kb asc). */
+static void walk_order(const double* mass, int qb, int32_t* order) {
+  int n = 0;
+  order[n++] = qb;
+  for (int kb = 0; kb < qb; ++kb) {
+    /* insertion into order[1..n) */
+    int p = n;
+    while (p > 1) {
+      const int o = order[p - 1];
+      const int before = mass[kb] > mass[o] || (mass[kb] == mass[o] && kb < o);
+      if (!before) break;
+      order[p] = o;
+      --p;
+    }
+    order[p] = kb;
+    ++n;
+  }
+}
+
+/*
+ * Block selection of one row (compression, step 2).  Writes the kept key-block
+ * indices ascending into kept[] and returns their count.  Optionally reports the
+ * row total, the running sum after the last kept block and before it, and the
+ * masses of the last kept and first dropped candidate (for boundary accounting;
+ * -1 where there is none).
+ */
+int mfo_select(const double* mass, int qb, double tau, int32_t* kept, double* info /*[5] or NULL*/) {
+  int32_t* order = (int32_t*)malloc(sizeof(int32_t) * (size_t)(qb + 1));
+  walk_order(mass, qb, order);
+  double total = 0.0;
+  for (int k = 0; k <= qb; ++k) total += mass[order[k]];
+  const double target = tau * total;
+  double S = 0.0, S_prev = 0.0;
+  int n_keep = qb + 1;
+  for (int k = 0; k <= qb; ++k) {
+    S_prev = S;
+    S += mass[order[k]];
+    if (S >= target) {
+      n_keep = k + 1;
+      break;
+    }
+  }
+  if (info) {
+    info[0] = total;
+    info[1] = S;
+    info[2] = n_keep >= 2 ? S_prev : -1.0;
+    info[3] = n_keep >= 2 ? mass[order[n_keep - 1]] : -1.0;
+    info[4] = n_keep <= qb ? mass[order[n_keep]] : -1.0;
+  }
+  /* ascending copy */
+  int n = 0;
+  for (int kb = 0; kb <= qb; ++kb)
+    for (int k = 0; k < n_keep; ++k)
+      if (order[k] == kb) {
+        kept[n++] = kb;
+        break;
+      }
+  free(order);
+  return n_keep;
+}
+
+/*
+ * Kept-block write (compression, step 3): out[s][ii][jj] = A_s[qb*B+ii][kb*B+jj]
+ * where that entry is causal and inside the sequence, else 0.  out has the input
+ * dtype; the copy is exact.
+ */
+void mfo_gather_block(const void* slab, int dtype, int h_s, int B, int64_t head_stride,
+                      int64_t row_stride, int qb, int kb, int L, void* out) {
+  for (int s = 0; s < h_s; ++s)
+    for (int ii = 0; ii < B; ++ii)
+      for (int jj = 0; jj < B; ++jj) {
+        const int i = qb * B + ii, j = kb * B + jj;
+        const int64_t o = ((int64_t)s * B + ii) * B + jj;
+        const int keep = i < L && j < L && j <= i;
+        const int64_t src = s * head_stride + ii * row_stride + j;
+        if (dtype == 0)
+          ((float*)out)[o] = keep ? ((const float*)slab)[src] : 0.0f;
+        else
+          ((uint16_t*)out)[o] = keep ? ((const uint16_t*)slab)[src] : (uint16_t)0;
+      }
+}
+
+/* where the receiver's V row of one key token lives (contiguous or paged). */
+typedef struct {
+  const void* V;               /* contiguous: [T, h_kv, d]; paged: [pages, page_size, h_kv, d] */
+  int dtype;                   /* 0 f32, 1 bf16 */
+  int paged, page_size;
+  const int32_t* block_table;  /* paged: this sequence's page list */
+  int64_t k_start;             /* contiguous: first token of this sequence in V */
+  int h_kv, d;
+} mfo_vref;
+
+static int64_t v_offset(const mfo_vref* v, int64_t tok, int g) {
+  if (v->paged) {
+    const int64_t page = v->block_table[tok / v->page_size];
+    return ((page * v->page_size + tok % v->page_size) * v->h_kv + g) * (int64_t)v->d;
+  }
+  return ((v->k_start + tok) * v->h_kv + g) * (int64_t)v->d;
+}
+
+/*
+ * Fused retrieval of one query block (retrieval, all steps), for block-local rows
+ * [i0, i1) of query block qb (the caller passes rows inside the sequence only).
+ * vals: the row's kept blocks [n][h_s][B][B] with key-block indices kb[n];
+ * W: [h_r][h_s] float32 of this receiver layer.  For each row i and receiver head r:
+ *   P_r[i, j] = sum_s W[r, s] * A_s[i, j]     over the keys j <= i of the kept blocks
+ *   O[i, r, :] = sum_j P_r[i, j] * V[j, g(r), :]
+ * O: [(i1 - i0)][h_r][d] double.
+ */
+void mfo_retrieve_block(const void* vals, int dtype, const int32_t* kb, int n, int qb, int B,
+                        int h_s, const float* W, int h_r, const mfo_vref* vref, int i0, int i1,
+                        double* O) {
+  const int d = vref->d;
+  double* P = (double*)malloc(sizeof(double) * (size_t)n * B);
+  for (int ii = i0; ii < i1; ++ii)
+    for (int r = 0; r < h_r; ++r) {
+      const int g = (int)(((int64_t)r * vref->h_kv) / h_r);
+      for (int t = 0; t < n; ++t)
+        for (int jj = 0; jj < B; ++jj) {
+          double p = 0.0;
+          for (int s = 0; s < h_s; ++s)
+            p += (double)W[r * h_s + s] *
+                 value_at(vals, dtype, (((int64_t)t * h_s + s) * B + ii) * B + jj);
+          P[t * B + jj] = p;
+        }
+      double* o = O + ((int64_t)(ii - i0) * h_r + r) * d;
+      for (int c = 0; c < d; ++c) o[c] = 0.0;
+      const int64_t i = (int64_t)qb * B + ii;
+      for (int t = 0; t < n; ++t)
+        for (int jj = 0; jj < B; ++jj) {
+          const double p = P[t * B + jj];
+          if ((int64_t)kb[t] * B + jj > i) continue; /* not a causal key of row i */
+          const int64_t base = v_offset(vref, (int64_t)kb[t] * B + jj, g);
+          for (int c = 0; c < d; ++c) o[c] += p * value_at(vref->V, vref->dtype, base + c);
+        }
+    }
+  free(P);
+}
