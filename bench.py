@@ -1,0 +1,388 @@
+#!/usr/bin/env python
+"""Benchmark of the MapFlow hot path on B200: one step = mf_compress of a sender layer
+followed by mf_map_retrieve of a receiver layer (the whole hot path) on the
+Ministral-like pair (L=8192, B=64, h_s=32, h_r=32, h_kv=8, d=128, bf16, tau=0.95).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+
+Prints ONE JSON line (rank 0).  With N > 1 (torchrun) every rank runs an independent
+replica of the workload (the path has no exchange step) and the value is the sum over
+ranks divided by the slowest rank's time.  `--impl reference` times the CPU oracle on a
+bounded sample of the same workload (there is no other implementation of this method
+to run).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "mf_map_retrieve GB/s & prefill tokens/s/layer; % of roofline on 1 B200"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------------ clocks
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+           0x100: "display_clock_setting"}
+
+
+def gpu_id(dev):
+    """nvidia-smi id of a CUDA device: its PCI bus id when torch reports it."""
+    p = torch.cuda.get_device_properties(dev)
+    try:
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except AttributeError:
+        return str(dev.index)
+
+
+class ClockSampler:
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 4:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+                bits = int(parts[3], 16)
+            except ValueError:
+                continue
+            for b, name in REASONS.items():
+                if bits & b and name != "gpu_idle":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------ workload
+def workload(name, reading):
+    import synth
+    w = synth.ALL[name]
+    return w.with_(reading=reading) if reading != w.reading else w
+
+
+def describe(w):
+    return (f"{w.name}: lens={list(w.lens) if len(w.lens) <= 4 else f'{len(w.lens)} seqs'} B={w.B} "
+            f"h_s={w.h_s} h_r={w.h_r} h_kv={w.h_kv} d={w.d} {w.dtype} tau={w.tau} "
+            f"heavy={w.n_heavy} map reading R{w.reading}")
+
+
+def algorithmic(w, nnz):
+    """Algorithmic bytes / FLOPs of one compress and one retrieve launch."""
+    e = 4 if w.dtype == "f32" else 2
+    blk = w.h_s * w.B * w.B * e
+    rows = sum(w.nqb)
+    comp_bytes = w.causal_blocks * blk + nnz * blk + 4 * nnz + 4 * (rows + 1)
+    ret_bytes = (nnz * blk + w.tokens * w.h_kv * w.d * e + w.tokens * w.h_r * w.d * e
+                 + 4 * nnz + 4 * (rows + 1) + 4 * w.h_r * w.h_s)
+    ret_flops = nnz * (2 * w.h_r * w.h_s * w.B * w.B + 2 * w.h_r * w.B * w.B * w.d)
+    return comp_bytes, ret_bytes, ret_flops
+
+
+# ------------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, dev):
+    import cross_model_attention_mf_b200 as mf
+    from synth import device as sdev
+
+    w = workload(args.workload, args.reading)
+    torch.cuda.set_device(dev)
+    pack = sdev.fill_maps(sdev.alloc_maps(w, dev), w, 0)
+    W = sdev.w_weights(w, dev)
+    V = sdev.v_contiguous(w, 0, dev)
+    cap = w.causal_blocks
+    bsr = mf.alloc_bsr(sum(w.nqb), cap, w.h_s, w.B, pack.maps.dtype, dev)
+    ws = torch.empty(mf.mf_compress_workspace_size(len(w.lens), max(w.lens), w.B, cap),
+                     dtype=torch.uint8, device=dev)
+    O = torch.empty((1, w.tokens, w.h_r, w.d), dtype=V.dtype, device=dev)
+    qbase = sdev.qblock_base(w, dev)
+    cu = pack.cu_seqlens
+    maxlen = max(w.lens)
+    st = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(st)
+        mf.mf_compress(pack.maps, pack.map_seq_offset, cu, maxlen, w.h_s, w.B, w.tau, bsr, ws)
+        if ev is not None:
+            ev[1].record(st)
+        mf.mf_map_retrieve([bsr], [0], W, V, cu, cu, qbase, maxlen, w.h_r, w.h_kv, O=O)
+        if ev is not None:
+            ev[2].record(st)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    rc, bits = mf.mf_get_status()
+    if rc != mf.MF_OK:
+        raise RuntimeError(f"device status {rc} bits {bits:#x}")
+    nnz = int(bsr.nnz.cpu()[0])
+
+    # per-kernel durations (CUDA events on the launching stream)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(min(args.steps, 200))]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for ev in evs:
+        step(ev)
+    torch.cuda.synchronize()
+    t_comp = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) * 1e-3
+    t_ret = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) * 1e-3
+
+    # the timed region: exactly K steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_id(dev)) as clk:
+        t0.record(st)
+        for _ in range(args.steps):
+            step()
+        t1.record(st)
+        torch.cuda.synchronize()
+    elapsed = t0.elapsed_time(t1) * 1e-3
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed = float(t.item())
+        torch.distributed.barrier()
+    rc, bits = mf.mf_get_status()
+    if rc != mf.MF_OK:
+        raise RuntimeError(f"device status {rc} bits {bits:#x}")
+
+    # end to end through the public API from pinned host buffers
+    e2e = None
+    if rank == 0 and not args.no_e2e:
+        e2e = run_e2e(args, w, mf, pack, W, V, bsr, ws, O, qbase, dev)
+
+    return dict(w=w, nnz=nnz, elapsed=elapsed, t_comp=t_comp, t_ret=t_ret, clocks=clk.summary(),
+                e2e=e2e)
+
+
+def run_e2e(args, w, mf, pack, W, V, bsr, ws, O, qbase, dev):
+    h_maps = torch.empty(pack.maps.shape, dtype=pack.maps.dtype, pin_memory=True)
+    h_maps.copy_(pack.maps)
+    h_V = torch.empty(V.shape, dtype=V.dtype, pin_memory=True)
+    h_V.copy_(V)
+    h_W = torch.empty(W.shape, dtype=W.dtype, pin_memory=True)
+    h_W.copy_(W)
+    h_O = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    st = torch.cuda.current_stream()
+    cu = pack.cu_seqlens
+    maxlen = max(w.lens)
+    n = max(1, min(args.steps, args.e2e_steps))
+
+    def e2e_step():
+        pack.maps.copy_(h_maps, non_blocking=True)
+        V.copy_(h_V, non_blocking=True)
+        W.copy_(h_W, non_blocking=True)
+        mf.mf_compress(pack.maps, pack.map_seq_offset, cu, maxlen, w.h_s, w.B, w.tau, bsr, ws)
+        mf.mf_map_retrieve([bsr], [0], W, V, cu, cu, qbase, maxlen, w.h_r, w.h_kv, O=O)
+        h_O.copy_(O, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(st)
+    for _ in range(n):
+        e2e_step()
+    t1.record(st)
+    torch.cuda.synchronize()
+    dt = t0.elapsed_time(t1) * 1e-3 / n
+    h2d = h_maps.numel() * h_maps.element_size() + h_V.numel() * h_V.element_size() + h_W.numel() * 4
+    d2h = h_O.numel() * h_O.element_size()
+    return {"value": w.tokens / dt, "unit": "tokens/s/layer", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": n}
+
+
+# ------------------------------------------------------------------------ oracle (CPU baseline)
+def oracle_sample(w, pack_host_rows, W_l, V_host, rows):
+    """Oracle compress + retrieve of the sampled query blocks (whole sequences)."""
+    import oracle
+    t0 = time.perf_counter()
+    for (qb, slab) in zip(rows, pack_host_rows):
+        m = oracle.row_masses(slab, w.lens[0], w.B, qb)
+        kept, _ = oracle.select(m, qb, w.tau)
+        vals = np.stack([oracle.gather_block(slab, w.lens[0], w.B, qb, int(kb)) for kb in kept])
+        lo, hi = 0, min(w.lens[0], (qb + 1) * w.B) - qb * w.B
+        oracle.retrieve_block(vals, kept, qb, w.B, W_l, V_host, w.h_kv, (lo, hi))
+    return time.perf_counter() - t0
+
+
+def cpu_sample_inputs(w, n_rows, dev):
+    """Host copies of n_rows query-block rows spread over the sequence (first sequence)."""
+    from synth import device as sdev
+    pack = sdev.fill_maps(sdev.alloc_maps(w, dev), w, 0)
+    W = sdev.w_weights(w, dev)
+    V = sdev.v_contiguous(w, 0, dev)
+    nqb = w.nqb[0]
+    rows = sorted(set(np.linspace(0, nqb - 1, n_rows).astype(int).tolist()))
+    view = pack.seq_view(0, w.h_s, w.B)
+    slabs = [view[:, qb * w.B:(qb + 1) * w.B, :(qb + 1) * w.B].cpu() for qb in rows]
+    out = (rows, slabs, W[0].cpu().numpy(), V[:w.lens[0]].cpu())
+    del pack
+    torch.cuda.empty_cache()
+    return out
+
+
+def cpu_baseline(w, dev, n_rows):
+    rows, slabs, W_l, V_host = cpu_sample_inputs(w, n_rows, dev)
+    dt = oracle_sample(w, slabs, W_l, V_host, rows)
+    toks = sum(min(w.lens[0], (qb + 1) * w.B) - qb * w.B for qb in rows)
+    return {"value": toks / dt, "unit": "tokens/s/layer", "cores": 1, "kind": "oracle",
+            "sample": f"{len(rows)} of {w.nqb[0]} query blocks ({toks} tokens) of sequence 0, "
+                      f"compress + retrieve, single-threaded C oracle, {dt:.1f} s"}
+
+
+# ------------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="ministral_pair")
+    ap.add_argument("--reading", type=int, default=1)
+    ap.add_argument("--cpu-rows", type=int, default=24)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = workload(args.workload, args.reading)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        # each step: the oracle on one query block of the workload (cycling over 8 blocks
+        # spread along the sequence); the run stops early after ~60 s of CPU time
+        rows, slabs, W_l, V_host = cpu_sample_inputs(w, 8, dev)
+        one = lambda t: oracle_sample(w, [slabs[t % len(rows)]], W_l, V_host, [rows[t % len(rows)]])
+        warm = min(args.warmup, 2)
+        for t in range(warm):
+            one(t)
+        spent, k, toks = 0.0, 0, 0
+        while k < max(args.steps, 1) and (spent < 60.0 or k == 0):
+            spent += one(k)
+            qb = rows[k % len(rows)]
+            toks += min(w.lens[0], (qb + 1) * w.B) - qb * w.B
+            k += 1
+        dt = spent / k
+        v = toks / spent
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s/layer",
+                "n_gpus": args.gpus, "steps": k, "warmup": warm, "ms_per_step": dt * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": {"workload": describe(w)},
+                "cpu_baseline": {"value": v, "unit": "tokens/s/layer", "cores": 1, "kind": "oracle",
+                                 "sample": f"{k} steps of one query block each ({toks} tokens), "
+                                           f"compress + retrieve, single-threaded C oracle"},
+                "e2e": {"value": v, "unit": "tokens/s/layer", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    res = run_ours(args, rank, world, dev)
+    if rank == 0:
+        hbm, tf_burst, tf_sus, src = peaks()
+        w = res["w"]
+        nnz = res["nnz"]
+        comp_b, ret_b, ret_f = algorithmic(w, nnz)
+        step_t = res["elapsed"] / args.steps
+        value = world * w.tokens / step_t
+        comp_gbs = comp_b / res["t_comp"] / 1e9
+        ret_gbs = ret_b / res["t_ret"] / 1e9
+        ret_tf = ret_f / res["t_ret"] / 1e12
+        ret_roof_t = max(ret_b / (hbm * 1e9), ret_f / (tf_burst * 1e12))
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s/layer", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_t * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": describe(w), "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (dense maps of 4.3 GB stream through every step)",
+                       "step": "mf_compress (sender layer) + mf_map_retrieve (receiver layer)"},
+            "density": nnz / w.causal_blocks, "nnz": nnz,
+            "compress": {"ms": res["t_comp"] * 1e3, "GB/s": comp_gbs, "bytes": comp_b,
+                         "frac_hbm": comp_gbs / hbm},
+            "retrieve": {"ms": res["t_ret"] * 1e3, "GB/s": ret_gbs, "TFLOP/s": ret_tf,
+                         "bytes": ret_b, "flops": ret_f,
+                         "tokens_per_s_layer": w.tokens / res["t_ret"],
+                         "roofline_frac": ret_roof_t / res["t_ret"],
+                         "bound": "hbm" if ret_b / (hbm * 1e9) >= ret_f / (tf_burst * 1e12) else "tensor"},
+            "roofline": {"bound": "hbm", "kernel": "mf_compress (block stats + select + gather)",
+                         "achieved": comp_gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": comp_gbs / hbm, "traffic": None, "peak_source": src},
+            "gpu_launches": 6 * args.steps,
+            "clocks": res["clocks"],
+        }
+        if res["e2e"] is not None:
+            line["e2e"] = res["e2e"]
+        if not args.no_cpu and world == 1:
+            line["cpu_baseline"] = cpu_baseline(w, dev, args.cpu_rows)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,248 @@
+"""Python binding of libmf (include/mf.h): MapFlow compression and fused retrieval on B200.
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+libmf.so.  PyTorch supplies device memory and the current stream.  Importing
+this package fails loudly when libmf.so is missing; there is no fallback.
+
+Functions mirror the C entry points:
+    mf_compress(...)        -> BSR (row_ptr, col_idx, values, nnz)
+    mf_map_retrieve(...)    -> O
+    mf_get_status()         -> (status, bits)
+    mf_compress_workspace_size(...), mf_retrieve_path(...), mf_version()
+"""
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import List, Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmf.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m cross_model_attention_mf_b200.build` "
+                      "(nvcc, sm_100a); this package has no CPU or library fallback")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+MF_OK, MF_ERR_INVALID, MF_ERR_UNSUPPORTED, MF_ERR_CAPACITY, MF_ERR_CUDA, MF_ERR_TIMEOUT, \
+    MF_ERR_DEVICE_INDEX = range(7)
+MF_F32, MF_BF16 = 0, 1
+MF_RETRIEVE_FORCE_SIMT = 1
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+
+
+class CompressDesc(ctypes.Structure):
+    _fields_ = [("maps", _P), ("dtype", ctypes.c_int), ("map_seq_offset", _P), ("cu_seqlens", _P),
+                ("nseq", _I32), ("max_seqlen", _I32), ("h_s", _I32), ("B", _I32),
+                ("tau", ctypes.c_double), ("row_ptr", _P), ("col_idx", _P), ("values", _P),
+                ("capacity_blocks", _I64), ("nnz_out", _P), ("block_mass_out", _P)]
+
+
+class BsrDesc(ctypes.Structure):
+    _fields_ = [("row_ptr", _P), ("col_idx", _P), ("values", _P), ("capacity_blocks", _I64)]
+
+
+class RetrieveDesc(ctypes.Structure):
+    _fields_ = [("layers", ctypes.POINTER(BsrDesc)), ("n_sender_layers", _I32),
+                ("map_dtype", ctypes.c_int), ("h_s", _I32), ("B", _I32), ("layer_map", _P),
+                ("l_r_begin", _I32), ("l_r_end", _I32), ("W", _P), ("V", _P),
+                ("v_dtype", ctypes.c_int), ("v_layer_stride", _I64), ("paged", _I32),
+                ("page_size", _I32), ("n_pages", _I32), ("max_pages", _I32), ("block_table", _P),
+                ("total_k", _I64), ("cu_seqlens_q", _P), ("cu_seqlens_k", _P),
+                ("qblock_base", _P), ("nseq", _I32), ("max_seqlen_q", _I32), ("h_r", _I32),
+                ("h_kv", _I32), ("d", _I32), ("O", _P), ("o_layer_stride", _I64),
+                ("total_q", _I32), ("flags", _I32)]
+
+
+_lib.mf_compress_workspace_size.argtypes = [ctypes.POINTER(CompressDesc), ctypes.POINTER(ctypes.c_size_t)]
+_lib.mf_compress_workspace_size.restype = ctypes.c_int
+_lib.mf_compress.argtypes = [ctypes.POINTER(CompressDesc), _P, ctypes.c_size_t, _P]
+_lib.mf_compress.restype = ctypes.c_int
+_lib.mf_map_retrieve.argtypes = [ctypes.POINTER(RetrieveDesc), _P]
+_lib.mf_map_retrieve.restype = ctypes.c_int
+_lib.mf_retrieve_path.argtypes = [ctypes.POINTER(RetrieveDesc)]
+_lib.mf_retrieve_path.restype = ctypes.c_int
+_lib.mf_get_status.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
+_lib.mf_get_status.restype = ctypes.c_int
+_lib.mf_last_error.argtypes = []
+_lib.mf_last_error.restype = ctypes.c_char_p
+_lib.mf_version.argtypes = []
+_lib.mf_version.restype = ctypes.c_char_p
+_lib.mf_abi_struct_size.argtypes = [ctypes.c_int]
+_lib.mf_abi_struct_size.restype = ctypes.c_size_t
+
+for _k, _s in ((0, CompressDesc), (1, BsrDesc), (2, RetrieveDesc)):
+    if _lib.mf_abi_struct_size(_k) != ctypes.sizeof(_s):
+        raise ImportError(f"libmf.so struct {_s.__name__} size mismatch: rebuild the library")
+
+
+class MFError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"mf status {status}: {msg}")
+        self.status = status
+
+
+def _check(rc):
+    if rc != MF_OK:
+        raise MFError(rc, _lib.mf_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _dt(t: torch.Tensor):
+    if t.dtype == torch.float32:
+        return MF_F32
+    if t.dtype == torch.bfloat16:
+        return MF_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def mf_version() -> str:
+    return _lib.mf_version().decode()
+
+
+@dataclass
+class BSR:
+    """Compressed sender layer (device tensors)."""
+    row_ptr: torch.Tensor   # int32 [R + 1]
+    col_idx: torch.Tensor   # int32 [capacity]
+    values: torch.Tensor    # [capacity, h_s, B, B]
+    nnz: torch.Tensor       # int32 [1]
+    block_mass: Optional[torch.Tensor] = None  # float64 [causal blocks]
+
+    @property
+    def capacity(self) -> int:
+        return self.values.shape[0]
+
+    def desc(self) -> BsrDesc:
+        return BsrDesc(self.row_ptr.data_ptr(), self.col_idx.data_ptr(), self.values.data_ptr(),
+                       self.capacity)
+
+
+def _compress_desc(maps, map_seq_offset, cu_seqlens, max_seqlen, h_s, B, tau, out: BSR):
+    return CompressDesc(_ptr(maps), _dt(maps), _ptr(map_seq_offset), _ptr(cu_seqlens),
+                        cu_seqlens.numel() - 1, int(max_seqlen), int(h_s), int(B), float(tau),
+                        _ptr(out.row_ptr), _ptr(out.col_idx), _ptr(out.values), out.capacity,
+                        _ptr(out.nnz), _ptr(out.block_mass))
+
+
+def mf_compress_workspace_size(nseq: int, max_seqlen: int, B: int, capacity: int) -> int:
+    d = CompressDesc()
+    d.nseq, d.max_seqlen, d.B, d.capacity_blocks = nseq, max_seqlen, B, capacity
+    n = ctypes.c_size_t(0)
+    _check(_lib.mf_compress_workspace_size(ctypes.byref(d), ctypes.byref(n)))
+    return n.value
+
+
+def alloc_bsr(n_rows: int, capacity: int, h_s: int, B: int, dtype, device, n_causal: int = 0) -> BSR:
+    """Output buffers of one compressed layer (PyTorch allocations)."""
+    return BSR(torch.empty(n_rows + 1, dtype=torch.int32, device=device),
+               torch.empty(max(capacity, 1), dtype=torch.int32, device=device),
+               torch.empty((max(capacity, 1), h_s, B, B), dtype=dtype, device=device),
+               torch.empty(1, dtype=torch.int32, device=device),
+               torch.empty(n_causal, dtype=torch.float64, device=device) if n_causal else None)
+
+
+def mf_compress(maps: torch.Tensor, map_seq_offset: torch.Tensor, cu_seqlens: torch.Tensor,
+                max_seqlen: int, h_s: int, B: int, tau: float, out: BSR,
+                workspace: Optional[torch.Tensor] = None, stream=None) -> BSR:
+    """Enqueue compression of one sender layer into `out` (see mf.h for the layout)."""
+    d = _compress_desc(maps, map_seq_offset, cu_seqlens, max_seqlen, h_s, B, tau, out)
+    need = ctypes.c_size_t(0)
+    _check(_lib.mf_compress_workspace_size(ctypes.byref(d), ctypes.byref(need)))
+    if workspace is None:
+        workspace = torch.empty(need.value, dtype=torch.uint8, device=maps.device)
+    _check(_lib.mf_compress(ctypes.byref(d), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+def _retrieve_desc(layers: Sequence[BSR], layer_map: Sequence[int], l_r_range, W, V, O,
+                   cu_seqlens_q, cu_seqlens_k, qblock_base, max_seqlen_q, h_s, B, h_r, h_kv,
+                   v_layer_stride=0, o_layer_stride=0, paged=None, flags=0):
+    arr = (BsrDesc * len(layers))(*[b.desc() for b in layers])
+    lm = (ctypes.c_int32 * len(layer_map))(*layer_map)
+    d = RetrieveDesc()
+    d.layers = arr
+    d.n_sender_layers = len(layers)
+    d.map_dtype = _dt(layers[0].values)
+    d.h_s, d.B = h_s, B
+    d.layer_map = ctypes.cast(lm, _P)
+    d.l_r_begin, d.l_r_end = l_r_range
+    d.W, d.V = _ptr(W), _ptr(V)
+    d.v_dtype = _dt(V)
+    d.v_layer_stride = v_layer_stride
+    if paged is not None:
+        block_table, page_size = paged
+        d.paged, d.page_size = 1, page_size
+        d.n_pages = V.shape[-4]
+        d.max_pages = block_table.shape[-1]
+        d.block_table = _ptr(block_table)
+    else:
+        d.total_k = V.shape[-3]
+    d.cu_seqlens_q, d.cu_seqlens_k, d.qblock_base = _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), _ptr(qblock_base)
+    d.nseq = cu_seqlens_q.numel() - 1
+    d.max_seqlen_q = int(max_seqlen_q)
+    d.h_r, d.h_kv, d.d = h_r, h_kv, V.shape[-1]
+    d.O = _ptr(O)
+    d.o_layer_stride = o_layer_stride
+    d.total_q = O.shape[-3]
+    d.flags = flags
+    return d, (arr, lm)  # keep the ctypes arrays alive
+
+
+def mf_map_retrieve(layers: Sequence[BSR], layer_map: Sequence[int], W: torch.Tensor,
+                    V: torch.Tensor, cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                    qblock_base: torch.Tensor, max_seqlen_q: int, h_r: int, h_kv: int,
+                    O: Optional[torch.Tensor] = None, l_r_range=None, total_q: Optional[int] = None,
+                    paged=None, v_layer_stride: int = 0, force_simt: bool = False,
+                    stream=None) -> torch.Tensor:
+    """Enqueue fused retrieval for receiver layers l_r_range (default: all of layer_map).
+    O: [n_layers, T_q, h_r, d] (allocated when None).  paged = (block_table, page_size)."""
+    if l_r_range is None:
+        l_r_range = (0, len(layer_map))
+    n_l = l_r_range[1] - l_r_range[0]
+    h_s, B = layers[0].values.shape[1], layers[0].values.shape[2]
+    if O is None:
+        if total_q is None:
+            raise ValueError("total_q is needed to allocate O")
+        O = torch.empty((n_l, total_q, h_r, V.shape[-1]), dtype=V.dtype, device=V.device)
+    d, keep = _retrieve_desc(layers, layer_map, l_r_range, W, V, O, cu_seqlens_q, cu_seqlens_k,
+                             qblock_base, max_seqlen_q, h_s, B, h_r, h_kv, v_layer_stride,
+                             0, paged, MF_RETRIEVE_FORCE_SIMT if force_simt else 0)
+    _check(_lib.mf_map_retrieve(ctypes.byref(d), _stream(stream)))
+    del keep
+    return O
+
+
+def mf_retrieve_path(layers, layer_map, W, V, cu_seqlens_q, cu_seqlens_k, qblock_base,
+                     max_seqlen_q, h_r, h_kv, O, paged=None, force_simt=False) -> int:
+    h_s, B = layers[0].values.shape[1], layers[0].values.shape[2]
+    d, keep = _retrieve_desc(layers, layer_map, (0, len(layer_map)), W, V, O, cu_seqlens_q,
+                             cu_seqlens_k, qblock_base, max_seqlen_q, h_s, B, h_r, h_kv, 0, 0,
+                             paged, MF_RETRIEVE_FORCE_SIMT if force_simt else 0)
+    return _lib.mf_retrieve_path(ctypes.byref(d))
+
+
+def mf_get_status(stream=None):
+    """Synchronise the stream; return (status, bits) of the device status word and clear it."""
+    bits = ctypes.c_uint32(0)
+    rc = _lib.mf_get_status(_stream(stream), ctypes.byref(bits))
+    return rc, bits.value
+
+
+def check_device_status(stream=None):
+    rc, bits = mf_get_status(stream)
+    if rc != MF_OK:
+        raise MFError(rc, f"{_lib.mf_last_error().decode()} (bits {bits:#x})")

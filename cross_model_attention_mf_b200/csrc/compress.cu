@@ -1,0 +1,423 @@
+// Block-sparse compression of one sender layer's attention maps.
+//
+// MapFlow page "MapFlow开源:大模型换班,Prefill为何能快20%?" (aitest123.com),
+// section "存不下、读得慢?三个工程优化手段", subsection 1 "只存重要的:块稀疏压缩":
+// the map is cut into regular 2-D blocks; block-level statistics are computed
+// first, then the blocks to keep are chosen by cumulative attention probability,
+// and only those are written -- no second dense matrix is assembled.
+//
+// Kernels (one launch each, all on the caller's stream):
+//   k_meta          per-sequence geometry of the varlen pack (one thread)
+//   k_stats         head-summed mass of every causal block: a streaming reduction
+//                   with 16-byte loads, float32 partials of 8 (bf16) or 4 (f32)
+//                   elements combined in float64, fixed order (deterministic)
+//   k_select        per query block: sort candidates (mass desc, kb asc), walk
+//                   the running float64 sum until it reaches tau * total
+//   k_scan_compact  row_ptr by exclusive scan, then col_idx in ascending order
+//   k_gather        copy each kept block with the causal/length mask applied
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "mf_internal.cuh"
+
+namespace mfi {
+namespace {
+
+constexpr int META_HDR = 4;
+
+__device__ inline int find_seq(const int64_t* meta, int nseq, int64_t x, int field) {
+  // last s with meta[seq s].field <= x (fields are non-decreasing in s)
+  int lo = 0, hi = nseq - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (meta[META_HDR + 4 * mid + field] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ inline int tri_row(int64_t c) {
+  int q = (int)((sqrt(8.0 * (double)c + 1.0) - 1.0) * 0.5);
+  while ((int64_t)(q + 1) * (q + 2) / 2 <= c) ++q;
+  while ((int64_t)q * (q + 1) / 2 > c) --q;
+  return q;
+}
+
+__global__ void k_meta(const int32_t* cu, const int64_t* off, int nseq, int max_seqlen, int B,
+                       int elem_bytes, int64_t* meta, uint32_t* status) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int64_t rows = 0, cb = 0;
+  uint32_t st = 0;
+  for (int s = 0; s < nseq; ++s) {
+    int64_t L = (int64_t)cu[s + 1] - cu[s];
+    if (L < 0 || L > max_seqlen) { st |= ST_INDEX; L = 0; }
+    if ((off[s] * elem_bytes) % 16 != 0 || off[s] < 0) { st |= ST_ALIGN; L = 0; }
+    const int64_t nqb = (L + B - 1) / B;
+    int64_t* m = meta + META_HDR + 4 * s;
+    m[0] = L; m[1] = nqb; m[2] = rows; m[3] = cb;
+    rows += nqb;
+    cb += nqb * (nqb + 1) / 2;
+  }
+  meta[0] = rows; meta[1] = cb; meta[2] = 0; meta[3] = 0;
+  if (st) atomicOr(status, st);
+}
+
+template <typename T> struct Vec;
+template <> struct Vec<float> {
+  static constexpr int EPV = 4;
+  __device__ static float get(const uint4& v, int e) {
+    const uint32_t w = e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w;
+    return __uint_as_float(w);
+  }
+};
+template <> struct Vec<__nv_bfloat16> {
+  static constexpr int EPV = 8;
+  __device__ static float get(const uint4& v, int e) {
+    const uint32_t w = (e >> 1) == 0 ? v.x : (e >> 1) == 1 ? v.y : (e >> 1) == 2 ? v.z : v.w;
+    return __uint_as_float((e & 1) ? (w & 0xffff0000u) : (w << 16));
+  }
+};
+
+template <int NT>
+__device__ inline double block_sum_f64(double v, double* red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  double t = 0.0;
+  if (threadIdx.x == 0)
+    for (int k = 0; k < NT / 32; ++k) t += red[k];
+  __syncthreads();
+  return t;  // valid in thread 0
+}
+
+// Masses of every causal block.  Item = (sequence, qb, kb) over all sender heads.
+template <typename T, int B, int NT>
+__global__ void __launch_bounds__(NT) k_stats(const T* __restrict__ maps,
+                                              const int64_t* __restrict__ seq_off,
+                                              const int64_t* __restrict__ meta, int nseq,
+                                              int h_s, double* __restrict__ mass) {
+  constexpr int EPV = Vec<T>::EPV, VPR = B / EPV, VPB = B * VPR;  // vectors per row / per head
+  constexpr int U = 4;
+  __shared__ double red[NT / 32];
+  const int64_t total = meta[1];
+  const int64_t nv = (int64_t)h_s * VPB;
+  for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
+    const int s = find_seq(meta, nseq, item, 3);
+    const int64_t* m = meta + META_HDR + 4 * s;
+    const int64_t L = m[0], Lp = m[1] * B, c = item - m[3];
+    const int qb = tri_row(c);
+    const int kb = (int)(c - (int64_t)qb * (qb + 1) / 2);
+    const T* base = maps + seq_off[s];
+    const bool full = kb < qb && (int64_t)(qb + 1) * B <= L;
+    double acc = 0.0;
+    for (int64_t v0 = threadIdx.x; v0 < nv; v0 += (int64_t)NT * U) {
+      uint4 r[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t v = v0 + (int64_t)u * NT;
+        if (v < nv) {
+          const int64_t hs = v / VPB;
+          const int rem = (int)(v - hs * VPB);
+          const int ii = rem / VPR, jv = rem % VPR;
+          const T* p = base + ((hs * Lp) + (int64_t)qb * B + ii) * Lp + (int64_t)kb * B + jv * EPV;
+          r[u] = __ldg(reinterpret_cast<const uint4*>(p));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t v = v0 + (int64_t)u * NT;
+        if (v < nv) {
+          float part = 0.0f;
+          if (full) {
+            float a[EPV];
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) a[e] = Vec<T>::get(r[u], e);
+            if constexpr (EPV == 8)
+              part = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+            else
+              part = (a[0] + a[1]) + (a[2] + a[3]);
+          } else {
+            const int64_t hs = v / VPB;
+            const int rem = (int)(v - hs * VPB);
+            const int ii = rem / VPR, jv = rem % VPR;
+            const int64_t i = (int64_t)qb * B + ii;
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) {
+              const int64_t j = (int64_t)kb * B + jv * EPV + e;
+              if (i < L && j <= i) part += Vec<T>::get(r[u], e);
+            }
+          }
+          acc += (double)part;
+        }
+      }
+    }
+    const double t = block_sum_f64<NT>(acc, red);
+    if (threadIdx.x == 0) mass[item] = t;
+  }
+}
+
+__device__ inline uint64_t order_key(double x) {
+  if (x == 0.0) x = 0.0;  // -0 sorts with +0
+  const uint64_t b = (uint64_t)__double_as_longlong(x);
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+// One CTA per query block (row).  Candidates kb < qb sorted by (mass desc, kb asc);
+// the walk starts from the diagonal block.
+template <int NT>
+__global__ void __launch_bounds__(NT) k_select(const int64_t* __restrict__ meta, int nseq,
+                                               const double* __restrict__ mass, double tau,
+                                               int32_t* __restrict__ counts,
+                                               uint8_t* __restrict__ flags) {
+  extern __shared__ uint64_t sm[];
+  __shared__ int s_nkeep;
+  const int64_t row = blockIdx.x;
+  if (row >= meta[0]) return;
+  const int s = find_seq(meta, nseq, row, 2);
+  const int64_t* m = meta + META_HDR + 4 * s;
+  const int qb = (int)(row - m[2]);
+  const int64_t tri = m[3] + (int64_t)qb * (qb + 1) / 2;
+  const double* mr = mass + tri;
+  const int n = qb;
+  int n2 = 1;
+  while (n2 < n) n2 <<= 1;
+  uint64_t* key = sm;
+  int* idx = reinterpret_cast<int*>(sm + n2);
+  for (int t = threadIdx.x; t < n2; t += NT) {
+    if (t < n) { key[t] = order_key(mr[t]); idx[t] = t; }
+    else { key[t] = 0ull; idx[t] = 0x7fffffff; }
+  }
+  __syncthreads();
+  // bitonic sort into (key desc, idx asc)
+  for (int k = 2; k <= n2; k <<= 1)
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int t = threadIdx.x; t < n2; t += NT) {
+        const int p = t ^ j;
+        if (p > t) {
+          const bool up = (t & k) == 0;  // this run sorts into the target order
+          const uint64_t ka = key[t], kb2 = key[p];
+          const int ia = idx[t], ib = idx[p];
+          const bool a_first = ka > kb2 || (ka == kb2 && ia < ib);
+          if (up != a_first) {
+            key[t] = kb2; key[p] = ka; idx[t] = ib; idx[p] = ia;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  if (threadIdx.x == 0) {
+    double total = 0.0;
+    total += mr[qb];
+    for (int t = 0; t < n; ++t) total += mr[idx[t]];
+    const double target = tau * total;
+    double S = 0.0;
+    int nk = n + 1;
+    S += mr[qb];
+    if (S >= target) {
+      nk = 1;
+    } else {
+      for (int t = 0; t < n; ++t) {
+        S += mr[idx[t]];
+        if (S >= target) { nk = t + 2; break; }
+      }
+    }
+    s_nkeep = nk;
+    counts[row] = nk;
+    flags[tri + qb] = 1;
+  }
+  __syncthreads();
+  const int nk = s_nkeep;
+  for (int t = threadIdx.x; t < n; t += NT) flags[tri + idx[t]] = (uint8_t)(t < nk - 1);
+}
+
+// One CTA: exclusive scan of counts into row_ptr, then ascending col_idx per row.
+constexpr int SCAN_NT = 1024;
+__global__ void __launch_bounds__(SCAN_NT) k_scan_compact(
+    const int64_t* __restrict__ meta, int nseq, const int32_t* __restrict__ counts,
+    const uint8_t* __restrict__ flags, int32_t* __restrict__ row_ptr,
+    int32_t* __restrict__ col_idx, int32_t* __restrict__ kept_row, int32_t* __restrict__ nnz_out,
+    int64_t capacity, uint32_t* status) {
+  __shared__ int64_t part[SCAN_NT];
+  const int64_t R = meta[0];
+  const int t = threadIdx.x;
+  const int64_t chunk = (R + SCAN_NT - 1) / SCAN_NT;
+  const int64_t r0 = t * chunk, r1 = min(R, r0 + chunk);
+  int64_t sum = 0;
+  for (int64_t r = r0; r < r1; ++r) sum += counts[r];
+  part[t] = sum;
+  __syncthreads();
+  for (int o = 1; o < SCAN_NT; o <<= 1) {  // inclusive Hillis-Steele scan
+    const int64_t v = t >= o ? part[t - o] : 0;
+    __syncthreads();
+    part[t] += v;
+    __syncthreads();
+  }
+  int64_t run = part[t] - sum;
+  for (int64_t r = r0; r < r1; ++r) {
+    row_ptr[r] = (int32_t)run;
+    run += counts[r];
+  }
+  const int64_t nnz = part[SCAN_NT - 1];
+  if (t == 0) {
+    row_ptr[R] = (int32_t)nnz;
+    *nnz_out = (int32_t)nnz;
+    if (nnz > capacity) atomicOr(status, ST_CAPACITY);
+  }
+  __syncthreads();
+  const int warp = t >> 5, lane = t & 31;
+  for (int64_t row = warp; row < R; row += SCAN_NT / 32) {
+    const int s = find_seq(meta, nseq, row, 2);
+    const int64_t* m = meta + META_HDR + 4 * s;
+    const int qb = (int)(row - m[2]);
+    const uint8_t* f = flags + m[3] + (int64_t)qb * (qb + 1) / 2;
+    int64_t base = row_ptr[row];
+    for (int k0 = 0; k0 <= qb; k0 += 32) {
+      const int kb = k0 + lane;
+      const bool fl = kb <= qb && f[kb];
+      const uint32_t bal = __ballot_sync(0xffffffffu, fl);
+      const int64_t n = base + __popc(bal & ((1u << lane) - 1u));
+      if (fl && n < capacity) {
+        col_idx[n] = kb;
+        kept_row[n] = (int32_t)row;
+      }
+      base += __popc(bal);
+    }
+  }
+}
+
+template <typename T, int B, int NT>
+__global__ void __launch_bounds__(NT) k_gather(const T* __restrict__ maps,
+                                               const int64_t* __restrict__ seq_off,
+                                               const int64_t* __restrict__ meta, int nseq,
+                                               int h_s, const int32_t* __restrict__ nnz_in,
+                                               int64_t capacity,
+                                               const int32_t* __restrict__ col_idx,
+                                               const int32_t* __restrict__ kept_row,
+                                               T* __restrict__ values) {
+  constexpr int EPV = Vec<T>::EPV, VPR = B / EPV, VPB = B * VPR;
+  constexpr int U = 4;
+  const int64_t nnz = min((int64_t)*nnz_in, capacity);
+  const int64_t nv = (int64_t)h_s * VPB;
+  for (int64_t n = blockIdx.x; n < nnz; n += gridDim.x) {
+    const int64_t row = kept_row[n];
+    const int kb = col_idx[n];
+    const int s = find_seq(meta, nseq, row, 2);
+    const int64_t* m = meta + META_HDR + 4 * s;
+    const int64_t L = m[0], Lp = m[1] * B;
+    const int qb = (int)(row - m[2]);
+    const T* base = maps + seq_off[s];
+    uint4* dst = reinterpret_cast<uint4*>(values + n * (int64_t)h_s * B * B);
+    const bool full = kb < qb && (int64_t)(qb + 1) * B <= L;
+    for (int64_t v0 = threadIdx.x; v0 < nv; v0 += (int64_t)NT * U) {
+      uint4 r[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t v = v0 + (int64_t)u * NT;
+        if (v < nv) {
+          const int64_t hs = v / VPB;
+          const int rem = (int)(v - hs * VPB);
+          const int ii = rem / VPR, jv = rem % VPR;
+          const T* p = base + ((hs * Lp) + (int64_t)qb * B + ii) * Lp + (int64_t)kb * B + jv * EPV;
+          r[u] = __ldg(reinterpret_cast<const uint4*>(p));
+          if (!full) {
+            const int64_t i = (int64_t)qb * B + ii;
+            uint32_t w[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) {
+              const int64_t j = (int64_t)kb * B + jv * EPV + e;
+              if (!(i < L && j <= i)) {
+                if (EPV == 4) w[e] = 0u;
+                else w[e >> 1] &= (e & 1) ? 0x0000ffffu : 0xffff0000u;
+              }
+            }
+            r[u] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t v = v0 + (int64_t)u * NT;
+        if (v < nv) __stcs(dst + v, r[u]);
+      }
+    }
+  }
+}
+
+template <typename T, int B>
+cudaError_t launch_typed(const mf_compress_desc& d, const CompressWs& ws, uint32_t* status,
+                         cudaStream_t st, int sms) {
+  constexpr int NT = 256;
+  const T* maps = static_cast<const T*>(d.maps);
+  double* mass = d.block_mass_out ? d.block_mass_out : ws.mass;
+  const int grid_stats = (int)std::min<int64_t>(ws.max_cb, (int64_t)sms * 8);
+  k_stats<T, B, NT><<<grid_stats, NT, 0, st>>>(maps, d.map_seq_offset, ws.meta, d.nseq, d.h_s,
+                                                mass);
+  int64_t nqb_max = (d.max_seqlen + B - 1) / B;
+  int n2 = 1;
+  while (n2 < nqb_max) n2 <<= 1;
+  const size_t smem_sel = (size_t)n2 * (sizeof(uint64_t) + sizeof(int));
+  if (smem_sel > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k_select<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem_sel);
+    if (e != cudaSuccess) return e;
+  }
+  k_select<128><<<(unsigned)ws.max_rows, 128, smem_sel, st>>>(ws.meta, d.nseq, mass, d.tau,
+                                                              ws.counts, ws.flags);
+  k_scan_compact<<<1, SCAN_NT, 0, st>>>(ws.meta, d.nseq, ws.counts, ws.flags, d.row_ptr,
+                                        d.col_idx, ws.kept_row, d.nnz_out, d.capacity_blocks,
+                                        status);
+  const int grid_g = (int)std::max<int64_t>(1, std::min<int64_t>(d.capacity_blocks, (int64_t)sms * 8));
+  k_gather<T, B, NT><<<grid_g, NT, 0, st>>>(maps, d.map_seq_offset, ws.meta, d.nseq, d.h_s,
+                                            d.nnz_out, d.capacity_blocks, d.col_idx, ws.kept_row,
+                                            static_cast<T*>(d.values));
+  return cudaGetLastError();
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+size_t compress_ws_layout(const mf_compress_desc& d, CompressWs* ws, void* base) {
+  const int64_t nqb_max = (d.max_seqlen + d.B - 1) / d.B;
+  const int64_t max_rows = (int64_t)d.nseq * nqb_max;
+  const int64_t max_cb = (int64_t)d.nseq * nqb_max * (nqb_max + 1) / 2;
+  size_t off = 0;
+  const size_t o_meta = off; off = align_up(off + sizeof(int64_t) * (META_HDR + 4 * (size_t)d.nseq), 256);
+  const size_t o_mass = off; off = align_up(off + sizeof(double) * (size_t)max_cb, 256);
+  const size_t o_flags = off; off = align_up(off + (size_t)max_cb, 256);
+  const size_t o_counts = off; off = align_up(off + sizeof(int32_t) * (size_t)max_rows, 256);
+  const size_t o_kept = off; off = align_up(off + sizeof(int32_t) * (size_t)std::max<int64_t>(d.capacity_blocks, 1), 256);
+  if (ws) {
+    char* b = static_cast<char*>(base);
+    ws->meta = reinterpret_cast<int64_t*>(b + o_meta);
+    ws->mass = reinterpret_cast<double*>(b + o_mass);
+    ws->flags = reinterpret_cast<uint8_t*>(b + o_flags);
+    ws->counts = reinterpret_cast<int32_t*>(b + o_counts);
+    ws->kept_row = reinterpret_cast<int32_t*>(b + o_kept);
+    ws->max_cb = max_cb;
+    ws->max_rows = max_rows;
+  }
+  return off;
+}
+
+cudaError_t launch_compress(const mf_compress_desc& d, const CompressWs& ws, uint32_t* status,
+                            cudaStream_t st) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int elem = d.dtype == MF_F32 ? 4 : 2;
+  k_meta<<<1, 32, 0, st>>>(d.cu_seqlens, d.map_seq_offset, d.nseq, d.max_seqlen, d.B, elem,
+                           ws.meta, status);
+  if (d.dtype == MF_F32) {
+    if (d.B == 32) return launch_typed<float, 32>(d, ws, status, st, sms);
+    if (d.B == 64) return launch_typed<float, 64>(d, ws, status, st, sms);
+    return launch_typed<float, 128>(d, ws, status, st, sms);
+  }
+  if (d.B == 32) return launch_typed<__nv_bfloat16, 32>(d, ws, status, st, sms);
+  if (d.B == 64) return launch_typed<__nv_bfloat16, 64>(d, ws, status, st, sms);
+  return launch_typed<__nv_bfloat16, 128>(d, ws, status, st, sms);
+}
+
+}  // namespace mfi

@@ -1,0 +1,184 @@
+// C ABI (include/mf.h): host-side validation, workspace carving, launches, status word.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstdio>
+#include <string>
+
+#include "mf.h"
+#include "mf_internal.cuh"
+
+namespace {
+
+// per-device status word (each device that loads the library has its own copy)
+__device__ uint32_t g_status;
+
+thread_local std::string t_err;
+
+mf_status fail(mf_status s, const std::string& msg) {
+  t_err = msg;
+  return s;
+}
+
+uint32_t* status_ptr() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+  return static_cast<uint32_t*>(p);
+}
+
+bool is_dtype(int d) { return d == MF_F32 || d == MF_BF16; }
+
+mf_status check_compress(const mf_compress_desc* d) {
+  if (!d) return fail(MF_ERR_INVALID, "desc is NULL");
+  if (!is_dtype(d->dtype)) return fail(MF_ERR_INVALID, "dtype must be MF_F32 or MF_BF16");
+  if (!d->maps || !d->map_seq_offset || !d->cu_seqlens || !d->row_ptr || !d->col_idx ||
+      !d->values || !d->nnz_out)
+    return fail(MF_ERR_INVALID, "a required pointer is NULL");
+  if (d->nseq < 1) return fail(MF_ERR_INVALID, "nseq must be >= 1");
+  if (d->max_seqlen < 0) return fail(MF_ERR_INVALID, "max_seqlen must be >= 0");
+  if (!(d->B == 32 || d->B == 64 || d->B == 128)) return fail(MF_ERR_INVALID, "B must be 32, 64 or 128");
+  if (d->h_s < 1 || d->h_s > 256) return fail(MF_ERR_INVALID, "h_s must be in [1, 256]");
+  if (!(d->tau >= 0.0 && d->tau <= 1.0)) return fail(MF_ERR_INVALID, "tau must be in [0, 1]");
+  if (d->capacity_blocks < 0) return fail(MF_ERR_INVALID, "capacity_blocks must be >= 0");
+  const int64_t nqb = ((int64_t)d->max_seqlen + d->B - 1) / d->B;
+  if (nqb > 4096) return fail(MF_ERR_UNSUPPORTED, "more than 4096 query blocks per sequence");
+  if ((int64_t)d->nseq * nqb >= (int64_t)1 << 31) return fail(MF_ERR_UNSUPPORTED, "too many rows");
+  const int64_t elem = d->dtype == MF_F32 ? 4 : 2;
+  if ((int64_t)d->h_s * d->B * d->B * elem * d->capacity_blocks < 0)
+    return fail(MF_ERR_INVALID, "capacity overflow");
+  if (reinterpret_cast<uintptr_t>(d->maps) % 16 || reinterpret_cast<uintptr_t>(d->values) % 16)
+    return fail(MF_ERR_INVALID, "maps and values must be 16-byte aligned");
+  return MF_OK;
+}
+
+mf_status check_retrieve(const mf_retrieve_desc* d) {
+  if (!d) return fail(MF_ERR_INVALID, "desc is NULL");
+  if (!is_dtype(d->map_dtype) || !is_dtype(d->v_dtype)) return fail(MF_ERR_INVALID, "bad dtype");
+  if (!d->layers || d->n_sender_layers < 1) return fail(MF_ERR_INVALID, "no sender layers");
+  if (!d->layer_map) return fail(MF_ERR_INVALID, "layer_map is NULL");
+  if (d->l_r_begin < 0 || d->l_r_end < d->l_r_begin) return fail(MF_ERR_INVALID, "bad layer range");
+  if (!d->W || !d->V || !d->O || !d->cu_seqlens_q || !d->cu_seqlens_k || !d->qblock_base)
+    return fail(MF_ERR_INVALID, "a required pointer is NULL");
+  if (d->nseq < 1 || d->max_seqlen_q < 0) return fail(MF_ERR_INVALID, "bad nseq / max_seqlen_q");
+  if (d->B < 1 || d->B > 128 || d->h_s < 1 || d->h_s > 256) return fail(MF_ERR_INVALID, "bad B / h_s");
+  if (d->h_r < 1 || d->h_kv < 1 || d->h_r % d->h_kv) return fail(MF_ERR_INVALID, "h_r must be a multiple of h_kv");
+  if (d->d < 1 || d->d > 256) return fail(MF_ERR_INVALID, "d must be in [1, 256]");
+  if (d->paged) {
+    if (!d->block_table || d->page_size < 1 || d->n_pages < 1 || d->max_pages < 1)
+      return fail(MF_ERR_INVALID, "paged V needs block_table, page_size, n_pages, max_pages");
+  } else if (d->total_k < 0) {
+    return fail(MF_ERR_INVALID, "total_k must be >= 0");
+  }
+  for (int l = d->l_r_begin; l < d->l_r_end; ++l) {
+    const int ls = d->layer_map[l];
+    if (ls < 0 || ls >= d->n_sender_layers) return fail(MF_ERR_INVALID, "layer_map entry out of range");
+    const mf_bsr& b = d->layers[ls];
+    if (!b.row_ptr || !b.col_idx || !b.values || b.capacity_blocks < 0)
+      return fail(MF_ERR_INVALID, "incomplete BSR for a mapped sender layer");
+  }
+  if (!mfi::tc_supported(*d) && (int64_t)d->B * d->d > 16384)
+    return fail(MF_ERR_UNSUPPORTED, "B * d > 16384 needs the tensor-core path");
+  return MF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+#pragma GCC visibility push(default)
+
+const char* mf_version(void) { return "mapflow-b200 0.1.0 (sm_100a)"; }
+
+const char* mf_last_error(void) { return t_err.c_str(); }
+
+size_t mf_abi_struct_size(int which) {
+  switch (which) {
+    case 0: return sizeof(mf_compress_desc);
+    case 1: return sizeof(mf_bsr);
+    case 2: return sizeof(mf_retrieve_desc);
+    default: return 0;
+  }
+}
+
+mf_status mf_compress_workspace_size(const mf_compress_desc* desc, size_t* bytes) {
+  if (!bytes) return fail(MF_ERR_INVALID, "bytes is NULL");
+  if (!desc) return fail(MF_ERR_INVALID, "desc is NULL");
+  if (desc->nseq < 1 || desc->max_seqlen < 0 || !(desc->B == 32 || desc->B == 64 || desc->B == 128) ||
+      desc->capacity_blocks < 0)
+    return fail(MF_ERR_INVALID, "bad nseq / max_seqlen / B / capacity");
+  *bytes = mfi::compress_ws_layout(*desc, nullptr, nullptr);
+  return MF_OK;
+}
+
+mf_status mf_compress(const mf_compress_desc* desc, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  mf_status s = check_compress(desc);
+  if (s != MF_OK) return s;
+  const size_t need = mfi::compress_ws_layout(*desc, nullptr, nullptr);
+  if (!workspace || workspace_bytes < need)
+    return fail(MF_ERR_INVALID, "workspace missing or smaller than mf_compress_workspace_size");
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(MF_ERR_INVALID, "workspace must be 256-byte aligned");
+  uint32_t* st = status_ptr();
+  if (!st) return fail(MF_ERR_CUDA, "cannot resolve the device status word");
+  mfi::CompressWs ws;
+  mfi::compress_ws_layout(*desc, &ws, workspace);
+  cudaError_t e = mfi::launch_compress(*desc, ws, st, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(MF_ERR_CUDA, std::string("mf_compress launch: ") + cudaGetErrorString(e));
+  return MF_OK;
+}
+
+int mf_retrieve_path(const mf_retrieve_desc* desc) {
+  if (check_retrieve(desc) != MF_OK) return -1;
+  return mfi::tc_supported(*desc) ? 1 : 0;
+}
+
+mf_status mf_map_retrieve(const mf_retrieve_desc* desc, void* stream) {
+  mf_status s = check_retrieve(desc);
+  if (s != MF_OK) return s;
+  uint32_t* st = status_ptr();
+  if (!st) return fail(MF_ERR_CUDA, "cannot resolve the device status word");
+  const bool tc = mfi::tc_supported(*desc);
+  const int64_t ve = desc->v_dtype == MF_F32 ? 4 : 2;
+  const int64_t o_stride = desc->o_layer_stride ? desc->o_layer_stride
+                                                : (int64_t)desc->total_q * desc->h_r * desc->d;
+  for (int l = desc->l_r_begin; l < desc->l_r_end; ++l) {
+    const mf_bsr& b = desc->layers[desc->layer_map[l]];
+    mfi::RetrieveLayer L;
+    L.row_ptr = b.row_ptr;
+    L.col_idx = b.col_idx;
+    L.values = b.values;
+    L.capacity = b.capacity_blocks;
+    L.W = desc->W + (int64_t)l * desc->h_r * desc->h_s;
+    L.V = static_cast<const char*>(desc->V) + (int64_t)l * desc->v_layer_stride * ve;
+    L.O = static_cast<char*>(desc->O) + (int64_t)(l - desc->l_r_begin) * o_stride * ve;
+    if (tc) {
+      std::string err;
+      if (!mfi::launch_retrieve_tc(*desc, L, st, static_cast<cudaStream_t>(stream), &err))
+        return fail(MF_ERR_CUDA, "mf_map_retrieve (tcgen05): " + err);
+    } else {
+      cudaError_t e = mfi::launch_retrieve_simt(*desc, L, st, static_cast<cudaStream_t>(stream));
+      if (e != cudaSuccess)
+        return fail(MF_ERR_CUDA, std::string("mf_map_retrieve (simt): ") + cudaGetErrorString(e));
+    }
+  }
+  return MF_OK;
+}
+
+mf_status mf_get_status(void* stream, uint32_t* bits) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(MF_ERR_CUDA, std::string("stream: ") + cudaGetErrorString(e));
+  uint32_t v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_status, sizeof v);
+  if (e != cudaSuccess) return fail(MF_ERR_CUDA, std::string("status read: ") + cudaGetErrorString(e));
+  const uint32_t zero = 0;
+  e = cudaMemcpyToSymbol(g_status, &zero, sizeof zero);
+  if (e != cudaSuccess) return fail(MF_ERR_CUDA, std::string("status clear: ") + cudaGetErrorString(e));
+  if (bits) *bits = v;
+  if (v == 0) return MF_OK;
+  if (v & mfi::ST_INDEX) return fail(MF_ERR_DEVICE_INDEX, "device: BSR index out of range");
+  if (v & mfi::ST_CAPACITY) return fail(MF_ERR_CAPACITY, "device: kept blocks exceed capacity");
+  if (v & mfi::ST_TIMEOUT) return fail(MF_ERR_TIMEOUT, "device: pipeline wait timed out");
+  if (v & mfi::ST_ALIGN) return fail(MF_ERR_INVALID, "device: misaligned map offset");
+  return fail(MF_ERR_DEVICE_INDEX, "device: page id out of range");
+}
+
+}  // extern "C"

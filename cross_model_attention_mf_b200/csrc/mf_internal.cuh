@@ -1,0 +1,59 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "mf.h"
+
+namespace mfi {
+
+// bits of the per-device status word
+enum : uint32_t {
+  ST_INDEX = 1u,     // BSR row/column index out of range
+  ST_CAPACITY = 2u,  // more kept blocks than capacity
+  ST_TIMEOUT = 4u,   // a pipeline wait gave up
+  ST_ALIGN = 8u,     // a sequence's map offset is not 16-byte aligned
+  ST_PAGE = 16u,     // a page id out of range
+};
+
+// scratch of mf_compress (carved out of the caller's workspace)
+struct CompressWs {
+  int64_t* meta;      // [4 + 4 * nseq]: total rows, total causal blocks, -, -, then per
+                      // sequence (L, nqb, row_base, cb_base)
+  double* mass;       // [max_cb] head-summed block masses
+  uint8_t* flags;     // [max_cb] kept flags
+  int32_t* counts;    // [max_rows] kept blocks per row
+  int32_t* kept_row;  // [capacity] BSR row of each kept block
+  int64_t max_cb, max_rows;
+};
+
+// Computes the layout; with base == nullptr only the size is returned.
+size_t compress_ws_layout(const mf_compress_desc& d, CompressWs* ws, void* base);
+
+cudaError_t launch_compress(const mf_compress_desc& d, const CompressWs& ws, uint32_t* status,
+                            cudaStream_t st);
+
+// one receiver layer's pointers
+struct RetrieveLayer {
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  const void* values;
+  int64_t capacity;
+  const float* W;  // [h_r][h_s] of this layer
+  const void* V;   // this layer's V
+  void* O;         // this layer's O
+};
+
+cudaError_t launch_retrieve_simt(const mf_retrieve_desc& d, const RetrieveLayer& l,
+                                 uint32_t* status, cudaStream_t st);
+
+bool tc_supported(const mf_retrieve_desc& d);
+
+// returns false and fills *err on a host-side failure (tensor-map encoding, launch)
+bool launch_retrieve_tc(const mf_retrieve_desc& d, const RetrieveLayer& l, uint32_t* status,
+                        cudaStream_t st, std::string* err);
+
+}  // namespace mfi

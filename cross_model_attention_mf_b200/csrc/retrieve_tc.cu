@@ -1,0 +1,576 @@
+// Fused map retrieval on sm_100a tensor cores (tcgen05 + TMA + TMEM).
+//
+// MapFlow page "MapFlow开源:大模型换班,Prefill为何能快20%?" (aitest123.com),
+// section "存不下、读得慢?三个工程优化手段", subsection 3 "算得省的:融合内核执行":
+// read the kept sparse blocks, mix sender heads into receiver heads on chip,
+// multiply by the receiver's V and accumulate, without materialising the
+// receiver's dense map.  The pages' kernel is Triton on A800; this one is a
+// new design for B200.
+//
+// CTA = (sequence, query block, 16-row chunk, 4 KV groups = 16 virtual receiver
+// heads; a group of gq <= 4 heads is padded to 4).  For each kept 64-key tile:
+//
+//   mixing  D1[pos][r] = sum_s A_s[pos] * W[r][s]       tcgen05 M=128 N=16 K=16
+//           pos = (row, key) of 2 rows x 64 keys, A tile MN-major SW128 from TMA,
+//           W^T K-major in smem (bf16).  D1 is double-buffered in TMEM.
+//   convert 4 epilogue warps read D1 (lane = position), apply the causal mask,
+//           round to bf16 and write P^T[key][(row, head)] (MN-major SW128) with
+//           one 8-byte store per (position, group).
+//   P.V     D2[dim][(row, head)] += V^T[dim][key] * P^T[key][(row, head)]
+//           tcgen05 M=128 (d) N=64 K=16 per group; V tile MN-major SW128 by TMA
+//           (contiguous or paged).  D2 stays in TMEM for the whole row chunk.
+//
+// Warp roles: warp 0 TMA producer, warp 1 MMA issuer (+ TMEM owner), warps 2-5
+// convert/epilogue.  TMEM: D2 in columns [0, 256), D1 in [256, 512).  Every
+// mbarrier wait is bounded by a timer: on expiry the CTA records ST_TIMEOUT, all
+// roles stop, in-flight copies and MMAs are drained (bounded) and TMEM is freed.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "mf_internal.cuh"
+
+namespace mfi {
+namespace {
+
+constexpr int NT = 192;
+constexpr int R = 16;          // query rows per CTA
+constexpr int KT = 64;         // keys per tile
+constexpr int NG = 4;          // KV groups per CTA
+constexpr int GQP = 4;         // virtual heads per group
+constexpr int HV = NG * GQP;   // virtual receiver heads per CTA
+constexpr int D = 128;         // head dim
+constexpr int SC = 16;         // sender heads per A chunk (one MMA K step)
+constexpr int A_STAGES = 3, V_STAGES = 3;
+constexpr uint32_t A_BYTES = R * SC * KT * 2;   // 32 KB
+constexpr uint32_t V_BYTES = KT * D * 2;        // 16 KB
+constexpr uint32_t PT_BYTES = KT * 64 * 2;      // 8 KB per group
+constexpr uint32_t PBUF_BYTES = NG * PT_BYTES;  // 32 KB per tile
+constexpr uint32_t OFF_A = 0;
+constexpr uint32_t OFF_V = OFF_A + A_STAGES * A_BYTES;
+constexpr uint32_t OFF_P = OFF_V + V_STAGES * V_BYTES;
+constexpr uint32_t OFF_W = OFF_P + 2 * PBUF_BYTES;
+constexpr uint32_t W_BYTES_MAX = 4 * 512;       // up to 4 chunks (h_s <= 64)
+constexpr uint32_t OFF_BAR = OFF_W + W_BYTES_MAX;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
+constexpr uint64_t TIMEOUT_NS = 2000000000ull;
+
+// barrier slots (8 bytes each)
+enum {
+  B_AFULL = 0, B_AEMPTY = B_AFULL + A_STAGES, B_VFULL = B_AEMPTY + A_STAGES,
+  B_VEMPTY = B_VFULL + V_STAGES, B_D1FULL = B_VEMPTY + V_STAGES, B_D1EMPTY = B_D1FULL + 2,
+  B_PFULL = B_D1EMPTY + 2, B_PEMPTY = B_PFULL + 2, B_OFULL = B_PEMPTY + 2, B_COUNT = B_OFULL + 1
+};
+
+// instruction descriptors (kind::f16): D f32, A/B bf16, majors, N >> 3, M >> 4
+constexpr uint32_t IDESC_MIX = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (0u << 16) |
+                               ((16u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t IDESC_PV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                              ((64u >> 3) << 17) | ((128u >> 4) << 24);
+
+struct TcParams {
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  int64_t capacity;
+  const float* W;  // [h_r][h_s]
+  __nv_bfloat16* O;
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  const int32_t* qblock_base;
+  const int32_t* block_table;
+  int paged, page_size, n_pages, max_pages;
+  int total_k;
+  int nqbq, rcs, hcs;  // query blocks, row chunks per block, head chunks
+  int h_s, nsc, B, h_r, h_kv, gq;
+  uint32_t* status;
+};
+
+// ------------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false if the CTA aborted or the wait ran out of time.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t* status) {
+  if (mbar_try(bar, parity)) return true;
+  uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > TIMEOUT_NS) {
+        *abort_flag = 1;
+        atomicOr(status, ST_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
+                                            int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// shared-memory matrix descriptor: start, leading/stride byte offsets, SM100 version bit,
+// layout (0 = no swizzle, 2 = 128-byte swizzle)
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// ------------------------------------------------------------------ kernel
+__global__ void __launch_bounds__(NT, 1)
+    k_retrieve_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmV,
+                  TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work item (uniform across the CTA)
+  int idx = blockIdx.x;
+  const int hc = idx % p.hcs; idx /= p.hcs;
+  const int rc = idx % p.rcs; idx /= p.rcs;
+  const int qbl = idx % p.nqbq;
+  const int s = idx / p.nqbq;
+  const int q_len = p.cu_q[s + 1] - p.cu_q[s];
+  const int k_len = p.cu_k[s + 1] - p.cu_k[s];
+  const int q0 = k_len - q_len;
+  if (q_len <= 0 || q0 < 0) return;
+  const int qb = q0 / p.B + qbl;
+  if ((int64_t)qb * p.B >= k_len) return;
+  const int i_begin = qb * p.B + rc * R;
+  const int row_lo = max(q0, i_begin), row_hi = min(k_len, i_begin + R);
+  if (row_lo >= row_hi) return;
+  const int64_t brow = (int64_t)p.qblock_base[s] + qb;
+  const int64_t rp0 = p.row_ptr[brow], rp1 = p.row_ptr[brow + 1];
+  const bool bsr_ok = rp0 >= 0 && rp1 >= rp0 && rp1 <= p.capacity && rp1 - rp0 <= qb + 1;
+  const int tpb = p.B / KT;
+  const int n_tiles = bsr_ok ? (int)(rp1 - rp0) * tpb : 0;
+  if (!bsr_ok && threadIdx.x == 0) atomicOr(p.status, ST_INDEX);
+
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t bar0 = sb + OFF_BAR;
+  auto bar = [&](int k) { return bar0 + 8u * (uint32_t)k; };
+
+  // ---- setup
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int k = 0; k < A_STAGES; ++k) { mbar_init(bar(B_AFULL + k), 1); mbar_init(bar(B_AEMPTY + k), 1); }
+    for (int k = 0; k < V_STAGES; ++k) { mbar_init(bar(B_VFULL + k), 1); mbar_init(bar(B_VEMPTY + k), 1); }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(bar(B_D1FULL + k), 1); mbar_init(bar(B_D1EMPTY + k), 128);
+      mbar_init(bar(B_PFULL + k), 128); mbar_init(bar(B_PEMPTY + k), 1);
+    }
+    mbar_init(bar(B_OFULL), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&s_tmem)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  // W^T of this CTA's 16 virtual heads, bf16, K-major without swizzle:
+  // element (r_v, s) at (s/8)*256 + (r_v/8)*128 + (r_v%8)*16 + (s%8)*2
+  {
+    const int ks = p.nsc * SC;
+    uint16_t* wt = reinterpret_cast<uint16_t*>(smem + OFF_W);
+    for (int e = threadIdx.x; e < HV * ks; e += NT) {
+      const int rv = e / ks, hs = e % ks;
+      const int G = hc * NG + rv / GQP, q = rv % GQP;
+      float w = 0.0f;
+      if (q < p.gq && G < p.h_kv && hs < p.h_s) w = p.W[(int64_t)(G * p.gq + q) * p.h_s + hs];
+      __nv_bfloat16 b = __float2bfloat16_rn(w);
+      wt[((hs >> 3) * 256 + (rv >> 3) * 128 + (rv & 7) * 16 + (hs & 7) * 2) >> 1] =
+          *reinterpret_cast<uint16_t*>(&b);
+    }
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  volatile int* abort_flag = &s_abort;
+
+  if (warp == 0) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      int as = 0, vs = 0;
+      uint32_t aph = 0, vph = 0;
+      int a_issued = 0, v_issued = 0;
+      bool ok = true;
+      for (int t = 0; t <= n_tiles && ok; ++t) {
+        if (t < n_tiles) {  // A chunks of tile t (consumed by the mixing of tile t)
+          const int64_t e = rp0 + t / tpb;
+          const int half = t % tpb;
+          for (int c = 0; c < p.nsc && ok; ++c) {
+            if (!(ok = mbar_wait(bar(B_AEMPTY + as), aph ^ 1, abort_flag, p.status))) break;
+            mbar_expect_tx(bar(B_AFULL + as), A_BYTES);
+            tma_load_4d(sb + OFF_A + as * A_BYTES, &tmA, bar(B_AFULL + as), half * KT, c * SC,
+                        rc * R, (int)e);
+            ++a_issued;
+            if (++as == A_STAGES) { as = 0; aph ^= 1; }
+          }
+        }
+        if (t >= 1 && ok) {  // V tiles of tile t-1 (consumed by P.V of tile t-1)
+          const int u = t - 1;
+          const int64_t e = rp0 + u / tpb;
+          const int half = u % tpb;
+          const int kb = p.col_idx[e];
+          const bool kb_ok = kb >= 0 && kb <= qb;
+          if (!kb_ok) atomicOr(p.status, ST_INDEX);
+          const int tok0 = kb * p.B + half * KT;
+          for (int g = 0; g < NG && ok; ++g) {
+            if (!(ok = mbar_wait(bar(B_VEMPTY + vs), vph ^ 1, abort_flag, p.status))) break;
+            mbar_expect_tx(bar(B_VFULL + vs), V_BYTES);
+            const uint32_t dst = sb + OFF_V + vs * V_BYTES;
+            const int G = hc * NG + g;
+            if (!p.paged) {
+              const int row = kb_ok ? p.cu_k[s] + tok0 : p.total_k;  // out of range reads 0
+              tma_load_3d(dst, &tmV, bar(B_VFULL + vs), 0, G, row);
+              tma_load_3d(dst + 8192, &tmV, bar(B_VFULL + vs), 64, G, row);
+            } else {
+              const int ps = p.page_size;
+              for (int q = 0; q < KT / ps; ++q) {
+                const int tok = tok0 + q * ps;
+                const int slot = tok / ps;
+                int page = p.n_pages;  // out of range: the copy reads zeros
+                if (kb_ok && tok < k_len && slot < p.max_pages) {
+                  const int pg = p.block_table[(int64_t)s * p.max_pages + slot];
+                  if (pg >= 0 && pg < p.n_pages) page = pg;
+                  else atomicOr(p.status, ST_PAGE);
+                }
+                tma_load_4d(dst + q * ps * 128, &tmV, bar(B_VFULL + vs), 0, G, 0, page);
+                tma_load_4d(dst + 8192 + q * ps * 128, &tmV, bar(B_VFULL + vs), 64, G, 0, page);
+              }
+            }
+            ++v_issued;
+            if (++vs == V_STAGES) { vs = 0; vph ^= 1; }
+          }
+        }
+      }
+      // drain: wait (bounded) for the last copy issued into every stage
+      for (int k = 0; k < A_STAGES; ++k) {
+        const int cnt = a_issued > k ? (a_issued - k - 1) / A_STAGES + 1 : 0;
+        if (cnt) {
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try(bar(B_AFULL + k), (cnt - 1) & 1) && globaltimer() - t0 < TIMEOUT_NS) {}
+        }
+      }
+      for (int k = 0; k < V_STAGES; ++k) {
+        const int cnt = v_issued > k ? (v_issued - k - 1) / V_STAGES + 1 : 0;
+        if (cnt) {
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try(bar(B_VFULL + k), (cnt - 1) & 1) && globaltimer() - t0 < TIMEOUT_NS) {}
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      int as = 0, vs = 0;
+      uint32_t aph = 0, vph = 0;
+      bool ok = true;
+      const uint32_t wbase = sb + OFF_W;
+      for (int t = 0; t <= n_tiles && ok; ++t) {
+        if (t < n_tiles) {  // mixing of tile t into D1[t & 1]
+          const int b = t & 1;
+          if (!(ok = mbar_wait(bar(B_D1EMPTY + b), ((t >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          const uint32_t d1 = tmem + 256u + 128u * (uint32_t)b;
+          for (int c = 0; c < p.nsc; ++c) {
+            if (!(ok = mbar_wait(bar(B_AFULL + as), aph, abort_flag, p.status))) break;
+            tc_fence_after();
+            const uint32_t abase = sb + OFF_A + as * A_BYTES;
+            const uint64_t bdesc = smem_desc(wbase + c * 512u, 256u, 128u, 0u);
+            for (int m = 0; m < 8; ++m)
+              tc_mma(d1 + 16u * m, smem_desc(abase + m * 4096u, 2048u, 1024u, 2u), bdesc,
+                     IDESC_MIX, c > 0 ? 1u : 0u);
+            tc_commit(bar(B_AEMPTY + as));
+            if (++as == A_STAGES) { as = 0; aph ^= 1; }
+          }
+          if (!ok) break;
+          tc_commit(bar(B_D1FULL + b));
+        }
+        if (t >= 1) {  // P.V of tile t-1 into D2
+          const int u = t - 1, b = u & 1;
+          if (!(ok = mbar_wait(bar(B_PFULL + b), (u >> 1) & 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          const uint32_t pbase = sb + OFF_P + b * PBUF_BYTES;
+          for (int g = 0; g < NG; ++g) {
+            if (!(ok = mbar_wait(bar(B_VFULL + vs), vph, abort_flag, p.status))) break;
+            tc_fence_after();
+            const uint32_t vbase = sb + OFF_V + vs * V_BYTES;
+            for (int k = 0; k < 4; ++k)
+              tc_mma(tmem + 64u * g, smem_desc(vbase + k * 2048u, 8192u, 1024u, 2u),
+                     smem_desc(pbase + g * PT_BYTES + k * 2048u, 8192u, 1024u, 2u), IDESC_PV,
+                     (u > 0 || k > 0) ? 1u : 0u);
+            tc_commit(bar(B_VEMPTY + vs));
+            if (++vs == V_STAGES) { vs = 0; vph ^= 1; }
+          }
+          if (!ok) break;
+          tc_commit(bar(B_PEMPTY + b));
+        }
+      }
+      tc_commit(bar(B_OFULL));
+      // drain our own MMAs before anyone frees TMEM
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try(bar(B_OFULL), 0) && globaltimer() - t0 < TIMEOUT_NS) {}
+    }
+  } else {
+    // ================================================================ convert + epilogue
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int lrow = quarter * 32 + lane;  // TMEM lane of this thread
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    bool ok = true;
+    for (int t = 0; t < n_tiles && ok; ++t) {
+      const int b = t & 1;
+      // warp-uniform control flow: tcgen05.ld is a warp-collective instruction
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_D1FULL + b), (t >> 1) & 1, abort_flag, p.status));
+      if (!ok) break;
+      tc_fence_after();
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(bar(B_PEMPTY + b), ((t >> 1) & 1) ^ 1, abort_flag, p.status));
+      if (!ok) break;
+      const int64_t e = rp0 + t / tpb;
+      const int half = t % tpb;
+      const int kb = p.col_idx[e];
+      const bool kb_ok = kb >= 0 && kb <= qb;
+      const int tok0 = kb * p.B + half * KT;
+      uint8_t* pt = smem + OFF_P + b * PBUF_BYTES;
+      const int j = lrow & 63;
+      for (int m = 0; m < 8; ++m) {
+        uint32_t v[16];
+        tmem_ld16(tl + 256u + 128u * (uint32_t)b + 16u * m, v);
+        tmem_wait_ld();
+        const int ii = 2 * m + (lrow >> 6);
+        const bool keep = kb_ok && tok0 + j <= i_begin + ii;
+        const uint32_t off = (uint32_t)j * 128u + ((((uint32_t)ii >> 1) ^ ((uint32_t)j & 7u)) << 4) +
+                             (((uint32_t)ii & 1u) << 3);
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+          uint32_t w0 = 0u, w1 = 0u;
+          if (keep) {
+            w0 = pack_bf16(__uint_as_float(v[4 * g + 0]), __uint_as_float(v[4 * g + 1]));
+            w1 = pack_bf16(__uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
+          }
+          asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(smem_u32(pt + g * PT_BYTES + off)),
+                       "r"(w0), "r"(w1)
+                       : "memory");
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_D1EMPTY + b));
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(bar(B_PFULL + b));
+    }
+    // ---- O epilogue: D2 lane = head dim, column = (group, row, head)
+    const bool have = __all_sync(0xffffffffu, ok && n_tiles > 0 &&
+                                                  mbar_wait(bar(B_OFULL), 0, abort_flag, p.status));
+    tc_fence_after();
+    const int dcol = lrow;  // head-dim index of this thread
+    for (int g = 0; g < NG; ++g) {
+      const int G = hc * NG + g;
+      if (G >= p.h_kv) break;
+      for (int k = 0; k < 4; ++k) {
+        uint32_t v[16];
+        if (have) {
+          tmem_ld16(tl + 64u * g + 16u * k, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) v[c] = 0u;
+        }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int ii = 4 * k + c / GQP, rv = c % GQP;
+          const int row = i_begin + ii;
+          if (rv < p.gq && row >= row_lo && row < row_hi) {
+            const int r = G * p.gq + rv;
+            const int64_t orow = (int64_t)p.cu_q[s] + (row - q0);
+            p.O[(orow * p.h_r + r) * D + dcol] = __float2bfloat16_rn(__uint_as_float(v[c]));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+bool encode(CUtensorMap* tm, const void* base, int rank, const uint64_t* dims,
+            const uint64_t* strides_bytes, const uint32_t* box, std::string* err) {
+  auto fn = get_encode();
+  if (!fn) { *err = "cuTensorMapEncodeTiled unavailable"; return false; }
+  uint32_t es[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                  dims, strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) { *err = "cuTensorMapEncodeTiled failed: " + std::to_string((int)r); return false; }
+  return true;
+}
+
+}  // namespace
+
+bool tc_supported(const mf_retrieve_desc& d) {
+  if (d.flags & MF_RETRIEVE_FORCE_SIMT) return false;
+  if (d.map_dtype != MF_BF16 || d.v_dtype != MF_BF16) return false;
+  if (!(d.B == 64 || d.B == 128) || d.d != D) return false;
+  if (d.h_kv <= 0 || d.h_r % d.h_kv != 0 || d.h_r / d.h_kv > GQP) return false;
+  if (d.h_s <= 0 || d.h_s > 64) return false;
+  if (d.paged && !(d.page_size == 8 || d.page_size == 16 || d.page_size == 32 || d.page_size == 64))
+    return false;
+  if (!d.paged && d.total_k >= (int64_t)1 << 31) return false;
+  return true;
+}
+
+bool launch_retrieve_tc(const mf_retrieve_desc& d, const RetrieveLayer& l, uint32_t* status,
+                        cudaStream_t st, std::string* err) {
+  const int B = d.B;
+  CUtensorMap tmA, tmV;
+  {  // kept blocks [capacity][h_s][B][B]: dims (key j, sender head s, row i, block n)
+    const uint64_t dims[4] = {(uint64_t)B, (uint64_t)d.h_s, (uint64_t)B,
+                              (uint64_t)std::max<int64_t>(l.capacity, 1)};
+    const uint64_t strides[3] = {(uint64_t)B * B * 2, (uint64_t)B * 2, (uint64_t)d.h_s * B * B * 2};
+    const uint32_t box[4] = {KT, SC, R, 1};
+    if (!encode(&tmA, l.values, 4, dims, strides, box, err)) return false;
+  }
+  if (!d.paged) {  // V [T][h_kv][d]: dims (dim, kv head, token)
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)d.h_kv, (uint64_t)std::max<int64_t>(d.total_k, 1)};
+    const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)d.h_kv * D * 2};
+    const uint32_t box[3] = {64, 1, KT};
+    if (!encode(&tmV, l.V, 3, dims, strides, box, err)) return false;
+  } else {  // V [pages][page][h_kv][d]: dims (dim, kv head, row in page, page)
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)d.h_kv, (uint64_t)d.page_size,
+                              (uint64_t)std::max(d.n_pages, 1)};
+    const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)d.h_kv * D * 2,
+                                 (uint64_t)d.page_size * d.h_kv * D * 2};
+    const uint32_t box[4] = {64, 1, (uint32_t)d.page_size, 1};
+    if (!encode(&tmV, l.V, 4, dims, strides, box, err)) return false;
+  }
+  TcParams p{};
+  p.row_ptr = l.row_ptr; p.col_idx = l.col_idx; p.capacity = l.capacity;
+  p.W = l.W; p.O = static_cast<__nv_bfloat16*>(l.O);
+  p.cu_q = d.cu_seqlens_q; p.cu_k = d.cu_seqlens_k; p.qblock_base = d.qblock_base;
+  p.block_table = d.block_table; p.paged = d.paged; p.page_size = d.page_size;
+  p.n_pages = d.n_pages; p.max_pages = d.max_pages; p.total_k = (int)d.total_k;
+  p.nqbq = (d.max_seqlen_q + B - 1) / B;
+  p.rcs = B / R;
+  p.hcs = (d.h_kv + NG - 1) / NG;
+  p.h_s = d.h_s; p.nsc = (d.h_s + SC - 1) / SC; p.B = B; p.h_r = d.h_r; p.h_kv = d.h_kv;
+  p.gq = d.h_r / d.h_kv;
+  p.status = status;
+  const int64_t grid = (int64_t)d.nseq * p.nqbq * p.rcs * p.hcs;
+  if (grid == 0) return true;
+  if (grid >= ((int64_t)1 << 31)) { *err = "grid too large"; return false; }
+  cudaError_t e = cudaFuncSetAttribute(k_retrieve_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SMEM_BYTES);
+  if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
+  k_retrieve_tc<<<(unsigned)grid, NT, SMEM_BYTES, st>>>(tmA, tmV, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
+  return true;
+}
+
+}  // namespace mfi

@@ -1,0 +1,212 @@
+/*
+ * mf.h -- C ABI of the MapFlow hot path on NVIDIA B200 (sm_100a).
+ *
+ * MapFlow ("Accelerating Cross-Model LLM Inference via Attention Map Reuse",
+ * Jin, Luo, Cui, Miao) lets a receiver LLM reuse the attention maps a sender
+ * LLM computed on the same context instead of recomputing its own prefill
+ * attention.  This library implements the two data-parallel kernels of that
+ * method:
+ *
+ *   mf_compress      block-sparse compression of one sender layer's maps.
+ *                    Page "MapFlow开源:大模型换班,Prefill为何能快20%?"
+ *                    (aitest123.com), section "存不下、读得慢?三个工程优化手段",
+ *                    subsection 1 "只存重要的:块稀疏压缩": the map is cut into
+ *                    regular 2-D blocks, block statistics are computed first and
+ *                    the important blocks are then chosen by cumulative
+ *                    attention probability, without assembling a second dense
+ *                    matrix.
+ *
+ *   mf_map_retrieve  the fused retrieval kernel.  Same page and section,
+ *                    subsection 3 "算得省的:融合内核执行": read the sparse blocks,
+ *                    form the linear combination of sender heads into receiver
+ *                    heads on chip, multiply by the receiver's own V and
+ *                    accumulate; layer and head mapping from the section
+ *                    "不传 KV Cache,改传注意力关系" ("层映射", "头映射");
+ *                    PagedAttention, chunked prefill and varlen packing from the
+ *                    closing paragraph of subsection 3.
+ *
+ * Conventions (all calls):
+ *   - The caller owns every buffer.  The library never allocates or frees
+ *     device memory; scratch space is passed in as `workspace`.
+ *   - Pointers documented "device" are CUDA device (or managed) pointers on
+ *     the current device; "host" pointers are read during the call only.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  The call returns after host-side validation and
+ *     launch.  Host-detectable errors return a status immediately and enqueue
+ *     nothing.
+ *   - Errors found on the device (a BSR index out of range, a page id out of
+ *     range, nnz above capacity, a pipeline wait that ran out of time) set a
+ *     per-device status word and never fault: the kernel skips the offending
+ *     access.  mf_get_status() reads and clears it.
+ *   - mf_last_error() returns a message for the calling host thread's last
+ *     failed call.
+ *   - All calls are thread-safe for distinct streams.
+ */
+#ifndef MF_H
+#define MF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MF_OK = 0,
+  MF_ERR_INVALID = 1,      /* a descriptor field is out of range or inconsistent */
+  MF_ERR_UNSUPPORTED = 2,  /* valid, but a shape this build does not handle */
+  MF_ERR_CAPACITY = 3,     /* device: more kept blocks than capacity_blocks */
+  MF_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+  MF_ERR_TIMEOUT = 5,      /* device: a pipeline wait ran out of time */
+  MF_ERR_DEVICE_INDEX = 6  /* device: a BSR row/column or page id was out of range */
+} mf_status;
+
+typedef enum { MF_F32 = 0, MF_BF16 = 1 } mf_dtype;
+
+/* ------------------------------------------------------------------------------
+ * Compression of one sender layer.
+ *
+ * For every sequence s of the varlen pack (length L_s = cu_seqlens[s+1] -
+ * cu_seqlens[s], nqb_s = ceil(L_s / B) query blocks, Lp_s = nqb_s * B) the dense
+ * maps are [h_s][Lp_s][Lp_s] row-major, starting at element map_seq_offset[s] of
+ * `maps`.  Only the causal blocks (kb <= qb) are read; entries with j > i, or
+ * i or j >= L_s, are ignored and stored as 0.
+ *
+ * For each query block qb (rows [qb*B, qb*B+B) of each sequence, in pack order):
+ *   mass[kb] = sum over sender heads s, rows i, keys j <= i of A_s[i][j], kb <= qb
+ *   the diagonal block is kept; the other blocks are taken in (mass desc, kb asc)
+ *   order until the running sum S reaches tau * total, where total is the row's
+ *   mass summed in that same order (float64).  Kept indices are stored ascending.
+ * Output is BSR over all query blocks of the pack:
+ *   row_ptr[r], r = 0..R (R = sum_s nqb_s), int32 device, row r = (s, qb) in order
+ *   col_idx[n], int32 device, key-block index local to the sequence
+ *   values[n][h_s][B][B], map dtype, device: exact copies of the kept blocks
+ *   *nnz_out (int32 device) = row_ptr[R]
+ * If more than capacity_blocks blocks are kept, the first capacity_blocks are
+ * written, *nnz_out holds the true count and the status word reports
+ * MF_ERR_CAPACITY.
+ * block_mass_out (optional, float64 device) receives every causal block's mass:
+ * sequence s, row qb, block kb at cb_base_s + qb*(qb+1)/2 + kb, where cb_base_s =
+ * sum over earlier sequences of nqb*(nqb+1)/2.
+ * Requirements: B in {32, 64, 128}; 0 <= tau <= 1; map_seq_offset[s] a multiple
+ * of 16 bytes; nqb_s <= 4096.
+ * ------------------------------------------------------------------------------ */
+typedef struct {
+  const void* maps;                /* device */
+  mf_dtype dtype;                  /* MF_F32 or MF_BF16 (maps and values) */
+  const int64_t* map_seq_offset;   /* device [nseq], element offsets */
+  const int32_t* cu_seqlens;       /* device [nseq + 1] */
+  int32_t nseq;                    /* >= 1 */
+  int32_t max_seqlen;              /* host bound: every L_s <= max_seqlen */
+  int32_t h_s;                     /* sender heads, 1..256 */
+  int32_t B;                       /* block size */
+  double tau;                      /* cumulative-mass threshold */
+  int32_t* row_ptr;                /* device out [R + 1] */
+  int32_t* col_idx;                /* device out [capacity_blocks] */
+  void* values;                    /* device out [capacity_blocks][h_s][B][B] */
+  int64_t capacity_blocks;
+  int32_t* nnz_out;                /* device out [1] */
+  double* block_mass_out;          /* device out, optional (NULL) */
+} mf_compress_desc;
+
+/* Bytes of scratch `mf_compress` needs for this descriptor (an upper bound computed
+ * from nseq, max_seqlen, B and capacity_blocks).  Returns MF_OK or MF_ERR_INVALID. */
+mf_status mf_compress_workspace_size(const mf_compress_desc* desc, size_t* bytes);
+
+/* Enqueue compression.  workspace: device, >= mf_compress_workspace_size bytes,
+ * 256-byte aligned, not used by any other call until this one completes. */
+mf_status mf_compress(const mf_compress_desc* desc, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/* ------------------------------------------------------------------------------
+ * Fused retrieval for receiver layers l = l_r_begin .. l_r_end-1.
+ *
+ * Receiver layer l reads sender layer layer_map[l] (a BSR from mf_compress).  For
+ * each sequence s of the batch, k_len = cu_seqlens_k[s+1] - cu_seqlens_k[s] is
+ * the prefix length and q_len = cu_seqlens_q[s+1] - cu_seqlens_q[s] the number of
+ * queries: the queries are the last q_len tokens of the prefix (chunked prefill;
+ * q_len = k_len for a whole sequence).  k_len - q_len must be a multiple of B.
+ * Query position i of sequence s lives in BSR row qblock_base[s] + i / B.  For
+ * every query i and receiver head r (g(r) = r * h_kv / h_r, contiguous GQA groups):
+ *   P_r[i][j] = sum_s W[l][r][s] * A_s[i][j]          over kept keys j <= i
+ *   O[l'][cu_seqlens_q[s] + (i - (k_len - q_len))][r][:] = sum_j P_r[i][j] * V_l[j][g(r)][:]
+ * with l' = l - l_r_begin.  V_l = V + l * v_layer_stride elements:
+ *   contiguous: [T_k][h_kv][d], key j of sequence s at token cu_seqlens_k[s] + j;
+ *   paged:      [n_pages][page_size][h_kv][d], key j at page
+ *               block_table[s * max_pages + j / page_size], row j % page_size.
+ * O (dtype v_dtype) is [l_r_end - l_r_begin][T_q][h_r][d] with layer stride
+ * o_layer_stride elements (0 = T_q * h_r * d).
+ * Arithmetic: MF_F32 maps/V run in float32 throughout.  MF_BF16 maps and V run on
+ * tcgen05 tensor cores: W is rounded to bf16, the mixed map P is accumulated in
+ * float32 and rounded to bf16, P.V is accumulated in float32 and O rounded to
+ * bf16 (round to nearest even).  Each output row's accumulation order depends
+ * only on its query block's kept blocks, so chunked, paged and varlen layouts give
+ * bit-identical rows.
+ * Requirements: h_r % h_kv == 0; layer_map[l] < n_sender_layers; d <= 256.
+ * The tensor-core path needs MF_BF16 maps and V, B in {64, 128}, d = 128,
+ * h_r / h_kv <= 4, h_s <= 64 and (if paged) page_size in {8, 16, 32, 64}; other
+ * shapes run a float32 SIMT kernel.
+ * ------------------------------------------------------------------------------ */
+typedef struct {
+  const int32_t* row_ptr;          /* device */
+  const int32_t* col_idx;          /* device */
+  const void* values;              /* device [capacity_blocks][h_s][B][B] */
+  int64_t capacity_blocks;
+} mf_bsr;
+
+#define MF_RETRIEVE_FORCE_SIMT 1   /* flags: run the SIMT kernel even where tensor cores apply */
+
+typedef struct {
+  const mf_bsr* layers;            /* host [n_sender_layers] */
+  int32_t n_sender_layers;
+  mf_dtype map_dtype;
+  int32_t h_s, B;
+  const int32_t* layer_map;        /* host [>= l_r_end] */
+  int32_t l_r_begin, l_r_end;
+  const float* W;                  /* device [L_r][h_r][h_s] float32, indexed by l */
+  const void* V;                   /* device, see above */
+  mf_dtype v_dtype;                /* V and O */
+  int64_t v_layer_stride;          /* elements; 0 = one V for every layer */
+  int32_t paged, page_size, n_pages, max_pages;
+  const int32_t* block_table;      /* device [nseq][max_pages] when paged */
+  int64_t total_k;                 /* contiguous: rows of V (T_k) */
+  const int32_t* cu_seqlens_q;     /* device [nseq + 1] */
+  const int32_t* cu_seqlens_k;     /* device [nseq + 1] */
+  const int32_t* qblock_base;      /* device [nseq] */
+  int32_t nseq, max_seqlen_q;      /* host bound: every q_len <= max_seqlen_q */
+  int32_t h_r, h_kv, d;
+  void* O;                         /* device out */
+  int64_t o_layer_stride;          /* elements */
+  int32_t total_q;                 /* T_q */
+  int32_t flags;
+} mf_retrieve_desc;
+
+mf_status mf_map_retrieve(const mf_retrieve_desc* desc, void* stream);
+
+/* Which kernel mf_map_retrieve would launch: 0 = float32 SIMT, 1 = tcgen05.
+ * Returns -1 for an invalid descriptor. */
+int mf_retrieve_path(const mf_retrieve_desc* desc);
+
+/* Synchronise `stream`, then read and clear this device's status word.  *bits
+ * (optional) receives the raw bits: 1 index out of range, 2 capacity, 4 wait
+ * timeout, 8 misaligned input, 16 page id out of range.  Returns MF_OK when no
+ * bit was set, else the status of the lowest set bit. */
+mf_status mf_get_status(void* stream, uint32_t* bits);
+
+/* Message for the calling thread's last failed call ("" if none). */
+const char* mf_last_error(void);
+
+/* Library version string. */
+const char* mf_version(void);
+
+/* sizeof of this header's structs as the library was compiled, for bindings that
+ * mirror them: which = 0 mf_compress_desc, 1 mf_bsr, 2 mf_retrieve_desc.
+ * Returns 0 for any other value. */
+size_t mf_abi_struct_size(int which);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MF_H */

@@ -1,0 +1,130 @@
+"""The C ABI library (no GPU needed): it loads, exports every function include/mf.h
+declares, mirrors its structs, and rejects bad descriptors on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def mf():
+    from cross_model_attention_mf_b200 import build
+    build.build()
+    import cross_model_attention_mf_b200 as mf
+    return mf
+
+
+def header_functions():
+    txt = open(os.path.join(ROOT, "include", "mf.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(mf_[a-z_]+)\s*\(", txt)))
+
+
+def test_exports_every_declared_function(mf):
+    lib = ctypes.CDLL(mf.LIB_PATH)
+    names = header_functions()
+    assert {"mf_compress", "mf_map_retrieve", "mf_compress_workspace_size", "mf_get_status"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_struct_mirrors(mf):
+    assert mf._lib.mf_abi_struct_size(0) == ctypes.sizeof(mf.CompressDesc)
+    assert mf._lib.mf_abi_struct_size(1) == ctypes.sizeof(mf.BsrDesc)
+    assert mf._lib.mf_abi_struct_size(2) == ctypes.sizeof(mf.RetrieveDesc)
+    assert mf._lib.mf_abi_struct_size(7) == 0
+    assert "sm_100a" in mf.mf_version()
+
+
+def test_workspace_size_bounds(mf):
+    small = mf.mf_compress_workspace_size(1, 256, 32, 10)
+    big = mf.mf_compress_workspace_size(16, 8192, 64, 100000)
+    assert 0 < small < big
+    # per-sequence meta + masses + flags of 128*129/2 blocks per sequence + kept rows
+    assert big >= 16 * (128 * 129 // 2) * 9 + 100000 * 4
+    assert mf.mf_compress_workspace_size(1, 100, 64, 0) % 256 == 0
+
+
+def _compress_desc(mf, **kw):
+    d = mf.CompressDesc()
+    d.maps = d.map_seq_offset = d.cu_seqlens = d.row_ptr = d.col_idx = d.values = d.nnz_out = 4096
+    d.dtype, d.nseq, d.max_seqlen, d.h_s, d.B, d.tau, d.capacity_blocks = 1, 1, 128, 4, 64, 0.9, 8
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+@pytest.mark.parametrize("field,value", [("B", 48), ("tau", 1.5), ("tau", -0.1), ("h_s", 0),
+                                         ("nseq", 0), ("dtype", 5), ("maps", 0),
+                                         ("capacity_blocks", -1), ("values", 4100)])
+def test_compress_rejects_bad_descriptor(mf, field, value):
+    d = _compress_desc(mf, **{field: value})
+    rc = mf._lib.mf_compress(ctypes.byref(d), ctypes.c_void_p(4096), 1 << 30, None)
+    assert rc == mf.MF_ERR_INVALID
+    assert mf._lib.mf_last_error().decode()
+
+
+def test_compress_rejects_small_workspace(mf):
+    d = _compress_desc(mf)
+    rc = mf._lib.mf_compress(ctypes.byref(d), ctypes.c_void_p(4096), 16, None)
+    assert rc == mf.MF_ERR_INVALID and b"workspace" in mf._lib.mf_last_error()
+    rc = mf._lib.mf_compress(ctypes.byref(d), ctypes.c_void_p(4096 + 8), 1 << 30, None)
+    assert rc == mf.MF_ERR_INVALID and b"aligned" in mf._lib.mf_last_error()
+
+
+def test_compress_rejects_too_many_blocks(mf):
+    d = _compress_desc(mf, max_seqlen=4097 * 64)
+    rc = mf._lib.mf_compress(ctypes.byref(d), ctypes.c_void_p(4096), 1 << 40, None)
+    assert rc == mf.MF_ERR_UNSUPPORTED
+
+
+def _retrieve_desc(mf, bsr_arr, lm, **kw):
+    d = mf.RetrieveDesc()
+    d.layers = bsr_arr
+    d.n_sender_layers = 1
+    d.map_dtype = d.v_dtype = 1
+    d.h_s, d.B = 32, 64
+    d.layer_map = ctypes.cast(lm, ctypes.c_void_p)
+    d.l_r_begin, d.l_r_end = 0, 1
+    d.W = d.V = d.O = d.cu_seqlens_q = d.cu_seqlens_k = d.qblock_base = 4096
+    d.total_k, d.nseq, d.max_seqlen_q = 8192, 1, 8192
+    d.h_r, d.h_kv, d.d = 32, 8, 128
+    d.total_q = 8192
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+def test_retrieve_path_selection(mf):
+    arr = (mf.BsrDesc * 1)(mf.BsrDesc(4096, 4096, 4096, 100))
+    lm = (ctypes.c_int32 * 1)(0)
+    P = mf._lib.mf_retrieve_path
+    assert P(ctypes.byref(_retrieve_desc(mf, arr, lm))) == 1                     # Ministral-like
+    assert P(ctypes.byref(_retrieve_desc(mf, arr, lm, B=128, h_r=24))) == 1      # long context, gq 3
+    assert P(ctypes.byref(_retrieve_desc(mf, arr, lm, h_s=40))) == 1             # Qwen-like
+    assert P(ctypes.byref(_retrieve_desc(mf, arr, lm, map_dtype=0, v_dtype=0, B=32, h_s=4,
+                                         h_r=2, h_kv=1, d=64))) == 0             # tiny float32
+    assert P(ctypes.byref(_retrieve_desc(mf, arr, lm, flags=mf.MF_RETRIEVE_FORCE_SIMT))) == 0
+    assert P(ctypes.byref(_retrieve_desc(mf, arr, lm, h_r=32, h_kv=4))) == 0      # gq 8: SIMT
+    assert P(ctypes.byref(_retrieve_desc(mf, arr, lm, paged=1, page_size=16, n_pages=10,
+                                         max_pages=4, block_table=4096))) == 1
+
+
+@pytest.mark.parametrize("field,value", [("h_r", 30), ("l_r_end", 2), ("d", 0), ("nseq", 0),
+                                         ("W", 0), ("map_dtype", 9), ("l_r_begin", -1)])
+def test_retrieve_rejects_bad_descriptor(mf, field, value):
+    arr = (mf.BsrDesc * 1)(mf.BsrDesc(4096, 4096, 4096, 100))
+    lm = (ctypes.c_int32 * 2)(0, 3)
+    d = _retrieve_desc(mf, arr, lm, **{field: value})
+    assert mf._lib.mf_map_retrieve(ctypes.byref(d), None) == mf.MF_ERR_INVALID
+    assert mf._lib.mf_retrieve_path(ctypes.byref(d)) == -1
+
+
+def test_retrieve_rejects_unmapped_layer(mf):
+    arr = (mf.BsrDesc * 1)(mf.BsrDesc(4096, 4096, 0, 100))
+    lm = (ctypes.c_int32 * 1)(0)
+    d = _retrieve_desc(mf, arr, lm)
+    assert mf._lib.mf_map_retrieve(ctypes.byref(d), None) == mf.MF_ERR_INVALID

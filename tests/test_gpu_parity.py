@@ -1,0 +1,293 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, on the same seeded inputs.
+
+Small cases compare every row; the full-size workloads compare sampled rows (the oracle
+is run on the exact device bytes of each sampled row) plus layout identities that hold
+at any size.  Block sets must match exactly except near-tie rows, which are counted and
+expected to be 0; O must match within max-abs 2e-2 and relative-L2 1e-2 (bf16) or
+1e-5 (float32).
+"""
+import numpy as np
+import pytest
+import torch
+
+import cross_model_attention_mf_b200 as mf
+import oracle
+import synth
+from synth import device as sdev
+from tests.gpu_common import assert_O_close, check_rows, host_bsr, oracle_O_rows, run_compress
+
+pytestmark = pytest.mark.gpu
+
+
+def _retrieve(w, pack, bsr, W, V, force_simt=False, layer_map=(0,), layers=None):
+    qbase = sdev.qblock_base(w)
+    cu = pack.cu_seqlens
+    return mf.mf_map_retrieve(layers or [bsr], list(layer_map), W, V, cu, cu, qbase, max(w.lens),
+                              w.h_r, w.h_kv, total_q=w.tokens, force_simt=force_simt)
+
+
+def _path(w, pack, bsr, W, V, force_simt=False):
+    qbase = sdev.qblock_base(w)
+    O = torch.empty((1, w.tokens, w.h_r, w.d), dtype=V.dtype, device=V.device)
+    return mf.mf_retrieve_path([bsr], [0], W, V, pack.cu_seqlens, pack.cu_seqlens, qbase,
+                               max(w.lens), w.h_r, w.h_kv, O, force_simt=force_simt)
+
+
+def _status_ok():
+    rc, bits = mf.mf_get_status()
+    assert rc == mf.MF_OK and bits == 0, (rc, bits)
+
+
+def _all_rows(w):
+    return [(s, qb) for s in range(len(w.lens)) for qb in range(w.nqb[s])]
+
+
+def _oracle_O_all(w, orows, W_l, V_host):
+    outs = []
+    starts = np.concatenate([[0], np.cumsum(w.lens)])
+    for s in range(len(w.lens)):
+        for qb in range(w.nqb[s]):
+            O, _ = oracle_O_rows(w, orows, s, qb, W_l, V_host, 0, k_start=int(starts[s]))
+            outs.append(O)
+    return np.concatenate(outs, axis=0)
+
+
+def _full_check(w, force_simt=False, expect_path=None):
+    pack = sdev.fill_maps(sdev.alloc_maps(w), w, 0)
+    bsr = run_compress(w, pack)
+    _status_ok()
+    orows, nb = check_rows(w, pack, bsr, _all_rows(w))
+    assert nb == 0
+    W = sdev.w_weights(w)
+    V = sdev.v_contiguous(w, 0)
+    if expect_path is not None:
+        assert _path(w, pack, bsr, W, V, force_simt) == expect_path
+    O = _retrieve(w, pack, bsr, W, V, force_simt)
+    _status_ok()
+    want = _oracle_O_all(w, orows, W[0].cpu().numpy(), V.cpu())
+    assert_O_close(O[0].float().cpu().numpy(), want, w.dtype, w.name)
+    return pack, bsr, W, V, O
+
+
+def test_gpu_generator_matches_cpu_recipe():
+    for dt in ("f32", "bf16"):
+        w = synth.Workload("g", (77, 40), B=32, h_s=3, h_r=1, h_kv=1, d=8, dtype=dt, tau=0.9, n_heavy=5)
+        pack = sdev.fill_maps(sdev.alloc_maps(w), w, 2)
+        for s, L in enumerate(w.lens):
+            g = pack.seq_view(s, w.h_s, w.B).float().cpu().numpy()
+            c = synth.gen_maps(L, w.B, w.h_s, 5, seed=0, layer=2, seq=s, dtype=dt).float().numpy()
+            Lp = c.shape[1]
+            causal = np.tril(np.ones((Lp, Lp), dtype=bool))
+            if dt == "f32":
+                np.testing.assert_allclose(g[:, causal], c[:, causal], rtol=2e-5, atol=1e-7)
+            else:  # at most one bf16 rounding step apart
+                np.testing.assert_allclose(g[:, causal], c[:, causal], rtol=2 ** -7, atol=1e-8)
+
+
+def test_tiny_fp32():
+    w = synth.ALL["tiny"]
+    _full_check(w, expect_path=0)
+
+
+def test_small_bf16_varlen_tcgen05():
+    w = synth.Workload("small", (300, 129, 64, 1), B=64, h_s=32, h_r=32, h_kv=8, d=128,
+                       dtype="bf16", tau=0.95, n_heavy=16, reading=3)
+    pack, bsr, W, V, O = _full_check(w, expect_path=1)
+    # the SIMT kernel on the same BSR agrees with the tensor-core kernel
+    O2 = _retrieve(w, pack, bsr, W, V, force_simt=True)
+    _status_ok()
+    assert_O_close(O[0].float().cpu().numpy(), O2[0].float().cpu().numpy(), "bf16", "tc vs simt")
+
+
+def test_small_bf16_simt_path():
+    w = synth.Workload("small_simt", (200, 70), B=64, h_s=32, h_r=32, h_kv=8, d=128,
+                       dtype="bf16", tau=0.9, n_heavy=16, reading=3)
+    _full_check(w, force_simt=True, expect_path=0)
+
+
+def test_long_block_gqa3_tcgen05():
+    w = synth.Workload("b128", (400, 130), B=128, h_s=32, h_r=24, h_kv=8, d=128, dtype="bf16",
+                       tau=0.9, n_heavy=8, reading=3)
+    _full_check(w, expect_path=1)
+
+
+def test_qwen_heads_40_tcgen05():
+    w = synth.Workload("hs40", (200, 77, 130), B=64, h_s=40, h_r=32, h_kv=8, d=128, dtype="bf16",
+                       tau=0.95, n_heavy=16, reading=3)
+    _full_check(w, expect_path=1)
+
+
+def test_uneven_kv_groups_tcgen05():
+    """h_kv = 6: the second head chunk holds two real groups and two empty ones."""
+    w = synth.Workload("kv6", (150,), B=64, h_s=16, h_r=12, h_kv=6, d=128, dtype="bf16",
+                       tau=0.9, n_heavy=4, reading=3)
+    _full_check(w, expect_path=1)
+
+
+@pytest.mark.parametrize("tau", [0.0, 1.0])
+def test_tau_extremes(tau):
+    w = synth.Workload("tau", (260,), B=64, h_s=8, h_r=8, h_kv=2, d=128, dtype="bf16", tau=tau,
+                       n_heavy=4, reading=3)
+    pack, bsr, W, V, O = _full_check(w, expect_path=1)
+    rp, ci, nnz = host_bsr(bsr)
+    if tau == 0.0:
+        assert nnz == w.nqb[0] and ci[:nnz].tolist() == list(range(w.nqb[0]))
+    else:
+        # tau = 1: O equals the dense receiver map times V (numpy, float64)
+        A = pack.seq_view(0, w.h_s, w.B).float().cpu().numpy().astype(np.float64)
+        L = w.lens[0]
+        A = np.tril(A[:, :L, :L])
+        P = np.einsum("rs,sij->rij", W[0].cpu().numpy().astype(np.float64), A)
+        Vr = np.repeat(V.float().cpu().numpy().astype(np.float64), w.h_r // w.h_kv, axis=1)
+        dense = np.einsum("rij,jrd->ird", P, Vr)
+        assert_O_close(O[0].float().cpu().numpy(), dense, "bf16", "tau=1 vs dense")
+
+
+def test_identity_W_is_causal_attention():
+    """W = I, maps = causal softmax(Q K^T / sqrt(dk)) stored in bf16, tau = 1: O is standard
+    causal attention (torch SDPA on the same Q, K, V)."""
+    torch.manual_seed(0)
+    H, L, B, dk = 8, 200, 64, 64
+    Q = torch.randn(H, L, dk, dtype=torch.float64)
+    K = torch.randn(H, L, dk, dtype=torch.float64)
+    Vh = torch.randn(L, H, 128, dtype=torch.float64)
+    S = torch.einsum("hid,hjd->hij", Q, K) / dk ** 0.5
+    S = S.masked_fill(~torch.tril(torch.ones(L, L, dtype=torch.bool)), float("-inf"))
+    Pm = torch.softmax(S, dim=-1)
+    Lp = 256
+    w = synth.Workload("qk", (L,), B=B, h_s=H, h_r=H, h_kv=H, d=128, dtype="bf16", tau=1.0, n_heavy=0)
+    pack = sdev.alloc_maps(w)
+    view = pack.seq_view(0, H, B)
+    view.zero_()
+    view[:, :L, :L] = Pm.to(torch.bfloat16).cuda()
+    bsr = run_compress(w, pack)
+    W = torch.eye(H, dtype=torch.float32, device="cuda")[None]
+    V = Vh.to(torch.bfloat16).cuda()
+    O = _retrieve(w, pack, bsr, W, V)
+    _status_ok()
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        Q[None], K[None], Vh.to(torch.bfloat16).double().permute(1, 0, 2)[None], is_causal=True)[0]
+    assert_O_close(O[0].float().cpu().numpy(), ref.permute(1, 0, 2).numpy(), "bf16", "W=I vs SDPA")
+
+
+def test_layouts_bitwise_identical():
+    """Chunked prefill over a shuffled paged V, a contiguous V, one call per sequence and the
+    varlen pack all give bit-identical O rows on the tensor-core path."""
+    w = synth.Workload("lay", (700, 333, 64), B=64, h_s=32, h_r=32, h_kv=8, d=128, dtype="bf16",
+                       tau=0.95, n_heavy=16, reading=3, chunk=256, page_size=16)
+    pack = sdev.fill_maps(sdev.alloc_maps(w), w, 0)
+    bsr = run_compress(w, pack)
+    W = sdev.w_weights(w)
+    V = sdev.v_contiguous(w, 0)
+    whole = _retrieve(w, pack, bsr, W, V)[0]
+    qbase = sdev.qblock_base(w)
+    starts = np.concatenate([[0], np.cumsum(w.lens)])
+    # per-sequence calls
+    for s, L in enumerate(w.lens):
+        cu = torch.tensor([0, L], dtype=torch.int32, device="cuda")
+        Os = mf.mf_map_retrieve([bsr], [0], W, V[starts[s]:starts[s] + L].contiguous(), cu, cu,
+                                qbase[s:s + 1].contiguous(), L, w.h_r, w.h_kv, total_q=L)[0]
+        assert torch.equal(Os, whole[starts[s]:starts[s] + L])
+    # paged, whole sequences
+    Vp, table = sdev.v_paged(w, V)
+    cu = pack.cu_seqlens
+    paged = mf.mf_map_retrieve([bsr], [0], W, Vp, cu, cu, qbase, max(w.lens), w.h_r, w.h_kv,
+                               total_q=w.tokens, paged=(table, w.page_size))[0]
+    assert torch.equal(paged, whole)
+    # chunked prefill, paged
+    parts = [[] for _ in w.lens]
+    for step in synth.chunks(w):
+        cu_q, cu_k, mq = sdev.step_tensors(step)
+        Oc = mf.mf_map_retrieve([bsr], [0], W, Vp, cu_q, cu_k, qbase, mq, w.h_r, w.h_kv,
+                                total_q=int(cu_q[-1]), paged=(table, w.page_size))[0]
+        q = cu_q.cpu().numpy()
+        for s in range(len(w.lens)):
+            if q[s + 1] > q[s]:
+                parts[s].append(Oc[q[s]:q[s + 1]])
+    chunked = torch.cat([torch.cat(p) for p in parts])
+    assert torch.equal(chunked, whole)
+    # chunked prefill, contiguous prefixes
+    for step in synth.chunks(w)[:2]:
+        cu_q, cu_k, mq = sdev.step_tensors(step)
+        Vc = sdev.pack_prefixes(V, w.lens, step)
+        Oc = mf.mf_map_retrieve([bsr], [0], W, Vc, cu_q, cu_k, qbase, mq, w.h_r, w.h_kv,
+                                total_q=int(cu_q[-1]))[0]
+        Op = mf.mf_map_retrieve([bsr], [0], W, Vp, cu_q, cu_k, qbase, mq, w.h_r, w.h_kv,
+                                total_q=int(cu_q[-1]), paged=(table, w.page_size))[0]
+        assert torch.equal(Oc, Op)
+    _status_ok()
+
+
+def test_layer_batch_and_layer_map():
+    """Three receiver layers over two sender layers in one call equal three single-layer calls."""
+    w = synth.Workload("lm", (200,), B=64, h_s=32, h_r=32, h_kv=8, d=128, dtype="bf16", tau=0.9,
+                       n_heavy=8, reading=3, n_sender_layers=2, n_receiver_layers=3)
+    bsrs = []
+    for l in range(2):
+        pack = sdev.fill_maps(sdev.alloc_maps(w), w, l)
+        bsrs.append(run_compress(w, pack))
+    W = sdev.w_weights(w)
+    V = torch.stack([sdev.v_contiguous(w, l) for l in range(3)])
+    lm = [0, 1, 1]
+    qbase = sdev.qblock_base(w)
+    cu = pack.cu_seqlens
+    Oall = mf.mf_map_retrieve(bsrs, lm, W, V, cu, cu, qbase, 200, w.h_r, w.h_kv, total_q=200,
+                              v_layer_stride=V[0].numel())
+    for l in range(3):
+        Ol = mf.mf_map_retrieve(bsrs, lm, W, V, cu, cu, qbase, 200, w.h_r, w.h_kv, total_q=200,
+                                l_r_range=(l, l + 1), v_layer_stride=V[0].numel())
+        assert torch.equal(Ol[0], Oall[l])
+    assert not torch.equal(Oall[0], Oall[1])
+    _status_ok()
+
+
+# ------------------------------------------------------------------ device-side error reporting
+
+def test_capacity_overflow_reported():
+    w = synth.Workload("cap", (300,), B=64, h_s=8, h_r=8, h_kv=2, d=128, dtype="bf16", tau=0.99,
+                       n_heavy=4, reading=3)
+    pack = sdev.fill_maps(sdev.alloc_maps(w), w, 0)
+    full = run_compress(w, pack)
+    _status_ok()
+    n = int(full.nnz.cpu()[0])
+    small = run_compress(w, pack, capacity=n - 2)
+    rc, bits = mf.mf_get_status()
+    assert rc == mf.MF_ERR_CAPACITY and bits & 2
+    assert int(small.nnz.cpu()[0]) == n
+    assert torch.equal(small.col_idx[:n - 2], full.col_idx[:n - 2])
+    assert torch.equal(small.values[:n - 2], full.values[:n - 2])
+
+
+@pytest.mark.parametrize("force_simt", [False, True])
+def test_bad_bsr_index_reported_not_faulted(force_simt):
+    w = synth.Workload("bad", (200,), B=64, h_s=32, h_r=32, h_kv=8, d=128, dtype="bf16", tau=0.9,
+                       n_heavy=8, reading=3)
+    pack = sdev.fill_maps(sdev.alloc_maps(w), w, 0)
+    bsr = run_compress(w, pack)
+    W = sdev.w_weights(w)
+    V = sdev.v_contiguous(w, 0)
+    _status_ok()
+    bsr.col_idx[0] = 7  # row 0 may only reference key block 0
+    _retrieve(w, pack, bsr, W, V, force_simt=force_simt)
+    rc, bits = mf.mf_get_status()
+    assert rc == mf.MF_ERR_DEVICE_INDEX and bits & 1
+    bsr.row_ptr[1] = 1 << 30  # a row pointer beyond capacity: the row is skipped
+    _retrieve(w, pack, bsr, W, V, force_simt=force_simt)
+    rc, bits = mf.mf_get_status()
+    assert rc == mf.MF_ERR_DEVICE_INDEX
+    torch.cuda.synchronize()
+
+
+def test_bad_page_reported():
+    w = synth.Workload("page", (200,), B=64, h_s=32, h_r=32, h_kv=8, d=128, dtype="bf16", tau=0.9,
+                       n_heavy=8, reading=3, page_size=16)
+    pack = sdev.fill_maps(sdev.alloc_maps(w), w, 0)
+    bsr = run_compress(w, pack)
+    V = sdev.v_contiguous(w, 0)
+    Vp, table = sdev.v_paged(w, V)
+    table[0, 3] = 10 ** 6
+    cu = pack.cu_seqlens
+    mf.mf_map_retrieve([bsr], [0], sdev.w_weights(w), Vp, cu, cu, sdev.qblock_base(w), 200,
+                       w.h_r, w.h_kv, total_q=200, paged=(table, 16))
+    rc, bits = mf.mf_get_status()
+    assert rc == mf.MF_ERR_DEVICE_INDEX and bits & 16
