@@ -141,7 +141,7 @@ def run_ours(args, rank, world, dev):
     pack = sdev.fill_maps(sdev.alloc_maps(w, dev), w, 0)
     W = sdev.w_weights(w, dev)
     V = sdev.v_contiguous(w, 0, dev)
-    cap = w.causal_blocks
+    cap = args.capacity if args.capacity > 0 else w.causal_blocks
     bsr = mf.alloc_bsr(sum(w.nqb), cap, w.h_s, w.B, pack.maps.dtype, dev)
     ws = torch.empty(mf.mf_compress_workspace_size(len(w.lens), max(w.lens), w.B, cap),
                      dtype=torch.uint8, device=dev)
@@ -298,6 +298,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--capacity", type=int, default=0,
+                    help="BSR capacity in blocks (0: every causal block, which never overflows)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -18,7 +18,8 @@ from typing import List, Optional, Sequence
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmf.so")
+# MF_LIBRARY may point at another build of the same ABI (for example a traced one)
+LIB_PATH = os.environ.get("MF_LIBRARY") or os.path.join(_HERE, "libmf.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python -m cross_model_attention_mf_b200.build` "

@@ -7,21 +7,33 @@
 // receiver's dense map.  The pages' kernel is Triton on A800; this one is a
 // new design for B200.
 //
-// CTA = (sequence, query block, 16-row chunk, 4 KV groups = 16 virtual receiver
-// heads; a group of gq <= 4 heads is padded to 4).  For each kept 64-key tile:
+// Work item = (sequence, query block, 16-row chunk, 4 KV groups = 16 virtual
+// receiver heads; a group of gq <= 4 heads is padded to 4).  The kernel is
+// persistent: each CTA walks items blockIdx.x, blockIdx.x + gridDim.x, ... (the grid
+// is a multiple of the head-chunk count, so a CTA keeps one head chunk and one W^T),
+// and the rings below run across item boundaries, so the loads and the mixing of
+// the next item overlap the tail of the current one.  For each kept 64-key tile:
 //
 //   mixing  D1[pos][r] = sum_s A_s[pos] * W[r][s]       tcgen05 M=128 N=16 K=16
 //           pos = (row, key) of 2 rows x 64 keys, A tile MN-major SW128 from TMA,
-//           W^T K-major in smem (bf16).  D1 is double-buffered in TMEM.
-//   convert 4 epilogue warps read D1 (lane = position), apply the causal mask,
-//           round to bf16 and write P^T[key][(row, head)] (MN-major SW128) with
-//           one 8-byte store per (position, group).
-//   P.V     D2[dim][(row, head)] += V^T[dim][key] * P^T[key][(row, head)]
-//           tcgen05 M=128 (d) N=64 K=16 per group; V tile MN-major SW128 by TMA
-//           (contiguous or paged).  D2 stays in TMEM for the whole row chunk.
+//           W^T K-major in smem.  W is split into bf16 hi + lo parts (two MMAs into
+//           the same accumulator), so the mixing keeps ~16 bits of W.  D1 is
+//           double-buffered in TMEM.
+//   convert 4 epilogue warps read D1 (lane = position), apply the causal mask and
+//           split P into bf16 hi + lo (P = hi + lo to ~16 bits), written as
+//           P^T[key][(row, head)] (MN-major SW128), one group at a time into a
+//           ring of shared-memory slots.
+//   P.V     D2[dim][(row, head)] += V^T[dim][key] * (P^T_hi + P^T_lo)[key][(row, head)]
+//           tcgen05 M=128 (d) N=64 K=16 per group, two MMAs per K step; V tile
+//           MN-major SW128 by TMA (contiguous or paged).  D2 stays in TMEM for the
+//           whole row chunk.
+// The hi/lo splits keep the only bf16 rounding that matters at the final O.
 //
-// Warp roles: warp 0 TMA producer, warp 1 MMA issuer (+ TMEM owner), warps 2-5
-// convert/epilogue.  TMEM: D2 in columns [0, 256), D1 in [256, 512).  Every
+// Warp roles: warp 0 TMA producer, warp 1 MMA issuer (+ TMEM owner), warps 2-9
+// convert P (two warps per TMEM lane quarter, each taking two of the four groups),
+// warps 10-13 O epilogue (they release D2 as soon as it is read, so the next item's
+// P.V can start while O is stored).  TMEM: D2 in columns [0, 256), D1
+// in [256, 512).  Every
 // mbarrier wait is bounded by a timer: on expiry the CTA records ST_TIMEOUT, all
 // roles stop, in-flight copies and MMAs are drained (bounded) and TMEM is freed.
 #include <cuda.h>
@@ -29,6 +41,7 @@
 #include <cudaTypedefs.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "mf_internal.cuh"
@@ -36,7 +49,7 @@
 namespace mfi {
 namespace {
 
-constexpr int NT = 192;
+constexpr int NT = 448;
 constexpr int R = 16;          // query rows per CTA
 constexpr int KT = 64;         // keys per tile
 constexpr int NG = 4;          // KV groups per CTA
@@ -44,17 +57,17 @@ constexpr int GQP = 4;         // virtual heads per group
 constexpr int HV = NG * GQP;   // virtual receiver heads per CTA
 constexpr int D = 128;         // head dim
 constexpr int SC = 16;         // sender heads per A chunk (one MMA K step)
-constexpr int A_STAGES = 3, V_STAGES = 3;
+constexpr int A_STAGES = 2, V_STAGES = 4, P_SLOTS = 5;
 constexpr uint32_t A_BYTES = R * SC * KT * 2;   // 32 KB
 constexpr uint32_t V_BYTES = KT * D * 2;        // 16 KB
-constexpr uint32_t PT_BYTES = KT * 64 * 2;      // 8 KB per group
-constexpr uint32_t PBUF_BYTES = NG * PT_BYTES;  // 32 KB per tile
+constexpr uint32_t PT_BYTES = KT * 64 * 2;      // 8 KB: one group's P^T (hi or lo)
+constexpr uint32_t PSLOT_BYTES = 2 * PT_BYTES;  // hi + lo
 constexpr uint32_t OFF_A = 0;
 constexpr uint32_t OFF_V = OFF_A + A_STAGES * A_BYTES;
 constexpr uint32_t OFF_P = OFF_V + V_STAGES * V_BYTES;
-constexpr uint32_t OFF_W = OFF_P + 2 * PBUF_BYTES;
-constexpr uint32_t W_BYTES_MAX = 4 * 512;       // up to 4 chunks (h_s <= 64)
-constexpr uint32_t OFF_BAR = OFF_W + W_BYTES_MAX;
+constexpr uint32_t OFF_W = OFF_P + P_SLOTS * PSLOT_BYTES;
+constexpr uint32_t W_BYTES_MAX = 4 * 512;       // up to 4 chunks (h_s <= 64), per part
+constexpr uint32_t OFF_BAR = OFF_W + 2 * W_BYTES_MAX;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
 constexpr uint64_t TIMEOUT_NS = 2000000000ull;
 
@@ -62,7 +75,8 @@ constexpr uint64_t TIMEOUT_NS = 2000000000ull;
 enum {
   B_AFULL = 0, B_AEMPTY = B_AFULL + A_STAGES, B_VFULL = B_AEMPTY + A_STAGES,
   B_VEMPTY = B_VFULL + V_STAGES, B_D1FULL = B_VEMPTY + V_STAGES, B_D1EMPTY = B_D1FULL + 2,
-  B_PFULL = B_D1EMPTY + 2, B_PEMPTY = B_PFULL + 2, B_OFULL = B_PEMPTY + 2, B_COUNT = B_OFULL + 1
+  B_PFULL = B_D1EMPTY + 2, B_PEMPTY = B_PFULL + P_SLOTS, B_OFULL = B_PEMPTY + P_SLOTS,
+  B_OEMPTY = B_OFULL + 1, B_DRAIN = B_OEMPTY + 1, B_COUNT = B_DRAIN + 1
 };
 
 // instruction descriptors (kind::f16): D f32, A/B bf16, majors, N >> 3, M >> 4
@@ -84,6 +98,7 @@ struct TcParams {
   int paged, page_size, n_pages, max_pages;
   int total_k;
   int nqbq, rcs, hcs;  // query blocks, row chunks per block, head chunks
+  int n_items;
   int h_s, nsc, B, h_r, h_kv, gq;
   uint32_t* status;
 };
@@ -194,7 +209,64 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Optional timeline trace (compile with -DMF_TRACE): per CTA and role, globaltimer
+// stamps of pipeline events, read back with mf_trace_dump().
+#ifdef MF_TRACE
+constexpr int TRACE_CTAS = 160, TRACE_N = 2048;
+__device__ uint64_t g_trace[TRACE_CTAS][4][TRACE_N];
+__device__ __forceinline__ void trace(int role, uint32_t code) {
+  if (blockIdx.x >= TRACE_CTAS) return;
+  uint64_t* b = g_trace[blockIdx.x][role];
+  const uint64_t n = b[0];
+  if (n < TRACE_N - 1) {
+    b[1 + n] = ((uint64_t)code << 56) | (globaltimer() & ((1ull << 56) - 1));
+    b[0] = n + 1;
+  }
+}
+#define TRACE(role, code) trace(role, code)
+#else
+#define TRACE(role, code)
+#endif
+
 // ------------------------------------------------------------------ kernel
+struct Item {
+  int s, qb, q0, i_begin, row_lo, row_hi, k_len, n_tiles;
+  int64_t rp0;
+  int64_t o_row0;  // O row of query position i_begin (cu_seqlens_q[s] + i_begin - q0)
+  bool valid, bsr_ok;
+};
+
+// item idx = ((s * nqbq + qbl) * rcs + rc) * hcs + hc; identical in every role
+__device__ __forceinline__ Item decode(const TcParams& p, int idx) {
+  Item it;
+  it.valid = false;
+  it.bsr_ok = true;
+  it.n_tiles = 0;
+  idx /= p.hcs;
+  const int rc = idx % p.rcs;
+  idx /= p.rcs;
+  const int qbl = idx % p.nqbq;
+  const int s = idx / p.nqbq;
+  const int q_len = p.cu_q[s + 1] - p.cu_q[s];
+  const int k_len = p.cu_k[s + 1] - p.cu_k[s];
+  const int q0 = k_len - q_len;
+  if (q_len <= 0 || q0 < 0) return it;
+  const int qb = q0 / p.B + qbl;
+  if ((int64_t)qb * p.B >= k_len) return it;
+  const int i_begin = qb * p.B + rc * R;
+  const int row_lo = max(q0, i_begin), row_hi = min(k_len, i_begin + R);
+  if (row_lo >= row_hi) return it;
+  const int64_t brow = (int64_t)p.qblock_base[s] + qb;
+  const int64_t rp0 = p.row_ptr[brow], rp1 = p.row_ptr[brow + 1];
+  it.bsr_ok = rp0 >= 0 && rp1 >= rp0 && rp1 <= p.capacity && rp1 - rp0 <= qb + 1;
+  it.n_tiles = it.bsr_ok ? (int)(rp1 - rp0) * (p.B / KT) : 0;
+  it.s = s; it.qb = qb; it.q0 = q0; it.i_begin = i_begin; it.row_lo = row_lo;
+  it.row_hi = row_hi; it.k_len = k_len; it.rp0 = rp0;
+  it.o_row0 = (int64_t)p.cu_q[s] + (i_begin - q0);
+  it.valid = true;
+  return it;
+}
+
 __global__ void __launch_bounds__(NT, 1)
     k_retrieve_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmV,
                   TcParams p) {
@@ -204,28 +276,8 @@ __global__ void __launch_bounds__(NT, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // ---- work item (uniform across the CTA)
-  int idx = blockIdx.x;
-  const int hc = idx % p.hcs; idx /= p.hcs;
-  const int rc = idx % p.rcs; idx /= p.rcs;
-  const int qbl = idx % p.nqbq;
-  const int s = idx / p.nqbq;
-  const int q_len = p.cu_q[s + 1] - p.cu_q[s];
-  const int k_len = p.cu_k[s + 1] - p.cu_k[s];
-  const int q0 = k_len - q_len;
-  if (q_len <= 0 || q0 < 0) return;
-  const int qb = q0 / p.B + qbl;
-  if ((int64_t)qb * p.B >= k_len) return;
-  const int i_begin = qb * p.B + rc * R;
-  const int row_lo = max(q0, i_begin), row_hi = min(k_len, i_begin + R);
-  if (row_lo >= row_hi) return;
-  const int64_t brow = (int64_t)p.qblock_base[s] + qb;
-  const int64_t rp0 = p.row_ptr[brow], rp1 = p.row_ptr[brow + 1];
-  const bool bsr_ok = rp0 >= 0 && rp1 >= rp0 && rp1 <= p.capacity && rp1 - rp0 <= qb + 1;
+  const int hc = blockIdx.x % p.hcs;  // constant per CTA (gridDim.x is a multiple of hcs)
   const int tpb = p.B / KT;
-  const int n_tiles = bsr_ok ? (int)(rp1 - rp0) * tpb : 0;
-  if (!bsr_ok && threadIdx.x == 0) atomicOr(p.status, ST_INDEX);
 
   const uint32_t sb = smem_u32(smem);
   const uint32_t bar0 = sb + OFF_BAR;
@@ -236,11 +288,11 @@ __global__ void __launch_bounds__(NT, 1)
     s_abort = 0;
     for (int k = 0; k < A_STAGES; ++k) { mbar_init(bar(B_AFULL + k), 1); mbar_init(bar(B_AEMPTY + k), 1); }
     for (int k = 0; k < V_STAGES; ++k) { mbar_init(bar(B_VFULL + k), 1); mbar_init(bar(B_VEMPTY + k), 1); }
-    for (int k = 0; k < 2; ++k) {
-      mbar_init(bar(B_D1FULL + k), 1); mbar_init(bar(B_D1EMPTY + k), 128);
-      mbar_init(bar(B_PFULL + k), 128); mbar_init(bar(B_PEMPTY + k), 1);
-    }
+    for (int k = 0; k < 2; ++k) { mbar_init(bar(B_D1FULL + k), 1); mbar_init(bar(B_D1EMPTY + k), 256); }
+    for (int k = 0; k < P_SLOTS; ++k) { mbar_init(bar(B_PFULL + k), 128); mbar_init(bar(B_PEMPTY + k), 1); }
     mbar_init(bar(B_OFULL), 1);
+    mbar_init(bar(B_OEMPTY), 128);
+    mbar_init(bar(B_DRAIN), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -250,8 +302,8 @@ __global__ void __launch_bounds__(NT, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  // W^T of this CTA's 16 virtual heads, bf16, K-major without swizzle:
-  // element (r_v, s) at (s/8)*256 + (r_v/8)*128 + (r_v%8)*16 + (s%8)*2
+  // W^T of this CTA's 16 virtual heads as bf16 hi + lo parts, K-major without swizzle:
+  // element (r_v, s) at (s/8)*256 + (r_v/8)*128 + (r_v%8)*16 + (s%8)*2; lo part at +W_BYTES_MAX
   {
     const int ks = p.nsc * SC;
     uint16_t* wt = reinterpret_cast<uint16_t*>(smem + OFF_W);
@@ -260,9 +312,11 @@ __global__ void __launch_bounds__(NT, 1)
       const int G = hc * NG + rv / GQP, q = rv % GQP;
       float w = 0.0f;
       if (q < p.gq && G < p.h_kv && hs < p.h_s) w = p.W[(int64_t)(G * p.gq + q) * p.h_s + hs];
-      __nv_bfloat16 b = __float2bfloat16_rn(w);
-      wt[((hs >> 3) * 256 + (rv >> 3) * 128 + (rv & 7) * 16 + (hs & 7) * 2) >> 1] =
-          *reinterpret_cast<uint16_t*>(&b);
+      __nv_bfloat16 hi = __float2bfloat16_rn(w);
+      __nv_bfloat16 lo = __float2bfloat16_rn(w - __bfloat162float(hi));
+      const int o = ((hs >> 3) * 256 + (rv >> 3) * 128 + (rv & 7) * 16 + (hs & 7) * 2) >> 1;
+      wt[o] = *reinterpret_cast<uint16_t*>(&hi);
+      wt[o + W_BYTES_MAX / 2] = *reinterpret_cast<uint16_t*>(&lo);
     }
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -279,34 +333,35 @@ __global__ void __launch_bounds__(NT, 1)
       uint32_t aph = 0, vph = 0;
       int a_issued = 0, v_issued = 0;
       bool ok = true;
-      for (int t = 0; t <= n_tiles && ok; ++t) {
-        if (t < n_tiles) {  // A chunks of tile t (consumed by the mixing of tile t)
-          const int64_t e = rp0 + t / tpb;
+      for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
+        const Item it = decode(p, idx);
+        if (!it.valid) continue;
+        TRACE(0, 1);
+        if (!it.bsr_ok) atomicOr(p.status, ST_INDEX);
+        const int rc = (idx / p.hcs) % p.rcs;
+        for (int t = 0; t < it.n_tiles && ok; ++t) {
+          const int64_t e = it.rp0 + t / tpb;
           const int half = t % tpb;
-          for (int c = 0; c < p.nsc && ok; ++c) {
+          for (int c = 0; c < p.nsc && ok; ++c) {  // A chunks (mixing of this tile)
             if (!(ok = mbar_wait(bar(B_AEMPTY + as), aph ^ 1, abort_flag, p.status))) break;
             mbar_expect_tx(bar(B_AFULL + as), A_BYTES);
             tma_load_4d(sb + OFF_A + as * A_BYTES, &tmA, bar(B_AFULL + as), half * KT, c * SC,
                         rc * R, (int)e);
+            TRACE(0, 2);
             ++a_issued;
             if (++as == A_STAGES) { as = 0; aph ^= 1; }
           }
-        }
-        if (t >= 1 && ok) {  // V tiles of tile t-1 (consumed by P.V of tile t-1)
-          const int u = t - 1;
-          const int64_t e = rp0 + u / tpb;
-          const int half = u % tpb;
           const int kb = p.col_idx[e];
-          const bool kb_ok = kb >= 0 && kb <= qb;
+          const bool kb_ok = kb >= 0 && kb <= it.qb;
           if (!kb_ok) atomicOr(p.status, ST_INDEX);
           const int tok0 = kb * p.B + half * KT;
-          for (int g = 0; g < NG && ok; ++g) {
+          for (int g = 0; g < NG && ok; ++g) {  // V tiles (P.V of this tile)
             if (!(ok = mbar_wait(bar(B_VEMPTY + vs), vph ^ 1, abort_flag, p.status))) break;
             mbar_expect_tx(bar(B_VFULL + vs), V_BYTES);
             const uint32_t dst = sb + OFF_V + vs * V_BYTES;
             const int G = hc * NG + g;
             if (!p.paged) {
-              const int row = kb_ok ? p.cu_k[s] + tok0 : p.total_k;  // out of range reads 0
+              const int row = kb_ok ? p.cu_k[it.s] + tok0 : p.total_k;  // out of range reads 0
               tma_load_3d(dst, &tmV, bar(B_VFULL + vs), 0, G, row);
               tma_load_3d(dst + 8192, &tmV, bar(B_VFULL + vs), 64, G, row);
             } else {
@@ -315,8 +370,8 @@ __global__ void __launch_bounds__(NT, 1)
                 const int tok = tok0 + q * ps;
                 const int slot = tok / ps;
                 int page = p.n_pages;  // out of range: the copy reads zeros
-                if (kb_ok && tok < k_len && slot < p.max_pages) {
-                  const int pg = p.block_table[(int64_t)s * p.max_pages + slot];
+                if (kb_ok && tok < it.k_len && slot < p.max_pages) {
+                  const int pg = p.block_table[(int64_t)it.s * p.max_pages + slot];
                   if (pg >= 0 && pg < p.n_pages) page = pg;
                   else atomicOr(p.status, ST_PAGE);
                 }
@@ -325,6 +380,7 @@ __global__ void __launch_bounds__(NT, 1)
               }
             }
             ++v_issued;
+            TRACE(0, 3);
             if (++vs == V_STAGES) { vs = 0; vph ^= 1; }
           }
         }
@@ -351,127 +407,203 @@ __global__ void __launch_bounds__(NT, 1)
       int as = 0, vs = 0;
       uint32_t aph = 0, vph = 0;
       bool ok = true;
+      int T = 0, K = 0;  // tiles and items processed so far
       const uint32_t wbase = sb + OFF_W;
-      for (int t = 0; t <= n_tiles && ok; ++t) {
-        if (t < n_tiles) {  // mixing of tile t into D1[t & 1]
-          const int b = t & 1;
-          if (!(ok = mbar_wait(bar(B_D1EMPTY + b), ((t >> 1) & 1) ^ 1, abort_flag, p.status))) break;
-          tc_fence_after();
-          const uint32_t d1 = tmem + 256u + 128u * (uint32_t)b;
-          for (int c = 0; c < p.nsc; ++c) {
-            if (!(ok = mbar_wait(bar(B_AFULL + as), aph, abort_flag, p.status))) break;
+      for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
+        const Item it = decode(p, idx);
+        if (!it.valid) continue;
+        TRACE(1, 1);
+        const int n = it.n_tiles;
+        for (int t = 0; t <= n && ok; ++t) {
+          if (t < n) {  // mixing of tile T+t into D1[(T+t) & 1]
+            const int tg = T + t, b = tg & 1;
+            if (!(ok = mbar_wait(bar(B_D1EMPTY + b), ((tg >> 1) & 1) ^ 1, abort_flag, p.status))) break;
             tc_fence_after();
-            const uint32_t abase = sb + OFF_A + as * A_BYTES;
-            const uint64_t bdesc = smem_desc(wbase + c * 512u, 256u, 128u, 0u);
-            for (int m = 0; m < 8; ++m)
-              tc_mma(d1 + 16u * m, smem_desc(abase + m * 4096u, 2048u, 1024u, 2u), bdesc,
-                     IDESC_MIX, c > 0 ? 1u : 0u);
-            tc_commit(bar(B_AEMPTY + as));
-            if (++as == A_STAGES) { as = 0; aph ^= 1; }
+            TRACE(1, 2);
+            const uint32_t d1 = tmem + 256u + 128u * (uint32_t)b;
+            for (int c = 0; c < p.nsc; ++c) {
+              if (!(ok = mbar_wait(bar(B_AFULL + as), aph, abort_flag, p.status))) break;
+              tc_fence_after();
+              TRACE(1, 3);
+              const uint32_t abase = sb + OFF_A + as * A_BYTES;
+              const uint64_t bhi = smem_desc(wbase + c * 512u, 256u, 128u, 0u);
+              const uint64_t blo = smem_desc(wbase + W_BYTES_MAX + c * 512u, 256u, 128u, 0u);
+              for (int m = 0; m < 8; ++m) {
+                const uint64_t adesc = smem_desc(abase + m * 4096u, 2048u, 1024u, 2u);
+                tc_mma(d1 + 16u * m, adesc, bhi, IDESC_MIX, c > 0 ? 1u : 0u);
+                tc_mma(d1 + 16u * m, adesc, blo, IDESC_MIX, 1u);
+              }
+              tc_commit(bar(B_AEMPTY + as));
+              if (++as == A_STAGES) { as = 0; aph ^= 1; }
+            }
+            if (!ok) break;
+            tc_commit(bar(B_D1FULL + b));
+            TRACE(1, 4);
           }
-          if (!ok) break;
-          tc_commit(bar(B_D1FULL + b));
-        }
-        if (t >= 1) {  // P.V of tile t-1 into D2
-          const int u = t - 1, b = u & 1;
-          if (!(ok = mbar_wait(bar(B_PFULL + b), (u >> 1) & 1, abort_flag, p.status))) break;
-          tc_fence_after();
-          const uint32_t pbase = sb + OFF_P + b * PBUF_BYTES;
-          for (int g = 0; g < NG; ++g) {
-            if (!(ok = mbar_wait(bar(B_VFULL + vs), vph, abort_flag, p.status))) break;
-            tc_fence_after();
-            const uint32_t vbase = sb + OFF_V + vs * V_BYTES;
-            for (int k = 0; k < 4; ++k)
-              tc_mma(tmem + 64u * g, smem_desc(vbase + k * 2048u, 8192u, 1024u, 2u),
-                     smem_desc(pbase + g * PT_BYTES + k * 2048u, 8192u, 1024u, 2u), IDESC_PV,
-                     (u > 0 || k > 0) ? 1u : 0u);
-            tc_commit(bar(B_VEMPTY + vs));
-            if (++vs == V_STAGES) { vs = 0; vph ^= 1; }
+          if (t >= 1) {  // P.V of tile T+t-1 into D2, one group (P slot, V stage) at a time
+            const int u = t - 1, ug = T + u;
+            if (u == 0 && K > 0) {  // D2 must have been read out by the previous item's epilogue
+              if (!(ok = mbar_wait(bar(B_OEMPTY), (K - 1) & 1, abort_flag, p.status))) break;
+              tc_fence_after();
+            }
+            for (int g = 0; g < NG; ++g) {
+              const int q = ug * NG + g, ps = q % P_SLOTS;
+              if (!(ok = mbar_wait(bar(B_PFULL + ps), (q / P_SLOTS) & 1, abort_flag, p.status))) break;
+              if (!(ok = mbar_wait(bar(B_VFULL + vs), vph, abort_flag, p.status))) break;
+              tc_fence_after();
+              TRACE(1, 5);
+              const uint32_t vbase = sb + OFF_V + vs * V_BYTES;
+              const uint32_t pbase = sb + OFF_P + ps * PSLOT_BYTES;
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t vdesc = smem_desc(vbase + k * 2048u, 8192u, 1024u, 2u);
+                tc_mma(tmem + 64u * g, vdesc, smem_desc(pbase + k * 2048u, 8192u, 1024u, 2u),
+                       IDESC_PV, (u > 0 || k > 0) ? 1u : 0u);
+                tc_mma(tmem + 64u * g, vdesc,
+                       smem_desc(pbase + PT_BYTES + k * 2048u, 8192u, 1024u, 2u), IDESC_PV, 1u);
+              }
+              tc_commit(bar(B_VEMPTY + vs));
+              tc_commit(bar(B_PEMPTY + ps));
+              if (++vs == V_STAGES) { vs = 0; vph ^= 1; }
+            }
+            if (!ok) break;
           }
-          if (!ok) break;
-          tc_commit(bar(B_PEMPTY + b));
         }
+        if (!ok) break;
+        tc_commit(bar(B_OFULL));  // D2 of this item complete (immediate when n == 0)
+        TRACE(1, 7);
+        T += n;
+        ++K;
       }
-      tc_commit(bar(B_OFULL));
       // drain our own MMAs before anyone frees TMEM
+      tc_commit(bar(B_DRAIN));
       const uint64_t t0 = globaltimer();
-      while (!mbar_try(bar(B_OFULL), 0) && globaltimer() - t0 < TIMEOUT_NS) {}
+      while (!mbar_try(bar(B_DRAIN), 0) && globaltimer() - t0 < TIMEOUT_NS) {}
+    }
+  } else if (warp < 10) {
+    // ================================================================ convert P (hi + lo)
+    const int quarter = warp & 3;
+    const int g0 = 2 * ((warp - 2) >> 2);  // this warp's groups: g0, g0 + 1
+    const int lrow = quarter * 32 + lane;  // TMEM lane = position in an M tile
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int j = lrow & 63;
+    const uint32_t swz = (uint32_t)j & 7u;
+    bool ok = true;
+    int T = 0;
+    for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
+      const Item it = decode(p, idx);
+      if (!it.valid) continue;
+      for (int t = 0; t < it.n_tiles && ok; ++t) {
+        const int tg = T + t, b = tg & 1;
+        // warp-uniform control flow: tcgen05.ld is a warp-collective instruction
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(bar(B_D1FULL + b), (tg >> 1) & 1, abort_flag, p.status));
+        if (!ok) break;
+        tc_fence_after();
+        if (warp == 2 && lane == 0) TRACE(2, 1);
+        const int64_t e = it.rp0 + t / tpb;
+        const int half = t % tpb;
+        const int kb = p.col_idx[e];
+        const bool kb_ok = kb >= 0 && kb <= it.qb;
+        const int tok0 = kb * p.B + half * KT;
+        for (int g = g0; g < g0 + 2 && ok; ++g) {
+          const int q = tg * NG + g, ps = q % P_SLOTS;
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PEMPTY + ps), ((q / P_SLOTS) & 1) ^ 1,
+                                                 abort_flag, p.status));
+          if (!ok) break;
+          uint32_t v[8][4];
+#pragma unroll
+          for (int m = 0; m < 8; ++m)
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v[m][0]), "=r"(v[m][1]), "=r"(v[m][2]), "=r"(v[m][3])
+                         : "r"(tl + 256u + 128u * (uint32_t)b + 16u * m + 4u * g));
+          tmem_wait_ld();
+          uint8_t* pt = smem + OFF_P + ps * PSLOT_BYTES;
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const int ii = 2 * m + (lrow >> 6);
+            const bool keep = kb_ok && tok0 + j <= it.i_begin + ii;
+            const uint32_t off = (uint32_t)j * 128u + ((((uint32_t)ii >> 1) ^ swz) << 4) +
+                                 (((uint32_t)ii & 1u) << 3);
+            float x[4], r[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              x[c] = keep ? __uint_as_float(v[m][c]) : 0.0f;
+              r[c] = x[c] - __bfloat162float(__float2bfloat16_rn(x[c]));
+            }
+            const uint32_t h0 = pack_bf16(x[0], x[1]), h1 = pack_bf16(x[2], x[3]);
+            const uint32_t l0 = pack_bf16(r[0], r[1]), l1 = pack_bf16(r[2], r[3]);
+            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(smem_u32(pt + off)), "r"(h0),
+                         "r"(h1)
+                         : "memory");
+            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(smem_u32(pt + PT_BYTES + off)),
+                         "r"(l0), "r"(l1)
+                         : "memory");
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          mbar_arrive(bar(B_PFULL + ps));
+          if (warp == 2 && lane == 0) TRACE(2, 2);
+        }
+        if (!ok) break;
+        tc_fence_before();
+        mbar_arrive(bar(B_D1EMPTY + b));
+      }
+      T += it.n_tiles;
     }
   } else {
-    // ================================================================ convert + epilogue
-    const int quarter = warp & 3;  // TMEM lanes this warp may access
-    const int lrow = quarter * 32 + lane;  // TMEM lane of this thread
+    // ================================================================ O epilogue
+    // D2 lane = head dim, column = (group, row, head)
+    const int quarter = warp & 3;
+    const int dcol = quarter * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int ng = min(NG, p.h_kv - hc * NG);  // real groups of this head chunk
     bool ok = true;
-    for (int t = 0; t < n_tiles && ok; ++t) {
-      const int b = t & 1;
-      // warp-uniform control flow: tcgen05.ld is a warp-collective instruction
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_D1FULL + b), (t >> 1) & 1, abort_flag, p.status));
+    int K = 0;
+    for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
+      const Item it = decode(p, idx);
+      if (!it.valid) continue;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OFULL), K & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait(bar(B_PEMPTY + b), ((t >> 1) & 1) ^ 1, abort_flag, p.status));
-      if (!ok) break;
-      const int64_t e = rp0 + t / tpb;
-      const int half = t % tpb;
-      const int kb = p.col_idx[e];
-      const bool kb_ok = kb >= 0 && kb <= qb;
-      const int tok0 = kb * p.B + half * KT;
-      uint8_t* pt = smem + OFF_P + b * PBUF_BYTES;
-      const int j = lrow & 63;
-      for (int m = 0; m < 8; ++m) {
-        uint32_t v[16];
-        tmem_ld16(tl + 256u + 128u * (uint32_t)b + 16u * m, v);
-        tmem_wait_ld();
-        const int ii = 2 * m + (lrow >> 6);
-        const bool keep = kb_ok && tok0 + j <= i_begin + ii;
-        const uint32_t off = (uint32_t)j * 128u + ((((uint32_t)ii >> 1) ^ ((uint32_t)j & 7u)) << 4) +
-                             (((uint32_t)ii & 1u) << 3);
+      if (warp == 10 && lane == 0) TRACE(3, 1);
+      const bool have = it.n_tiles > 0;
+      // rows [ilo, ihi) of this chunk are inside the query range; O row stride h_r * D
+      const int ilo = it.row_lo - it.i_begin, ihi = it.row_hi - it.i_begin, gq = p.gq;
+      const int64_t rs = (int64_t)p.h_r * D;
+      for (int g = 0; g < ng; ++g) {
+        __nv_bfloat16* ob = p.O + (it.o_row0 * p.h_r + (int64_t)(hc * NG + g) * gq) * D + dcol;
+        for (int kh = 0; kh < 2; ++kh) {  // 32 of the group's 64 columns at a time
+          uint32_t v[2][16];
+          if (have) {
+            tmem_ld16(tl + 64u * g + 32u * kh, v[0]);
+            tmem_ld16(tl + 64u * g + 32u * kh + 16u, v[1]);
+            tmem_wait_ld();
+          } else {
 #pragma unroll
-        for (int g = 0; g < NG; ++g) {
-          uint32_t w0 = 0u, w1 = 0u;
-          if (keep) {
-            w0 = pack_bf16(__uint_as_float(v[4 * g + 0]), __uint_as_float(v[4 * g + 1]));
-            w1 = pack_bf16(__uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
+            for (int k = 0; k < 2; ++k)
+#pragma unroll
+              for (int c = 0; c < 16; ++c) v[k][c] = 0u;
           }
-          asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(smem_u32(pt + g * PT_BYTES + off)),
-                       "r"(w0), "r"(w1)
-                       : "memory");
+          if (g == ng - 1 && kh == 1) {  // D2 fully read: the next item may overwrite it
+            tc_fence_before();
+            mbar_arrive(bar(B_OEMPTY));
+            if (warp == 10 && lane == 0) TRACE(3, 2);
+          }
+#pragma unroll
+          for (int k = 0; k < 2; ++k)
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int ii = 8 * kh + 4 * k + c / GQP, rv = c % GQP;
+              if (rv < gq && ii >= ilo && ii < ihi)
+                ob[ii * rs + rv * D] = __float2bfloat16_rn(__uint_as_float(v[k][c]));
+            }
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar(B_D1EMPTY + b));
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(bar(B_PFULL + b));
-    }
-    // ---- O epilogue: D2 lane = head dim, column = (group, row, head)
-    const bool have = __all_sync(0xffffffffu, ok && n_tiles > 0 &&
-                                                  mbar_wait(bar(B_OFULL), 0, abort_flag, p.status));
-    tc_fence_after();
-    const int dcol = lrow;  // head-dim index of this thread
-    for (int g = 0; g < NG; ++g) {
-      const int G = hc * NG + g;
-      if (G >= p.h_kv) break;
-      for (int k = 0; k < 4; ++k) {
-        uint32_t v[16];
-        if (have) {
-          tmem_ld16(tl + 64u * g + 16u * k, v);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) v[c] = 0u;
-        }
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int ii = 4 * k + c / GQP, rv = c % GQP;
-          const int row = i_begin + ii;
-          if (rv < p.gq && row >= row_lo && row < row_hi) {
-            const int r = G * p.gq + rv;
-            const int64_t orow = (int64_t)p.cu_q[s] + (row - q0);
-            p.O[(orow * p.h_r + r) * D + dcol] = __float2bfloat16_rn(__uint_as_float(v[c]));
-          }
-        }
+      if (ng <= 0) {
+        tc_fence_before();
+        mbar_arrive(bar(B_OEMPTY));
       }
+      if (warp == 10 && lane == 0) TRACE(3, 3);
+      ++K;
     }
   }
   tc_fence_before();
@@ -561,9 +693,16 @@ bool launch_retrieve_tc(const mf_retrieve_desc& d, const RetrieveLayer& l, uint3
   p.h_s = d.h_s; p.nsc = (d.h_s + SC - 1) / SC; p.B = B; p.h_r = d.h_r; p.h_kv = d.h_kv;
   p.gq = d.h_r / d.h_kv;
   p.status = status;
-  const int64_t grid = (int64_t)d.nseq * p.nqbq * p.rcs * p.hcs;
-  if (grid == 0) return true;
-  if (grid >= ((int64_t)1 << 31)) { *err = "grid too large"; return false; }
+  const int64_t n_items = (int64_t)d.nseq * p.nqbq * p.rcs * p.hcs;
+  if (n_items == 0) return true;
+  if (n_items >= ((int64_t)1 << 31)) { *err = "too many work items"; return false; }
+  p.n_items = (int)n_items;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // persistent grid, a multiple of the head-chunk count (one W^T per CTA)
+  int64_t grid = std::min<int64_t>(n_items, sms);
+  grid = std::max<int64_t>(p.hcs, grid / p.hcs * p.hcs);
   cudaError_t e = cudaFuncSetAttribute(k_retrieve_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SMEM_BYTES);
   if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
@@ -574,3 +713,13 @@ bool launch_retrieve_tc(const mf_retrieve_desc& d, const RetrieveLayer& l, uint3
 }
 
 }  // namespace mfi
+
+#ifdef MF_TRACE
+extern "C" __attribute__((visibility("default"))) int mf_trace_dump(void* host, size_t bytes) {
+  if (bytes < sizeof(mfi::g_trace)) return -1;
+  if (cudaMemcpyFromSymbol(host, mfi::g_trace, sizeof(mfi::g_trace)) != cudaSuccess) return -2;
+  static uint64_t zero[mfi::TRACE_CTAS][4][mfi::TRACE_N];
+  if (cudaMemcpyToSymbol(mfi::g_trace, zero, sizeof(zero)) != cudaSuccess) return -3;
+  return 0;
+}
+#endif

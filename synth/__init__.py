@@ -56,12 +56,13 @@ def gen_maps_gpu(out, L, B, h_s, n_heavy, seed=0, layer=0, seq=0, reading=1, dty
     code, tdt = _dt(dtype)
     Lp = -(-L // B) * B
     assert out.is_cuda and out.dtype == tdt and out.numel() >= h_s * Lp * Lp
-    heavy = np.stack([heavy_columns(seed, layer, seq, s, L, n_heavy) for s in range(h_s)]) \
-        if n_heavy > 0 else np.zeros((h_s, 1), dtype=np.int32)
+    nh = min(n_heavy, L)
+    heavy = np.stack([heavy_columns(seed, layer, seq, s, L, nh) for s in range(h_s)]) \
+        if nh > 0 else np.zeros((h_s, 1), dtype=np.int32)
     heavy_t = torch.from_numpy(heavy.astype(np.int32)).to(out.device)
     st = torch.cuda.current_stream(out.device).cuda_stream
     rc = _load().mfsynth_gen_maps(out.data_ptr(), code, L, Lp, B, h_s, heavy_t.data_ptr(),
-                                  n_heavy, seed, layer, seq, reading, st)
+                                  nh, seed, layer, seq, reading, st)
     if rc != 0:
         raise RuntimeError(f"mfsynth_gen_maps failed: {rc}")
     torch.cuda.current_stream(out.device).synchronize()  # heavy_t lifetime

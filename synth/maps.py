@@ -10,8 +10,8 @@ Map recipe (one (layer, sequence, sender head) at a time), for query row i and k
 
 and the map row is the causal softmax of that row (subtract the row max, exp, divide
 by the sum), rounded to the map dtype.  Entries with j > i, and every entry of a
-padding row i >= L, are 0.  Heavy columns are n_heavy distinct keys drawn uniformly
-from [0, L) (rejection of repeats, TAG_HEAVY stream).
+padding row i >= L, are 0.  Heavy columns are min(n_heavy, L) distinct keys drawn
+uniformly from [0, L) (rejection of repeats, TAG_HEAVY stream).
 
 Nothing here computes block statistics, selection, head mixing or P.V: this module
 only makes inputs.  `synth/csrc/gen_maps.cu` follows the same recipe on the GPU for
@@ -30,8 +30,8 @@ DECAY = 0.05
 
 
 def heavy_columns(seed, layer, seq, head, L, n_heavy):
-    if n_heavy > L:
-        raise ValueError("n_heavy > L")
+    """min(n_heavy, L) distinct heavy columns of one (layer, sequence, sender head)."""
+    n_heavy = min(n_heavy, L)
     key = rng.stream_key(seed, rng.TAG_HEAVY, layer, seq, head)
     chosen, seen, n = [], set(), 0
     while len(chosen) < n_heavy:

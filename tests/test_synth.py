@@ -59,6 +59,7 @@ def test_heavy_columns_distinct_and_seeded():
     assert len(set(a.tolist())) == 64 and a.min() >= 0 and a.max() < 1000
     assert (a == b).all() and not (a == c).all()
     assert sorted(smaps.heavy_columns(0, 0, 0, 0, 5, 5).tolist()) == [0, 1, 2, 3, 4]
+    assert sorted(smaps.heavy_columns(0, 0, 0, 0, 3, 16).tolist()) == [0, 1, 2]
 
 
 def test_v_and_w_distributions():
