@@ -11,31 +11,33 @@
 // receiver heads; a group of gq <= 4 heads is padded to 4).  The kernel is
 // persistent: each CTA walks items blockIdx.x, blockIdx.x + gridDim.x, ... (the grid
 // is a multiple of the head-chunk count, so a CTA keeps one head chunk and one W^T),
-// and the rings below run across item boundaries, so the loads and the mixing of
-// the next item overlap the tail of the current one.  For each kept 64-key tile:
+// and every ring runs across item boundaries, so the loads and the mixing of the
+// next item overlap the tail of the current one.  For each kept 64-key tile:
 //
-//   mixing  D1[pos][r] = sum_s A_s[pos] * W[r][s]       tcgen05 M=128 N=16 K=16
-//           pos = (row, key) of 2 rows x 64 keys, A tile MN-major SW128 from TMA,
-//           W^T K-major in smem.  W is split into bf16 hi + lo parts (two MMAs into
-//           the same accumulator), so the mixing keeps ~16 bits of W.  D1 is
-//           double-buffered in TMEM.
-//   convert 4 epilogue warps read D1 (lane = position), apply the causal mask and
-//           split P into bf16 hi + lo (P = hi + lo to ~16 bits), written as
-//           P^T[key][(row, head)] (MN-major SW128), one group at a time into a
-//           ring of shared-memory slots.
+//   mixing  D1[pos][(part, r)] = sum_s A_s[pos] * W_part[r][s]   tcgen05 M=128 N=32 K=16
+//           pos = (row, key) of 2 rows x 64 keys (one M tile), A tile MN-major SW128
+//           from TMA; B = W^T with W split into bf16 hi and lo parts stacked along N,
+//           so one MMA per M tile and s-chunk keeps ~16 bits of W.  D1 is a ring of
+//           eight 32-column M-tile slots in TMEM.
+//   convert 8 warps read D1 (lane = position), form P = hi part + lo part (float32),
+//           apply the causal mask and split P into bf16 hi + lo (P = hi + lo to ~16
+//           bits), written as P^T[key][(row, head)] (MN-major SW128) per group.
 //   P.V     D2[dim][(row, head)] += V^T[dim][key] * (P^T_hi + P^T_lo)[key][(row, head)]
 //           tcgen05 M=128 (d) N=64 K=16 per group, two MMAs per K step; V tile
 //           MN-major SW128 by TMA (contiguous or paged).  D2 stays in TMEM for the
 //           whole row chunk.
-// The hi/lo splits keep the only bf16 rounding that matters at the final O.
+// The hi/lo splits leave the final bf16 rounding of O as the only rounding that
+// matters.
 //
-// Warp roles: warp 0 TMA producer, warp 1 MMA issuer (+ TMEM owner), warps 2-9
-// convert P (two warps per TMEM lane quarter, each taking two of the four groups),
-// warps 10-13 O epilogue (they release D2 as soon as it is read, so the next item's
-// P.V can start while O is stored).  TMEM: D2 in columns [0, 256), D1
-// in [256, 512).  Every
-// mbarrier wait is bounded by a timer: on expiry the CTA records ST_TIMEOUT, all
-// roles stop, in-flight copies and MMAs are drained (bounded) and TMEM is freed.
+// Warp roles: 0 TMA producer of the map tiles; 1 mixing MMA issuer (+ TMEM owner);
+// 2 P.V MMA issuer; 3 TMA producer of the V tiles (separate producers and issuers, so
+// no stream waits behind another); 4-19 convert (four sets of four warps, one warp per
+// TMEM lane quarter; set k converts the M tiles m = k, k + 4 for all 16 heads);
+// 20-23 O epilogue (they release D2 as soon as it is read, so the next item's P.V can
+// start while O is stored).  Consumer warps signal barriers once per warp (lane 0
+// after __syncwarp).  TMEM: D2 in columns [0, 256), D1 slots in [256, 512).  Every mbarrier
+// wait is bounded by a timer: on expiry the CTA records ST_TIMEOUT, all roles stop,
+// in-flight copies and MMAs are drained (bounded) and TMEM is freed.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -49,7 +51,8 @@
 namespace mfi {
 namespace {
 
-constexpr int NT = 448;
+constexpr int NT = 768;        // 24 warps
+constexpr int CONV_SETS = 4;   // convert warp sets
 constexpr int R = 16;          // query rows per CTA
 constexpr int KT = 64;         // keys per tile
 constexpr int NG = 4;          // KV groups per CTA
@@ -57,7 +60,8 @@ constexpr int GQP = 4;         // virtual heads per group
 constexpr int HV = NG * GQP;   // virtual receiver heads per CTA
 constexpr int D = 128;         // head dim
 constexpr int SC = 16;         // sender heads per A chunk (one MMA K step)
-constexpr int A_STAGES = 2, V_STAGES = 4, P_SLOTS = 5;
+constexpr int MT = R * KT / 128;  // M tiles (of 128 positions) per tile: 8
+constexpr int A_STAGES = 2, V_STAGES = 3, P_SLOTS = 6;
 constexpr uint32_t A_BYTES = R * SC * KT * 2;   // 32 KB
 constexpr uint32_t V_BYTES = KT * D * 2;        // 16 KB
 constexpr uint32_t PT_BYTES = KT * 64 * 2;      // 8 KB: one group's P^T (hi or lo)
@@ -66,22 +70,24 @@ constexpr uint32_t OFF_A = 0;
 constexpr uint32_t OFF_V = OFF_A + A_STAGES * A_BYTES;
 constexpr uint32_t OFF_P = OFF_V + V_STAGES * V_BYTES;
 constexpr uint32_t OFF_W = OFF_P + P_SLOTS * PSLOT_BYTES;
-constexpr uint32_t W_BYTES_MAX = 4 * 512;       // up to 4 chunks (h_s <= 64), per part
-constexpr uint32_t OFF_BAR = OFF_W + 2 * W_BYTES_MAX;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
+constexpr uint32_t W_CHUNK = 1024;              // W^T (32 rows = hi, lo) per s-chunk
+constexpr uint32_t W_BYTES_MAX = 4 * W_CHUNK;   // up to 4 chunks (h_s <= 64)
+constexpr uint32_t OFF_BAR = OFF_W + W_BYTES_MAX;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;  // + alignment slack
 constexpr uint64_t TIMEOUT_NS = 2000000000ull;
 
 // barrier slots (8 bytes each)
 enum {
   B_AFULL = 0, B_AEMPTY = B_AFULL + A_STAGES, B_VFULL = B_AEMPTY + A_STAGES,
-  B_VEMPTY = B_VFULL + V_STAGES, B_D1FULL = B_VEMPTY + V_STAGES, B_D1EMPTY = B_D1FULL + 2,
-  B_PFULL = B_D1EMPTY + 2, B_PEMPTY = B_PFULL + P_SLOTS, B_OFULL = B_PEMPTY + P_SLOTS,
-  B_OEMPTY = B_OFULL + 1, B_DRAIN = B_OEMPTY + 1, B_COUNT = B_DRAIN + 1
+  B_VEMPTY = B_VFULL + V_STAGES, B_D1FULL = B_VEMPTY + V_STAGES, B_D1EMPTY = B_D1FULL + MT,
+  B_PFULL = B_D1EMPTY + MT, B_PEMPTY = B_PFULL + P_SLOTS, B_OFULL = B_PEMPTY + P_SLOTS,
+  B_OEMPTY = B_OFULL + 1, B_DRAIN1 = B_OEMPTY + 1, B_DRAIN2 = B_DRAIN1 + 1, B_COUNT = B_DRAIN2 + 1
 };
+static_assert(B_COUNT * 8 <= 512, "barrier area");
 
 // instruction descriptors (kind::f16): D f32, A/B bf16, majors, N >> 3, M >> 4
 constexpr uint32_t IDESC_MIX = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (0u << 16) |
-                               ((16u >> 3) << 17) | ((128u >> 4) << 24);
+                               ((32u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t IDESC_PV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                               ((64u >> 3) << 17) | ((128u >> 4) << 24);
 
@@ -213,7 +219,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // stamps of pipeline events, read back with mf_trace_dump().
 #ifdef MF_TRACE
 constexpr int TRACE_CTAS = 160, TRACE_N = 2048;
-__device__ uint64_t g_trace[TRACE_CTAS][4][TRACE_N];
+__device__ uint64_t g_trace[TRACE_CTAS][5][TRACE_N];
 __device__ __forceinline__ void trace(int role, uint32_t code) {
   if (blockIdx.x >= TRACE_CTAS) return;
   uint64_t* b = g_trace[blockIdx.x][role];
@@ -288,11 +294,12 @@ __global__ void __launch_bounds__(NT, 1)
     s_abort = 0;
     for (int k = 0; k < A_STAGES; ++k) { mbar_init(bar(B_AFULL + k), 1); mbar_init(bar(B_AEMPTY + k), 1); }
     for (int k = 0; k < V_STAGES; ++k) { mbar_init(bar(B_VFULL + k), 1); mbar_init(bar(B_VEMPTY + k), 1); }
-    for (int k = 0; k < 2; ++k) { mbar_init(bar(B_D1FULL + k), 1); mbar_init(bar(B_D1EMPTY + k), 256); }
-    for (int k = 0; k < P_SLOTS; ++k) { mbar_init(bar(B_PFULL + k), 128); mbar_init(bar(B_PEMPTY + k), 1); }
+    for (int k = 0; k < MT; ++k) { mbar_init(bar(B_D1FULL + k), 1); mbar_init(bar(B_D1EMPTY + k), 4); }
+    for (int k = 0; k < P_SLOTS; ++k) { mbar_init(bar(B_PFULL + k), 4 * CONV_SETS); mbar_init(bar(B_PEMPTY + k), 1); }
     mbar_init(bar(B_OFULL), 1);
-    mbar_init(bar(B_OEMPTY), 128);
-    mbar_init(bar(B_DRAIN), 1);
+    mbar_init(bar(B_OEMPTY), 4);
+    mbar_init(bar(B_DRAIN1), 1);
+    mbar_init(bar(B_DRAIN2), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -302,8 +309,9 @@ __global__ void __launch_bounds__(NT, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  // W^T of this CTA's 16 virtual heads as bf16 hi + lo parts, K-major without swizzle:
-  // element (r_v, s) at (s/8)*256 + (r_v/8)*128 + (r_v%8)*16 + (s%8)*2; lo part at +W_BYTES_MAX
+  // W^T of this CTA's 16 virtual heads, bf16, K-major without swizzle, 32 rows per s:
+  // row n < 16 is the hi part of head n, row 16 + n its lo part.  Element (n, s) at
+  // (s/8)*512 + (n/8)*128 + (n%8)*16 + (s%8)*2.
   {
     const int ks = p.nsc * SC;
     uint16_t* wt = reinterpret_cast<uint16_t*>(smem + OFF_W);
@@ -314,9 +322,9 @@ __global__ void __launch_bounds__(NT, 1)
       if (q < p.gq && G < p.h_kv && hs < p.h_s) w = p.W[(int64_t)(G * p.gq + q) * p.h_s + hs];
       __nv_bfloat16 hi = __float2bfloat16_rn(w);
       __nv_bfloat16 lo = __float2bfloat16_rn(w - __bfloat162float(hi));
-      const int o = ((hs >> 3) * 256 + (rv >> 3) * 128 + (rv & 7) * 16 + (hs & 7) * 2) >> 1;
-      wt[o] = *reinterpret_cast<uint16_t*>(&hi);
-      wt[o + W_BYTES_MAX / 2] = *reinterpret_cast<uint16_t*>(&lo);
+      const int base = (hs >> 3) * 512 + (hs & 7) * 2;
+      wt[(base + (rv >> 3) * 128 + (rv & 7) * 16) >> 1] = *reinterpret_cast<uint16_t*>(&hi);
+      wt[(base + ((rv + 16) >> 3) * 128 + (rv & 7) * 16) >> 1] = *reinterpret_cast<uint16_t*>(&lo);
     }
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -326,9 +334,11 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t tmem = s_tmem;
   volatile int* abort_flag = &s_abort;
 
-  if (warp == 0) {
-    // ================================================================ TMA producer
+  if (warp == 0 || warp == 3) {
+    // ================================================================ TMA producers
+    // warp 0: map tiles (A chunks) in mixing order; warp 3: V tiles in P.V order
     if (lane == 0) {
+      const bool is_a = warp == 0;
       int as = 0, vs = 0;
       uint32_t aph = 0, vph = 0;
       int a_issued = 0, v_issued = 0;
@@ -336,26 +346,29 @@ __global__ void __launch_bounds__(NT, 1)
       for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
         const Item it = decode(p, idx);
         if (!it.valid) continue;
-        TRACE(0, 1);
-        if (!it.bsr_ok) atomicOr(p.status, ST_INDEX);
+        if (is_a) TRACE(0, 1);
+        if (is_a && !it.bsr_ok) atomicOr(p.status, ST_INDEX);
         const int rc = (idx / p.hcs) % p.rcs;
         for (int t = 0; t < it.n_tiles && ok; ++t) {
           const int64_t e = it.rp0 + t / tpb;
           const int half = t % tpb;
-          for (int c = 0; c < p.nsc && ok; ++c) {  // A chunks (mixing of this tile)
-            if (!(ok = mbar_wait(bar(B_AEMPTY + as), aph ^ 1, abort_flag, p.status))) break;
-            mbar_expect_tx(bar(B_AFULL + as), A_BYTES);
-            tma_load_4d(sb + OFF_A + as * A_BYTES, &tmA, bar(B_AFULL + as), half * KT, c * SC,
-                        rc * R, (int)e);
-            TRACE(0, 2);
-            ++a_issued;
-            if (++as == A_STAGES) { as = 0; aph ^= 1; }
+          if (is_a) {
+            for (int c = 0; c < p.nsc && ok; ++c) {
+              if (!(ok = mbar_wait(bar(B_AEMPTY + as), aph ^ 1, abort_flag, p.status))) break;
+              mbar_expect_tx(bar(B_AFULL + as), A_BYTES);
+              tma_load_4d(sb + OFF_A + as * A_BYTES, &tmA, bar(B_AFULL + as), half * KT, c * SC,
+                          rc * R, (int)e);
+              TRACE(0, 2);
+              ++a_issued;
+              if (++as == A_STAGES) { as = 0; aph ^= 1; }
+            }
+            continue;
           }
           const int kb = p.col_idx[e];
           const bool kb_ok = kb >= 0 && kb <= it.qb;
           if (!kb_ok) atomicOr(p.status, ST_INDEX);
           const int tok0 = kb * p.B + half * KT;
-          for (int g = 0; g < NG && ok; ++g) {  // V tiles (P.V of this tile)
+          for (int g = 0; g < NG && ok; ++g) {
             if (!(ok = mbar_wait(bar(B_VEMPTY + vs), vph ^ 1, abort_flag, p.status))) break;
             mbar_expect_tx(bar(B_VFULL + vs), V_BYTES);
             const uint32_t dst = sb + OFF_V + vs * V_BYTES;
@@ -402,87 +415,100 @@ __global__ void __launch_bounds__(NT, 1)
       }
     }
   } else if (warp == 1) {
-    // ================================================================ MMA issuer
+    // ================================================================ mixing MMA issuer
     if (lane == 0) {
-      int as = 0, vs = 0;
-      uint32_t aph = 0, vph = 0;
+      int as = 0;
+      uint32_t aph = 0;
       bool ok = true;
-      int T = 0, K = 0;  // tiles and items processed so far
-      const uint32_t wbase = sb + OFF_W;
+      int T = 0;  // tiles processed so far
+      const uint64_t wdesc0 = smem_desc(sb + OFF_W, 512u, 128u, 0u);
+      const uint64_t adesc0 = smem_desc(sb + OFF_A, 2048u, 1024u, 2u);
       for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
         const Item it = decode(p, idx);
         if (!it.valid) continue;
         TRACE(1, 1);
-        const int n = it.n_tiles;
-        for (int t = 0; t <= n && ok; ++t) {
-          if (t < n) {  // mixing of tile T+t into D1[(T+t) & 1]
-            const int tg = T + t, b = tg & 1;
-            if (!(ok = mbar_wait(bar(B_D1EMPTY + b), ((tg >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+        for (int t = 0; t < it.n_tiles && ok; ++t, ++T) {
+          // chunk-major: each s-chunk is mixed into all eight M-tile slots and released;
+          // the last chunk commits each slot as soon as its final MMA is issued
+          for (int c = 0; c < p.nsc && ok; ++c) {
+            if (!(ok = mbar_wait(bar(B_AFULL + as), aph, abort_flag, p.status))) break;
             tc_fence_after();
-            TRACE(1, 2);
-            const uint32_t d1 = tmem + 256u + 128u * (uint32_t)b;
-            for (int c = 0; c < p.nsc; ++c) {
-              if (!(ok = mbar_wait(bar(B_AFULL + as), aph, abort_flag, p.status))) break;
-              tc_fence_after();
-              TRACE(1, 3);
-              const uint32_t abase = sb + OFF_A + as * A_BYTES;
-              const uint64_t bhi = smem_desc(wbase + c * 512u, 256u, 128u, 0u);
-              const uint64_t blo = smem_desc(wbase + W_BYTES_MAX + c * 512u, 256u, 128u, 0u);
-              for (int m = 0; m < 8; ++m) {
-                const uint64_t adesc = smem_desc(abase + m * 4096u, 2048u, 1024u, 2u);
-                tc_mma(d1 + 16u * m, adesc, bhi, IDESC_MIX, c > 0 ? 1u : 0u);
-                tc_mma(d1 + 16u * m, adesc, blo, IDESC_MIX, 1u);
+            if (c == 0) TRACE(1, 3);
+            const uint64_t ad = adesc0 + (((uint32_t)as * A_BYTES) >> 4);
+            const uint64_t wd = wdesc0 + ((c * W_CHUNK) >> 4);
+            for (int m = 0; m < MT && ok; ++m) {
+              if (c == 0) {  // the slot must have been read out by the previous tile's converters
+                if (!(ok = mbar_wait(bar(B_D1EMPTY + m), (T & 1) ^ 1, abort_flag, p.status))) break;
+                tc_fence_after();
               }
-              tc_commit(bar(B_AEMPTY + as));
-              if (++as == A_STAGES) { as = 0; aph ^= 1; }
+              tc_mma(tmem + 256u + 32u * (uint32_t)m, ad + ((m * 4096u) >> 4), wd, IDESC_MIX,
+                     c > 0 ? 1u : 0u);
+              if (c == p.nsc - 1) tc_commit(bar(B_D1FULL + m));
+              if (c == 0) TRACE(1, 5);
             }
-            if (!ok) break;
-            tc_commit(bar(B_D1FULL + b));
-            TRACE(1, 4);
+            tc_commit(bar(B_AEMPTY + as));
+            if (++as == A_STAGES) { as = 0; aph ^= 1; }
           }
-          if (t >= 1) {  // P.V of tile T+t-1 into D2, one group (P slot, V stage) at a time
-            const int u = t - 1, ug = T + u;
-            if (u == 0 && K > 0) {  // D2 must have been read out by the previous item's epilogue
-              if (!(ok = mbar_wait(bar(B_OEMPTY), (K - 1) & 1, abort_flag, p.status))) break;
-              tc_fence_after();
+          if (!ok) break;
+          TRACE(1, 4);
+        }
+      }
+      tc_commit(bar(B_DRAIN1));
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try(bar(B_DRAIN1), 0) && globaltimer() - t0 < TIMEOUT_NS) {}
+    }
+  } else if (warp == 2) {
+    // ================================================================ P.V MMA issuer
+    if (lane == 0) {
+      int vs = 0;
+      uint32_t vph = 0;
+      bool ok = true;
+      int T = 0, K = 0;  // tiles and items processed so far
+      const uint64_t vdesc0 = smem_desc(sb + OFF_V, 8192u, 1024u, 2u);
+      const uint64_t pdesc0 = smem_desc(sb + OFF_P, 8192u, 1024u, 2u);
+      for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
+        const Item it = decode(p, idx);
+        if (!it.valid) continue;
+        // D2 must have been read out by the previous item's epilogue (waited for every
+        // item, also one without tiles, so the phases of the barrier are taken in order)
+        if (K > 0) {
+          if (!(ok = mbar_wait(bar(B_OEMPTY), (K - 1) & 1, abort_flag, p.status))) break;
+          tc_fence_after();
+        }
+        for (int t = 0; t < it.n_tiles && ok; ++t, ++T) {
+          for (int g = 0; g < NG; ++g) {
+            const int q = T * NG + g, ps = q % P_SLOTS;
+            if (!(ok = mbar_wait(bar(B_PFULL + ps), (q / P_SLOTS) & 1, abort_flag, p.status))) break;
+            if (!(ok = mbar_wait(bar(B_VFULL + vs), vph, abort_flag, p.status))) break;
+            tc_fence_after();
+            TRACE(4, 5);
+            const uint64_t vd = vdesc0 + ((vs * V_BYTES) >> 4);
+            const uint64_t pd = pdesc0 + ((ps * PSLOT_BYTES) >> 4);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              tc_mma(tmem + 64u * g, vd + ((k * 2048u) >> 4), pd + ((k * 2048u) >> 4), IDESC_PV,
+                     (t > 0 || k > 0) ? 1u : 0u);
+              tc_mma(tmem + 64u * g, vd + ((k * 2048u) >> 4), pd + ((PT_BYTES + k * 2048u) >> 4),
+                     IDESC_PV, 1u);
             }
-            for (int g = 0; g < NG; ++g) {
-              const int q = ug * NG + g, ps = q % P_SLOTS;
-              if (!(ok = mbar_wait(bar(B_PFULL + ps), (q / P_SLOTS) & 1, abort_flag, p.status))) break;
-              if (!(ok = mbar_wait(bar(B_VFULL + vs), vph, abort_flag, p.status))) break;
-              tc_fence_after();
-              TRACE(1, 5);
-              const uint32_t vbase = sb + OFF_V + vs * V_BYTES;
-              const uint32_t pbase = sb + OFF_P + ps * PSLOT_BYTES;
-              for (int k = 0; k < 4; ++k) {
-                const uint64_t vdesc = smem_desc(vbase + k * 2048u, 8192u, 1024u, 2u);
-                tc_mma(tmem + 64u * g, vdesc, smem_desc(pbase + k * 2048u, 8192u, 1024u, 2u),
-                       IDESC_PV, (u > 0 || k > 0) ? 1u : 0u);
-                tc_mma(tmem + 64u * g, vdesc,
-                       smem_desc(pbase + PT_BYTES + k * 2048u, 8192u, 1024u, 2u), IDESC_PV, 1u);
-              }
-              tc_commit(bar(B_VEMPTY + vs));
-              tc_commit(bar(B_PEMPTY + ps));
-              if (++vs == V_STAGES) { vs = 0; vph ^= 1; }
-            }
-            if (!ok) break;
+            tc_commit(bar(B_VEMPTY + vs));
+            tc_commit(bar(B_PEMPTY + ps));
+            if (++vs == V_STAGES) { vs = 0; vph ^= 1; }
           }
         }
         if (!ok) break;
-        tc_commit(bar(B_OFULL));  // D2 of this item complete (immediate when n == 0)
-        TRACE(1, 7);
-        T += n;
+        tc_commit(bar(B_OFULL));  // D2 of this item complete (immediate when it has no tile)
+        TRACE(4, 7);
         ++K;
       }
-      // drain our own MMAs before anyone frees TMEM
-      tc_commit(bar(B_DRAIN));
+      tc_commit(bar(B_DRAIN2));
       const uint64_t t0 = globaltimer();
-      while (!mbar_try(bar(B_DRAIN), 0) && globaltimer() - t0 < TIMEOUT_NS) {}
+      while (!mbar_try(bar(B_DRAIN2), 0) && globaltimer() - t0 < TIMEOUT_NS) {}
     }
-  } else if (warp < 10) {
+  } else if (warp < 4 + 4 * CONV_SETS) {
     // ================================================================ convert P (hi + lo)
     const int quarter = warp & 3;
-    const int g0 = 2 * ((warp - 2) >> 2);  // this warp's groups: g0, g0 + 1
+    const int set = (warp - 4) >> 2;       // M tiles set, set + CONV_SETS, ...
     const int lrow = quarter * 32 + lane;  // TMEM lane = position in an M tile
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
     const int j = lrow & 63;
@@ -492,46 +518,56 @@ __global__ void __launch_bounds__(NT, 1)
     for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
       const Item it = decode(p, idx);
       if (!it.valid) continue;
-      for (int t = 0; t < it.n_tiles && ok; ++t) {
-        const int tg = T + t, b = tg & 1;
-        // warp-uniform control flow: tcgen05.ld is a warp-collective instruction
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(bar(B_D1FULL + b), (tg >> 1) & 1, abort_flag, p.status));
-        if (!ok) break;
-        tc_fence_after();
-        if (warp == 2 && lane == 0) TRACE(2, 1);
+      for (int t = 0; t < it.n_tiles && ok; ++t, ++T) {
         const int64_t e = it.rp0 + t / tpb;
         const int half = t % tpb;
         const int kb = p.col_idx[e];
         const bool kb_ok = kb >= 0 && kb <= it.qb;
         const int tok0 = kb * p.B + half * KT;
-        for (int g = g0; g < g0 + 2 && ok; ++g) {
-          const int q = tg * NG + g, ps = q % P_SLOTS;
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PEMPTY + ps), ((q / P_SLOTS) & 1) ^ 1,
-                                                 abort_flag, p.status));
+        const int q0 = T * NG;  // P slots of this tile's four groups: (q0 + g) % P_SLOTS
+        // warp-uniform control flow: tcgen05.ld is a warp-collective instruction
+        for (int g = 0; g < NG && ok; ++g)
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PEMPTY + (q0 + g) % P_SLOTS),
+                                                 (((q0 + g) / P_SLOTS) & 1) ^ 1, abort_flag, p.status));
+        if (!ok) break;
+        if (warp == 4 && lane == 0) TRACE(2, 1);
+        for (int m = set; m < MT && ok; m += CONV_SETS) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_D1FULL + m), T & 1, abort_flag, p.status));
           if (!ok) break;
-          uint32_t v[8][4];
-#pragma unroll
-          for (int m = 0; m < 8; ++m)
-            asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(v[m][0]), "=r"(v[m][1]), "=r"(v[m][2]), "=r"(v[m][3])
-                         : "r"(tl + 256u + 128u * (uint32_t)b + 16u * m + 4u * g));
+          tc_fence_after();
+          uint32_t v[32];  // columns 0-15: A.W_hi of the 16 heads, 16-31: A.W_lo
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, "
+              "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, "
+              "%26, %27, %28, %29, %30, %31}, [%32];"
+              : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+                "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+                "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+                "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+                "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+                "=r"(v[31])
+              : "r"(tl + 256u + 32u * (uint32_t)m));
           tmem_wait_ld();
-          uint8_t* pt = smem + OFF_P + ps * PSLOT_BYTES;
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_D1EMPTY + m));  // this warp is done with the M-tile slot
+          if (warp == 4 && lane == 0) TRACE(2, 3);
+          const int ii = 2 * m + (lrow >> 6);
+          const bool keep = kb_ok && tok0 + j <= it.i_begin + ii;
+          const uint32_t off = (uint32_t)j * 128u + ((((uint32_t)ii >> 1) ^ swz) << 4) +
+                               (((uint32_t)ii & 1u) << 3);
 #pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const int ii = 2 * m + (lrow >> 6);
-            const bool keep = kb_ok && tok0 + j <= it.i_begin + ii;
-            const uint32_t off = (uint32_t)j * 128u + ((((uint32_t)ii >> 1) ^ swz) << 4) +
-                                 (((uint32_t)ii & 1u) << 3);
+          for (int g = 0; g < NG; ++g) {
             float x[4], r[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-              x[c] = keep ? __uint_as_float(v[m][c]) : 0.0f;
+              const float pv = __uint_as_float(v[4 * g + c]) + __uint_as_float(v[16 + 4 * g + c]);
+              x[c] = keep ? pv : 0.0f;
               r[c] = x[c] - __bfloat162float(__float2bfloat16_rn(x[c]));
             }
             const uint32_t h0 = pack_bf16(x[0], x[1]), h1 = pack_bf16(x[2], x[3]);
             const uint32_t l0 = pack_bf16(r[0], r[1]), l1 = pack_bf16(r[2], r[3]);
+            uint8_t* pt = smem + OFF_P + ((q0 + g) % P_SLOTS) * PSLOT_BYTES;
             asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(smem_u32(pt + off)), "r"(h0),
                          "r"(h1)
                          : "memory");
@@ -539,15 +575,14 @@ __global__ void __launch_bounds__(NT, 1)
                          "r"(l0), "r"(l1)
                          : "memory");
           }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          mbar_arrive(bar(B_PFULL + ps));
-          if (warp == 2 && lane == 0) TRACE(2, 2);
         }
         if (!ok) break;
-        tc_fence_before();
-        mbar_arrive(bar(B_D1EMPTY + b));
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0)
+          for (int g = 0; g < NG; ++g) mbar_arrive(bar(B_PFULL + (q0 + g) % P_SLOTS));
+        if (warp == 4 && lane == 0) TRACE(2, 2);
       }
-      T += it.n_tiles;
     }
   } else {
     // ================================================================ O epilogue
@@ -564,7 +599,7 @@ __global__ void __launch_bounds__(NT, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OFULL), K & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
-      if (warp == 10 && lane == 0) TRACE(3, 1);
+      if (warp == 20 && lane == 0) TRACE(3, 1);
       const bool have = it.n_tiles > 0;
       // rows [ilo, ihi) of this chunk are inside the query range; O row stride h_r * D
       const int ilo = it.row_lo - it.i_begin, ihi = it.row_hi - it.i_begin, gq = p.gq;
@@ -585,8 +620,9 @@ __global__ void __launch_bounds__(NT, 1)
           }
           if (g == ng - 1 && kh == 1) {  // D2 fully read: the next item may overwrite it
             tc_fence_before();
-            mbar_arrive(bar(B_OEMPTY));
-            if (warp == 10 && lane == 0) TRACE(3, 2);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_OEMPTY));
+            if (warp == 20 && lane == 0) TRACE(3, 2);
           }
 #pragma unroll
           for (int k = 0; k < 2; ++k)
@@ -600,9 +636,10 @@ __global__ void __launch_bounds__(NT, 1)
       }
       if (ng <= 0) {
         tc_fence_before();
-        mbar_arrive(bar(B_OEMPTY));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_OEMPTY));
       }
-      if (warp == 10 && lane == 0) TRACE(3, 3);
+      if (warp == 20 && lane == 0) TRACE(3, 3);
       ++K;
     }
   }
@@ -718,7 +755,7 @@ bool launch_retrieve_tc(const mf_retrieve_desc& d, const RetrieveLayer& l, uint3
 extern "C" __attribute__((visibility("default"))) int mf_trace_dump(void* host, size_t bytes) {
   if (bytes < sizeof(mfi::g_trace)) return -1;
   if (cudaMemcpyFromSymbol(host, mfi::g_trace, sizeof(mfi::g_trace)) != cudaSuccess) return -2;
-  static uint64_t zero[mfi::TRACE_CTAS][4][mfi::TRACE_N];
+  static uint64_t zero[mfi::TRACE_CTAS][5][mfi::TRACE_N];
   if (cudaMemcpyToSymbol(mfi::g_trace, zero, sizeof(zero)) != cudaSuccess) return -3;
   return 0;
 }
