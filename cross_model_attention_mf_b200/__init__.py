@@ -64,6 +64,8 @@ _lib.mf_compress_workspace_size.argtypes = [ctypes.POINTER(CompressDesc), ctypes
 _lib.mf_compress_workspace_size.restype = ctypes.c_int
 _lib.mf_compress.argtypes = [ctypes.POINTER(CompressDesc), _P, ctypes.c_size_t, _P]
 _lib.mf_compress.restype = ctypes.c_int
+_lib.mf_compress_static.argtypes = [ctypes.POINTER(CompressDesc), _P]
+_lib.mf_compress_static.restype = ctypes.c_int
 _lib.mf_map_retrieve.argtypes = [ctypes.POINTER(RetrieveDesc), _P]
 _lib.mf_map_retrieve.restype = ctypes.c_int
 _lib.mf_retrieve_path.argtypes = [ctypes.POINTER(RetrieveDesc)]
@@ -166,6 +168,19 @@ def mf_compress(maps: torch.Tensor, map_seq_offset: torch.Tensor, cu_seqlens: to
     if workspace is None:
         workspace = torch.empty(need.value, dtype=torch.uint8, device=maps.device)
     _check(_lib.mf_compress(ctypes.byref(d), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+MF_STATIC_WORKSPACE_BYTES = 8 << 20
+
+
+def mf_compress_static(maps: torch.Tensor, map_seq_offset: torch.Tensor, cu_seqlens: torch.Tensor,
+                       max_seqlen: int, h_s: int, B: int, tau: float, out: BSR,
+                       stream=None) -> BSR:
+    """Same as mf_compress, for callers that cannot allocate device memory: the scratch
+    comes from the library's static device array (see mf.h); nothing is allocated here."""
+    d = _compress_desc(maps, map_seq_offset, cu_seqlens, max_seqlen, h_s, B, tau, out)
+    _check(_lib.mf_compress_static(ctypes.byref(d), _stream(stream)))
     return out
 
 

@@ -3,6 +3,7 @@
 #include <stdint.h>
 
 #include <cstdio>
+#include <mutex>
 #include <string>
 
 #include "mf.h"
@@ -81,6 +82,34 @@ mf_status check_retrieve(const mf_retrieve_desc* d) {
   return MF_OK;
 }
 
+// Scratch of mf_compress_static: a file-scope device array, so that entry point never
+// allocates.  Each device that loads this library holds MF_STATIC_WORKSPACE_BYTES of it
+// until the process exits.  In host code `g_static_ws` is only a stand-in for the
+// symbol, never a device address: the address is looked up per device below.
+static __device__ __align__(256) unsigned char g_static_ws[MF_STATIC_WORKSPACE_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_ptr[kMaxDevices];  // device address of g_static_ws, per device (null: not yet)
+
+// Device address of the static scratch on the current device; looked up once per device.
+mf_status static_ws_ptr(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(MF_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(MF_ERR_UNSUPPORTED, "device ordinal above 63");
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_ws);
+    if (e != cudaSuccess || !p)
+      return fail(MF_ERR_CUDA, std::string("cudaGetSymbolAddress(static scratch): ") + cudaGetErrorString(e));
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return MF_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -123,6 +152,30 @@ mf_status mf_compress(const mf_compress_desc* desc, void* workspace, size_t work
   mfi::compress_ws_layout(*desc, &ws, workspace);
   cudaError_t e = mfi::launch_compress(*desc, ws, st, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(MF_ERR_CUDA, std::string("mf_compress launch: ") + cudaGetErrorString(e));
+  return MF_OK;
+}
+
+mf_status mf_compress_static(const mf_compress_desc* desc, void* stream) {
+  mf_status s = check_compress(desc);
+  if (s != MF_OK) return s;
+  const size_t need = mfi::compress_ws_layout(*desc, nullptr, nullptr);
+  if (need > (size_t)MF_STATIC_WORKSPACE_BYTES)
+    return fail(MF_ERR_UNSUPPORTED, "mf_compress_static: this descriptor needs " + std::to_string(need) +
+                                        " bytes of scratch, more than the static " +
+                                        std::to_string((size_t)MF_STATIC_WORKSPACE_BYTES) +
+                                        " bytes; use mf_compress with a caller workspace");
+  void* ws_ptr = nullptr;
+  s = static_ws_ptr(&ws_ptr);
+  if (s != MF_OK) return s;
+  uint32_t* st = status_ptr();
+  if (!st) return fail(MF_ERR_CUDA, "cannot resolve the device status word");
+  // Every scratch word the kernels read is written earlier in the same call, so the
+  // contents left by a previous call need no clearing.
+  mfi::CompressWs ws;
+  mfi::compress_ws_layout(*desc, &ws, ws_ptr);
+  cudaError_t e = mfi::launch_compress(*desc, ws, st, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess)
+    return fail(MF_ERR_CUDA, std::string("mf_compress_static launch: ") + cudaGetErrorString(e));
   return MF_OK;
 }
 

@@ -119,6 +119,26 @@ mf_status mf_compress_workspace_size(const mf_compress_desc* desc, size_t* bytes
 mf_status mf_compress(const mf_compress_desc* desc, void* workspace, size_t workspace_bytes,
                       void* stream);
 
+/* Compression for callers that cannot allocate device memory.  (This entry point is
+ * a property of this library, not of the MapFlow method: the pages have no
+ * counterpart.)  Some callers may not call cudaMalloc at all: a plugin inside a host
+ * program that owns every byte of device memory through its own pool, or a
+ * latency-critical path where an allocation's implicit device synchronisation is
+ * not acceptable.  Such a caller passes only the inputs and outputs; the scratch
+ * space mf_compress takes as `workspace` comes instead from a file-scope device
+ * array of MF_STATIC_WORKSPACE_BYTES that every device loading this library holds
+ * until the process exits.  Nothing is allocated or freed by this call.
+ *   - The first call on a device looks up the array's device address on the current
+ *     device (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - A descriptor whose scratch need (mf_compress_workspace_size) exceeds
+ *     MF_STATIC_WORKSPACE_BYTES is rejected with MF_ERR_UNSUPPORTED and a message.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents (each call writes every scratch word before reading it).  Calls whose
+ *     work overlaps on the GPU race on it: issue them on one stream, or order them.
+ * Outputs and errors are those of mf_compress. */
+#define MF_STATIC_WORKSPACE_BYTES (8u << 20)
+mf_status mf_compress_static(const mf_compress_desc* desc, void* stream);
+
 /* ------------------------------------------------------------------------------
  * Fused retrieval for receiver layers l = l_r_begin .. l_r_end-1.
  *
