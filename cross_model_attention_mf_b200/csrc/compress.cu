@@ -12,9 +12,12 @@
 //                   with 16-byte loads, float32 partials of 8 (bf16) or 4 (f32)
 //                   elements combined in float64, fixed order (deterministic)
 //   k_select        per query block: sort candidates (mass desc, kb asc), walk
-//                   the running float64 sum until it reaches tau * total
-//   k_scan_compact  row_ptr by exclusive scan, then col_idx in ascending order
-//   k_gather        copy each kept block with the causal/length mask applied
+//                   the running float64 sum until it reaches tau * total, write the
+//                   row's kept indices in ascending order to a per-row list
+//   k_scan_compact  row_ptr by exclusive scan of the counts, then copy the per-row
+//                   lists into col_idx
+//   k_gather        copy each kept block with the causal/length mask applied, one
+//                   (block, sender head) unit per CTA iteration
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -45,7 +48,8 @@ __device__ inline int tri_row(int64_t c) {
 }
 
 __global__ void k_meta(const int32_t* cu, const int64_t* off, int nseq, int max_seqlen, int B,
-                       int elem_bytes, int64_t* meta, uint32_t* status) {
+                       int elem_bytes, int64_t* meta, uint32_t* status, int32_t* row_ptr,
+                       int32_t* nnz_out) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   int64_t rows = 0, cb = 0;
   uint32_t st = 0;
@@ -59,7 +63,11 @@ __global__ void k_meta(const int32_t* cu, const int64_t* off, int nseq, int max_
     rows += nqb;
     cb += nqb * (nqb + 1) / 2;
   }
-  meta[0] = rows; meta[1] = cb; meta[2] = 0; meta[3] = 0;
+  meta[0] = rows; meta[1] = cb; meta[2] = 0; meta[3] = 0;  // meta[2]: rows selected so far
+  if (rows == 0) {  // no query block at all: an empty BSR
+    row_ptr[0] = 0;
+    *nnz_out = 0;
+  }
   if (st) atomicOr(status, st);
 }
 
@@ -170,7 +178,7 @@ template <int NT>
 __global__ void __launch_bounds__(NT) k_select(const int64_t* __restrict__ meta, int nseq,
                                                const double* __restrict__ mass, double tau,
                                                int32_t* __restrict__ counts,
-                                               uint8_t* __restrict__ flags) {
+                                               int32_t* __restrict__ kept_local) {
   extern __shared__ uint64_t sm[];
   __shared__ int s_nkeep;
   const int64_t row = blockIdx.x;
@@ -225,41 +233,79 @@ __global__ void __launch_bounds__(NT) k_select(const int64_t* __restrict__ meta,
     }
     s_nkeep = nk;
     counts[row] = nk;
-    flags[tri + qb] = 1;
   }
   __syncthreads();
+  // kept flags by key-block index (reusing the key array), then an ordered compaction:
+  // the row's kept indices in ascending order at kept_local[tri ...]
   const int nk = s_nkeep;
-  for (int t = threadIdx.x; t < n; t += NT) flags[tri + idx[t]] = (uint8_t)(t < nk - 1);
+  uint8_t* kept = reinterpret_cast<uint8_t*>(key);
+  for (int t = threadIdx.x; t <= n; t += NT) kept[t] = 0;
+  __syncthreads();
+  for (int t = threadIdx.x; t < nk - 1; t += NT) kept[idx[t]] = 1;
+  if (threadIdx.x == 0) kept[qb] = 1;
+  __syncthreads();
+  __shared__ int s_warp[NT / 32];
+  __shared__ int s_base;
+  if (threadIdx.x == 0) s_base = 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int k0 = 0; k0 <= n; k0 += NT) {
+    const int kb = k0 + threadIdx.x;
+    const bool f = kb <= n && kept[kb];
+    const uint32_t bal = __ballot_sync(0xffffffffu, f);
+    __syncthreads();
+    if (lane == 0) s_warp[warp] = __popc(bal);
+    __syncthreads();
+    int before = s_base;
+    for (int w = 0; w < warp; ++w) before += s_warp[w];
+    if (f) kept_local[tri + before + __popc(bal & ((1u << lane) - 1u))] = kb;
+    __syncthreads();
+    if (threadIdx.x == 0)
+      for (int w = 0; w < NT / 32; ++w) s_base += s_warp[w];
+  }
 }
 
-// One CTA: exclusive scan of counts into row_ptr, then ascending col_idx per row.
-constexpr int SCAN_NT = 1024;
+// One CTA: exclusive scan of the counts into row_ptr (independent loads, so their
+// latencies overlap), then each row's list is copied into col_idx (warp per row).
+constexpr int SCAN_NT = 1024, SCAN_PER = 8;
 __global__ void __launch_bounds__(SCAN_NT) k_scan_compact(
     const int64_t* __restrict__ meta, int nseq, const int32_t* __restrict__ counts,
-    const uint8_t* __restrict__ flags, int32_t* __restrict__ row_ptr,
+    const int32_t* __restrict__ kept_local, int32_t* __restrict__ row_ptr,
     int32_t* __restrict__ col_idx, int32_t* __restrict__ kept_row, int32_t* __restrict__ nnz_out,
     int64_t capacity, uint32_t* status) {
   __shared__ int64_t part[SCAN_NT];
+  __shared__ int64_t carry;
   const int64_t R = meta[0];
   const int t = threadIdx.x;
-  const int64_t chunk = (R + SCAN_NT - 1) / SCAN_NT;
-  const int64_t r0 = t * chunk, r1 = min(R, r0 + chunk);
-  int64_t sum = 0;
-  for (int64_t r = r0; r < r1; ++r) sum += counts[r];
-  part[t] = sum;
+  if (t == 0) carry = 0;
   __syncthreads();
-  for (int o = 1; o < SCAN_NT; o <<= 1) {  // inclusive Hillis-Steele scan
-    const int64_t v = t >= o ? part[t - o] : 0;
+  for (int64_t base = 0; base < R; base += (int64_t)SCAN_NT * SCAN_PER) {
+    const int64_t r0 = base + (int64_t)t * SCAN_PER;
+    int32_t c[SCAN_PER];
+#pragma unroll
+    for (int k = 0; k < SCAN_PER; ++k) c[k] = r0 + k < R ? counts[r0 + k] : 0;
+    int64_t sum = 0;
+#pragma unroll
+    for (int k = 0; k < SCAN_PER; ++k) sum += c[k];
+    part[t] = sum;
     __syncthreads();
-    part[t] += v;
+    for (int o = 1; o < SCAN_NT; o <<= 1) {  // inclusive Hillis-Steele scan
+      const int64_t v = t >= o ? part[t - o] : 0;
+      __syncthreads();
+      part[t] += v;
+      __syncthreads();
+    }
+    int64_t run = carry + part[t] - sum;
+#pragma unroll
+    for (int k = 0; k < SCAN_PER; ++k)
+      if (r0 + k < R) {
+        row_ptr[r0 + k] = (int32_t)run;
+        run += c[k];
+      }
+    __syncthreads();
+    if (t == SCAN_NT - 1) carry += part[SCAN_NT - 1];
     __syncthreads();
   }
-  int64_t run = part[t] - sum;
-  for (int64_t r = r0; r < r1; ++r) {
-    row_ptr[r] = (int32_t)run;
-    run += counts[r];
-  }
-  const int64_t nnz = part[SCAN_NT - 1];
+  const int64_t nnz = carry;
   if (t == 0) {
     row_ptr[R] = (int32_t)nnz;
     *nnz_out = (int32_t)nnz;
@@ -271,19 +317,14 @@ __global__ void __launch_bounds__(SCAN_NT) k_scan_compact(
     const int s = find_seq(meta, nseq, row, 2);
     const int64_t* m = meta + META_HDR + 4 * s;
     const int qb = (int)(row - m[2]);
-    const uint8_t* f = flags + m[3] + (int64_t)qb * (qb + 1) / 2;
-    int64_t base = row_ptr[row];
-    for (int k0 = 0; k0 <= qb; k0 += 32) {
-      const int kb = k0 + lane;
-      const bool fl = kb <= qb && f[kb];
-      const uint32_t bal = __ballot_sync(0xffffffffu, fl);
-      const int64_t n = base + __popc(bal & ((1u << lane) - 1u));
-      if (fl && n < capacity) {
-        col_idx[n] = kb;
-        kept_row[n] = (int32_t)row;
+    const int32_t* kl = kept_local + m[3] + (int64_t)qb * (qb + 1) / 2;
+    const int64_t n0 = row_ptr[row];
+    const int cnt = counts[row];
+    for (int k = lane; k < cnt; k += 32)
+      if (n0 + k < capacity) {
+        col_idx[n0 + k] = kl[k];
+        kept_row[n0 + k] = (int32_t)row;
       }
-      base += __popc(bal);
-    }
   }
 }
 
@@ -296,51 +337,48 @@ __global__ void __launch_bounds__(NT) k_gather(const T* __restrict__ maps,
                                                const int32_t* __restrict__ col_idx,
                                                const int32_t* __restrict__ kept_row,
                                                T* __restrict__ values) {
-  constexpr int EPV = Vec<T>::EPV, VPR = B / EPV, VPB = B * VPR;
-  constexpr int U = 4;
+  constexpr int EPV = Vec<T>::EPV, VPR = B / EPV, VPB = B * VPR;  // vectors per row / per head
+  constexpr int U = (VPB + NT - 1) / NT;
   const int64_t nnz = min((int64_t)*nnz_in, capacity);
-  const int64_t nv = (int64_t)h_s * VPB;
-  for (int64_t n = blockIdx.x; n < nnz; n += gridDim.x) {
+  const int64_t units = nnz * h_s;
+  for (int64_t u0 = blockIdx.x; u0 < units; u0 += gridDim.x) {
+    const int64_t n = u0 / h_s;
+    const int hs = (int)(u0 - n * h_s);
     const int64_t row = kept_row[n];
     const int kb = col_idx[n];
     const int s = find_seq(meta, nseq, row, 2);
     const int64_t* m = meta + META_HDR + 4 * s;
     const int64_t L = m[0], Lp = m[1] * B;
     const int qb = (int)(row - m[2]);
-    const T* base = maps + seq_off[s];
-    uint4* dst = reinterpret_cast<uint4*>(values + n * (int64_t)h_s * B * B);
+    const T* src = maps + seq_off[s] + ((int64_t)hs * Lp + (int64_t)qb * B) * Lp + (int64_t)kb * B;
+    uint4* dst = reinterpret_cast<uint4*>(values + (n * h_s + hs) * (int64_t)B * B);
     const bool full = kb < qb && (int64_t)(qb + 1) * B <= L;
-    for (int64_t v0 = threadIdx.x; v0 < nv; v0 += (int64_t)NT * U) {
-      uint4 r[U];
+    uint4 r[U];
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t v = v0 + (int64_t)u * NT;
-        if (v < nv) {
-          const int64_t hs = v / VPB;
-          const int rem = (int)(v - hs * VPB);
-          const int ii = rem / VPR, jv = rem % VPR;
-          const T* p = base + ((hs * Lp) + (int64_t)qb * B + ii) * Lp + (int64_t)kb * B + jv * EPV;
-          r[u] = __ldg(reinterpret_cast<const uint4*>(p));
-          if (!full) {
-            const int64_t i = (int64_t)qb * B + ii;
-            uint32_t w[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
+    for (int k = 0; k < U; ++k) {
+      const int v = threadIdx.x + k * NT;
+      if (v < VPB) {
+        const int ii = v / VPR, jv = v % VPR;
+        r[k] = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)ii * Lp + jv * EPV));
+        if (!full) {
+          const int64_t i = (int64_t)qb * B + ii;
+          uint32_t w[4] = {r[k].x, r[k].y, r[k].z, r[k].w};
 #pragma unroll
-            for (int e = 0; e < EPV; ++e) {
-              const int64_t j = (int64_t)kb * B + jv * EPV + e;
-              if (!(i < L && j <= i)) {
-                if (EPV == 4) w[e] = 0u;
-                else w[e >> 1] &= (e & 1) ? 0x0000ffffu : 0xffff0000u;
-              }
+          for (int e = 0; e < EPV; ++e) {
+            const int64_t j = (int64_t)kb * B + jv * EPV + e;
+            if (!(i < L && j <= i)) {
+              if (EPV == 4) w[e] = 0u;
+              else w[e >> 1] &= (e & 1) ? 0x0000ffffu : 0xffff0000u;
             }
-            r[u] = make_uint4(w[0], w[1], w[2], w[3]);
           }
+          r[k] = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
+    }
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t v = v0 + (int64_t)u * NT;
-        if (v < nv) __stcs(dst + v, r[u]);
-      }
+    for (int k = 0; k < U; ++k) {
+      const int v = threadIdx.x + k * NT;
+      if (v < VPB) __stcs(dst + v, r[k]);
     }
   }
 }
@@ -364,11 +402,12 @@ cudaError_t launch_typed(const mf_compress_desc& d, const CompressWs& ws, uint32
     if (e != cudaSuccess) return e;
   }
   k_select<128><<<(unsigned)ws.max_rows, 128, smem_sel, st>>>(ws.meta, d.nseq, mass, d.tau,
-                                                              ws.counts, ws.flags);
-  k_scan_compact<<<1, SCAN_NT, 0, st>>>(ws.meta, d.nseq, ws.counts, ws.flags, d.row_ptr,
+                                                              ws.counts, ws.kept_local);
+  k_scan_compact<<<1, SCAN_NT, 0, st>>>(ws.meta, d.nseq, ws.counts, ws.kept_local, d.row_ptr,
                                         d.col_idx, ws.kept_row, d.nnz_out, d.capacity_blocks,
                                         status);
-  const int grid_g = (int)std::max<int64_t>(1, std::min<int64_t>(d.capacity_blocks, (int64_t)sms * 8));
+  const int grid_g = (int)std::max<int64_t>(
+      1, std::min<int64_t>(std::max<int64_t>(d.capacity_blocks, 1) * d.h_s, (int64_t)sms * 8));
   k_gather<T, B, NT><<<grid_g, NT, 0, st>>>(maps, d.map_seq_offset, ws.meta, d.nseq, d.h_s,
                                             d.nnz_out, d.capacity_blocks, d.col_idx, ws.kept_row,
                                             static_cast<T*>(d.values));
@@ -386,14 +425,14 @@ size_t compress_ws_layout(const mf_compress_desc& d, CompressWs* ws, void* base)
   size_t off = 0;
   const size_t o_meta = off; off = align_up(off + sizeof(int64_t) * (META_HDR + 4 * (size_t)d.nseq), 256);
   const size_t o_mass = off; off = align_up(off + sizeof(double) * (size_t)max_cb, 256);
-  const size_t o_flags = off; off = align_up(off + (size_t)max_cb, 256);
+  const size_t o_kept_local = off; off = align_up(off + sizeof(int32_t) * (size_t)max_cb, 256);
   const size_t o_counts = off; off = align_up(off + sizeof(int32_t) * (size_t)max_rows, 256);
   const size_t o_kept = off; off = align_up(off + sizeof(int32_t) * (size_t)std::max<int64_t>(d.capacity_blocks, 1), 256);
   if (ws) {
     char* b = static_cast<char*>(base);
     ws->meta = reinterpret_cast<int64_t*>(b + o_meta);
     ws->mass = reinterpret_cast<double*>(b + o_mass);
-    ws->flags = reinterpret_cast<uint8_t*>(b + o_flags);
+    ws->kept_local = reinterpret_cast<int32_t*>(b + o_kept_local);
     ws->counts = reinterpret_cast<int32_t*>(b + o_counts);
     ws->kept_row = reinterpret_cast<int32_t*>(b + o_kept);
     ws->max_cb = max_cb;
@@ -409,7 +448,7 @@ cudaError_t launch_compress(const mf_compress_desc& d, const CompressWs& ws, uin
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int elem = d.dtype == MF_F32 ? 4 : 2;
   k_meta<<<1, 32, 0, st>>>(d.cu_seqlens, d.map_seq_offset, d.nseq, d.max_seqlen, d.B, elem,
-                           ws.meta, status);
+                           ws.meta, status, d.row_ptr, d.nnz_out);
   if (d.dtype == MF_F32) {
     if (d.B == 32) return launch_typed<float, 32>(d, ws, status, st, sms);
     if (d.B == 64) return launch_typed<float, 64>(d, ws, status, st, sms);

@@ -24,7 +24,7 @@ struct CompressWs {
   int64_t* meta;      // [4 + 4 * nseq]: total rows, total causal blocks, -, -, then per
                       // sequence (L, nqb, row_base, cb_base)
   double* mass;       // [max_cb] head-summed block masses
-  uint8_t* flags;     // [max_cb] kept flags
+  int32_t* kept_local;  // [max_cb] each row's kept key blocks, ascending, at its causal base
   int32_t* counts;    // [max_rows] kept blocks per row
   int32_t* kept_row;  // [capacity] BSR row of each kept block
   int64_t max_cb, max_rows;
