@@ -37,6 +37,23 @@ def peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def measured_traffic(entry, workload):
+    """DRAM bytes per launch from the last ncu capture of this entry point's kernels
+    (profiles/traffic.txt), or None when the kernel source changed since the capture."""
+    import hashlib
+    src = {"mf_compress": "compress.cu", "mf_map_retrieve": "retrieve_tc.cu"}[entry]
+    path = os.path.join(ROOT, "cross_model_attention_mf_b200", "csrc", src)
+    sha = hashlib.sha1(open(path, "rb").read()).hexdigest()[:12]
+    tpath = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(tpath):
+        return None
+    for line in open(tpath):
+        f = line.split()
+        if len(f) >= 4 and not line.startswith("#") and f[0] == entry and f[1] == sha and f[3] == workload:
+            return int(f[2])
+    return None
+
+
 # ------------------------------------------------------------------------ clocks
 REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
@@ -373,7 +390,16 @@ def main():
                          "bound": "hbm" if ret_b / (hbm * 1e9) >= ret_f / (tf_burst * 1e12) else "tensor"},
             "roofline": {"bound": "hbm", "kernel": "mf_compress (block stats + select + gather)",
                          "achieved": comp_gbs, "peak": hbm, "unit": "GB/s",
-                         "frac": comp_gbs / hbm, "traffic": None, "peak_source": src},
+                         "frac": comp_gbs / hbm,
+                         "traffic": measured_traffic("mf_compress", w.name),
+                         "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)"},
+            "roofline_retrieve": {
+                "bound": "hbm", "kernel": "mf_map_retrieve (k_retrieve_tc)",
+                "achieved": ret_gbs, "peak": hbm, "unit": "GB/s",
+                "frac": ret_roof_t / res["t_ret"],
+                "tensor_TFLOP/s": ret_tf, "tensor_peak": tf_burst,
+                "traffic": measured_traffic("mf_map_retrieve", w.name),
+                "peak_source": f"{src} (hbm_gbs; bf16_tflops burst for the tensor side)"},
             "gpu_launches": 6 * args.steps,
             "clocks": res["clocks"],
         }
