@@ -17,9 +17,9 @@
 //   mixing  D1[pos][(part, r)] = sum_s A_s[pos] * W_part[r][s]   tcgen05 M=128 N=32 K=16
 //           pos = (row, key) of 2 rows x 64 keys (one M tile), A tile MN-major SW128
 //           from TMA; B = W^T with W split into bf16 hi and lo parts stacked along N,
-//           so one MMA per M tile and s-chunk keeps ~16 bits of W.  D1 is a ring of
-//           eight 32-column M-tile slots in TMEM.
-//   convert 8 warps read D1 (lane = position), form P = hi part + lo part (float32),
+//           so one MMA per M tile and s-chunk keeps ~16 bits of W.  D1 holds the eight
+//           32-column M tiles of one key tile in TMEM.
+//   convert 16 warps read D1 (lane = position), form P = hi part + lo part (float32),
 //           apply the causal mask and split P into bf16 hi + lo (P = hi + lo to ~16
 //           bits), written as P^T[key][(row, head)] (MN-major SW128) per group.
 //   P.V     D2[dim][(row, head)] += V^T[dim][key] * (P^T_hi + P^T_lo)[key][(row, head)]
@@ -34,8 +34,12 @@
 // no stream waits behind another); 4-19 convert (four sets of four warps, one warp per
 // TMEM lane quarter; set k converts the M tiles m = k, k + 4 for all 16 heads);
 // 20-23 O epilogue (they release D2 as soon as it is read, so the next item's P.V can
-// start while O is stored).  Consumer warps signal barriers once per warp (lane 0
-// after __syncwarp).  TMEM: D2 in columns [0, 256), D1 slots in [256, 512).  Every mbarrier
+// start while O is stored; O goes out through a small shared staging buffer as
+// 16-byte stores).  Barriers are tile-granular: one wait and one signal per role and
+// key tile where the data allows, since a barrier operation costs hundreds of cycles.
+// Converters release D1 as soon as it is in registers, so the next tile's mixing
+// overlaps this tile's P.V.  Consumer warps signal once per warp (lane 0 after
+// __syncwarp).  TMEM: D2 in columns [0, 256), D1 slots in [256, 512).  Every mbarrier
 // wait is bounded by a timer: on expiry the CTA records ST_TIMEOUT, all roles stop,
 // in-flight copies and MMAs are drained (bounded) and TMEM is freed.
 #include <cuda.h>
@@ -51,7 +55,7 @@
 namespace mfi {
 namespace {
 
-constexpr int NT = 768;        // 24 warps
+constexpr int NT = 640;        // 20 warps
 constexpr int CONV_SETS = 4;   // convert warp sets
 constexpr int R = 16;          // query rows per CTA
 constexpr int KT = 64;         // keys per tile
@@ -61,27 +65,31 @@ constexpr int HV = NG * GQP;   // virtual receiver heads per CTA
 constexpr int D = 128;         // head dim
 constexpr int SC = 16;         // sender heads per A chunk (one MMA K step)
 constexpr int MT = R * KT / 128;  // M tiles (of 128 positions) per tile: 8
-constexpr int A_STAGES = 2, V_STAGES = 3, P_SLOTS = 6;
+constexpr int A_STAGES = 2, V_STAGES = 2, VG = 2;  // a V stage holds VG groups
 constexpr uint32_t A_BYTES = R * SC * KT * 2;   // 32 KB
-constexpr uint32_t V_BYTES = KT * D * 2;        // 16 KB
+constexpr uint32_t VGRP_BYTES = KT * D * 2;     // 16 KB: one group's V tile
+constexpr uint32_t V_BYTES = VG * VGRP_BYTES;   // 32 KB per V stage
 constexpr uint32_t PT_BYTES = KT * 64 * 2;      // 8 KB: one group's P^T (hi or lo)
-constexpr uint32_t PSLOT_BYTES = 2 * PT_BYTES;  // hi + lo
+constexpr uint32_t PSLOT_BYTES = 2 * PT_BYTES;  // hi + lo of one group
 constexpr uint32_t OFF_A = 0;
 constexpr uint32_t OFF_V = OFF_A + A_STAGES * A_BYTES;
-constexpr uint32_t OFF_P = OFF_V + V_STAGES * V_BYTES;
-constexpr uint32_t OFF_W = OFF_P + P_SLOTS * PSLOT_BYTES;
+constexpr uint32_t OFF_P = OFF_V + V_STAGES * V_BYTES;  // one key tile: NG group slots
+constexpr uint32_t OFF_W = OFF_P + NG * PSLOT_BYTES;
 constexpr uint32_t W_CHUNK = 1024;              // W^T (32 rows = hi, lo) per s-chunk
 constexpr uint32_t W_BYTES_MAX = 4 * W_CHUNK;   // up to 4 chunks (h_s <= 64)
-constexpr uint32_t OFF_BAR = OFF_W + W_BYTES_MAX;
+constexpr int ITEMS_MAX = 64;                     // work items per CTA decoded up front
+constexpr uint32_t ITEM_BYTES = 64;
+constexpr uint32_t OFF_ITEMS = OFF_W + W_BYTES_MAX;
+constexpr uint32_t OFF_BAR = OFF_ITEMS + ITEMS_MAX * ITEM_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;  // + alignment slack
 constexpr uint64_t TIMEOUT_NS = 2000000000ull;
 
 // barrier slots (8 bytes each)
 enum {
   B_AFULL = 0, B_AEMPTY = B_AFULL + A_STAGES, B_VFULL = B_AEMPTY + A_STAGES,
-  B_VEMPTY = B_VFULL + V_STAGES, B_D1FULL = B_VEMPTY + V_STAGES, B_D1EMPTY = B_D1FULL + MT,
-  B_PFULL = B_D1EMPTY + MT, B_PEMPTY = B_PFULL + P_SLOTS, B_OFULL = B_PEMPTY + P_SLOTS,
-  B_OEMPTY = B_OFULL + 1, B_DRAIN1 = B_OEMPTY + 1, B_DRAIN2 = B_DRAIN1 + 1, B_COUNT = B_DRAIN2 + 1
+  B_VEMPTY = B_VFULL + V_STAGES, B_D1FULL = B_VEMPTY + V_STAGES, B_D1EMPTY = B_D1FULL + 1,
+  B_PFULL = B_D1EMPTY + 1, B_PEMPTY = B_PFULL + 2, B_OFULL = B_PEMPTY + 2,
+  B_OEMPTY = B_OFULL + 1, B_DRAIN1 = B_OEMPTY + 2, B_DRAIN2 = B_DRAIN1 + 1, B_COUNT = B_DRAIN2 + 1
 };
 static_assert(B_COUNT * 8 <= 512, "barrier area");
 
@@ -198,13 +206,16 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
   return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
 }
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
       : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
         "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-        "=r"(v[14]), "=r"(v[15])
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_wait_ld() {
@@ -215,21 +226,20 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Optional timeline trace (compile with -DMF_TRACE): per CTA and role, globaltimer
-// stamps of pipeline events, read back with mf_trace_dump().
+// Optional timeline trace (compile with -DMF_TRACE): per CTA and role, SM-clock stamps of
+// pipeline events kept in shared memory and copied out at the end, read back with
+// mf_trace_dump().  Each role has a single writing thread.
 #ifdef MF_TRACE
-constexpr int TRACE_CTAS = 160, TRACE_N = 2048;
-__device__ uint64_t g_trace[TRACE_CTAS][5][TRACE_N];
-__device__ __forceinline__ void trace(int role, uint32_t code) {
-  if (blockIdx.x >= TRACE_CTAS) return;
-  uint64_t* b = g_trace[blockIdx.x][role];
-  const uint64_t n = b[0];
-  if (n < TRACE_N - 1) {
-    b[1 + n] = ((uint64_t)code << 56) | (globaltimer() & ((1ull << 56) - 1));
-    b[0] = n + 1;
-  }
-}
-#define TRACE(role, code) trace(role, code)
+constexpr int TRACE_CTAS = 160, TRACE_N = 256, TRACE_ROLES = 6;
+__device__ uint64_t g_trace[TRACE_CTAS][TRACE_ROLES][TRACE_N];
+#define TRACE(role, code)                                                            \
+  do {                                                                               \
+    const int n_ = s_tn[role];                                                       \
+    if (n_ < TRACE_N - 1) {                                                          \
+      s_tr[role][1 + n_] = ((uint64_t)(code) << 56) | ((uint64_t)clock64() & ((1ull << 56) - 1)); \
+      s_tn[role] = n_ + 1;                                                           \
+    }                                                                                \
+  } while (0)
 #else
 #define TRACE(role, code)
 #endif
@@ -241,6 +251,7 @@ struct Item {
   int64_t o_row0;  // O row of query position i_begin (cu_seqlens_q[s] + i_begin - q0)
   bool valid, bsr_ok;
 };
+static_assert(sizeof(Item) <= ITEM_BYTES, "item table slot");
 
 // item idx = ((s * nqbq + qbl) * rcs + rc) * hcs + hc; identical in every role
 __device__ __forceinline__ Item decode(const TcParams& p, int idx) {
@@ -279,6 +290,11 @@ __global__ void __launch_bounds__(NT, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
+#ifdef MF_TRACE
+  __shared__ uint64_t s_tr[TRACE_ROLES][TRACE_N];
+  __shared__ volatile int s_tn[TRACE_ROLES];
+  if (threadIdx.x < TRACE_ROLES) s_tn[threadIdx.x] = 0;
+#endif
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -288,16 +304,24 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t sb = smem_u32(smem);
   const uint32_t bar0 = sb + OFF_BAR;
   auto bar = [&](int k) { return bar0 + 8u * (uint32_t)k; };
+  // item k of this CTA (idx = blockIdx.x + k * gridDim.x): the first ITEMS_MAX come from the
+  // table decoded once below, later ones are decoded where they are needed
+  Item* s_items = reinterpret_cast<Item*>(smem + OFF_ITEMS);
+  auto item = [&](int k, int idx) -> Item { return k < ITEMS_MAX ? s_items[k] : decode(p, idx); };
 
   // ---- setup
   if (threadIdx.x == 0) {
     s_abort = 0;
     for (int k = 0; k < A_STAGES; ++k) { mbar_init(bar(B_AFULL + k), 1); mbar_init(bar(B_AEMPTY + k), 1); }
     for (int k = 0; k < V_STAGES; ++k) { mbar_init(bar(B_VFULL + k), 1); mbar_init(bar(B_VEMPTY + k), 1); }
-    for (int k = 0; k < MT; ++k) { mbar_init(bar(B_D1FULL + k), 1); mbar_init(bar(B_D1EMPTY + k), 4); }
-    for (int k = 0; k < P_SLOTS; ++k) { mbar_init(bar(B_PFULL + k), 4 * CONV_SETS); mbar_init(bar(B_PEMPTY + k), 1); }
+    mbar_init(bar(B_D1FULL), 1);
+    mbar_init(bar(B_D1EMPTY), 4 * CONV_SETS);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(bar(B_PFULL + h), 4 * CONV_SETS);
+      mbar_init(bar(B_PEMPTY + h), 1);
+      mbar_init(bar(B_OEMPTY + h), 4 * VG);  // the epilogue warps of the half's groups
+    }
     mbar_init(bar(B_OFULL), 1);
-    mbar_init(bar(B_OEMPTY), 4);
     mbar_init(bar(B_DRAIN1), 1);
     mbar_init(bar(B_DRAIN2), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -327,6 +351,11 @@ __global__ void __launch_bounds__(NT, 1)
       wt[(base + ((rv + 16) >> 3) * 128 + (rv & 7) * 16) >> 1] = *reinterpret_cast<uint16_t*>(&lo);
     }
   }
+  // the item table: one decode per item instead of one per item and role
+  for (int k = threadIdx.x; k < ITEMS_MAX; k += NT) {
+    const int idx = blockIdx.x + k * gridDim.x;
+    if (idx < p.n_items) s_items[k] = decode(p, idx);
+  }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   tc_fence_before();
   __syncthreads();
@@ -336,15 +365,16 @@ __global__ void __launch_bounds__(NT, 1)
 
   if (warp == 0 || warp == 3) {
     // ================================================================ TMA producers
-    // warp 0: map tiles (A chunks) in mixing order; warp 3: V tiles in P.V order
+    // warp 0: map tiles (A chunks) in mixing order; warp 3: V tiles in P.V order (one stage
+    // per half tile = groups 2h, 2h + 1)
     if (lane == 0) {
       const bool is_a = warp == 0;
       int as = 0, vs = 0;
       uint32_t aph = 0, vph = 0;
       int a_issued = 0, v_issued = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
-        const Item it = decode(p, idx);
+      for (int idx = blockIdx.x, ik = 0; idx < p.n_items && ok; idx += gridDim.x, ++ik) {
+        const Item it = item(ik, idx);
         if (!it.valid) continue;
         if (is_a) TRACE(0, 1);
         if (is_a && !it.bsr_ok) atomicOr(p.status, ST_INDEX);
@@ -368,32 +398,34 @@ __global__ void __launch_bounds__(NT, 1)
           const bool kb_ok = kb >= 0 && kb <= it.qb;
           if (!kb_ok) atomicOr(p.status, ST_INDEX);
           const int tok0 = kb * p.B + half * KT;
-          for (int g = 0; g < NG && ok; ++g) {
+          for (int h = 0; h < NG / VG && ok; ++h) {
             if (!(ok = mbar_wait(bar(B_VEMPTY + vs), vph ^ 1, abort_flag, p.status))) break;
             mbar_expect_tx(bar(B_VFULL + vs), V_BYTES);
-            const uint32_t dst = sb + OFF_V + vs * V_BYTES;
-            const int G = hc * NG + g;
-            if (!p.paged) {
-              const int row = kb_ok ? p.cu_k[it.s] + tok0 : p.total_k;  // out of range reads 0
-              tma_load_3d(dst, &tmV, bar(B_VFULL + vs), 0, G, row);
-              tma_load_3d(dst + 8192, &tmV, bar(B_VFULL + vs), 64, G, row);
-            } else {
-              const int ps = p.page_size;
-              for (int q = 0; q < KT / ps; ++q) {
-                const int tok = tok0 + q * ps;
-                const int slot = tok / ps;
-                int page = p.n_pages;  // out of range: the copy reads zeros
-                if (kb_ok && tok < it.k_len && slot < p.max_pages) {
-                  const int pg = p.block_table[(int64_t)it.s * p.max_pages + slot];
-                  if (pg >= 0 && pg < p.n_pages) page = pg;
-                  else atomicOr(p.status, ST_PAGE);
+            for (int gl = 0; gl < VG; ++gl) {
+              const uint32_t dst = sb + OFF_V + vs * V_BYTES + gl * VGRP_BYTES;
+              const int G = hc * NG + h * VG + gl;
+              if (!p.paged) {
+                const int row = kb_ok ? p.cu_k[it.s] + tok0 : p.total_k;  // out of range reads 0
+                tma_load_3d(dst, &tmV, bar(B_VFULL + vs), 0, G, row);
+                tma_load_3d(dst + 8192, &tmV, bar(B_VFULL + vs), 64, G, row);
+              } else {
+                const int ps = p.page_size;
+                for (int q = 0; q < KT / ps; ++q) {
+                  const int tok = tok0 + q * ps;
+                  const int slot = tok / ps;
+                  int page = p.n_pages;  // out of range: the copy reads zeros
+                  if (kb_ok && tok < it.k_len && slot < p.max_pages) {
+                    const int pg = p.block_table[(int64_t)it.s * p.max_pages + slot];
+                    if (pg >= 0 && pg < p.n_pages) page = pg;
+                    else atomicOr(p.status, ST_PAGE);
+                  }
+                  tma_load_4d(dst + q * ps * 128, &tmV, bar(B_VFULL + vs), 0, G, 0, page);
+                  tma_load_4d(dst + 8192 + q * ps * 128, &tmV, bar(B_VFULL + vs), 64, G, 0, page);
                 }
-                tma_load_4d(dst + q * ps * 128, &tmV, bar(B_VFULL + vs), 0, G, 0, page);
-                tma_load_4d(dst + 8192 + q * ps * 128, &tmV, bar(B_VFULL + vs), 64, G, 0, page);
               }
             }
             ++v_issued;
-            TRACE(0, 3);
+            TRACE(5, 3);
             if (++vs == V_STAGES) { vs = 0; vph ^= 1; }
           }
         }
@@ -423,33 +455,30 @@ __global__ void __launch_bounds__(NT, 1)
       int T = 0;  // tiles processed so far
       const uint64_t wdesc0 = smem_desc(sb + OFF_W, 512u, 128u, 0u);
       const uint64_t adesc0 = smem_desc(sb + OFF_A, 2048u, 1024u, 2u);
-      for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
-        const Item it = decode(p, idx);
+      for (int idx = blockIdx.x, ik = 0; idx < p.n_items && ok; idx += gridDim.x, ++ik) {
+        const Item it = item(ik, idx);
         if (!it.valid) continue;
         TRACE(1, 1);
         for (int t = 0; t < it.n_tiles && ok; ++t, ++T) {
-          // chunk-major: each s-chunk is mixed into all eight M-tile slots and released;
-          // the last chunk commits each slot as soon as its final MMA is issued
+          // D1 must have been read out by the previous tile's converters
+          if (!(ok = mbar_wait(bar(B_D1EMPTY), (T & 1) ^ 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          // chunk-major: each s-chunk is mixed into all eight M tiles, then its stage is freed
           for (int c = 0; c < p.nsc && ok; ++c) {
             if (!(ok = mbar_wait(bar(B_AFULL + as), aph, abort_flag, p.status))) break;
             tc_fence_after();
             if (c == 0) TRACE(1, 3);
             const uint64_t ad = adesc0 + (((uint32_t)as * A_BYTES) >> 4);
             const uint64_t wd = wdesc0 + ((c * W_CHUNK) >> 4);
-            for (int m = 0; m < MT && ok; ++m) {
-              if (c == 0) {  // the slot must have been read out by the previous tile's converters
-                if (!(ok = mbar_wait(bar(B_D1EMPTY + m), (T & 1) ^ 1, abort_flag, p.status))) break;
-                tc_fence_after();
-              }
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
               tc_mma(tmem + 256u + 32u * (uint32_t)m, ad + ((m * 4096u) >> 4), wd, IDESC_MIX,
                      c > 0 ? 1u : 0u);
-              if (c == p.nsc - 1) tc_commit(bar(B_D1FULL + m));
-              if (c == 0) TRACE(1, 5);
-            }
             tc_commit(bar(B_AEMPTY + as));
             if (++as == A_STAGES) { as = 0; aph ^= 1; }
           }
           if (!ok) break;
+          tc_commit(bar(B_D1FULL));
           TRACE(1, 4);
         }
       }
@@ -466,37 +495,43 @@ __global__ void __launch_bounds__(NT, 1)
       int T = 0, K = 0;  // tiles and items processed so far
       const uint64_t vdesc0 = smem_desc(sb + OFF_V, 8192u, 1024u, 2u);
       const uint64_t pdesc0 = smem_desc(sb + OFF_P, 8192u, 1024u, 2u);
-      for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
-        const Item it = decode(p, idx);
+      for (int idx = blockIdx.x, ik = 0; idx < p.n_items && ok; idx += gridDim.x, ++ik) {
+        const Item it = item(ik, idx);
         if (!it.valid) continue;
-        // D2 must have been read out by the previous item's epilogue (waited for every
-        // item, also one without tiles, so the phases of the barrier are taken in order)
-        if (K > 0) {
-          if (!(ok = mbar_wait(bar(B_OEMPTY), (K - 1) & 1, abort_flag, p.status))) break;
-          tc_fence_after();
-        }
+        TRACE(4, 6);
         for (int t = 0; t < it.n_tiles && ok; ++t, ++T) {
-          for (int g = 0; g < NG; ++g) {
-            const int q = T * NG + g, ps = q % P_SLOTS;
-            if (!(ok = mbar_wait(bar(B_PFULL + ps), (q / P_SLOTS) & 1, abort_flag, p.status))) break;
+          for (int h = 0; h < NG / VG && ok; ++h) {
+            if (!(ok = mbar_wait(bar(B_PFULL + h), T & 1, abort_flag, p.status))) break;
+            // the previous item's epilogue must have read this half of D2 out
+            if (t == 0 && K > 0)
+              if (!(ok = mbar_wait(bar(B_OEMPTY + h), (K - 1) & 1, abort_flag, p.status))) break;
             if (!(ok = mbar_wait(bar(B_VFULL + vs), vph, abort_flag, p.status))) break;
             tc_fence_after();
             TRACE(4, 5);
-            const uint64_t vd = vdesc0 + ((vs * V_BYTES) >> 4);
-            const uint64_t pd = pdesc0 + ((ps * PSLOT_BYTES) >> 4);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              tc_mma(tmem + 64u * g, vd + ((k * 2048u) >> 4), pd + ((k * 2048u) >> 4), IDESC_PV,
-                     (t > 0 || k > 0) ? 1u : 0u);
-              tc_mma(tmem + 64u * g, vd + ((k * 2048u) >> 4), pd + ((PT_BYTES + k * 2048u) >> 4),
-                     IDESC_PV, 1u);
+            for (int gl = 0; gl < VG; ++gl) {
+              const int g = h * VG + gl;
+              const uint64_t vd = vdesc0 + ((vs * V_BYTES + gl * VGRP_BYTES) >> 4);
+              const uint64_t pd = pdesc0 + ((g * PSLOT_BYTES) >> 4);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                tc_mma(tmem + 64u * g, vd + ((k * 2048u) >> 4), pd + ((k * 2048u) >> 4), IDESC_PV,
+                       (t > 0 || k > 0) ? 1u : 0u);
+                tc_mma(tmem + 64u * g, vd + ((k * 2048u) >> 4), pd + ((PT_BYTES + k * 2048u) >> 4),
+                       IDESC_PV, 1u);
+              }
             }
             tc_commit(bar(B_VEMPTY + vs));
-            tc_commit(bar(B_PEMPTY + ps));
+            tc_commit(bar(B_PEMPTY + h));
             if (++vs == V_STAGES) { vs = 0; vph ^= 1; }
           }
         }
         if (!ok) break;
+        if (it.n_tiles == 0 && K > 0) {  // take the epilogue's phases in order all the same
+          for (int h = 0; h < NG / VG && ok; ++h)
+            ok = mbar_wait(bar(B_OEMPTY + h), (K - 1) & 1, abort_flag, p.status);
+          if (!ok) break;
+        }
         tc_commit(bar(B_OFULL));  // D2 of this item complete (immediate when it has no tile)
         TRACE(4, 7);
         ++K;
@@ -507,34 +542,89 @@ __global__ void __launch_bounds__(NT, 1)
     }
   } else if (warp < 4 + 4 * CONV_SETS) {
     // ================================================================ convert P (hi + lo)
+    // Warp (set, quarter) owns TMEM lanes of its quarter in M tiles set and set + 4, i.e.
+    // key j of rows 2 set + rb and 2 set + 8 + rb, which is exactly one 16-byte chunk of the
+    // P^T row of key j (D2 column n = 8 (2 set + rb) + 4 mi + head): one conflict-free
+    // 16-byte store per group for the hi part and one for the lo part.
     const int quarter = warp & 3;
-    const int set = (warp - 4) >> 2;       // M tiles set, set + CONV_SETS, ...
+    const int set = (warp - 4) >> 2;
     const int lrow = quarter * 32 + lane;  // TMEM lane = position in an M tile
     const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-    const int j = lrow & 63;
-    const uint32_t swz = (uint32_t)j & 7u;
+    const int j = lrow & 63, rb = lrow >> 6;
+    const uint32_t choff =
+        (uint32_t)j * 128u + ((((uint32_t)(2 * set + rb)) ^ ((uint32_t)j & 7u)) << 4);
+    // O epilogue of an item, shared by the 16 warps: warp (set, quarter) reads D2 group g = set
+    // (64 columns) for head dims [32 quarter, 32 quarter + 32), releases it and stores O
+    const int ng = min(NG, p.h_kv - hc * NG);  // real groups of this head chunk
+    const int64_t rs = (int64_t)p.h_r * D;     // O row stride
+    struct Pend { int64_t o_row0; int ilo, ihi; bool have; };
+    auto epilogue = [&](const Pend& q, int K) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_OFULL), K & 1, abort_flag, p.status)))
+        return false;
+      tc_fence_after();
+      if (warp == 4 && lane == 0) TRACE(3, 1);
+      const int g = set;
+      uint32_t o[64];
+      if (q.have) {
+        tmem_ld32(tl + 64u * g, *reinterpret_cast<uint32_t(*)[32]>(o));
+        tmem_ld32(tl + 64u * g + 32u, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) o[c] = 0u;
+      }
+      // D2 of this group is in registers: the next item's P.V may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_OEMPTY + g / VG));
+      if (warp == 4 && lane == 0) TRACE(3, 2);
+      if (g < ng) {
+        __nv_bfloat16* ob = p.O + (q.o_row0 * p.h_r + (int64_t)(hc * NG + g) * p.gq) * D +
+                            quarter * 32 + lane;
+        // column n = 8 c + 4 mi + head holds row 2 (c / 2) + 8 mi + c % 2
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          const uint32_t pr = pack_bf16(__uint_as_float(o[2 * u]), __uint_as_float(o[2 * u + 1]));
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            const int n = 2 * u + b, c8 = n >> 3;
+            const int ii = 2 * (c8 >> 1) + 8 * ((n >> 2) & 1) + (c8 & 1), rv = n & 3;
+            if (rv < p.gq && ii >= q.ilo && ii < q.ihi)
+              *reinterpret_cast<uint16_t*>(ob + ii * rs + rv * D) =
+                  (uint16_t)(b ? pr >> 16 : pr & 0xFFFFu);
+          }
+        }
+      }
+      return true;
+    };
     bool ok = true;
-    int T = 0;
-    for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
-      const Item it = decode(p, idx);
+    int T = 0, K = 0;     // tiles converted, epilogues done
+    bool pend = false;    // an item whose O epilogue is still to run: it runs after the
+    Pend pq{0, 0, 0, false};  // next item's first tile is converted, so P.V never starves
+    for (int idx = blockIdx.x, ik = 0; idx < p.n_items && ok; idx += gridDim.x, ++ik) {
+      const Item it = item(ik, idx);
       if (!it.valid) continue;
       for (int t = 0; t < it.n_tiles && ok; ++t, ++T) {
+        if (t == 1 && pend) {  // the previous item's epilogue, after this item's first tile
+          ok = epilogue(pq, K++);
+          pend = false;
+          if (!ok) break;
+        }
         const int64_t e = it.rp0 + t / tpb;
         const int half = t % tpb;
         const int kb = p.col_idx[e];
         const bool kb_ok = kb >= 0 && kb <= it.qb;
         const int tok0 = kb * p.B + half * KT;
-        const int q0 = T * NG;  // P slots of this tile's four groups: (q0 + g) % P_SLOTS
         // warp-uniform control flow: tcgen05.ld is a warp-collective instruction
-        for (int g = 0; g < NG && ok; ++g)
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PEMPTY + (q0 + g) % P_SLOTS),
-                                                 (((q0 + g) / P_SLOTS) & 1) ^ 1, abort_flag, p.status));
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_D1FULL), T & 1, abort_flag, p.status));
         if (!ok) break;
+        tc_fence_after();
         if (warp == 4 && lane == 0) TRACE(2, 1);
-        for (int m = set; m < MT && ok; m += CONV_SETS) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_D1FULL + m), T & 1, abort_flag, p.status));
-          if (!ok) break;
-          tc_fence_after();
+        // P = hi + lo with hi = P truncated to bf16 and lo = bf16(P - hi), P - hi exact in f32
+        uint32_t hw[NG][4], lw[NG][4];  // per group: the chunk's packed hi and lo words
+#pragma unroll
+        for (int mi = 0; mi < MT / CONV_SETS; ++mi) {
+          const int m = set + mi * CONV_SETS;
           uint32_t v[32];  // columns 0-15: A.W_hi of the 16 heads, 16-31: A.W_lo
           asm volatile(
               "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, "
@@ -548,103 +638,72 @@ __global__ void __launch_bounds__(NT, 1)
                 "=r"(v[31])
               : "r"(tl + 256u + 32u * (uint32_t)m));
           tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_D1EMPTY + m));  // this warp is done with the M-tile slot
-          if (warp == 4 && lane == 0) TRACE(2, 3);
-          const int ii = 2 * m + (lrow >> 6);
+          const int ii = 2 * m + rb;
           const bool keep = kb_ok && tok0 + j <= it.i_begin + ii;
-          const uint32_t off = (uint32_t)j * 128u + ((((uint32_t)ii >> 1) ^ swz) << 4) +
-                               (((uint32_t)ii & 1u) << 3);
 #pragma unroll
           for (int g = 0; g < NG; ++g) {
-            float x[4], r[4];
+            uint32_t xb[4];
+            float lo[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-              const float pv = __uint_as_float(v[4 * g + c]) + __uint_as_float(v[16 + 4 * g + c]);
-              x[c] = keep ? pv : 0.0f;
-              r[c] = x[c] - __bfloat162float(__float2bfloat16_rn(x[c]));
+              const float x =
+                  keep ? __uint_as_float(v[4 * g + c]) + __uint_as_float(v[16 + 4 * g + c]) : 0.0f;
+              xb[c] = __float_as_uint(x) & 0xFFFF0000u;
+              lo[c] = x - __uint_as_float(xb[c]);
             }
-            const uint32_t h0 = pack_bf16(x[0], x[1]), h1 = pack_bf16(x[2], x[3]);
-            const uint32_t l0 = pack_bf16(r[0], r[1]), l1 = pack_bf16(r[2], r[3]);
-            uint8_t* pt = smem + OFF_P + ((q0 + g) % P_SLOTS) * PSLOT_BYTES;
-            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(smem_u32(pt + off)), "r"(h0),
-                         "r"(h1)
-                         : "memory");
-            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(smem_u32(pt + PT_BYTES + off)),
-                         "r"(l0), "r"(l1)
-                         : "memory");
+            hw[g][2 * mi] = __byte_perm(xb[0], xb[1], 0x7632);
+            hw[g][2 * mi + 1] = __byte_perm(xb[2], xb[3], 0x7632);
+            lw[g][2 * mi] = pack_bf16(lo[0], lo[1]);
+            lw[g][2 * mi + 1] = pack_bf16(lo[2], lo[3]);
           }
         }
-        if (!ok) break;
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0)
-          for (int g = 0; g < NG; ++g) mbar_arrive(bar(B_PFULL + (q0 + g) % P_SLOTS));
-        if (warp == 4 && lane == 0) TRACE(2, 2);
-      }
-    }
-  } else {
-    // ================================================================ O epilogue
-    // D2 lane = head dim, column = (group, row, head)
-    const int quarter = warp & 3;
-    const int dcol = quarter * 32 + lane;
-    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-    const int ng = min(NG, p.h_kv - hc * NG);  // real groups of this head chunk
-    bool ok = true;
-    int K = 0;
-    for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
-      const Item it = decode(p, idx);
-      if (!it.valid) continue;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OFULL), K & 1, abort_flag, p.status));
-      if (!ok) break;
-      tc_fence_after();
-      if (warp == 20 && lane == 0) TRACE(3, 1);
-      const bool have = it.n_tiles > 0;
-      // rows [ilo, ihi) of this chunk are inside the query range; O row stride h_r * D
-      const int ilo = it.row_lo - it.i_begin, ihi = it.row_hi - it.i_begin, gq = p.gq;
-      const int64_t rs = (int64_t)p.h_r * D;
-      for (int g = 0; g < ng; ++g) {
-        __nv_bfloat16* ob = p.O + (it.o_row0 * p.h_r + (int64_t)(hc * NG + g) * gq) * D + dcol;
-        for (int kh = 0; kh < 2; ++kh) {  // 32 of the group's 64 columns at a time
-          uint32_t v[2][16];
-          if (have) {
-            tmem_ld16(tl + 64u * g + 32u * kh, v[0]);
-            tmem_ld16(tl + 64u * g + 32u * kh + 16u, v[1]);
-            tmem_wait_ld();
-          } else {
-#pragma unroll
-            for (int k = 0; k < 2; ++k)
-#pragma unroll
-              for (int c = 0; c < 16; ++c) v[k][c] = 0u;
-          }
-          if (g == ng - 1 && kh == 1) {  // D2 fully read: the next item may overwrite it
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_OEMPTY));
-            if (warp == 20 && lane == 0) TRACE(3, 2);
-          }
-#pragma unroll
-          for (int k = 0; k < 2; ++k)
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const int ii = 8 * kh + 4 * k + c / GQP, rv = c % GQP;
-              if (rv < gq && ii >= ilo && ii < ihi)
-                ob[ii * rs + rv * D] = __float2bfloat16_rn(__uint_as_float(v[k][c]));
-            }
-        }
-      }
-      if (ng <= 0) {
+        // D1 is in registers: the next tile's mixing may overwrite it
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_OEMPTY));
+        if (lane == 0) mbar_arrive(bar(B_D1EMPTY));
+        if (warp == 4 && lane == 0) TRACE(2, 3);
+#pragma unroll
+        for (int h = 0; h < NG / VG; ++h) {
+          // this half of the P buffer must have been consumed by the previous tile's P.V
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PEMPTY + h), (T & 1) ^ 1, abort_flag, p.status));
+          if (!ok) break;
+#pragma unroll
+          for (int gl = 0; gl < VG; ++gl) {
+            const int g = h * VG + gl;
+            const uint32_t pt = sb + OFF_P + g * PSLOT_BYTES + choff;
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pt), "r"(hw[g][0]),
+                         "r"(hw[g][1]), "r"(hw[g][2]), "r"(hw[g][3])
+                         : "memory");
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pt + PT_BYTES),
+                         "r"(lw[g][0]), "r"(lw[g][1]), "r"(lw[g][2]), "r"(lw[g][3])
+                         : "memory");
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_PFULL + h));
+        }
+        if (!ok) break;
+        if (warp == 4 && lane == 0) TRACE(2, 2);
       }
-      if (warp == 20 && lane == 0) TRACE(3, 3);
-      ++K;
+      if (!ok) break;
+      if (pend) {
+        ok = epilogue(pq, K++);
+        if (!ok) break;
+      }
+      pq = Pend{it.o_row0, it.row_lo - it.i_begin, it.row_hi - it.i_begin, it.n_tiles > 0};
+      pend = true;
     }
+    if (ok && pend) ok = epilogue(pq, K++);
   }
   tc_fence_before();
   __syncthreads();
+#ifdef MF_TRACE
+  if (blockIdx.x < TRACE_CTAS)
+    for (int e = threadIdx.x; e < TRACE_ROLES * TRACE_N; e += NT) {
+      const int r = e / TRACE_N, k = e % TRACE_N;
+      g_trace[blockIdx.x][r][k] = k == 0 ? (uint64_t)s_tn[r] : s_tr[r][k];
+    }
+#endif
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
@@ -755,7 +814,7 @@ bool launch_retrieve_tc(const mf_retrieve_desc& d, const RetrieveLayer& l, uint3
 extern "C" __attribute__((visibility("default"))) int mf_trace_dump(void* host, size_t bytes) {
   if (bytes < sizeof(mfi::g_trace)) return -1;
   if (cudaMemcpyFromSymbol(host, mfi::g_trace, sizeof(mfi::g_trace)) != cudaSuccess) return -2;
-  static uint64_t zero[mfi::TRACE_CTAS][5][mfi::TRACE_N];
+  static uint64_t zero[mfi::TRACE_CTAS][mfi::TRACE_ROLES][mfi::TRACE_N];
   if (cudaMemcpyToSymbol(mfi::g_trace, zero, sizeof(zero)) != cudaSuccess) return -3;
   return 0;
 }
