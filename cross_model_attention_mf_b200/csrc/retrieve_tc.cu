@@ -32,16 +32,17 @@
 // Warp roles: 0 TMA producer of the map tiles; 1 mixing MMA issuer (+ TMEM owner);
 // 2 P.V MMA issuer; 3 TMA producer of the V tiles (separate producers and issuers, so
 // no stream waits behind another); 4-19 convert (four sets of four warps, one warp per
-// TMEM lane quarter; set k converts the M tiles m = k, k + 4 for all 16 heads);
-// 20-23 O epilogue (they release D2 as soon as it is read, so the next item's P.V can
-// start while O is stored; O goes out through a small shared staging buffer as
-// 16-byte stores).  Barriers are tile-granular: one wait and one signal per role and
-// key tile where the data allows, since a barrier operation costs hundreds of cycles.
-// Converters release D1 as soon as it is in registers, so the next tile's mixing
-// overlaps this tile's P.V.  Consumer warps signal once per warp (lane 0 after
-// __syncwarp).  TMEM: D2 in columns [0, 256), D1 slots in [256, 512).  Every mbarrier
-// wait is bounded by a timer: on expiry the CTA records ST_TIMEOUT, all roles stop,
-// in-flight copies and MMAs are drained (bounded) and TMEM is freed.
+// TMEM lane quarter; set k converts the M tiles m = k, k + 4 for all 16 heads) and, once
+// per item, run the O epilogue (set k reads D2 group k, releases it for the next item's
+// P.V and stores O).  Barriers are tile- or half-tile-granular: a barrier operation costs
+// hundreds of cycles.  Converters release D1 as soon as it is in registers, so the next
+// tile's mixing overlaps the conversion; P^T and the V ring work in half tiles (groups
+// 0-1, 2-3), so P.V of one half overlaps the conversion of the other.  Consumer warps
+// wait with all 32 lanes (the hardware suspends such a warp; a lone polling lane would
+// spin) and signal once per warp (lane 0 after __syncwarp).  TMEM: D2 in columns
+// [0, 256), D1 in [256, 512).  Every mbarrier wait is bounded by a timer: on expiry the
+// CTA records ST_TIMEOUT, all roles stop, in-flight copies and MMAs are drained (bounded)
+// and TMEM is freed.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -65,7 +66,19 @@ constexpr int HV = NG * GQP;   // virtual receiver heads per CTA
 constexpr int D = 128;         // head dim
 constexpr int SC = 16;         // sender heads per A chunk (one MMA K step)
 constexpr int MT = R * KT / 128;  // M tiles (of 128 positions) per tile: 8
-constexpr int A_STAGES = 2, V_STAGES = 2, VG = 2;  // a V stage holds VG groups
+#ifndef MF_TC_A_STAGES
+#define MF_TC_A_STAGES 2
+#endif
+#ifndef MF_TC_P_SLOTS
+#define MF_TC_P_SLOTS 2
+#endif
+#ifndef MF_TC_V_STAGES
+#define MF_TC_V_STAGES 2
+#endif
+constexpr int A_STAGES = MF_TC_A_STAGES, V_STAGES = MF_TC_V_STAGES;
+constexpr int VG = 2;  // a V stage holds the V tiles of VG groups
+// P^T buffer: a ring of half-tile slots (one half = groups 2h, 2h + 1, hi and lo parts)
+constexpr int P_SLOTS = MF_TC_P_SLOTS;
 constexpr uint32_t A_BYTES = R * SC * KT * 2;   // 32 KB
 constexpr uint32_t VGRP_BYTES = KT * D * 2;     // 16 KB: one group's V tile
 constexpr uint32_t V_BYTES = VG * VGRP_BYTES;   // 32 KB per V stage
@@ -73,8 +86,9 @@ constexpr uint32_t PT_BYTES = KT * 64 * 2;      // 8 KB: one group's P^T (hi or 
 constexpr uint32_t PSLOT_BYTES = 2 * PT_BYTES;  // hi + lo of one group
 constexpr uint32_t OFF_A = 0;
 constexpr uint32_t OFF_V = OFF_A + A_STAGES * A_BYTES;
-constexpr uint32_t OFF_P = OFF_V + V_STAGES * V_BYTES;  // one key tile: NG group slots
-constexpr uint32_t OFF_W = OFF_P + NG * PSLOT_BYTES;
+constexpr uint32_t OFF_P = OFF_V + V_STAGES * V_BYTES;
+constexpr uint32_t PHALF_BYTES = VG * PSLOT_BYTES;  // 32 KB
+constexpr uint32_t OFF_W = OFF_P + P_SLOTS * PHALF_BYTES;
 constexpr uint32_t W_CHUNK = 1024;              // W^T (32 rows = hi, lo) per s-chunk
 constexpr uint32_t W_BYTES_MAX = 4 * W_CHUNK;   // up to 4 chunks (h_s <= 64)
 constexpr int ITEMS_MAX = 64;                     // work items per CTA decoded up front
@@ -82,13 +96,14 @@ constexpr uint32_t ITEM_BYTES = 64;
 constexpr uint32_t OFF_ITEMS = OFF_W + W_BYTES_MAX;
 constexpr uint32_t OFF_BAR = OFF_ITEMS + ITEMS_MAX * ITEM_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;  // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "dynamic shared memory of one CTA");
 constexpr uint64_t TIMEOUT_NS = 2000000000ull;
 
 // barrier slots (8 bytes each)
 enum {
   B_AFULL = 0, B_AEMPTY = B_AFULL + A_STAGES, B_VFULL = B_AEMPTY + A_STAGES,
   B_VEMPTY = B_VFULL + V_STAGES, B_D1FULL = B_VEMPTY + V_STAGES, B_D1EMPTY = B_D1FULL + 1,
-  B_PFULL = B_D1EMPTY + 1, B_PEMPTY = B_PFULL + 2, B_OFULL = B_PEMPTY + 2,
+  B_PFULL = B_D1EMPTY + 1, B_PEMPTY = B_PFULL + P_SLOTS, B_OFULL = B_PEMPTY + P_SLOTS,
   B_OEMPTY = B_OFULL + 1, B_DRAIN1 = B_OEMPTY + 2, B_DRAIN2 = B_DRAIN1 + 1, B_COUNT = B_DRAIN2 + 1
 };
 static_assert(B_COUNT * 8 <= 512, "barrier area");
@@ -221,6 +236,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// Register fence: the compiler sees v redefined here, so no use of v moves above this point
+// (above the tcgen05.wait::ld that makes v valid, or above a barrier signal that should go
+// out before the arithmetic on v).
+__device__ __forceinline__ void reg_fence(uint32_t (&v)[32]) {
+  asm volatile(""
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]), "+r"(v[16]), "+r"(v[17]),
+                 "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]), "+r"(v[22]), "+r"(v[23]),
+                 "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]), "+r"(v[29]),
+                 "+r"(v[30]), "+r"(v[31]));
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -247,6 +274,7 @@ __device__ uint64_t g_trace[TRACE_CTAS][TRACE_ROLES][TRACE_N];
 // ------------------------------------------------------------------ kernel
 struct Item {
   int s, qb, q0, i_begin, row_lo, row_hi, k_len, n_tiles;
+  int k0;  // first key row of the sequence (cu_seqlens_k[s])
   int64_t rp0;
   int64_t o_row0;  // O row of query position i_begin (cu_seqlens_q[s] + i_begin - q0)
   bool valid, bsr_ok;
@@ -278,7 +306,7 @@ __device__ __forceinline__ Item decode(const TcParams& p, int idx) {
   it.bsr_ok = rp0 >= 0 && rp1 >= rp0 && rp1 <= p.capacity && rp1 - rp0 <= qb + 1;
   it.n_tiles = it.bsr_ok ? (int)(rp1 - rp0) * (p.B / KT) : 0;
   it.s = s; it.qb = qb; it.q0 = q0; it.i_begin = i_begin; it.row_lo = row_lo;
-  it.row_hi = row_hi; it.k_len = k_len; it.rp0 = rp0;
+  it.row_hi = row_hi; it.k_len = k_len; it.rp0 = rp0; it.k0 = p.cu_k[s];
   it.o_row0 = (int64_t)p.cu_q[s] + (i_begin - q0);
   it.valid = true;
   return it;
@@ -316,11 +344,11 @@ __global__ void __launch_bounds__(NT, 1)
     for (int k = 0; k < V_STAGES; ++k) { mbar_init(bar(B_VFULL + k), 1); mbar_init(bar(B_VEMPTY + k), 1); }
     mbar_init(bar(B_D1FULL), 1);
     mbar_init(bar(B_D1EMPTY), 4 * CONV_SETS);
-    for (int h = 0; h < 2; ++h) {
-      mbar_init(bar(B_PFULL + h), 4 * CONV_SETS);
-      mbar_init(bar(B_PEMPTY + h), 1);
-      mbar_init(bar(B_OEMPTY + h), 4 * VG);  // the epilogue warps of the half's groups
+    for (int k = 0; k < P_SLOTS; ++k) {
+      mbar_init(bar(B_PFULL + k), 4 * CONV_SETS);
+      mbar_init(bar(B_PEMPTY + k), 1);
     }
+    for (int h = 0; h < NG / VG; ++h) mbar_init(bar(B_OEMPTY + h), 4 * VG);  // epilogue warps
     mbar_init(bar(B_OFULL), 1);
     mbar_init(bar(B_DRAIN1), 1);
     mbar_init(bar(B_DRAIN2), 1);
@@ -385,6 +413,7 @@ __global__ void __launch_bounds__(NT, 1)
           if (is_a) {
             for (int c = 0; c < p.nsc && ok; ++c) {
               if (!(ok = mbar_wait(bar(B_AEMPTY + as), aph ^ 1, abort_flag, p.status))) break;
+              TRACE(0, 3);
               mbar_expect_tx(bar(B_AFULL + as), A_BYTES);
               tma_load_4d(sb + OFF_A + as * A_BYTES, &tmA, bar(B_AFULL + as), half * KT, c * SC,
                           rc * R, (int)e);
@@ -400,12 +429,13 @@ __global__ void __launch_bounds__(NT, 1)
           const int tok0 = kb * p.B + half * KT;
           for (int h = 0; h < NG / VG && ok; ++h) {
             if (!(ok = mbar_wait(bar(B_VEMPTY + vs), vph ^ 1, abort_flag, p.status))) break;
+            TRACE(5, 4);
             mbar_expect_tx(bar(B_VFULL + vs), V_BYTES);
             for (int gl = 0; gl < VG; ++gl) {
               const uint32_t dst = sb + OFF_V + vs * V_BYTES + gl * VGRP_BYTES;
               const int G = hc * NG + h * VG + gl;
               if (!p.paged) {
-                const int row = kb_ok ? p.cu_k[it.s] + tok0 : p.total_k;  // out of range reads 0
+                const int row = kb_ok ? it.k0 + tok0 : p.total_k;  // out of range reads 0
                 tma_load_3d(dst, &tmV, bar(B_VFULL + vs), 0, G, row);
                 tma_load_3d(dst + 8192, &tmV, bar(B_VFULL + vs), 64, G, row);
               } else {
@@ -474,6 +504,7 @@ __global__ void __launch_bounds__(NT, 1)
             for (int m = 0; m < MT; ++m)
               tc_mma(tmem + 256u + 32u * (uint32_t)m, ad + ((m * 4096u) >> 4), wd, IDESC_MIX,
                      c > 0 ? 1u : 0u);
+            TRACE(1, 5);
             tc_commit(bar(B_AEMPTY + as));
             if (++as == A_STAGES) { as = 0; aph ^= 1; }
           }
@@ -501,10 +532,14 @@ __global__ void __launch_bounds__(NT, 1)
         TRACE(4, 6);
         for (int t = 0; t < it.n_tiles && ok; ++t, ++T) {
           for (int h = 0; h < NG / VG && ok; ++h) {
-            if (!(ok = mbar_wait(bar(B_PFULL + h), T & 1, abort_flag, p.status))) break;
+            const int hq = T * (NG / VG) + h, ps = hq % P_SLOTS;  // half-tile count, P slot
+            if (!(ok = mbar_wait(bar(B_PFULL + ps), (hq / P_SLOTS) & 1, abort_flag, p.status))) break;
+            TRACE(4, 8);
             // the previous item's epilogue must have read this half of D2 out
-            if (t == 0 && K > 0)
+            if (t == 0 && K > 0) {
               if (!(ok = mbar_wait(bar(B_OEMPTY + h), (K - 1) & 1, abort_flag, p.status))) break;
+              TRACE(4, 9);
+            }
             if (!(ok = mbar_wait(bar(B_VFULL + vs), vph, abort_flag, p.status))) break;
             tc_fence_after();
             TRACE(4, 5);
@@ -512,7 +547,7 @@ __global__ void __launch_bounds__(NT, 1)
             for (int gl = 0; gl < VG; ++gl) {
               const int g = h * VG + gl;
               const uint64_t vd = vdesc0 + ((vs * V_BYTES + gl * VGRP_BYTES) >> 4);
-              const uint64_t pd = pdesc0 + ((g * PSLOT_BYTES) >> 4);
+              const uint64_t pd = pdesc0 + ((ps * PHALF_BYTES + gl * PSLOT_BYTES) >> 4);
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
                 tc_mma(tmem + 64u * g, vd + ((k * 2048u) >> 4), pd + ((k * 2048u) >> 4), IDESC_PV,
@@ -521,8 +556,9 @@ __global__ void __launch_bounds__(NT, 1)
                        IDESC_PV, 1u);
               }
             }
+            TRACE(4, 10);
             tc_commit(bar(B_VEMPTY + vs));
-            tc_commit(bar(B_PEMPTY + h));
+            tc_commit(bar(B_PEMPTY + ps));
             if (++vs == V_STAGES) { vs = 0; vph ^= 1; }
           }
         }
@@ -557,23 +593,33 @@ __global__ void __launch_bounds__(NT, 1)
     // (64 columns) for head dims [32 quarter, 32 quarter + 32), releases it and stores O
     const int ng = min(NG, p.h_kv - hc * NG);  // real groups of this head chunk
     const int64_t rs = (int64_t)p.h_r * D;     // O row stride
-    struct Pend { int64_t o_row0; int ilo, ihi; bool have; };
-    auto epilogue = [&](const Pend& q, int K) -> bool {
+    // the item (table slot ek, index eidx) is re-read from the item table here
+    auto epilogue = [&](int ek, int eidx, int K) -> bool {
+      const Item q = item(ek, eidx);
+      const bool have = q.n_tiles > 0;
+      const int ilo = q.row_lo - q.i_begin, ihi = q.row_hi - q.i_begin;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_OFULL), K & 1, abort_flag, p.status)))
         return false;
       tc_fence_after();
       if (warp == 4 && lane == 0) TRACE(3, 1);
       const int g = set;
-      uint32_t o[64];
-      if (q.have) {
-        tmem_ld32(tl + 64u * g, *reinterpret_cast<uint32_t(*)[32]>(o));
-        tmem_ld32(tl + 64u * g + 32u, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
-        tmem_wait_ld();
-      } else {
+      uint32_t pr[32];  // the group's 64 columns rounded to bf16, as pairs (2u, 2u + 1)
 #pragma unroll
-        for (int c = 0; c < 64; ++c) o[c] = 0u;
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t o[32];
+        if (have) {
+          tmem_ld32(tl + 64u * g + 32u * hh, o);
+          tmem_wait_ld();
+          reg_fence(o);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          pr[16 * hh + u] = pack_bf16(__uint_as_float(o[2 * u]), __uint_as_float(o[2 * u + 1]));
       }
-      // D2 of this group is in registers: the next item's P.V may overwrite it
+      // D2 of this group is read: the next item's P.V may overwrite it
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_OEMPTY + g / VG));
@@ -584,14 +630,13 @@ __global__ void __launch_bounds__(NT, 1)
         // column n = 8 c + 4 mi + head holds row 2 (c / 2) + 8 mi + c % 2
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
-          const uint32_t pr = pack_bf16(__uint_as_float(o[2 * u]), __uint_as_float(o[2 * u + 1]));
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
             const int n = 2 * u + b, c8 = n >> 3;
             const int ii = 2 * (c8 >> 1) + 8 * ((n >> 2) & 1) + (c8 & 1), rv = n & 3;
-            if (rv < p.gq && ii >= q.ilo && ii < q.ihi)
+            if (rv < p.gq && ii >= ilo && ii < ihi)
               *reinterpret_cast<uint16_t*>(ob + ii * rs + rv * D) =
-                  (uint16_t)(b ? pr >> 16 : pr & 0xFFFFu);
+                  (uint16_t)(b ? pr[u] >> 16 : pr[u] & 0xFFFFu);
           }
         }
       }
@@ -599,15 +644,18 @@ __global__ void __launch_bounds__(NT, 1)
     };
     bool ok = true;
     int T = 0, K = 0;     // tiles converted, epilogues done
-    bool pend = false;    // an item whose O epilogue is still to run: it runs after the
-    Pend pq{0, 0, 0, false};  // next item's first tile is converted, so P.V never starves
+    // an item whose O epilogue is still to run (pk < 0: none): it runs after the next item's
+    // first tile is converted, so P.V never waits for the stores
+    int pk = -1, pidx = 0;
     for (int idx = blockIdx.x, ik = 0; idx < p.n_items && ok; idx += gridDim.x, ++ik) {
       const Item it = item(ik, idx);
       if (!it.valid) continue;
       for (int t = 0; t < it.n_tiles && ok; ++t, ++T) {
-        if (t == 1 && pend) {  // the previous item's epilogue, after this item's first tile
-          ok = epilogue(pq, K++);
-          pend = false;
+        // the previous item's epilogue, after this item's first tile (with a single P slot
+        // before it: that tile's second half cannot be written before P.V, which needs D2)
+        if (t == (P_SLOTS > 1 ? 1 : 0) && pk >= 0) {
+          ok = epilogue(pk, pidx, K++);
+          pk = -1;
           if (!ok) break;
         }
         const int64_t e = it.rp0 + t / tpb;
@@ -620,57 +668,60 @@ __global__ void __launch_bounds__(NT, 1)
         if (!ok) break;
         tc_fence_after();
         if (warp == 4 && lane == 0) TRACE(2, 1);
-        // P = hi + lo with hi = P truncated to bf16 and lo = bf16(P - hi), P - hi exact in f32
-        uint32_t hw[NG][4], lw[NG][4];  // per group: the chunk's packed hi and lo words
+        // both M tiles into registers first, so that D1 is released as early as possible
+        // (columns 0-15: A.W_hi of the 16 heads, 16-31: A.W_lo)
+        uint32_t v[MT / CONV_SETS][32];
 #pragma unroll
-        for (int mi = 0; mi < MT / CONV_SETS; ++mi) {
-          const int m = set + mi * CONV_SETS;
-          uint32_t v[32];  // columns 0-15: A.W_hi of the 16 heads, 16-31: A.W_lo
-          asm volatile(
-              "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, "
-              "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, "
-              "%26, %27, %28, %29, %30, %31}, [%32];"
-              : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-                "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
-                "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
-                "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
-                "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
-                "=r"(v[31])
-              : "r"(tl + 256u + 32u * (uint32_t)m));
-          tmem_wait_ld();
-          const int ii = 2 * m + rb;
-          const bool keep = kb_ok && tok0 + j <= it.i_begin + ii;
-#pragma unroll
-          for (int g = 0; g < NG; ++g) {
-            uint32_t xb[4];
-            float lo[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const float x =
-                  keep ? __uint_as_float(v[4 * g + c]) + __uint_as_float(v[16 + 4 * g + c]) : 0.0f;
-              xb[c] = __float_as_uint(x) & 0xFFFF0000u;
-              lo[c] = x - __uint_as_float(xb[c]);
-            }
-            hw[g][2 * mi] = __byte_perm(xb[0], xb[1], 0x7632);
-            hw[g][2 * mi + 1] = __byte_perm(xb[2], xb[3], 0x7632);
-            lw[g][2 * mi] = pack_bf16(lo[0], lo[1]);
-            lw[g][2 * mi + 1] = pack_bf16(lo[2], lo[3]);
-          }
-        }
+        for (int mi = 0; mi < MT / CONV_SETS; ++mi)
+          tmem_ld32(tl + 256u + 32u * (uint32_t)(set + mi * CONV_SETS), v[mi]);
+        tmem_wait_ld();
+        if (warp == 4 && lane == 0) TRACE(2, 5);
         // D1 is in registers: the next tile's mixing may overwrite it
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_D1EMPTY));
+#pragma unroll
+        for (int mi = 0; mi < MT / CONV_SETS; ++mi) reg_fence(v[mi]);
+        // P = hi + lo with hi = P truncated to bf16 and lo = bf16(P - hi); a tile wholly below
+        // the diagonal of every row needs no causal mask
+        const bool full = kb_ok && tok0 + KT - 1 <= it.i_begin;
+        uint32_t hw[NG][4], lw[NG][4];  // per group: the chunk's packed hi and lo words
+#pragma unroll
+        for (int mi = 0; mi < MT / CONV_SETS; ++mi) {
+          const int ii = 2 * (set + mi * CONV_SETS) + rb;
+          const float mk = kb_ok && tok0 + j <= it.i_begin + ii ? 1.0f : 0.0f;
+#pragma unroll
+          for (int g = 0; g < NG; ++g) {
+#pragma unroll
+            for (int c = 0; c < 4; c += 2) {
+              float x0 = __uint_as_float(v[mi][4 * g + c]) + __uint_as_float(v[mi][16 + 4 * g + c]);
+              float x1 =
+                  __uint_as_float(v[mi][4 * g + c + 1]) + __uint_as_float(v[mi][16 + 4 * g + c + 1]);
+              if (!full) {
+                x0 *= mk;
+                x1 *= mk;
+              }
+              const uint32_t b0 = __float_as_uint(x0) & 0xFFFF0000u;
+              const uint32_t b1 = __float_as_uint(x1) & 0xFFFF0000u;
+              hw[g][2 * mi + c / 2] = __byte_perm(b0, b1, 0x7632);
+              // P - hi is exact in f32; one rounding to bf16 for the pair
+              lw[g][2 * mi + c / 2] = pack_bf16(x0 - __uint_as_float(b0), x1 - __uint_as_float(b1));
+            }
+          }
+        }
         if (warp == 4 && lane == 0) TRACE(2, 3);
 #pragma unroll
         for (int h = 0; h < NG / VG; ++h) {
           // this half of the P buffer must have been consumed by the previous tile's P.V
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PEMPTY + h), (T & 1) ^ 1, abort_flag, p.status));
+          const int hq = T * (NG / VG) + h, ps = hq % P_SLOTS;  // half-tile count, P slot
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PEMPTY + ps), ((hq / P_SLOTS) & 1) ^ 1,
+                                                 abort_flag, p.status));
           if (!ok) break;
+          if (warp == 4 && lane == 0) TRACE(2, 4);
 #pragma unroll
           for (int gl = 0; gl < VG; ++gl) {
             const int g = h * VG + gl;
-            const uint32_t pt = sb + OFF_P + g * PSLOT_BYTES + choff;
+            const uint32_t pt = sb + OFF_P + ps * PHALF_BYTES + gl * PSLOT_BYTES + choff;
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pt), "r"(hw[g][0]),
                          "r"(hw[g][1]), "r"(hw[g][2]), "r"(hw[g][3])
                          : "memory");
@@ -680,20 +731,20 @@ __global__ void __launch_bounds__(NT, 1)
           }
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_PFULL + h));
+          if (lane == 0) mbar_arrive(bar(B_PFULL + ps));
         }
         if (!ok) break;
         if (warp == 4 && lane == 0) TRACE(2, 2);
       }
       if (!ok) break;
-      if (pend) {
-        ok = epilogue(pq, K++);
+      if (pk >= 0) {
+        ok = epilogue(pk, pidx, K++);
         if (!ok) break;
       }
-      pq = Pend{it.o_row0, it.row_lo - it.i_begin, it.row_hi - it.i_begin, it.n_tiles > 0};
-      pend = true;
+      pk = ik;
+      pidx = idx;
     }
-    if (ok && pend) ok = epilogue(pq, K++);
+    if (ok && pk >= 0) ok = epilogue(pk, pidx, K++);
   }
   tc_fence_before();
   __syncthreads();
