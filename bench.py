@@ -311,7 +311,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="ministral_pair")
     ap.add_argument("--reading", type=int, default=1)
-    ap.add_argument("--cpu-rows", type=int, default=24)
+    ap.add_argument("--cpu-rows", type=int, default=128,
+                    help="query blocks of sequence 0 the CPU oracle runs (default: all of them for the Ministral-like pair)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")

@@ -69,26 +69,21 @@ constexpr int MT = R * KT / 128;  // M tiles (of 128 positions) per tile: 8
 #ifndef MF_TC_A_STAGES
 #define MF_TC_A_STAGES 2
 #endif
-#ifndef MF_TC_P_SLOTS
-#define MF_TC_P_SLOTS 2
-#endif
-#ifndef MF_TC_V_STAGES
-#define MF_TC_V_STAGES 2
-#endif
-constexpr int A_STAGES = MF_TC_A_STAGES, V_STAGES = MF_TC_V_STAGES;
-constexpr int VG = 2;  // a V stage holds the V tiles of VG groups
-// P^T buffer: a ring of half-tile slots (one half = groups 2h, 2h + 1, hi and lo parts)
-constexpr int P_SLOTS = MF_TC_P_SLOTS;
+constexpr int A_STAGES = MF_TC_A_STAGES;
+// Half tiles (KV groups 2h, 2h + 1) flow through a ring of HS slots; a slot holds the half's
+// V tiles (loaded by TMA) and its P^T (written by the converters), filled and freed together.
+constexpr int PH = 2;   // groups per half tile
+constexpr int HS = 2;   // half-tile slots: one key tile
 constexpr uint32_t A_BYTES = R * SC * KT * 2;   // 32 KB
 constexpr uint32_t VGRP_BYTES = KT * D * 2;     // 16 KB: one group's V tile
-constexpr uint32_t V_BYTES = VG * VGRP_BYTES;   // 32 KB per V stage
+constexpr uint32_t V_BYTES = PH * VGRP_BYTES;   // 32 KB: V of one half tile
 constexpr uint32_t PT_BYTES = KT * 64 * 2;      // 8 KB: one group's P^T (hi or lo)
 constexpr uint32_t PSLOT_BYTES = 2 * PT_BYTES;  // hi + lo of one group
 constexpr uint32_t OFF_A = 0;
 constexpr uint32_t OFF_V = OFF_A + A_STAGES * A_BYTES;
-constexpr uint32_t OFF_P = OFF_V + V_STAGES * V_BYTES;
-constexpr uint32_t PHALF_BYTES = VG * PSLOT_BYTES;  // 32 KB
-constexpr uint32_t OFF_W = OFF_P + P_SLOTS * PHALF_BYTES;
+constexpr uint32_t OFF_P = OFF_V + HS * V_BYTES;
+constexpr uint32_t PHALF_BYTES = PH * PSLOT_BYTES;  // 32 KB
+constexpr uint32_t OFF_W = OFF_P + HS * PHALF_BYTES;
 constexpr uint32_t W_CHUNK = 1024;              // W^T (32 rows = hi, lo) per s-chunk
 constexpr uint32_t W_BYTES_MAX = 4 * W_CHUNK;   // up to 4 chunks (h_s <= 64)
 constexpr int ITEMS_MAX = 64;                     // work items per CTA decoded up front
@@ -101,9 +96,9 @@ constexpr uint64_t TIMEOUT_NS = 2000000000ull;
 
 // barrier slots (8 bytes each)
 enum {
-  B_AFULL = 0, B_AEMPTY = B_AFULL + A_STAGES, B_VFULL = B_AEMPTY + A_STAGES,
-  B_VEMPTY = B_VFULL + V_STAGES, B_D1FULL = B_VEMPTY + V_STAGES, B_D1EMPTY = B_D1FULL + 1,
-  B_PFULL = B_D1EMPTY + 1, B_PEMPTY = B_PFULL + P_SLOTS, B_OFULL = B_PEMPTY + P_SLOTS,
+  B_AFULL = 0, B_AEMPTY = B_AFULL + A_STAGES, B_HFULL = B_AEMPTY + A_STAGES,
+  B_HEMPTY = B_HFULL + HS, B_D1FULL = B_HEMPTY + HS, B_D1EMPTY = B_D1FULL + 1,
+  B_OFULL = B_D1EMPTY + 1,
   B_OEMPTY = B_OFULL + 1, B_DRAIN1 = B_OEMPTY + 2, B_DRAIN2 = B_DRAIN1 + 1, B_COUNT = B_DRAIN2 + 1
 };
 static_assert(B_COUNT * 8 <= 512, "barrier area");
@@ -274,7 +269,8 @@ __device__ uint64_t g_trace[TRACE_CTAS][TRACE_ROLES][TRACE_N];
 // ------------------------------------------------------------------ kernel
 struct Item {
   int s, qb, q0, i_begin, row_lo, row_hi, k_len, n_tiles;
-  int k0;  // first key row of the sequence (cu_seqlens_k[s])
+  int k0;   // first key row of the sequence (cu_seqlens_k[s])
+  int kb0;  // key block of the row's first kept block (col_idx[rp0]), -1 without tiles
   int64_t rp0;
   int64_t o_row0;  // O row of query position i_begin (cu_seqlens_q[s] + i_begin - q0)
   bool valid, bsr_ok;
@@ -307,6 +303,7 @@ __device__ __forceinline__ Item decode(const TcParams& p, int idx) {
   it.n_tiles = it.bsr_ok ? (int)(rp1 - rp0) * (p.B / KT) : 0;
   it.s = s; it.qb = qb; it.q0 = q0; it.i_begin = i_begin; it.row_lo = row_lo;
   it.row_hi = row_hi; it.k_len = k_len; it.rp0 = rp0; it.k0 = p.cu_k[s];
+  it.kb0 = it.n_tiles > 0 ? p.col_idx[rp0] : -1;
   it.o_row0 = (int64_t)p.cu_q[s] + (i_begin - q0);
   it.valid = true;
   return it;
@@ -341,14 +338,13 @@ __global__ void __launch_bounds__(NT, 1)
   if (threadIdx.x == 0) {
     s_abort = 0;
     for (int k = 0; k < A_STAGES; ++k) { mbar_init(bar(B_AFULL + k), 1); mbar_init(bar(B_AEMPTY + k), 1); }
-    for (int k = 0; k < V_STAGES; ++k) { mbar_init(bar(B_VFULL + k), 1); mbar_init(bar(B_VEMPTY + k), 1); }
+    for (int k = 0; k < HS; ++k) {
+      mbar_init(bar(B_HFULL + k), 1 + 4 * CONV_SETS);  // V producer + converter warps
+      mbar_init(bar(B_HEMPTY + k), 1);
+    }
     mbar_init(bar(B_D1FULL), 1);
     mbar_init(bar(B_D1EMPTY), 4 * CONV_SETS);
-    for (int k = 0; k < P_SLOTS; ++k) {
-      mbar_init(bar(B_PFULL + k), 4 * CONV_SETS);
-      mbar_init(bar(B_PEMPTY + k), 1);
-    }
-    for (int h = 0; h < NG / VG; ++h) mbar_init(bar(B_OEMPTY + h), 4 * VG);  // epilogue warps
+    for (int h = 0; h < NG / PH; ++h) mbar_init(bar(B_OEMPTY + h), 4 * PH);  // epilogue warps
     mbar_init(bar(B_OFULL), 1);
     mbar_init(bar(B_DRAIN1), 1);
     mbar_init(bar(B_DRAIN2), 1);
@@ -407,9 +403,16 @@ __global__ void __launch_bounds__(NT, 1)
         if (is_a) TRACE(0, 1);
         if (is_a && !it.bsr_ok) atomicOr(p.status, ST_INDEX);
         const int rc = (idx / p.hcs) % p.rcs;
+        // key block of the current kept block and, loaded one block ahead, of the next one
+        const int nblk = it.n_tiles / tpb;
+        int kb_cur = it.kb0, kb_nxt = (!is_a && nblk > 1) ? p.col_idx[it.rp0 + 1] : -1;
         for (int t = 0; t < it.n_tiles && ok; ++t) {
           const int64_t e = it.rp0 + t / tpb;
           const int half = t % tpb;
+          if (!is_a && t > 0 && half == 0) {
+            kb_cur = kb_nxt;
+            if (t / tpb + 1 < nblk) kb_nxt = p.col_idx[e + 1];
+          }
           if (is_a) {
             for (int c = 0; c < p.nsc && ok; ++c) {
               if (!(ok = mbar_wait(bar(B_AEMPTY + as), aph ^ 1, abort_flag, p.status))) break;
@@ -423,21 +426,21 @@ __global__ void __launch_bounds__(NT, 1)
             }
             continue;
           }
-          const int kb = p.col_idx[e];
+          const int kb = kb_cur;
           const bool kb_ok = kb >= 0 && kb <= it.qb;
           if (!kb_ok) atomicOr(p.status, ST_INDEX);
           const int tok0 = kb * p.B + half * KT;
-          for (int h = 0; h < NG / VG && ok; ++h) {
-            if (!(ok = mbar_wait(bar(B_VEMPTY + vs), vph ^ 1, abort_flag, p.status))) break;
+          for (int h = 0; h < NG / PH && ok; ++h) {
+            if (!(ok = mbar_wait(bar(B_HEMPTY + vs), vph ^ 1, abort_flag, p.status))) break;
             TRACE(5, 4);
-            mbar_expect_tx(bar(B_VFULL + vs), V_BYTES);
-            for (int gl = 0; gl < VG; ++gl) {
+            mbar_expect_tx(bar(B_HFULL + vs), V_BYTES);
+            for (int gl = 0; gl < PH; ++gl) {
               const uint32_t dst = sb + OFF_V + vs * V_BYTES + gl * VGRP_BYTES;
-              const int G = hc * NG + h * VG + gl;
+              const int G = hc * NG + h * PH + gl;
               if (!p.paged) {
                 const int row = kb_ok ? it.k0 + tok0 : p.total_k;  // out of range reads 0
-                tma_load_3d(dst, &tmV, bar(B_VFULL + vs), 0, G, row);
-                tma_load_3d(dst + 8192, &tmV, bar(B_VFULL + vs), 64, G, row);
+                tma_load_3d(dst, &tmV, bar(B_HFULL + vs), 0, G, row);
+                tma_load_3d(dst + 8192, &tmV, bar(B_HFULL + vs), 64, G, row);
               } else {
                 const int ps = p.page_size;
                 for (int q = 0; q < KT / ps; ++q) {
@@ -449,14 +452,14 @@ __global__ void __launch_bounds__(NT, 1)
                     if (pg >= 0 && pg < p.n_pages) page = pg;
                     else atomicOr(p.status, ST_PAGE);
                   }
-                  tma_load_4d(dst + q * ps * 128, &tmV, bar(B_VFULL + vs), 0, G, 0, page);
-                  tma_load_4d(dst + 8192 + q * ps * 128, &tmV, bar(B_VFULL + vs), 64, G, 0, page);
+                  tma_load_4d(dst + q * ps * 128, &tmV, bar(B_HFULL + vs), 0, G, 0, page);
+                  tma_load_4d(dst + 8192 + q * ps * 128, &tmV, bar(B_HFULL + vs), 64, G, 0, page);
                 }
               }
             }
             ++v_issued;
             TRACE(5, 3);
-            if (++vs == V_STAGES) { vs = 0; vph ^= 1; }
+            if (++vs == HS) { vs = 0; vph ^= 1; }
           }
         }
       }
@@ -468,11 +471,13 @@ __global__ void __launch_bounds__(NT, 1)
           while (!mbar_try(bar(B_AFULL + k), (cnt - 1) & 1) && globaltimer() - t0 < TIMEOUT_NS) {}
         }
       }
-      for (int k = 0; k < V_STAGES; ++k) {
-        const int cnt = v_issued > k ? (v_issued - k - 1) / V_STAGES + 1 : 0;
+      // (a V slot's phase also needs the converters' arrivals: after an abort this wait runs
+      // out its bounded time)
+      for (int k = 0; k < HS; ++k) {
+        const int cnt = v_issued > k ? (v_issued - k - 1) / HS + 1 : 0;
         if (cnt) {
           const uint64_t t0 = globaltimer();
-          while (!mbar_try(bar(B_VFULL + k), (cnt - 1) & 1) && globaltimer() - t0 < TIMEOUT_NS) {}
+          while (!mbar_try(bar(B_HFULL + k), (cnt - 1) & 1) && globaltimer() - t0 < TIMEOUT_NS) {}
         }
       }
     }
@@ -531,40 +536,39 @@ __global__ void __launch_bounds__(NT, 1)
         if (!it.valid) continue;
         TRACE(4, 6);
         for (int t = 0; t < it.n_tiles && ok; ++t, ++T) {
-          for (int h = 0; h < NG / VG && ok; ++h) {
-            const int hq = T * (NG / VG) + h, ps = hq % P_SLOTS;  // half-tile count, P slot
-            if (!(ok = mbar_wait(bar(B_PFULL + ps), (hq / P_SLOTS) & 1, abort_flag, p.status))) break;
+          for (int h = 0; h < NG / PH && ok; ++h) {
+            // the half's V tiles and P^T are in slot vs
+            if (!(ok = mbar_wait(bar(B_HFULL + vs), vph, abort_flag, p.status))) break;
             TRACE(4, 8);
             // the previous item's epilogue must have read this half of D2 out
             if (t == 0 && K > 0) {
               if (!(ok = mbar_wait(bar(B_OEMPTY + h), (K - 1) & 1, abort_flag, p.status))) break;
               TRACE(4, 9);
             }
-            if (!(ok = mbar_wait(bar(B_VFULL + vs), vph, abort_flag, p.status))) break;
             tc_fence_after();
             TRACE(4, 5);
+            // the MMAs of the half's two groups are interleaved, so consecutive MMAs accumulate
+            // into different D2 columns
+            const uint64_t pd = pdesc0 + ((vs * PHALF_BYTES) >> 4);
+            const uint64_t vd = vdesc0 + ((vs * V_BYTES) >> 4);
 #pragma unroll
-            for (int gl = 0; gl < VG; ++gl) {
-              const int g = h * VG + gl;
-              const uint64_t vd = vdesc0 + ((vs * V_BYTES + gl * VGRP_BYTES) >> 4);
-              const uint64_t pd = pdesc0 + ((ps * PHALF_BYTES + gl * PSLOT_BYTES) >> 4);
+            for (int k = 0; k < 4; ++k)
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                tc_mma(tmem + 64u * g, vd + ((k * 2048u) >> 4), pd + ((k * 2048u) >> 4), IDESC_PV,
-                       (t > 0 || k > 0) ? 1u : 0u);
-                tc_mma(tmem + 64u * g, vd + ((k * 2048u) >> 4), pd + ((PT_BYTES + k * 2048u) >> 4),
-                       IDESC_PV, 1u);
-              }
-            }
+              for (int part = 0; part < 2; ++part)
+#pragma unroll
+                for (int gl = 0; gl < PH; ++gl)
+                  tc_mma(tmem + 64u * (uint32_t)(h * PH + gl),
+                         vd + ((gl * VGRP_BYTES + k * 2048u) >> 4),
+                         pd + ((gl * PSLOT_BYTES + part * PT_BYTES + k * 2048u) >> 4), IDESC_PV,
+                         (t > 0 || k > 0 || part > 0) ? 1u : 0u);
             TRACE(4, 10);
-            tc_commit(bar(B_VEMPTY + vs));
-            tc_commit(bar(B_PEMPTY + ps));
-            if (++vs == V_STAGES) { vs = 0; vph ^= 1; }
+            tc_commit(bar(B_HEMPTY + vs));  // V and P^T of the slot consumed
+            if (++vs == HS) { vs = 0; vph ^= 1; }
           }
         }
         if (!ok) break;
         if (it.n_tiles == 0 && K > 0) {  // take the epilogue's phases in order all the same
-          for (int h = 0; h < NG / VG && ok; ++h)
+          for (int h = 0; h < NG / PH && ok; ++h)
             ok = mbar_wait(bar(B_OEMPTY + h), (K - 1) & 1, abort_flag, p.status);
           if (!ok) break;
         }
@@ -622,7 +626,7 @@ __global__ void __launch_bounds__(NT, 1)
       // D2 of this group is read: the next item's P.V may overwrite it
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_OEMPTY + g / VG));
+      if (lane == 0) mbar_arrive(bar(B_OEMPTY + g / PH));
       if (warp == 4 && lane == 0) TRACE(3, 2);
       if (g < ng) {
         __nv_bfloat16* ob = p.O + (q.o_row0 * p.h_r + (int64_t)(hc * NG + g) * p.gq) * D +
@@ -647,20 +651,21 @@ __global__ void __launch_bounds__(NT, 1)
     // an item whose O epilogue is still to run (pk < 0: none): it runs after the next item's
     // first tile is converted, so P.V never waits for the stores
     int pk = -1, pidx = 0;
+    int kb_prev = -1;  // key block of the previous tile (tiles of one kept block share it)
     for (int idx = blockIdx.x, ik = 0; idx < p.n_items && ok; idx += gridDim.x, ++ik) {
       const Item it = item(ik, idx);
       if (!it.valid) continue;
       for (int t = 0; t < it.n_tiles && ok; ++t, ++T) {
-        // the previous item's epilogue, after this item's first tile (with a single P slot
-        // before it: that tile's second half cannot be written before P.V, which needs D2)
-        if (t == (P_SLOTS > 1 ? 1 : 0) && pk >= 0) {
+        // the previous item's epilogue, after this item's first tile
+        if (t == 1 && pk >= 0) {
           ok = epilogue(pk, pidx, K++);
           pk = -1;
           if (!ok) break;
         }
         const int64_t e = it.rp0 + t / tpb;
         const int half = t % tpb;
-        const int kb = p.col_idx[e];
+        const int kb = half == 0 && t == 0 ? it.kb0 : (half == 0 ? p.col_idx[e] : kb_prev);
+        kb_prev = kb;
         const bool kb_ok = kb >= 0 && kb <= it.qb;
         const int tok0 = kb * p.B + half * KT;
         // warp-uniform control flow: tcgen05.ld is a warp-collective instruction
@@ -711,16 +716,16 @@ __global__ void __launch_bounds__(NT, 1)
         }
         if (warp == 4 && lane == 0) TRACE(2, 3);
 #pragma unroll
-        for (int h = 0; h < NG / VG; ++h) {
+        for (int h = 0; h < NG / PH; ++h) {
           // this half of the P buffer must have been consumed by the previous tile's P.V
-          const int hq = T * (NG / VG) + h, ps = hq % P_SLOTS;  // half-tile count, P slot
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PEMPTY + ps), ((hq / P_SLOTS) & 1) ^ 1,
+          const int hq = T * (NG / PH) + h, ps = hq % HS;  // half-tile count, slot
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_HEMPTY + ps), ((hq / HS) & 1) ^ 1,
                                                  abort_flag, p.status));
           if (!ok) break;
           if (warp == 4 && lane == 0) TRACE(2, 4);
 #pragma unroll
-          for (int gl = 0; gl < VG; ++gl) {
-            const int g = h * VG + gl;
+          for (int gl = 0; gl < PH; ++gl) {
+            const int g = h * PH + gl;
             const uint32_t pt = sb + OFF_P + ps * PHALF_BYTES + gl * PSLOT_BYTES + choff;
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pt), "r"(hw[g][0]),
                          "r"(hw[g][1]), "r"(hw[g][2]), "r"(hw[g][3])
@@ -731,7 +736,7 @@ __global__ void __launch_bounds__(NT, 1)
           }
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_PFULL + ps));
+          if (lane == 0) mbar_arrive(bar(B_HFULL + ps));
         }
         if (!ok) break;
         if (warp == 4 && lane == 0) TRACE(2, 2);
