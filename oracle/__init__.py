@@ -27,7 +27,8 @@ BOUNDARY_EPS = 1e-5
 def build(force=False):
     if not force and os.path.exists(_LIB_PATH) and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC):
         return _LIB_PATH
-    subprocess.run(["gcc", "-O2", "-std=c99", "-shared", "-fPIC", "-o", _LIB_PATH, _SRC], check=True)
+    subprocess.run(["gcc", "-O2", "-std=c99", "-shared", "-fPIC", "-o", _LIB_PATH, _SRC, "-lm"],
+                   check=True)
     return _LIB_PATH
 
 
@@ -51,6 +52,10 @@ def _load():
         lib.mfo_gather_block.restype = None
         lib.mfo_retrieve_block.argtypes = [P, I, P, I, I, I, I, P, I, ctypes.POINTER(_VRef), I, I, P]
         lib.mfo_retrieve_block.restype = None
+        lib.mfo_calib_gram.argtypes = [P, P, I, I, I, I, I64, P]
+        lib.mfo_calib_gram.restype = None
+        lib.mfo_calib_solve.argtypes = [P, I, I, D, P, P]
+        lib.mfo_calib_solve.restype = I
         _lib = lib
     return _lib
 
@@ -203,3 +208,32 @@ def retrieve_step(bsr_rows, B, W_l, V, h_kv, step, qblock_base, k_starts=None,
             O.append(retrieve_block(vals, kept, qb, B, W_l, V, h_kv, (lo, hi), ks, bt, page_size))
         outs.append(np.concatenate(O, axis=0))
     return np.concatenate(outs, axis=0)
+
+
+# ----------------------------------------------------------------------------- calibration
+
+def calib_gram(X, Y, L, gram=None):
+    """Gram [F, F] (float64, F = h_s + h_r) of the stacked sender / receiver maps of one
+    sequence over its causal positions (i < L, j <= i), added to `gram` when given.
+    X: [h_s, Lp, Lp], Y: [h_r, Lp, Lp], same dtype (float32 or bfloat16)."""
+    xa, xc = as_raw(X)
+    ya, yc = as_raw(Y)
+    assert xc == yc and xa.shape[1:] == ya.shape[1:]
+    h_s, h_r, Lp = xa.shape[0], ya.shape[0], xa.shape[1]
+    F = h_s + h_r
+    g = np.zeros((F, F), dtype=np.float64) if gram is None else gram
+    assert g.shape == (F, F) and g.dtype == np.float64 and g.flags["C_CONTIGUOUS"]
+    _load().mfo_calib_gram(_ptr(xa), _ptr(ya), xc, h_s, h_r, L, Lp, _ptr(g))
+    return g
+
+
+def calib_solve(gram, h_s, h_r, ridge=0.0):
+    """Least-squares head map from a Gram: W [h_r, h_s] float64 and the residual sum of
+    squares per receiver head; raises ValueError when the sender Gram (+ ridge) is not
+    positive definite."""
+    g = np.ascontiguousarray(gram, dtype=np.float64)
+    W = np.zeros((h_r, h_s), dtype=np.float64)
+    res = np.zeros(h_r, dtype=np.float64)
+    if _load().mfo_calib_solve(_ptr(g), h_s, h_r, float(ridge), _ptr(W), _ptr(res)) != 0:
+        raise ValueError("sender Gram is not positive definite")
+    return W, res

@@ -31,6 +31,7 @@
  *   - kept blocks are stored raw (no renormalisation), col_idx ascending;
  *   - receiver head r reads KV head g(r) = floor(r * h_kv / h_r).
  */
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -204,4 +205,83 @@ void mfo_retrieve_block(const void* vals, int dtype, const int32_t* kb, int n, i
         }
     }
   free(P);
+}
+
+/*
+ * Head-map calibration (offline step of the head mapping).  The pages say the linear-
+ * combination weights that map sender heads onto receiver heads are learned once, offline,
+ * with both models frozen ("头映射:学习一组线性组合权重" and "这些映射关系离线校准一次",
+ * section "MapFlow 的核心思路"), but give no objective.  Reading taken: ordinary least squares
+ * of each receiver head's map on the sender heads' maps over the causal positions of the
+ * calibration sequences, with an optional ridge term:
+ *   w_r = argmin_w  sum_{i < L, j <= i} (Y_r[i, j] - sum_s w[s] X_s[i, j])^2 + ridge * |w|^2.
+ *
+ * mfo_calib_gram accumulates, for one sequence, the Gram matrix of the stacked features
+ * f = (X_0 .. X_{h_s-1}, Y_0 .. Y_{h_r-1}) at every causal position (i < L, j <= i) into
+ * gram[F][F] (F = h_s + h_r, double).  X: [h_s][Lp][Lp], Y: [h_r][Lp][Lp] raw (dtype 0 f32,
+ * 1 bf16); entries with j > i or in the padding are never read.
+ */
+void mfo_calib_gram(const void* X, const void* Y, int dtype, int h_s, int h_r, int L,
+                    int64_t Lp, double* gram) {
+  const int F = h_s + h_r;
+  double* f = (double*)malloc(sizeof(double) * (size_t)F);
+  for (int64_t i = 0; i < L; ++i)
+    for (int64_t j = 0; j <= i; ++j) {
+      for (int s = 0; s < h_s; ++s) f[s] = value_at(X, dtype, ((int64_t)s * Lp + i) * Lp + j);
+      for (int r = 0; r < h_r; ++r) f[h_s + r] = value_at(Y, dtype, ((int64_t)r * Lp + i) * Lp + j);
+      for (int a = 0; a < F; ++a)
+        for (int b = 0; b < F; ++b) gram[a * F + b] += f[a] * f[b];
+    }
+  free(f);
+}
+
+/*
+ * The least-squares solve from an accumulated Gram: G = gram[0:h_s][0:h_s] + ridge * I is
+ * factored as L L^T (Cholesky, the textbook column algorithm); for every receiver head r the
+ * right-hand side is c_r = gram[0:h_s][h_s + r], and w_r solves G w_r = c_r.  residual[r] is
+ * sum (Y_r - w_r . X)^2 = gram[h_s+r][h_s+r] - 2 w_r . c_r + w_r^T G0 w_r with G0 the Gram
+ * without the ridge term.  W: [h_r][h_s] double.  Returns 0, or -1 when G is not positive
+ * definite.
+ */
+int mfo_calib_solve(const double* gram, int h_s, int h_r, double ridge, double* W,
+                    double* residual) {
+  const int F = h_s + h_r;
+  double* Lf = (double*)calloc((size_t)h_s * h_s, sizeof(double));
+  for (int c = 0; c < h_s; ++c) {
+    double d = gram[c * F + c] + ridge;
+    for (int k = 0; k < c; ++k) d -= Lf[c * h_s + k] * Lf[c * h_s + k];
+    if (!(d > 0.0)) { free(Lf); return -1; }
+    Lf[c * h_s + c] = sqrt(d);
+    for (int r = c + 1; r < h_s; ++r) {
+      double v = gram[r * F + c];
+      for (int k = 0; k < c; ++k) v -= Lf[r * h_s + k] * Lf[c * h_s + k];
+      Lf[r * h_s + c] = v / Lf[c * h_s + c];
+    }
+  }
+  double* z = (double*)malloc(sizeof(double) * (size_t)h_s);
+  for (int r = 0; r < h_r; ++r) {
+    /* forward: L z = c_r, backward: L^T w = z */
+    for (int a = 0; a < h_s; ++a) {
+      double v = gram[a * F + h_s + r];
+      for (int k = 0; k < a; ++k) v -= Lf[a * h_s + k] * z[k];
+      z[a] = v / Lf[a * h_s + a];
+    }
+    double* w = W + (int64_t)r * h_s;
+    for (int a = h_s - 1; a >= 0; --a) {
+      double v = z[a];
+      for (int k = a + 1; k < h_s; ++k) v -= Lf[k * h_s + a] * w[k];
+      w[a] = v / Lf[a * h_s + a];
+    }
+    if (residual) {
+      double res = gram[(h_s + r) * F + h_s + r];
+      for (int a = 0; a < h_s; ++a) {
+        res -= 2.0 * w[a] * gram[a * F + h_s + r];
+        for (int b = 0; b < h_s; ++b) res += w[a] * gram[a * F + b] * w[b];
+      }
+      residual[r] = res;
+    }
+  }
+  free(z);
+  free(Lf);
+  return 0;
 }
