@@ -9,6 +9,7 @@ Functions mirror the C entry points:
     mf_map_retrieve(...)    -> O
     mf_get_status()         -> (status, bits)
     mf_compress_workspace_size(...), mf_retrieve_path(...), mf_version()
+    mf_calib_gram(...), mf_calib_solve(...), mf_calib_path(...)   (head-map calibration)
 """
 import ctypes
 import os
@@ -60,6 +61,12 @@ class RetrieveDesc(ctypes.Structure):
                 ("total_q", _I32), ("flags", _I32)]
 
 
+class CalibDesc(ctypes.Structure):
+    _fields_ = [("sender_maps", _P), ("receiver_maps", _P), ("dtype", ctypes.c_int),
+                ("sender_seq_offset", _P), ("receiver_seq_offset", _P), ("seqlens", _P),
+                ("nseq", _I32), ("h_s", _I32), ("h_r", _I32), ("B", _I32), ("gram", _P)]
+
+
 _lib.mf_compress_workspace_size.argtypes = [ctypes.POINTER(CompressDesc), ctypes.POINTER(ctypes.c_size_t)]
 _lib.mf_compress_workspace_size.restype = ctypes.c_int
 _lib.mf_compress.argtypes = [ctypes.POINTER(CompressDesc), _P, ctypes.c_size_t, _P]
@@ -78,8 +85,16 @@ _lib.mf_version.argtypes = []
 _lib.mf_version.restype = ctypes.c_char_p
 _lib.mf_abi_struct_size.argtypes = [ctypes.c_int]
 _lib.mf_abi_struct_size.restype = ctypes.c_size_t
+_lib.mf_calib_workspace_size.argtypes = [ctypes.POINTER(CalibDesc), ctypes.POINTER(ctypes.c_size_t)]
+_lib.mf_calib_workspace_size.restype = ctypes.c_int
+_lib.mf_calib_gram.argtypes = [ctypes.POINTER(CalibDesc), _P, ctypes.c_size_t, _P]
+_lib.mf_calib_gram.restype = ctypes.c_int
+_lib.mf_calib_solve.argtypes = [_P, _I32, _I32, ctypes.c_double, _P, _P, _P]
+_lib.mf_calib_solve.restype = ctypes.c_int
+_lib.mf_calib_path.argtypes = [ctypes.POINTER(CalibDesc)]
+_lib.mf_calib_path.restype = ctypes.c_int
 
-for _k, _s in ((0, CompressDesc), (1, BsrDesc), (2, RetrieveDesc)):
+for _k, _s in ((0, CompressDesc), (1, BsrDesc), (2, RetrieveDesc), (3, CalibDesc)):
     if _lib.mf_abi_struct_size(_k) != ctypes.sizeof(_s):
         raise ImportError(f"libmf.so struct {_s.__name__} size mismatch: rebuild the library")
 
@@ -262,3 +277,61 @@ def check_device_status(stream=None):
     rc, bits = mf_get_status(stream)
     if rc != MF_OK:
         raise MFError(rc, f"{_lib.mf_last_error().decode()} (bits {bits:#x})")
+
+
+# ----------------------------------------------------------------------------- calibration
+
+def _calib_desc(sender_maps, receiver_maps, seq_offsets, lens, h_s, h_r, B, gram):
+    """The host arrays are returned too: they must outlive the call."""
+    n = len(lens)
+    so = (ctypes.c_int64 * n)(*[int(o[0]) for o in seq_offsets])
+    ro = (ctypes.c_int64 * n)(*[int(o[1]) for o in seq_offsets])
+    ln = (ctypes.c_int32 * n)(*[int(L) for L in lens])
+    d = CalibDesc(_ptr(sender_maps), _ptr(receiver_maps), _dt(sender_maps),
+                  ctypes.cast(so, _P), ctypes.cast(ro, _P), ctypes.cast(ln, _P), n, h_s, h_r, B,
+                  _ptr(gram))
+    return d, (so, ro, ln)
+
+
+def mf_calib_gram(sender_maps: torch.Tensor, receiver_maps: torch.Tensor, seq_offsets, lens,
+                  h_s: int, h_r: int, B: int, gram: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Add the Gram of the stacked sender / receiver maps over the causal positions of every
+    sequence to `gram` (float64 [h_s + h_r, h_s + h_r] on the device, created as zeros when
+    None).  seq_offsets[s] = (sender element offset, receiver element offset) of sequence s;
+    both map tensors are flat, [h][Lp][Lp] per sequence as for mf_compress."""
+    if receiver_maps.dtype != sender_maps.dtype:
+        raise ValueError("sender and receiver maps must share a dtype")
+    F = h_s + h_r
+    if gram is None:
+        gram = torch.zeros((F, F), dtype=torch.float64, device=sender_maps.device)
+    d, keep = _calib_desc(sender_maps, receiver_maps, seq_offsets, lens, h_s, h_r, B, gram)
+    nb = ctypes.c_size_t(0)
+    _check(_lib.mf_calib_workspace_size(ctypes.byref(d), ctypes.byref(nb)))
+    if workspace is None or workspace.numel() < nb.value:
+        workspace = torch.empty(max(nb.value, 256), dtype=torch.uint8, device=sender_maps.device)
+    _check(_lib.mf_calib_gram(ctypes.byref(d), _ptr(workspace), workspace.numel(), _stream(stream)))
+    del keep
+    return gram
+
+
+def mf_calib_path(sender_maps, receiver_maps, seq_offsets, lens, h_s, h_r, B) -> int:
+    d, keep = _calib_desc(sender_maps, receiver_maps, seq_offsets, lens, h_s, h_r, B, None)
+    d.gram = 16  # any non-null pointer: only the shape is examined
+    return _lib.mf_calib_path(ctypes.byref(d))
+
+
+def mf_calib_solve(gram: torch.Tensor, h_s: int, h_r: int, ridge: float = 0.0, stream=None):
+    """Least-squares head map from a Gram: (W float32 [h_r, h_s], residual float64 [h_r]) on the
+    device.  A singular sender Gram (ridge 0) is reported by mf_get_status."""
+    W = torch.zeros((h_r, h_s), dtype=torch.float32, device=gram.device)
+    res = torch.zeros(h_r, dtype=torch.float64, device=gram.device)
+    _check(_lib.mf_calib_solve(_ptr(gram), h_s, h_r, float(ridge), _ptr(W), _ptr(res), _stream(stream)))
+    return W, res
+
+
+def choose_sender_layer(residuals_per_candidate: Sequence[torch.Tensor]) -> int:
+    """Layer map for one receiver layer: the candidate sender layer whose fitted head map leaves
+    the smallest total residual (one residual vector per candidate, from mf_calib_solve)."""
+    totals = [float(r.double().sum()) for r in residuals_per_candidate]
+    return min(range(len(totals)), key=lambda k: (totals[k], k))

@@ -112,6 +112,32 @@ mf_status static_ws_ptr(void** out) {
 
 }  // namespace
 
+namespace {
+mf_status check_calib(const mf_calib_desc* d) {
+  if (!d) return fail(MF_ERR_INVALID, "desc is NULL");
+  if (!is_dtype(d->dtype)) return fail(MF_ERR_INVALID, "dtype must be MF_F32 or MF_BF16");
+  if (!d->sender_maps || !d->receiver_maps || !d->sender_seq_offset || !d->receiver_seq_offset ||
+      !d->seqlens || !d->gram)
+    return fail(MF_ERR_INVALID, "a required pointer is NULL");
+  if (d->nseq < 1) return fail(MF_ERR_INVALID, "nseq must be >= 1");
+  if (d->h_s < 1 || d->h_s > 64 || d->h_r < 1 || d->h_r > 64)
+    return fail(MF_ERR_UNSUPPORTED, "h_s and h_r must lie in [1, 64]");
+  if (!(d->B == 32 || d->B == 64 || d->B == 128)) return fail(MF_ERR_INVALID, "B must be 32, 64 or 128");
+  if (mfi::calib_path(*d) == 0 && d->h_s + d->h_r > 64)
+    return fail(MF_ERR_UNSUPPORTED, "h_s + h_r > 64 needs bf16 maps with h_s % 8 == 0");
+  for (int s = 0; s < d->nseq; ++s) {
+    if (d->seqlens[s] < 0 || d->seqlens[s] > 65536) return fail(MF_ERR_INVALID, "a sequence length is out of [0, 65536]");
+    if (d->sender_seq_offset[s] < 0 || d->receiver_seq_offset[s] < 0)
+      return fail(MF_ERR_INVALID, "negative map offset");
+    if (d->sender_seq_offset[s] % 8 || d->receiver_seq_offset[s] % 8)
+      return fail(MF_ERR_INVALID, "map offsets must be multiples of 8 elements (16-byte aligned rows)");
+  }
+  if (reinterpret_cast<uintptr_t>(d->sender_maps) % 16 || reinterpret_cast<uintptr_t>(d->receiver_maps) % 16)
+    return fail(MF_ERR_INVALID, "maps must be 16-byte aligned");
+  return MF_OK;
+}
+}  // namespace
+
 extern "C" {
 #pragma GCC visibility push(default)
 
@@ -124,6 +150,7 @@ size_t mf_abi_struct_size(int which) {
     case 0: return sizeof(mf_compress_desc);
     case 1: return sizeof(mf_bsr);
     case 2: return sizeof(mf_retrieve_desc);
+    case 3: return sizeof(mf_calib_desc);
     default: return 0;
   }
 }
@@ -216,6 +243,47 @@ mf_status mf_map_retrieve(const mf_retrieve_desc* desc, void* stream) {
   return MF_OK;
 }
 
+mf_status mf_calib_workspace_size(const mf_calib_desc* desc, size_t* bytes) {
+  if (!bytes) return fail(MF_ERR_INVALID, "bytes is NULL");
+  mf_status s = check_calib(desc);
+  if (s != MF_OK) return s;
+  *bytes = mfi::calib_ws_bytes(*desc);
+  return MF_OK;
+}
+
+int mf_calib_path(const mf_calib_desc* desc) {
+  if (check_calib(desc) != MF_OK) return -1;
+  return mfi::calib_path(*desc);
+}
+
+mf_status mf_calib_gram(const mf_calib_desc* desc, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  mf_status s = check_calib(desc);
+  if (s != MF_OK) return s;
+  if (!workspace || workspace_bytes < mfi::calib_ws_bytes(*desc))
+    return fail(MF_ERR_INVALID, "workspace missing or smaller than mf_calib_workspace_size");
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(MF_ERR_INVALID, "workspace must be 256-byte aligned");
+  uint32_t* st = status_ptr();
+  if (!st) return fail(MF_ERR_CUDA, "cannot resolve the device status word");
+  std::string err;
+  if (!mfi::launch_calib_gram(*desc, workspace, st, static_cast<cudaStream_t>(stream), &err))
+    return fail(MF_ERR_CUDA, err);
+  return MF_OK;
+}
+
+mf_status mf_calib_solve(const double* gram, int h_s, int h_r, double ridge, float* W,
+                         double* residual, void* stream) {
+  if (!gram || !W) return fail(MF_ERR_INVALID, "gram and W are required");
+  if (h_s < 1 || h_s > 64 || h_r < 1 || h_r > 64) return fail(MF_ERR_UNSUPPORTED, "h_s and h_r must lie in [1, 64]");
+  if (!(ridge >= 0.0)) return fail(MF_ERR_INVALID, "ridge must be >= 0");
+  uint32_t* st = status_ptr();
+  if (!st) return fail(MF_ERR_CUDA, "cannot resolve the device status word");
+  cudaError_t e = mfi::launch_calib_solve(gram, h_s, h_r, ridge, W, residual, st,
+                                          static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(MF_ERR_CUDA, std::string("calib solve launch: ") + cudaGetErrorString(e));
+  return MF_OK;
+}
+
 mf_status mf_get_status(void* stream, uint32_t* bits) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(MF_ERR_CUDA, std::string("stream: ") + cudaGetErrorString(e));
@@ -231,7 +299,8 @@ mf_status mf_get_status(void* stream, uint32_t* bits) {
   if (v & mfi::ST_CAPACITY) return fail(MF_ERR_CAPACITY, "device: kept blocks exceed capacity");
   if (v & mfi::ST_TIMEOUT) return fail(MF_ERR_TIMEOUT, "device: pipeline wait timed out");
   if (v & mfi::ST_ALIGN) return fail(MF_ERR_INVALID, "device: misaligned map offset");
-  return fail(MF_ERR_DEVICE_INDEX, "device: page id out of range");
+  if (v & mfi::ST_PAGE) return fail(MF_ERR_DEVICE_INDEX, "device: page id out of range");
+  return fail(MF_ERR_INVALID, "device: calibration Gram is not positive definite");
 }
 
 }  // extern "C"

@@ -17,6 +17,7 @@ enum : uint32_t {
   ST_TIMEOUT = 4u,   // a pipeline wait gave up
   ST_ALIGN = 8u,     // a sequence's map offset is not 16-byte aligned
   ST_PAGE = 16u,     // a page id out of range
+  ST_SINGULAR = 32u, // a calibration Gram that is not positive definite
 };
 
 // scratch of mf_compress (carved out of the caller's workspace)
@@ -55,5 +56,14 @@ bool tc_supported(const mf_retrieve_desc& d);
 // returns false and fills *err on a host-side failure (tensor-map encoding, launch)
 bool launch_retrieve_tc(const mf_retrieve_desc& d, const RetrieveLayer& l, uint32_t* status,
                         cudaStream_t st, std::string* err);
+
+// head-map calibration
+size_t calib_ws_bytes(const mf_calib_desc& d);
+int calib_path(const mf_calib_desc& d);
+// returns false and fills *err on a host-side failure
+bool launch_calib_gram(const mf_calib_desc& d, void* ws, uint32_t* status, cudaStream_t st,
+                       std::string* err);
+cudaError_t launch_calib_solve(const double* gram, int h_s, int h_r, double ridge, float* W,
+                               double* residual, uint32_t* status, cudaStream_t st);
 
 }  // namespace mfi

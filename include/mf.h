@@ -208,9 +208,60 @@ mf_status mf_map_retrieve(const mf_retrieve_desc* desc, void* stream);
  * Returns -1 for an invalid descriptor. */
 int mf_retrieve_path(const mf_retrieve_desc* desc);
 
+/* ------------------------------------------------------------------------
+ * Head-map calibration (offline).  MapFlow page "MapFlow开源:大模型换班,Prefill为何能快20%?",
+ * section "MapFlow 的核心思路": the weights that map sender heads onto receiver heads are
+ * learned once, offline, with both models frozen ("头映射:学习一组线性组合权重",
+ * "这些映射关系离线校准一次"); the page states no objective.  Reading taken: least squares of
+ * every receiver head's map on the sender heads' maps over the causal positions (i < L,
+ * j <= i) of the calibration sequences, with an optional ridge term.  The layer map is then
+ * chosen by the smallest residual (caller side: one Gram per candidate sender layer).
+ *
+ * mf_calib_gram adds, for each sequence, the Gram matrix of the stacked features
+ * (X_0 .. X_{h_s-1}, Y_0 .. Y_{h_r-1}) over its causal positions into `gram`
+ * (device, double [F][F], F = h_s + h_r, row-major, not cleared by the call).
+ * Maps are dense, as for mf_compress: sequence s has [h][Lp][Lp] elements
+ * (Lp = ceil(L / B) * B) at element offset *_seq_offset[s] (HOST arrays here: the
+ * calibration is offline and its launches are planned on the host).  Entries with
+ * j > i or in the padding are never used.  bf16 maps with h_s % 8 == 0 and
+ * F <= 128 run on tcgen05 tensor cores; other shapes and float32 on a SIMT kernel.
+ * Limits: 1 <= h_s <= 64, 1 <= h_r <= 64, B in {32, 64, 128}, L <= 65536.
+ * The caller owns every buffer; the workspace (mf_calib_workspace_size bytes,
+ * 256-byte aligned) holds per-CTA partial Grams.  Asynchronous on `stream`.
+ */
+typedef struct {
+  const void* sender_maps;              /* device: maps of one sender layer */
+  const void* receiver_maps;            /* device: maps of one receiver layer, same dtype */
+  mf_dtype dtype;
+  const int64_t* sender_seq_offset;     /* HOST [nseq] element offsets into sender_maps */
+  const int64_t* receiver_seq_offset;   /* HOST [nseq] element offsets into receiver_maps */
+  const int32_t* seqlens;               /* HOST [nseq] sequence lengths L */
+  int nseq;
+  int h_s, h_r, B;
+  double* gram;                         /* device [F][F] double, accumulated into */
+} mf_calib_desc;
+
+mf_status mf_calib_workspace_size(const mf_calib_desc* desc, size_t* bytes);
+mf_status mf_calib_gram(const mf_calib_desc* desc, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* Least-squares head map from an accumulated Gram (device, double [F][F]):
+ * W (device, float [h_r][h_s]) solves (G_ss + ridge I) W^T = G_sr by Cholesky in
+ * double; residual (device, double [h_r], may be NULL) receives
+ * sum (Y_r - W_r . X)^2 over the positions of the Gram.  A sender Gram that is not
+ * positive definite (a silent sender head with ridge = 0) sets status bit 32
+ * (MF_ERR_INVALID from mf_get_status) and leaves W and residual at 0.
+ * Asynchronous on `stream`. */
+mf_status mf_calib_solve(const double* gram, int h_s, int h_r, double ridge, float* W,
+                         double* residual, void* stream);
+
+/* Which Gram kernel mf_calib_gram launches: 0 = SIMT, 1 = tcgen05; -1 invalid. */
+int mf_calib_path(const mf_calib_desc* desc);
+
 /* Synchronise `stream`, then read and clear this device's status word.  *bits
  * (optional) receives the raw bits: 1 index out of range, 2 capacity, 4 wait
- * timeout, 8 misaligned input, 16 page id out of range.  Returns MF_OK when no
+ * timeout, 8 misaligned input, 16 page id out of range, 32 singular
+ * calibration Gram.  Returns MF_OK when no
  * bit was set, else the status of the lowest set bit. */
 mf_status mf_get_status(void* stream, uint32_t* bits);
 
@@ -221,7 +272,8 @@ const char* mf_last_error(void);
 const char* mf_version(void);
 
 /* sizeof of this header's structs as the library was compiled, for bindings that
- * mirror them: which = 0 mf_compress_desc, 1 mf_bsr, 2 mf_retrieve_desc.
+ * mirror them: which = 0 mf_compress_desc, 1 mf_bsr, 2 mf_retrieve_desc,
+ * 3 mf_calib_desc.
  * Returns 0 for any other value. */
 size_t mf_abi_struct_size(int which);
 

@@ -128,3 +128,29 @@ def test_retrieve_rejects_unmapped_layer(mf):
     lm = (ctypes.c_int32 * 1)(0)
     d = _retrieve_desc(mf, arr, lm)
     assert mf._lib.mf_map_retrieve(ctypes.byref(d), None) == mf.MF_ERR_INVALID
+
+
+def test_calib_host_validation(mf):
+    d = mf.CalibDesc()
+    assert mf._lib.mf_calib_gram(None, None, 0, None) == mf.MF_ERR_INVALID
+    nb = ctypes.c_size_t(0)
+    assert mf._lib.mf_calib_workspace_size(ctypes.byref(d), ctypes.byref(nb)) == mf.MF_ERR_INVALID
+    so = (ctypes.c_int64 * 1)(0)
+    ro = (ctypes.c_int64 * 1)(3)  # not a multiple of 8 elements
+    ln = (ctypes.c_int32 * 1)(100)
+    d = mf.CalibDesc(4096, 4096, mf.MF_BF16, ctypes.cast(so, ctypes.c_void_p), ctypes.cast(ro, ctypes.c_void_p),
+                     ctypes.cast(ln, ctypes.c_void_p), 1, 32, 32, 64, 4096)
+    assert mf._lib.mf_calib_gram(ctypes.byref(d), None, 0, None) == mf.MF_ERR_INVALID
+    assert b"multiples of 8" in mf._lib.mf_last_error()
+    ro[0] = 0
+    d.h_s = 65
+    assert mf._lib.mf_calib_path(ctypes.byref(d)) == -1
+    d.h_s = 32
+    assert mf._lib.mf_calib_path(ctypes.byref(d)) == 1
+    d.h_s = 12
+    assert mf._lib.mf_calib_path(ctypes.byref(d)) == 0
+    d.h_s, d.h_r, d.dtype = 40, 40, mf.MF_F32  # F = 80 needs the tensor-core path
+    assert mf._lib.mf_calib_gram(ctypes.byref(d), None, 0, None) == mf.MF_ERR_UNSUPPORTED
+    assert mf._lib.mf_calib_solve(None, 4, 4, 0.0, None, None, None) == mf.MF_ERR_INVALID
+    assert mf._lib.mf_calib_solve(4096, 4, 4, -1.0, 4096, None, None) == mf.MF_ERR_INVALID
+    assert mf._lib.mf_calib_solve(4096, 65, 4, 0.0, 4096, None, None) == mf.MF_ERR_UNSUPPORTED
