@@ -222,8 +222,53 @@ def run_ours(args, rank, world, dev):
     if rank == 0 and not args.no_e2e:
         e2e = run_e2e(args, w, mf, pack, W, V, bsr, ws, O, qbase, dev)
 
+    calib = None
+    if rank == 0 and not args.no_calib:
+        calib = run_calib(w, mf, pack, dev, args.calib_len)
+
     return dict(w=w, nnz=nnz, elapsed=elapsed, t_comp=t_comp, t_ret=t_ret, clocks=clk.summary(),
-                e2e=e2e)
+                e2e=e2e, calib=calib)
+
+
+def run_calib(w, mf, pack, dev, calib_len=0, reps=5):
+    """Head-map calibration of the workload's receiver (h_r heads) on the sender layer: the Gram
+    of the stacked maps over the causal positions (tcgen05 kernel), CUDA-event timed; the
+    receiver maps are the recipe's maps of another layer.  Algorithmic bytes: every causal
+    position of every sender and receiver head read once."""
+    from synth import device as sdev
+    if calib_len and calib_len < max(w.lens):  # a shorter calibration sequence (small captures)
+        w = w.with_(lens=(calib_len,))
+        pack = sdev.fill_maps(sdev.alloc_maps(w, dev), w, 0)
+    wr = w.with_(h_s=w.h_r)
+    rmaps = sdev.fill_maps(sdev.alloc_maps(wr, dev), wr, 1)
+    offs = list(zip(pack.offsets, rmaps.offsets))
+    F = w.h_s + w.h_r
+    gram = torch.zeros((F, F), dtype=torch.float64, device=dev)
+    wsb = torch.empty(64 << 20, dtype=torch.uint8, device=dev)
+    path = mf.mf_calib_path(pack.maps, rmaps.maps, offs, w.lens, w.h_s, w.h_r, w.B)
+    mf.mf_calib_gram(pack.maps, rmaps.maps, offs, w.lens, w.h_s, w.h_r, w.B, gram=gram, workspace=wsb)
+    ts = []
+    for _ in range(reps):
+        gram.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mf.mf_calib_gram(pack.maps, rmaps.maps, offs, w.lens, w.h_s, w.h_r, w.B, gram=gram, workspace=wsb)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e-3)
+    Wm, res = mf.mf_calib_solve(gram, w.h_s, w.h_r, 0.0)
+    rc, bits = mf.mf_get_status()
+    if rc != mf.MF_OK:
+        raise RuntimeError(f"calibration status {rc} bits {bits:#x}")
+    pos = sum(L * (L + 1) // 2 for L in w.lens)
+    t = statistics.median(ts)
+    del rmaps
+    torch.cuda.empty_cache()
+    return {"kernel": "mf_calib_gram (" + ("k_calib_gram_tc" if path == 1 else "k_calib_gram_simt") + ")",
+            "workload": f"sender {w.h_s} heads, receiver {w.h_r} heads, lens={list(w.lens)}, B={w.B}",
+            "ms": t * 1e3, "bytes": pos * F * 2, "GB/s": pos * F * 2 / t / 1e9,
+            "TFLOP/s": 2.0 * F * F * pos / t / 1e12, "reps": reps,
+            "fit_rel_residual": float(res.sum() / torch.diagonal(gram)[w.h_s:].sum())}
 
 
 def run_e2e(args, w, mf, pack, W, V, bsr, ws, O, qbase, dev):
@@ -315,6 +360,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-calib", action="store_true", help="skip the head-map calibration line")
+    ap.add_argument("--calib-len", type=int, default=0,
+                    help="calibrate on a sequence of this many tokens (0: the workload's own)")
     ap.add_argument("--capacity", type=int, default=0,
                     help="BSR capacity in blocks (0: every causal block, which never overflows)")
     args = ap.parse_args()
@@ -405,6 +453,11 @@ def main():
         }
         if res["e2e"] is not None:
             line["e2e"] = res["e2e"]
+        if res["calib"] is not None:
+            c = res["calib"]
+            c.update({"bound": "hbm", "peak": hbm, "unit": "GB/s", "frac": c["GB/s"] / hbm,
+                      "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)"})
+            line["calibration"] = c
         if not args.no_cpu and world == 1:
             line["cpu_baseline"] = cpu_baseline(w, dev, args.cpu_rows)
         print(json.dumps(line), flush=True)
