@@ -222,12 +222,16 @@ def run_ours(args, rank, world, dev):
     if rank == 0 and not args.no_e2e:
         e2e = run_e2e(args, w, mf, pack, W, V, bsr, ws, O, qbase, dev)
 
+    multi = None
+    if rank == 0 and not args.no_multi:
+        multi = run_multi(w, mf, bsr, nnz, qbase, dev)
+
     calib = None
     if rank == 0 and not args.no_calib:
         calib = run_calib(w, mf, pack, dev, args.calib_len)
 
     return dict(w=w, nnz=nnz, elapsed=elapsed, t_comp=t_comp, t_ret=t_ret, clocks=clk.summary(),
-                e2e=e2e, calib=calib)
+                e2e=e2e, calib=calib, multi=multi)
 
 
 def run_calib(w, mf, pack, dev, calib_len=0, reps=5):
@@ -269,6 +273,61 @@ def run_calib(w, mf, pack, dev, calib_len=0, reps=5):
             "ms": t * 1e3, "bytes": pos * F * 2, "GB/s": pos * F * 2 / t / 1e9,
             "TFLOP/s": 2.0 * F * F * pos / t / 1e12, "reps": reps,
             "fit_rel_residual": float(res.sum() / torch.diagonal(gram)[w.h_s:].sum())}
+
+
+def run_multi(w, mf, bsr, nnz, qbase, dev, reps=20):
+    """One sender layer's blocks serving three receivers (the workload's receiver and two more,
+    the second with half the heads), once in shared launches (mf_map_retrieve_multi) and once
+    receiver by receiver; CUDA events on the launching stream.  Algorithmic bytes of the shared
+    launch: the kept blocks once, plus every receiver's V, O and W."""
+    from synth import device as sdev
+    specs = [(w.h_r, w.h_kv, w.seed), (w.h_r, w.h_kv, w.seed + 101), (w.h_r // 2, w.h_kv // 2, w.seed + 202)]
+    rs = []
+    for h_r, h_kv, seed in specs:
+        wr = w.with_(h_r=h_r, h_kv=h_kv, seed=seed)
+        rs.append(mf.Receiver([0], sdev.w_weights(wr, dev), sdev.v_contiguous(wr, 0, dev)[None], h_r, h_kv,
+                              O=torch.empty((1, w.tokens, h_r, w.d), dtype=torch.bfloat16, device=dev)))
+    cu = torch.tensor([0] + list(np.cumsum(w.lens)), dtype=torch.int32, device=dev)
+    maxlen = max(w.lens)
+    fused = mf.mf_retrieve_multi_fused([bsr], rs, cu, cu, qbase, maxlen)
+    st = torch.cuda.current_stream()
+
+    def shared():
+        mf.mf_map_retrieve_multi([bsr], rs, cu, cu, qbase, maxlen)
+
+    def separate():
+        for r in rs:
+            mf.mf_map_retrieve([bsr], [0], r.W, r.V, cu, cu, qbase, maxlen, r.h_r, r.h_kv, O=r.O)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            fn()
+            e1.record(st)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e-3)
+        return statistics.median(ts)
+
+    t_sh, t_sep = timed(shared), timed(separate)
+    rc, bits = mf.mf_get_status()
+    if rc != mf.MF_OK:
+        raise RuntimeError(f"multi-receiver status {rc} bits {bits:#x}")
+    blk = w.h_s * w.B * w.B * 2
+    per_r = sum(w.tokens * h_kv * w.d * 2 + w.tokens * h_r * w.d * 2 + 4 * h_r * w.h_s
+                for h_r, h_kv, _ in specs)
+    b_shared = nnz * blk + 4 * nnz + 4 * (sum(w.nqb) + 1) + per_r
+    b_sep = len(specs) * (nnz * blk + 4 * nnz + 4 * (sum(w.nqb) + 1)) + per_r
+    del rs
+    torch.cuda.empty_cache()
+    return {"kernel": "mf_map_retrieve_multi (k_retrieve_tc, " + ("one launch" if fused == 1 else "one launch per receiver") + ")",
+            "workload": "one sender layer, receivers " + ", ".join(f"{a}/{b} heads" for a, b, _ in specs),
+            "ms_shared": t_sh * 1e3, "ms_separate": t_sep * 1e3, "speedup": t_sep / t_sh,
+            "bytes_shared": b_shared, "bytes_separate": b_sep,
+            "GB/s": b_shared / t_sh / 1e9, "reps": reps}
 
 
 def run_e2e(args, w, mf, pack, W, V, bsr, ws, O, qbase, dev):
@@ -360,6 +419,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-multi", action="store_true", help="skip the several-receivers line")
     ap.add_argument("--no-calib", action="store_true", help="skip the head-map calibration line")
     ap.add_argument("--calib-len", type=int, default=0,
                     help="calibrate on a sequence of this many tokens (0: the workload's own)")
@@ -453,6 +513,11 @@ def main():
         }
         if res["e2e"] is not None:
             line["e2e"] = res["e2e"]
+        if res["multi"] is not None:
+            m = res["multi"]
+            m.update({"bound": "hbm", "peak": hbm, "unit": "GB/s", "frac": m["GB/s"] / hbm,
+                      "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)"})
+            line["multi_receiver"] = m
         if res["calib"] is not None:
             c = res["calib"]
             c.update({"bound": "hbm", "peak": hbm, "unit": "GB/s", "frac": c["GB/s"] / hbm,

@@ -7,6 +7,7 @@ this package fails loudly when libmf.so is missing; there is no fallback.
 Functions mirror the C entry points:
     mf_compress(...)        -> BSR (row_ptr, col_idx, values, nnz)
     mf_map_retrieve(...)    -> O
+    mf_map_retrieve_multi(...) -> [O]   (one sender, several receivers)
     mf_get_status()         -> (status, bits)
     mf_compress_workspace_size(...), mf_retrieve_path(...), mf_version()
     mf_calib_gram(...), mf_calib_solve(...), mf_calib_path(...)   (head-map calibration)
@@ -75,6 +76,10 @@ _lib.mf_compress_static.argtypes = [ctypes.POINTER(CompressDesc), _P]
 _lib.mf_compress_static.restype = ctypes.c_int
 _lib.mf_map_retrieve.argtypes = [ctypes.POINTER(RetrieveDesc), _P]
 _lib.mf_map_retrieve.restype = ctypes.c_int
+_lib.mf_map_retrieve_multi.argtypes = [ctypes.POINTER(RetrieveDesc), ctypes.c_int, _P]
+_lib.mf_map_retrieve_multi.restype = ctypes.c_int
+_lib.mf_retrieve_multi_fused.argtypes = [ctypes.POINTER(RetrieveDesc), ctypes.c_int]
+_lib.mf_retrieve_multi_fused.restype = ctypes.c_int
 _lib.mf_retrieve_path.argtypes = [ctypes.POINTER(RetrieveDesc)]
 _lib.mf_retrieve_path.restype = ctypes.c_int
 _lib.mf_get_status.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
@@ -255,6 +260,63 @@ def mf_map_retrieve(layers: Sequence[BSR], layer_map: Sequence[int], W: torch.Te
     _check(_lib.mf_map_retrieve(ctypes.byref(d), _stream(stream)))
     del keep
     return O
+
+
+@dataclass
+class Receiver:
+    """One receiver model of a shared sender: its layer map, head map W [L_r, h_r, h_s],
+    V ([L_r, T_k, h_kv, d] or paged [L_r, pages, page, h_kv, d]) and output O."""
+    layer_map: Sequence[int]
+    W: torch.Tensor
+    V: torch.Tensor
+    h_r: int
+    h_kv: int
+    O: Optional[torch.Tensor] = None
+    paged: Optional[tuple] = None
+    v_layer_stride: int = 0
+
+
+def _multi_descs(layers, receivers, cu_seqlens_q, cu_seqlens_k, qblock_base, max_seqlen_q,
+                 total_q, l_r_range):
+    h_s, B = layers[0].values.shape[1], layers[0].values.shape[2]
+    arr = (RetrieveDesc * len(receivers))()
+    keep, outs = [], []
+    for k, r in enumerate(receivers):
+        rng = l_r_range if l_r_range is not None else (0, len(r.layer_map))
+        O = r.O
+        if O is None:
+            if total_q is None:
+                raise ValueError("total_q is needed to allocate O")
+            O = torch.empty((rng[1] - rng[0], total_q, r.h_r, r.V.shape[-1]), dtype=r.V.dtype,
+                            device=r.V.device)
+        d, kp = _retrieve_desc(layers, r.layer_map, rng, r.W, r.V, O, cu_seqlens_q, cu_seqlens_k,
+                               qblock_base, max_seqlen_q, h_s, B, r.h_r, r.h_kv, r.v_layer_stride,
+                               0, r.paged, 0)
+        arr[k] = d
+        keep.append(kp)
+        outs.append(O)
+    return arr, keep, outs
+
+
+def mf_map_retrieve_multi(layers: Sequence[BSR], receivers: Sequence[Receiver],
+                          cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                          qblock_base: torch.Tensor, max_seqlen_q: int,
+                          total_q: Optional[int] = None, l_r_range=None,
+                          stream=None) -> List[torch.Tensor]:
+    """Retrieval for several receivers of one sender's compressed layers (one O per receiver);
+    up to four receivers share each launch when they can (mf_retrieve_multi_fused)."""
+    arr, keep, outs = _multi_descs(layers, receivers, cu_seqlens_q, cu_seqlens_k, qblock_base,
+                                   max_seqlen_q, total_q, l_r_range)
+    _check(_lib.mf_map_retrieve_multi(arr, len(receivers), _stream(stream)))
+    del keep
+    return outs
+
+
+def mf_retrieve_multi_fused(layers, receivers, cu_seqlens_q, cu_seqlens_k, qblock_base,
+                            max_seqlen_q, total_q=None, l_r_range=None) -> int:
+    arr, keep, _ = _multi_descs(layers, receivers, cu_seqlens_q, cu_seqlens_k, qblock_base,
+                                max_seqlen_q, total_q, l_r_range)
+    return _lib.mf_retrieve_multi_fused(arr, len(receivers))
 
 
 def mf_retrieve_path(layers, layer_map, W, V, cu_seqlens_q, cu_seqlens_k, qblock_base,

@@ -113,6 +113,45 @@ mf_status static_ws_ptr(void** out) {
 }  // namespace
 
 namespace {
+// receiver layer l of a retrieval descriptor
+mfi::RetrieveLayer layer_of(const mf_retrieve_desc& d, int l) {
+  const int64_t ve = d.v_dtype == MF_F32 ? 4 : 2;
+  const int64_t o_stride = d.o_layer_stride ? d.o_layer_stride : (int64_t)d.total_q * d.h_r * d.d;
+  const mf_bsr& b = d.layers[d.layer_map[l]];
+  mfi::RetrieveLayer L;
+  L.row_ptr = b.row_ptr;
+  L.col_idx = b.col_idx;
+  L.values = b.values;
+  L.capacity = b.capacity_blocks;
+  L.W = d.W + (int64_t)l * d.h_r * d.h_s;
+  L.V = static_cast<const char*>(d.V) + (int64_t)l * d.v_layer_stride * ve;
+  L.O = static_cast<char*>(d.O) + (int64_t)(l - d.l_r_begin) * o_stride * ve;
+  return L;
+}
+
+// receivers that can share launches: all on the tensor-core path, the same sender blocks at
+// every layer step, the same query / key packing
+bool can_fuse(const mf_retrieve_desc* ds, int n) {
+  const mf_retrieve_desc& a = ds[0];
+  for (int k = 0; k < n; ++k) {
+    const mf_retrieve_desc& b = ds[k];
+    if (!mfi::tc_supported(b)) return false;
+    if (b.map_dtype != a.map_dtype || b.h_s != a.h_s || b.B != a.B || b.nseq != a.nseq ||
+        b.max_seqlen_q != a.max_seqlen_q || b.cu_seqlens_q != a.cu_seqlens_q ||
+        b.cu_seqlens_k != a.cu_seqlens_k || b.qblock_base != a.qblock_base ||
+        b.l_r_end - b.l_r_begin != a.l_r_end - a.l_r_begin)
+      return false;
+    for (int j = 0; j < a.l_r_end - a.l_r_begin; ++j) {
+      const mf_bsr& x = a.layers[a.layer_map[a.l_r_begin + j]];
+      const mf_bsr& y = b.layers[b.layer_map[b.l_r_begin + j]];
+      if (x.row_ptr != y.row_ptr || x.col_idx != y.col_idx || x.values != y.values ||
+          x.capacity_blocks != y.capacity_blocks)
+        return false;
+    }
+  }
+  return true;
+}
+
 mf_status check_calib(const mf_calib_desc* d) {
   if (!d) return fail(MF_ERR_INVALID, "desc is NULL");
   if (!is_dtype(d->dtype)) return fail(MF_ERR_INVALID, "dtype must be MF_F32 or MF_BF16");
@@ -217,22 +256,11 @@ mf_status mf_map_retrieve(const mf_retrieve_desc* desc, void* stream) {
   uint32_t* st = status_ptr();
   if (!st) return fail(MF_ERR_CUDA, "cannot resolve the device status word");
   const bool tc = mfi::tc_supported(*desc);
-  const int64_t ve = desc->v_dtype == MF_F32 ? 4 : 2;
-  const int64_t o_stride = desc->o_layer_stride ? desc->o_layer_stride
-                                                : (int64_t)desc->total_q * desc->h_r * desc->d;
   for (int l = desc->l_r_begin; l < desc->l_r_end; ++l) {
-    const mf_bsr& b = desc->layers[desc->layer_map[l]];
-    mfi::RetrieveLayer L;
-    L.row_ptr = b.row_ptr;
-    L.col_idx = b.col_idx;
-    L.values = b.values;
-    L.capacity = b.capacity_blocks;
-    L.W = desc->W + (int64_t)l * desc->h_r * desc->h_s;
-    L.V = static_cast<const char*>(desc->V) + (int64_t)l * desc->v_layer_stride * ve;
-    L.O = static_cast<char*>(desc->O) + (int64_t)(l - desc->l_r_begin) * o_stride * ve;
+    const mfi::RetrieveLayer L = layer_of(*desc, l);
     if (tc) {
       std::string err;
-      if (!mfi::launch_retrieve_tc(*desc, L, st, static_cast<cudaStream_t>(stream), &err))
+      if (!mfi::launch_retrieve_tc(&desc, &L, 1, st, static_cast<cudaStream_t>(stream), &err))
         return fail(MF_ERR_CUDA, "mf_map_retrieve (tcgen05): " + err);
     } else {
       cudaError_t e = mfi::launch_retrieve_simt(*desc, L, st, static_cast<cudaStream_t>(stream));
@@ -240,6 +268,45 @@ mf_status mf_map_retrieve(const mf_retrieve_desc* desc, void* stream) {
         return fail(MF_ERR_CUDA, std::string("mf_map_retrieve (simt): ") + cudaGetErrorString(e));
     }
   }
+  return MF_OK;
+}
+
+int mf_retrieve_multi_fused(const mf_retrieve_desc* descs, int n) {
+  if (!descs || n < 1) return -1;
+  for (int k = 0; k < n; ++k)
+    if (check_retrieve(&descs[k]) != MF_OK) return -1;
+  return can_fuse(descs, n) ? 1 : 0;
+}
+
+mf_status mf_map_retrieve_multi(const mf_retrieve_desc* descs, int n, void* stream) {
+  if (!descs || n < 1) return fail(MF_ERR_INVALID, "descs is NULL or n < 1");
+  for (int k = 0; k < n; ++k) {
+    mf_status s = check_retrieve(&descs[k]);
+    if (s != MF_OK) return s;
+  }
+  if (!can_fuse(descs, n)) {  // one receiver at a time
+    for (int k = 0; k < n; ++k) {
+      mf_status s = mf_map_retrieve(&descs[k], stream);
+      if (s != MF_OK) return s;
+    }
+    return MF_OK;
+  }
+  uint32_t* st = status_ptr();
+  if (!st) return fail(MF_ERR_CUDA, "cannot resolve the device status word");
+  const int steps = descs[0].l_r_end - descs[0].l_r_begin;
+  for (int j = 0; j < steps; ++j)
+    for (int k0 = 0; k0 < n; k0 += 4) {  // up to four receivers share a launch
+      const int cnt = n - k0 < 4 ? n - k0 : 4;
+      const mf_retrieve_desc* ptrs[4];
+      mfi::RetrieveLayer Ls[4];
+      for (int k = 0; k < cnt; ++k) {
+        ptrs[k] = &descs[k0 + k];
+        Ls[k] = layer_of(descs[k0 + k], descs[k0 + k].l_r_begin + j);
+      }
+      std::string err;
+      if (!mfi::launch_retrieve_tc(ptrs, Ls, cnt, st, static_cast<cudaStream_t>(stream), &err))
+        return fail(MF_ERR_CUDA, "mf_map_retrieve_multi (tcgen05): " + err);
+    }
   return MF_OK;
 }
 

@@ -53,9 +53,10 @@ cudaError_t launch_retrieve_simt(const mf_retrieve_desc& d, const RetrieveLayer&
 
 bool tc_supported(const mf_retrieve_desc& d);
 
-// returns false and fills *err on a host-side failure (tensor-map encoding, launch)
-bool launch_retrieve_tc(const mf_retrieve_desc& d, const RetrieveLayer& l, uint32_t* status,
-                        cudaStream_t st, std::string* err);
+// one launch for n (1..4) receivers that share the sender BSR layer and the query / key
+// packing; returns false and fills *err on a host-side failure (tensor-map encoding, launch)
+bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* ls, int n,
+                        uint32_t* status, cudaStream_t st, std::string* err);
 
 // head-map calibration
 size_t calib_ws_bytes(const mf_calib_desc& d);

@@ -49,6 +49,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 #include "mf_internal.cuh"
@@ -109,22 +110,35 @@ constexpr uint32_t IDESC_MIX = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) |
 constexpr uint32_t IDESC_PV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                               ((64u >> 3) << 17) | ((128u >> 4) << 24);
 
+constexpr int NRMAX = 4;  // receivers served by one launch (one BSR, several W / V / O)
+
+// one receiver: its head map, V and O (and its V paging)
+struct RecvParams {
+  const float* W;  // [h_r][h_s]
+  __nv_bfloat16* O;
+  const int32_t* block_table;
+  int paged, page_size, n_pages, max_pages;
+  int total_k;     // V rows (contiguous V): the out-of-range row that reads zeros
+  int h_r, h_kv, gq, hcs;
+};
 struct TcParams {
   const int32_t* row_ptr;
   const int32_t* col_idx;
   int64_t capacity;
-  const float* W;  // [h_r][h_s]
-  __nv_bfloat16* O;
   const int32_t* cu_q;
   const int32_t* cu_k;
   const int32_t* qblock_base;
-  const int32_t* block_table;
-  int paged, page_size, n_pages, max_pages;
-  int total_k;
-  int nqbq, rcs, hcs;  // query blocks, row chunks per block, head chunks
+  int nqbq, rcs;    // query blocks, row chunks per block
+  int NH;           // head chunks of all receivers together
+  int hh_base[NRMAX + 1];  // first head chunk of each receiver
+  int nrecv;
   int n_items;
-  int h_s, nsc, B, h_r, h_kv, gq;
+  int h_s, nsc, B;
+  RecvParams rv[NRMAX];
   uint32_t* status;
+};
+struct VMaps {
+  CUtensorMap m[NRMAX];
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -277,13 +291,14 @@ struct Item {
 };
 static_assert(sizeof(Item) <= ITEM_BYTES, "item table slot");
 
-// item idx = ((s * nqbq + qbl) * rcs + rc) * hcs + hc; identical in every role
+// item idx = ((s * nqbq + qbl) * rcs + rc) * NH + hh, hh = a receiver's head chunk;
+// identical in every role
 __device__ __forceinline__ Item decode(const TcParams& p, int idx) {
   Item it;
   it.valid = false;
   it.bsr_ok = true;
   it.n_tiles = 0;
-  idx /= p.hcs;
+  idx /= p.NH;
   const int rc = idx % p.rcs;
   idx /= p.rcs;
   const int qbl = idx % p.nqbq;
@@ -310,8 +325,8 @@ __device__ __forceinline__ Item decode(const TcParams& p, int idx) {
 }
 
 __global__ void __launch_bounds__(NT, 1)
-    k_retrieve_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmV,
-                  TcParams p) {
+    k_retrieve_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ VMaps tmVs,
+                  const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
@@ -323,7 +338,13 @@ __global__ void __launch_bounds__(NT, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hc = blockIdx.x % p.hcs;  // constant per CTA (gridDim.x is a multiple of hcs)
+  // receiver and head chunk: constant per CTA (gridDim.x is a multiple of NH)
+  const int hh = blockIdx.x % p.NH;
+  int ri = 0;
+  while (ri + 1 < p.nrecv && hh >= p.hh_base[ri + 1]) ++ri;
+  const RecvParams& q_r = p.rv[ri];
+  const CUtensorMap* tmV = &tmVs.m[ri];
+  const int hc = hh - p.hh_base[ri];
   const int tpb = p.B / KT;
 
   const uint32_t sb = smem_u32(smem);
@@ -367,7 +388,7 @@ __global__ void __launch_bounds__(NT, 1)
       const int rv = e / ks, hs = e % ks;
       const int G = hc * NG + rv / GQP, q = rv % GQP;
       float w = 0.0f;
-      if (q < p.gq && G < p.h_kv && hs < p.h_s) w = p.W[(int64_t)(G * p.gq + q) * p.h_s + hs];
+      if (q < q_r.gq && G < q_r.h_kv && hs < p.h_s) w = q_r.W[(int64_t)(G * q_r.gq + q) * p.h_s + hs];
       __nv_bfloat16 hi = __float2bfloat16_rn(w);
       __nv_bfloat16 lo = __float2bfloat16_rn(w - __bfloat162float(hi));
       const int base = (hs >> 3) * 512 + (hs & 7) * 2;
@@ -402,7 +423,7 @@ __global__ void __launch_bounds__(NT, 1)
         if (!it.valid) continue;
         if (is_a) TRACE(0, 1);
         if (is_a && !it.bsr_ok) atomicOr(p.status, ST_INDEX);
-        const int rc = (idx / p.hcs) % p.rcs;
+        const int rc = (idx / p.NH) % p.rcs;
         // key block of the current kept block and, loaded one block ahead, of the next one
         const int nblk = it.n_tiles / tpb;
         int kb_cur = it.kb0, kb_nxt = (!is_a && nblk > 1) ? p.col_idx[it.rp0 + 1] : -1;
@@ -437,23 +458,23 @@ __global__ void __launch_bounds__(NT, 1)
             for (int gl = 0; gl < PH; ++gl) {
               const uint32_t dst = sb + OFF_V + vs * V_BYTES + gl * VGRP_BYTES;
               const int G = hc * NG + h * PH + gl;
-              if (!p.paged) {
-                const int row = kb_ok ? it.k0 + tok0 : p.total_k;  // out of range reads 0
-                tma_load_3d(dst, &tmV, bar(B_HFULL + vs), 0, G, row);
-                tma_load_3d(dst + 8192, &tmV, bar(B_HFULL + vs), 64, G, row);
+              if (!q_r.paged) {
+                const int row = kb_ok ? it.k0 + tok0 : q_r.total_k;  // out of range reads 0
+                tma_load_3d(dst, tmV, bar(B_HFULL + vs), 0, G, row);
+                tma_load_3d(dst + 8192, tmV, bar(B_HFULL + vs), 64, G, row);
               } else {
-                const int ps = p.page_size;
+                const int ps = q_r.page_size;
                 for (int q = 0; q < KT / ps; ++q) {
                   const int tok = tok0 + q * ps;
                   const int slot = tok / ps;
-                  int page = p.n_pages;  // out of range: the copy reads zeros
-                  if (kb_ok && tok < it.k_len && slot < p.max_pages) {
-                    const int pg = p.block_table[(int64_t)it.s * p.max_pages + slot];
-                    if (pg >= 0 && pg < p.n_pages) page = pg;
+                  int page = q_r.n_pages;  // out of range: the copy reads zeros
+                  if (kb_ok && tok < it.k_len && slot < q_r.max_pages) {
+                    const int pg = q_r.block_table[(int64_t)it.s * q_r.max_pages + slot];
+                    if (pg >= 0 && pg < q_r.n_pages) page = pg;
                     else atomicOr(p.status, ST_PAGE);
                   }
-                  tma_load_4d(dst + q * ps * 128, &tmV, bar(B_HFULL + vs), 0, G, 0, page);
-                  tma_load_4d(dst + 8192 + q * ps * 128, &tmV, bar(B_HFULL + vs), 64, G, 0, page);
+                  tma_load_4d(dst + q * ps * 128, tmV, bar(B_HFULL + vs), 0, G, 0, page);
+                  tma_load_4d(dst + 8192 + q * ps * 128, tmV, bar(B_HFULL + vs), 64, G, 0, page);
                 }
               }
             }
@@ -595,8 +616,8 @@ __global__ void __launch_bounds__(NT, 1)
         (uint32_t)j * 128u + ((((uint32_t)(2 * set + rb)) ^ ((uint32_t)j & 7u)) << 4);
     // O epilogue of an item, shared by the 16 warps: warp (set, quarter) reads D2 group g = set
     // (64 columns) for head dims [32 quarter, 32 quarter + 32), releases it and stores O
-    const int ng = min(NG, p.h_kv - hc * NG);  // real groups of this head chunk
-    const int64_t rs = (int64_t)p.h_r * D;     // O row stride
+    const int ng = min(NG, q_r.h_kv - hc * NG);  // real groups of this head chunk
+    const int64_t rs = (int64_t)q_r.h_r * D;     // O row stride
     // the item (table slot ek, index eidx) is re-read from the item table here
     auto epilogue = [&](int ek, int eidx, int K) -> bool {
       const Item q = item(ek, eidx);
@@ -629,7 +650,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (lane == 0) mbar_arrive(bar(B_OEMPTY + g / PH));
       if (warp == 4 && lane == 0) TRACE(3, 2);
       if (g < ng) {
-        __nv_bfloat16* ob = p.O + (q.o_row0 * p.h_r + (int64_t)(hc * NG + g) * p.gq) * D +
+        __nv_bfloat16* ob = q_r.O + (q.o_row0 * q_r.h_r + (int64_t)(hc * NG + g) * q_r.gq) * D +
                             quarter * 32 + lane;
         // column n = 8 c + 4 mi + head holds row 2 (c / 2) + 8 mi + c % 2
 #pragma unroll
@@ -638,7 +659,7 @@ __global__ void __launch_bounds__(NT, 1)
           for (int b = 0; b < 2; ++b) {
             const int n = 2 * u + b, c8 = n >> 3;
             const int ii = 2 * (c8 >> 1) + 8 * ((n >> 2) & 1) + (c8 & 1), rv = n & 3;
-            if (rv < p.gq && ii >= ilo && ii < ihi)
+            if (rv < q_r.gq && ii >= ilo && ii < ihi)
               *reinterpret_cast<uint16_t*>(ob + ii * rs + rv * D) =
                   (uint16_t)(b ? pr[u] >> 16 : pr[u] & 0xFFFFu);
           }
@@ -809,56 +830,72 @@ bool tc_supported(const mf_retrieve_desc& d) {
   return true;
 }
 
-bool launch_retrieve_tc(const mf_retrieve_desc& d, const RetrieveLayer& l, uint32_t* status,
-                        cudaStream_t st, std::string* err) {
-  const int B = d.B;
-  CUtensorMap tmA, tmV;
+bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* ls, int n,
+                        uint32_t* status, cudaStream_t st, std::string* err) {
+  if (n < 1 || n > NRMAX) { *err = "1 to 4 receivers per launch"; return false; }
+  const mf_retrieve_desc& d0 = *ds[0];
+  const RetrieveLayer& l0 = ls[0];
+  const int B = d0.B;
+  CUtensorMap tmA;
   {  // kept blocks [capacity][h_s][B][B]: dims (key j, sender head s, row i, block n)
-    const uint64_t dims[4] = {(uint64_t)B, (uint64_t)d.h_s, (uint64_t)B,
-                              (uint64_t)std::max<int64_t>(l.capacity, 1)};
-    const uint64_t strides[3] = {(uint64_t)B * B * 2, (uint64_t)B * 2, (uint64_t)d.h_s * B * B * 2};
+    const uint64_t dims[4] = {(uint64_t)B, (uint64_t)d0.h_s, (uint64_t)B,
+                              (uint64_t)std::max<int64_t>(l0.capacity, 1)};
+    const uint64_t strides[3] = {(uint64_t)B * B * 2, (uint64_t)B * 2, (uint64_t)d0.h_s * B * B * 2};
     const uint32_t box[4] = {KT, SC, R, 1};
-    if (!encode(&tmA, l.values, 4, dims, strides, box, err)) return false;
+    if (!encode(&tmA, l0.values, 4, dims, strides, box, err)) return false;
   }
-  if (!d.paged) {  // V [T][h_kv][d]: dims (dim, kv head, token)
-    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)d.h_kv, (uint64_t)std::max<int64_t>(d.total_k, 1)};
-    const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)d.h_kv * D * 2};
-    const uint32_t box[3] = {64, 1, KT};
-    if (!encode(&tmV, l.V, 3, dims, strides, box, err)) return false;
-  } else {  // V [pages][page][h_kv][d]: dims (dim, kv head, row in page, page)
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)d.h_kv, (uint64_t)d.page_size,
-                              (uint64_t)std::max(d.n_pages, 1)};
-    const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)d.h_kv * D * 2,
-                                 (uint64_t)d.page_size * d.h_kv * D * 2};
-    const uint32_t box[4] = {64, 1, (uint32_t)d.page_size, 1};
-    if (!encode(&tmV, l.V, 4, dims, strides, box, err)) return false;
-  }
+  VMaps vm;
+  memset(&vm, 0, sizeof vm);
   TcParams p{};
-  p.row_ptr = l.row_ptr; p.col_idx = l.col_idx; p.capacity = l.capacity;
-  p.W = l.W; p.O = static_cast<__nv_bfloat16*>(l.O);
-  p.cu_q = d.cu_seqlens_q; p.cu_k = d.cu_seqlens_k; p.qblock_base = d.qblock_base;
-  p.block_table = d.block_table; p.paged = d.paged; p.page_size = d.page_size;
-  p.n_pages = d.n_pages; p.max_pages = d.max_pages; p.total_k = (int)d.total_k;
-  p.nqbq = (d.max_seqlen_q + B - 1) / B;
+  p.row_ptr = l0.row_ptr; p.col_idx = l0.col_idx; p.capacity = l0.capacity;
+  p.cu_q = d0.cu_seqlens_q; p.cu_k = d0.cu_seqlens_k; p.qblock_base = d0.qblock_base;
+  p.nqbq = (d0.max_seqlen_q + B - 1) / B;
   p.rcs = B / R;
-  p.hcs = (d.h_kv + NG - 1) / NG;
-  p.h_s = d.h_s; p.nsc = (d.h_s + SC - 1) / SC; p.B = B; p.h_r = d.h_r; p.h_kv = d.h_kv;
-  p.gq = d.h_r / d.h_kv;
+  p.h_s = d0.h_s; p.nsc = (d0.h_s + SC - 1) / SC; p.B = B;
+  p.nrecv = n;
   p.status = status;
-  const int64_t n_items = (int64_t)d.nseq * p.nqbq * p.rcs * p.hcs;
+  int NH = 0;
+  for (int k = 0; k < n; ++k) {
+    const mf_retrieve_desc& d = *ds[k];
+    const RetrieveLayer& l = ls[k];
+    if (!d.paged) {  // V [T][h_kv][d]: dims (dim, kv head, token)
+      const uint64_t dims[3] = {(uint64_t)D, (uint64_t)d.h_kv, (uint64_t)std::max<int64_t>(d.total_k, 1)};
+      const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)d.h_kv * D * 2};
+      const uint32_t box[3] = {64, 1, KT};
+      if (!encode(&vm.m[k], l.V, 3, dims, strides, box, err)) return false;
+    } else {  // V [pages][page][h_kv][d]: dims (dim, kv head, row in page, page)
+      const uint64_t dims[4] = {(uint64_t)D, (uint64_t)d.h_kv, (uint64_t)d.page_size,
+                                (uint64_t)std::max(d.n_pages, 1)};
+      const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)d.h_kv * D * 2,
+                                   (uint64_t)d.page_size * d.h_kv * D * 2};
+      const uint32_t box[4] = {64, 1, (uint32_t)d.page_size, 1};
+      if (!encode(&vm.m[k], l.V, 4, dims, strides, box, err)) return false;
+    }
+    RecvParams& r = p.rv[k];
+    r.W = l.W; r.O = static_cast<__nv_bfloat16*>(l.O);
+    r.block_table = d.block_table; r.paged = d.paged; r.page_size = d.page_size;
+    r.n_pages = d.n_pages; r.max_pages = d.max_pages; r.total_k = (int)d.total_k;
+    r.h_r = d.h_r; r.h_kv = d.h_kv; r.gq = d.h_r / d.h_kv;
+    r.hcs = (d.h_kv + NG - 1) / NG;
+    p.hh_base[k] = NH;
+    NH += r.hcs;
+  }
+  p.hh_base[n] = NH;
+  p.NH = NH;
+  const int64_t n_items = (int64_t)d0.nseq * p.nqbq * p.rcs * NH;
   if (n_items == 0) return true;
   if (n_items >= ((int64_t)1 << 31)) { *err = "too many work items"; return false; }
   p.n_items = (int)n_items;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // persistent grid, a multiple of the head-chunk count (one W^T per CTA)
+  // persistent grid, a multiple of the head-chunk count (one receiver and one W^T per CTA)
   int64_t grid = std::min<int64_t>(n_items, sms);
-  grid = std::max<int64_t>(p.hcs, grid / p.hcs * p.hcs);
+  grid = std::max<int64_t>(NH, grid / NH * NH);
   cudaError_t e = cudaFuncSetAttribute(k_retrieve_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SMEM_BYTES);
   if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
-  k_retrieve_tc<<<(unsigned)grid, NT, SMEM_BYTES, st>>>(tmA, tmV, p);
+  k_retrieve_tc<<<(unsigned)grid, NT, SMEM_BYTES, st>>>(tmA, vm, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
   return true;

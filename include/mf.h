@@ -204,6 +204,22 @@ typedef struct {
 
 mf_status mf_map_retrieve(const mf_retrieve_desc* desc, void* stream);
 
+/* Several receivers of one sender in shared launches (the pages' one-sender, several-
+ * receivers workflow, MapFlow page "MapFlow开源:大模型换班,Prefill为何能快20%?", section
+ * "它能做什么:三种典型工作流": one sender's compressed maps serve several receiver models).
+ * Same results as calling mf_map_retrieve on descs[0..n-1] in order (bitwise).  When every
+ * receiver takes the tensor-core path and all share the sender blocks of every layer step
+ * (the same mf_bsr pointers), the query / key packing (cu_seqlens_q/k and qblock_base
+ * pointers, nseq, max_seqlen_q) and the number of receiver layers, up to four receivers share
+ * each launch: the CTAs of all receivers walk the same query blocks together, so the kept
+ * map tiles are read from HBM once per step and reused from L2.  Otherwise the receivers run
+ * one after another.  Errors as for mf_map_retrieve (the first failing descriptor). */
+mf_status mf_map_retrieve_multi(const mf_retrieve_desc* descs, int n, void* stream);
+
+/* 1 when mf_map_retrieve_multi would share launches among descs, 0 when it would run them
+ * one by one, -1 for an invalid descriptor. */
+int mf_retrieve_multi_fused(const mf_retrieve_desc* descs, int n);
+
 /* Which kernel mf_map_retrieve would launch: 0 = float32 SIMT, 1 = tcgen05.
  * Returns -1 for an invalid descriptor. */
 int mf_retrieve_path(const mf_retrieve_desc* desc);

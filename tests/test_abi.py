@@ -154,3 +154,29 @@ def test_calib_host_validation(mf):
     assert mf._lib.mf_calib_solve(None, 4, 4, 0.0, None, None, None) == mf.MF_ERR_INVALID
     assert mf._lib.mf_calib_solve(4096, 4, 4, -1.0, 4096, None, None) == mf.MF_ERR_INVALID
     assert mf._lib.mf_calib_solve(4096, 65, 4, 0.0, 4096, None, None) == mf.MF_ERR_UNSUPPORTED
+
+
+def test_retrieve_multi_fusing_rules(mf):
+    """Receivers of one sender share launches only when they share its blocks and the packing."""
+    arr = (mf.BsrDesc * 1)(mf.BsrDesc(4096, 4096, 4096, 100))
+    other = (mf.BsrDesc * 1)(mf.BsrDesc(4096, 8192, 4096, 100))
+    lm = (ctypes.c_int32 * 1)(0)
+    F = mf._lib.mf_retrieve_multi_fused
+
+    def many(*ds):
+        a = (mf.RetrieveDesc * len(ds))()
+        for k, d in enumerate(ds):
+            a[k] = d
+        return a
+
+    base = _retrieve_desc(mf, arr, lm)
+    small = _retrieve_desc(mf, arr, lm, h_r=8, h_kv=2, W=8192, V=8192, O=16384)  # another receiver
+    assert F(many(base, small), 2) == 1
+    assert F(many(base, small, small, base, small), 5) == 1          # two launches per step
+    assert F(many(base, _retrieve_desc(mf, other, lm)), 2) == 0       # other sender blocks
+    assert F(many(base, _retrieve_desc(mf, arr, lm, cu_seqlens_q=12288)), 2) == 0  # other packing
+    assert F(many(base, _retrieve_desc(mf, arr, lm, h_r=32, h_kv=4)), 2) == 0      # SIMT receiver
+    assert F(many(base, _retrieve_desc(mf, arr, lm, h_r=30)), 2) == -1             # invalid
+    assert mf._lib.mf_map_retrieve_multi(many(base), 0, None) == mf.MF_ERR_INVALID
+    assert mf._lib.mf_map_retrieve_multi(many(base, _retrieve_desc(mf, arr, lm, d=0)), 2,
+                                         None) == mf.MF_ERR_INVALID
