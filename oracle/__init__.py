@@ -56,6 +56,10 @@ def _load():
         lib.mfo_calib_gram.restype = None
         lib.mfo_calib_solve.argtypes = [P, I, I, D, P, P]
         lib.mfo_calib_solve.restype = I
+        lib.mfo_qk_maps.argtypes = [P, P, I, I, I, I, I, I64, D, P]
+        lib.mfo_qk_maps.restype = None
+        lib.mfo_qk_rows.argtypes = [P, P, I, I, I, I, I, I, I, I64, D, P]
+        lib.mfo_qk_rows.restype = None
         _lib = lib
     return _lib
 
@@ -63,19 +67,24 @@ def _load():
 # ----------------------------------------------------------------------------- dtypes
 
 def as_raw(t):
-    """(numpy array of the raw elements, dtype code): float32 -> (f32, 0), bf16 -> (uint16, 1)."""
+    """(numpy array of the raw elements, dtype code): float32 -> (f32, 0), bf16 -> (uint16, 1),
+    float64 -> (f64, 2)."""
     if isinstance(t, torch.Tensor):
         t = t.detach().cpu().contiguous()
         if t.dtype == torch.bfloat16:
             return t.view(torch.int16).numpy().view(np.uint16), 1
         if t.dtype == torch.float32:
             return t.numpy(), 0
+        if t.dtype == torch.float64:
+            return t.numpy(), 2
         raise TypeError(t.dtype)
     a = np.ascontiguousarray(t)
     if a.dtype == np.uint16:
         return a, 1
     if a.dtype == np.float32:
         return a, 0
+    if a.dtype == np.float64:
+        return a, 2
     raise TypeError(a.dtype)
 
 
@@ -208,6 +217,52 @@ def retrieve_step(bsr_rows, B, W_l, V, h_kv, step, qblock_base, k_starts=None,
             O.append(retrieve_block(vals, kept, qb, B, W_l, V, h_kv, (lo, hi), ks, bt, page_size))
         outs.append(np.concatenate(O, axis=0))
     return np.concatenate(outs, axis=0)
+
+
+# ----------------------------------------------------------------------------- maps from Q, K
+
+def qk_maps(Q, K, L, B, scale):
+    """The sender's causal attention maps of one sequence from its queries Q [L, h_s, d] and
+    keys K [L, h_kv, d] (float32 or bfloat16, read exactly): float64 [h_s, Lp, Lp] (Lp = L
+    rounded up to B), zero outside j <= i < L.  Query head s reads key head s * h_kv // h_s."""
+    qa, qc = as_raw(Q)
+    ka, kc = as_raw(K)
+    assert qc == kc and qa.shape[0] >= L and ka.shape[0] >= L and qa.shape[2] == ka.shape[2]
+    h_s, h_kv, d = qa.shape[1], ka.shape[1], qa.shape[2]
+    assert h_s % h_kv == 0
+    Lp = -(-L // B) * B
+    A = np.empty((h_s, Lp, Lp), dtype=np.float64)
+    _load().mfo_qk_maps(_ptr(qa), _ptr(ka), qc, L, h_s, h_kv, d, Lp, float(scale), _ptr(A))
+    return A
+
+
+def qk_slab(Q, K, L, B, qb, scale):
+    """Rows of query block qb of the maps of qk_maps: float64 [h_s, B, (qb + 1) * B]."""
+    qa, qc = as_raw(Q)
+    ka, kc = as_raw(K)
+    assert qc == kc
+    h_s, h_kv, d = qa.shape[1], ka.shape[1], qa.shape[2]
+    width = (qb + 1) * B
+    out = np.empty((h_s, B, width), dtype=np.float64)
+    _load().mfo_qk_rows(_ptr(qa), _ptr(ka), qc, L, h_s, h_kv, d, qb * B, (qb + 1) * B, width,
+                        float(scale), _ptr(out))
+    return out
+
+
+def compress_qk_row(Q, K, L, B, qb, tau, scale):
+    """One query block of compression from Q, K: (masses, kept, walk info, values float64)."""
+    slab = qk_slab(Q, K, L, B, qb, scale)
+    m = row_masses(slab, L, B, qb)
+    kept, info = select(m, qb, tau)
+    vals = np.stack([gather_block(slab, L, B, qb, int(kb)) for kb in kept])
+    return m, kept, info, vals
+
+
+def compress_qk_seq(Q, K, L, B, tau, scale, rows=None):
+    """Compression of one sequence straight from its queries and keys: the maps of qk_maps,
+    then the block statistics, selection and kept-block values of compress_seq (values
+    float64)."""
+    return compress_seq(qk_maps(Q, K, L, B, scale), L, B, tau, rows)
 
 
 # ----------------------------------------------------------------------------- calibration

@@ -36,9 +36,10 @@
 #include <stdlib.h>
 #include <string.h>
 
-/* dtype codes: 0 = float32, 1 = bfloat16 (stored as its upper 16 bits). */
+/* dtype codes: 0 = float32, 1 = bfloat16 (stored as its upper 16 bits), 2 = float64. */
 static double value_at(const void* p, int dtype, int64_t idx) {
   if (dtype == 0) return (double)((const float*)p)[idx];
+  if (dtype == 2) return ((const double*)p)[idx];
   uint32_t bits = (uint32_t)((const uint16_t*)p)[idx] << 16;
   float f;
   memcpy(&f, &bits, sizeof f);
@@ -145,6 +146,8 @@ void mfo_gather_block(const void* slab, int dtype, int h_s, int B, int64_t head_
         const int64_t src = s * head_stride + ii * row_stride + j;
         if (dtype == 0)
           ((float*)out)[o] = keep ? ((const float*)slab)[src] : 0.0f;
+        else if (dtype == 2)
+          ((double*)out)[o] = keep ? ((const double*)slab)[src] : 0.0;
         else
           ((uint16_t*)out)[o] = keep ? ((const uint16_t*)slab)[src] : (uint16_t)0;
       }
@@ -284,4 +287,53 @@ int mfo_calib_solve(const double* gram, int h_s, int h_r, double ridge, double* 
   free(z);
   free(Lf);
   return 0;
+}
+
+/*
+ * Sender attention maps from the sender's own queries and keys, for compression without a
+ * dense map (MapFlow page "MapFlow开源:大模型换班,Prefill为何能快20%?", section
+ * "存不下、读得慢?三个工程优化手段", subsection 1: block statistics first, then the kept
+ * blocks, with no dense matrix assembled).  The map is the sender's causal attention
+ * distribution:
+ *   A_s[i][j] = exp(scale * <q_{i,s}, k_{j,g}>) / sum_{j' <= i} exp(scale * <q_{i,s}, k_{j',g}>)
+ * for j <= i < L and 0 elsewhere, with g = floor(s * h_kv / h_s) (contiguous grouping of query
+ * heads onto key heads).  The row maximum of the scaled products is subtracted before the
+ * exponentials (the ratio is unchanged).  Q: [L][h_s][d], K: [L][h_kv][d] raw (dtype 0 f32,
+ * 1 bf16); A: [h_s][Lp][Lp] double, fully written.
+ */
+static void qk_row(const void* Q, const void* K, int dtype, int h_s, int h_kv, int d, int s,
+                   int i, double scale, double* z, double* out) {
+  const int g = (int)((int64_t)s * h_kv / h_s);
+  double zmax = -HUGE_VAL;
+  for (int j = 0; j <= i; ++j) {
+    double dot = 0.0;
+    for (int c = 0; c < d; ++c)
+      dot += value_at(Q, dtype, ((int64_t)i * h_s + s) * d + c) *
+             value_at(K, dtype, ((int64_t)j * h_kv + g) * d + c);
+    z[j] = scale * dot;
+    if (z[j] > zmax) zmax = z[j];
+  }
+  double denom = 0.0;
+  for (int j = 0; j <= i; ++j) denom += exp(z[j] - zmax);
+  for (int j = 0; j <= i; ++j) out[j] = exp(z[j] - zmax) / denom;
+}
+
+void mfo_qk_maps(const void* Q, const void* K, int dtype, int L, int h_s, int h_kv, int d,
+                 int64_t Lp, double scale, double* A) {
+  double* z = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+  for (int64_t e = 0; e < (int64_t)h_s * Lp * Lp; ++e) A[e] = 0.0;
+  for (int s = 0; s < h_s; ++s)
+    for (int i = 0; i < L; ++i) qk_row(Q, K, dtype, h_s, h_kv, d, s, i, scale, z, A + ((int64_t)s * Lp + i) * Lp);
+  free(z);
+}
+
+/* Rows [i0, i1) of the same maps (rows >= L are 0): out[s][i - i0][0 .. width), width >= i1. */
+void mfo_qk_rows(const void* Q, const void* K, int dtype, int L, int h_s, int h_kv, int d,
+                 int i0, int i1, int64_t width, double scale, double* out) {
+  double* z = (double*)malloc(sizeof(double) * (size_t)(i1 > 0 ? i1 : 1));
+  for (int64_t e = 0; e < (int64_t)h_s * (i1 - i0) * width; ++e) out[e] = 0.0;
+  for (int s = 0; s < h_s; ++s)
+    for (int i = i0; i < i1 && i < L; ++i)
+      qk_row(Q, K, dtype, h_s, h_kv, d, s, i, scale, z, out + ((int64_t)s * (i1 - i0) + (i - i0)) * width);
+  free(z);
 }
