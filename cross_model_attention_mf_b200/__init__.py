@@ -6,6 +6,7 @@ this package fails loudly when libmf.so is missing; there is no fallback.
 
 Functions mirror the C entry points:
     mf_compress(...)        -> BSR (row_ptr, col_idx, values, nnz)
+    mf_compress_qk(...)     -> BSR, straight from the sender's Q and K (no dense map)
     mf_map_retrieve(...)    -> O
     mf_map_retrieve_multi(...) -> [O]   (one sender, several receivers)
     mf_get_status()         -> (status, bits)
@@ -46,6 +47,14 @@ class CompressDesc(ctypes.Structure):
                 ("capacity_blocks", _I64), ("nnz_out", _P), ("block_mass_out", _P)]
 
 
+class CompressQkDesc(ctypes.Structure):
+    _fields_ = [("Q", _P), ("K", _P), ("dtype", ctypes.c_int), ("cu_seqlens", _P),
+                ("nseq", _I32), ("max_seqlen", _I32), ("T", _I64), ("h_s", _I32), ("h_kv", _I32),
+                ("d", _I32), ("scale", ctypes.c_float), ("B", _I32), ("tau", ctypes.c_double),
+                ("row_ptr", _P), ("col_idx", _P), ("values", _P), ("capacity_blocks", _I64),
+                ("nnz_out", _P), ("block_mass_out", _P), ("lse_out", _P)]
+
+
 class BsrDesc(ctypes.Structure):
     _fields_ = [("row_ptr", _P), ("col_idx", _P), ("values", _P), ("capacity_blocks", _I64)]
 
@@ -74,6 +83,10 @@ _lib.mf_compress.argtypes = [ctypes.POINTER(CompressDesc), _P, ctypes.c_size_t, 
 _lib.mf_compress.restype = ctypes.c_int
 _lib.mf_compress_static.argtypes = [ctypes.POINTER(CompressDesc), _P]
 _lib.mf_compress_static.restype = ctypes.c_int
+_lib.mf_compress_qk_workspace_size.argtypes = [ctypes.POINTER(CompressQkDesc), ctypes.POINTER(ctypes.c_size_t)]
+_lib.mf_compress_qk_workspace_size.restype = ctypes.c_int
+_lib.mf_compress_qk.argtypes = [ctypes.POINTER(CompressQkDesc), _P, ctypes.c_size_t, _P]
+_lib.mf_compress_qk.restype = ctypes.c_int
 _lib.mf_map_retrieve.argtypes = [ctypes.POINTER(RetrieveDesc), _P]
 _lib.mf_map_retrieve.restype = ctypes.c_int
 _lib.mf_map_retrieve_multi.argtypes = [ctypes.POINTER(RetrieveDesc), ctypes.c_int, _P]
@@ -189,6 +202,41 @@ def mf_compress(maps: torch.Tensor, map_seq_offset: torch.Tensor, cu_seqlens: to
         workspace = torch.empty(need.value, dtype=torch.uint8, device=maps.device)
     _check(_lib.mf_compress(ctypes.byref(d), _ptr(workspace), workspace.numel(), _stream(stream)))
     return out
+
+
+def _compress_qk_desc(Q, K, cu_seqlens, max_seqlen, B, tau, out: BSR, scale=0.0, lse=None):
+    return CompressQkDesc(_ptr(Q), _ptr(K), _dt(Q), _ptr(cu_seqlens), cu_seqlens.numel() - 1,
+                          int(max_seqlen), Q.shape[0], Q.shape[1], K.shape[1], Q.shape[2],
+                          float(scale), int(B), float(tau), _ptr(out.row_ptr), _ptr(out.col_idx),
+                          _ptr(out.values), out.capacity, _ptr(out.nnz), _ptr(out.block_mass),
+                          _ptr(lse))
+
+
+def mf_compress_qk(Q: torch.Tensor, K: torch.Tensor, cu_seqlens: torch.Tensor, max_seqlen: int,
+                   B: int, tau: float, out: BSR, scale: float = 0.0,
+                   lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                   stream=None) -> BSR:
+    """Enqueue compression straight from the sender's Q [T, h_s, d] and K [T, h_kv, d]
+    (bfloat16) into `out` (values bfloat16); scale 0 means 1 / sqrt(d); lse (optional float32
+    [h_s, T]) receives each row's log2-sum-exp of the scaled scores."""
+    d = _compress_qk_desc(Q, K, cu_seqlens, max_seqlen, B, tau, out, scale, lse)
+    need = ctypes.c_size_t(0)
+    _check(_lib.mf_compress_qk_workspace_size(ctypes.byref(d), ctypes.byref(need)))
+    if workspace is None:
+        workspace = torch.empty(need.value, dtype=torch.uint8, device=Q.device)
+    _check(_lib.mf_compress_qk(ctypes.byref(d), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+def mf_compress_qk_workspace_size(nseq: int, max_seqlen: int, T: int, h_s: int, h_kv: int,
+                                  capacity: int, B: int = 64, d: int = 128) -> int:
+    desc = CompressQkDesc()
+    desc.Q = desc.K = desc.cu_seqlens = desc.row_ptr = desc.col_idx = desc.values = desc.nnz_out = 256
+    desc.dtype, desc.nseq, desc.max_seqlen, desc.T = MF_BF16, nseq, max_seqlen, T
+    desc.h_s, desc.h_kv, desc.d, desc.B, desc.tau, desc.capacity_blocks = h_s, h_kv, d, B, 0.5, capacity
+    n = ctypes.c_size_t(0)
+    _check(_lib.mf_compress_qk_workspace_size(ctypes.byref(desc), ctypes.byref(n)))
+    return n.value
 
 
 MF_STATIC_WORKSPACE_BYTES = 8 << 20

@@ -1,4 +1,7 @@
-"""Build libmf.so (the C-ABI library) in-tree for sm_100a with nvcc."""
+"""Build libmf.so (the C-ABI library) in-tree for sm_100a with nvcc.
+
+This file imports nothing from the package (whose import needs the built library): load it
+by path with `load_builder()` of the repository's `__graft_entry__`, or run it as a script."""
 import glob
 import os
 import subprocess

@@ -56,7 +56,7 @@ __global__ void k_meta(const int32_t* cu, const int64_t* off, int nseq, int max_
   for (int s = 0; s < nseq; ++s) {
     int64_t L = (int64_t)cu[s + 1] - cu[s];
     if (L < 0 || L > max_seqlen) { st |= ST_INDEX; L = 0; }
-    if ((off[s] * elem_bytes) % 16 != 0 || off[s] < 0) { st |= ST_ALIGN; L = 0; }
+    if (off && ((off[s] * elem_bytes) % 16 != 0 || off[s] < 0)) { st |= ST_ALIGN; L = 0; }
     const int64_t nqb = (L + B - 1) / B;
     int64_t* m = meta + META_HDR + 4 * s;
     m[0] = L; m[1] = nqb; m[2] = rows; m[3] = cb;
@@ -392,20 +392,9 @@ cudaError_t launch_typed(const mf_compress_desc& d, const CompressWs& ws, uint32
   const int grid_stats = (int)std::min<int64_t>(ws.max_cb, (int64_t)sms * 8);
   k_stats<T, B, NT><<<grid_stats, NT, 0, st>>>(maps, d.map_seq_offset, ws.meta, d.nseq, d.h_s,
                                                 mass);
-  int64_t nqb_max = (d.max_seqlen + B - 1) / B;
-  int n2 = 1;
-  while (n2 < nqb_max) n2 <<= 1;
-  const size_t smem_sel = (size_t)n2 * (sizeof(uint64_t) + sizeof(int));
-  if (smem_sel > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k_select<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem_sel);
-    if (e != cudaSuccess) return e;
-  }
-  k_select<128><<<(unsigned)ws.max_rows, 128, smem_sel, st>>>(ws.meta, d.nseq, mass, d.tau,
-                                                              ws.counts, ws.kept_local);
-  k_scan_compact<<<1, SCAN_NT, 0, st>>>(ws.meta, d.nseq, ws.counts, ws.kept_local, d.row_ptr,
-                                        d.col_idx, ws.kept_row, d.nnz_out, d.capacity_blocks,
-                                        status);
+  cudaError_t e = launch_select(ws, d.nseq, d.max_seqlen, B, mass, d.tau, d.row_ptr, d.col_idx,
+                                d.nnz_out, d.capacity_blocks, status, st);
+  if (e != cudaSuccess) return e;
   const int grid_g = (int)std::max<int64_t>(
       1, std::min<int64_t>(std::max<int64_t>(d.capacity_blocks, 1) * d.h_s, (int64_t)sms * 8));
   k_gather<T, B, NT><<<grid_g, NT, 0, st>>>(maps, d.map_seq_offset, ws.meta, d.nseq, d.h_s,
@@ -417,6 +406,33 @@ cudaError_t launch_typed(const mf_compress_desc& d, const CompressWs& ws, uint32
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace
+
+cudaError_t launch_meta(const int32_t* cu, const int64_t* off, int nseq, int max_seqlen, int B,
+                        int elem_bytes, const CompressWs& ws, uint32_t* status, int32_t* row_ptr,
+                        int32_t* nnz_out, cudaStream_t st) {
+  k_meta<<<1, 32, 0, st>>>(cu, off, nseq, max_seqlen, B, elem_bytes, ws.meta, status, row_ptr,
+                           nnz_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const CompressWs& ws, int nseq, int max_seqlen, int B, const double* mass,
+                          double tau, int32_t* row_ptr, int32_t* col_idx, int32_t* nnz_out,
+                          int64_t capacity, uint32_t* status, cudaStream_t st) {
+  const int64_t nqb_max = (max_seqlen + B - 1) / B;
+  int n2 = 1;
+  while (n2 < nqb_max) n2 <<= 1;
+  const size_t smem_sel = (size_t)n2 * (sizeof(uint64_t) + sizeof(int));
+  if (smem_sel > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k_select<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem_sel);
+    if (e != cudaSuccess) return e;
+  }
+  k_select<128><<<(unsigned)ws.max_rows, 128, smem_sel, st>>>(ws.meta, nseq, mass, tau, ws.counts,
+                                                              ws.kept_local);
+  k_scan_compact<<<1, SCAN_NT, 0, st>>>(ws.meta, nseq, ws.counts, ws.kept_local, row_ptr, col_idx,
+                                        ws.kept_row, nnz_out, capacity, status);
+  return cudaGetLastError();
+}
 
 size_t compress_ws_layout(const mf_compress_desc& d, CompressWs* ws, void* base) {
   const int64_t nqb_max = (d.max_seqlen + d.B - 1) / d.B;
@@ -447,8 +463,9 @@ cudaError_t launch_compress(const mf_compress_desc& d, const CompressWs& ws, uin
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int elem = d.dtype == MF_F32 ? 4 : 2;
-  k_meta<<<1, 32, 0, st>>>(d.cu_seqlens, d.map_seq_offset, d.nseq, d.max_seqlen, d.B, elem,
-                           ws.meta, status, d.row_ptr, d.nnz_out);
+  cudaError_t e = launch_meta(d.cu_seqlens, d.map_seq_offset, d.nseq, d.max_seqlen, d.B, elem, ws,
+                              status, d.row_ptr, d.nnz_out, st);
+  if (e != cudaSuccess) return e;
   if (d.dtype == MF_F32) {
     if (d.B == 32) return launch_typed<float, 32>(d, ws, status, st, sms);
     if (d.B == 64) return launch_typed<float, 64>(d, ws, status, st, sms);

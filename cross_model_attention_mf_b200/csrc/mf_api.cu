@@ -4,6 +4,7 @@
 
 #include <cstdio>
 #include <mutex>
+#include <cmath>
 #include <string>
 
 #include "mf.h"
@@ -152,6 +153,29 @@ bool can_fuse(const mf_retrieve_desc* ds, int n) {
   return true;
 }
 
+mf_status check_compress_qk(const mf_compress_qk_desc* d) {
+  if (!d) return fail(MF_ERR_INVALID, "desc is NULL");
+  if (!d->Q || !d->K || !d->cu_seqlens || !d->row_ptr || !d->nnz_out ||
+      (d->capacity_blocks > 0 && (!d->col_idx || !d->values)))
+    return fail(MF_ERR_INVALID, "a required pointer is NULL");
+  if (d->nseq < 1) return fail(MF_ERR_INVALID, "nseq must be >= 1");
+  if (d->max_seqlen < 0 || d->T < 0) return fail(MF_ERR_INVALID, "max_seqlen and T must be >= 0");
+  if (d->h_s < 1 || d->h_s > 256 || d->h_kv < 1 || d->h_s % d->h_kv != 0)
+    return fail(MF_ERR_INVALID, "h_s must be in [1, 256] and a multiple of h_kv");
+  if (!(d->tau >= 0.0 && d->tau <= 1.0)) return fail(MF_ERR_INVALID, "tau must be in [0, 1]");
+  if (d->capacity_blocks < 0) return fail(MF_ERR_INVALID, "capacity_blocks must be >= 0");
+  if (!(d->scale >= 0.0f) || std::isinf(d->scale)) return fail(MF_ERR_INVALID, "scale must be finite and >= 0");
+  if (d->dtype != MF_BF16) return fail(MF_ERR_UNSUPPORTED, "mf_compress_qk takes bfloat16 Q and K");
+  if (d->d != 128) return fail(MF_ERR_UNSUPPORTED, "mf_compress_qk needs d = 128");
+  if (d->B != 64) return fail(MF_ERR_UNSUPPORTED, "mf_compress_qk needs B = 64");
+  if (d->T >= ((int64_t)1 << 31) - 256) return fail(MF_ERR_UNSUPPORTED, "T too large");
+  if ((d->max_seqlen + 63) / 64 > 4096) return fail(MF_ERR_UNSUPPORTED, "more than 4096 query blocks per sequence");
+  if ((reinterpret_cast<uintptr_t>(d->Q) | reinterpret_cast<uintptr_t>(d->K) |
+       reinterpret_cast<uintptr_t>(d->values)) % 16)
+    return fail(MF_ERR_INVALID, "Q, K and values must be 16-byte aligned");
+  return MF_OK;
+}
+
 mf_status check_calib(const mf_calib_desc* d) {
   if (!d) return fail(MF_ERR_INVALID, "desc is NULL");
   if (!is_dtype(d->dtype)) return fail(MF_ERR_INVALID, "dtype must be MF_F32 or MF_BF16");
@@ -190,6 +214,7 @@ size_t mf_abi_struct_size(int which) {
     case 1: return sizeof(mf_bsr);
     case 2: return sizeof(mf_retrieve_desc);
     case 3: return sizeof(mf_calib_desc);
+    case 4: return sizeof(mf_compress_qk_desc);
     default: return 0;
   }
 }
@@ -242,6 +267,33 @@ mf_status mf_compress_static(const mf_compress_desc* desc, void* stream) {
   cudaError_t e = mfi::launch_compress(*desc, ws, st, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess)
     return fail(MF_ERR_CUDA, std::string("mf_compress_static launch: ") + cudaGetErrorString(e));
+  return MF_OK;
+}
+
+mf_status mf_compress_qk_workspace_size(const mf_compress_qk_desc* desc, size_t* bytes) {
+  if (!bytes) return fail(MF_ERR_INVALID, "bytes is NULL");
+  mf_status s = check_compress_qk(desc);
+  if (s != MF_OK) return s;
+  *bytes = mfi::compress_qk_ws_layout(*desc, nullptr, nullptr, nullptr);
+  return MF_OK;
+}
+
+mf_status mf_compress_qk(const mf_compress_qk_desc* desc, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  mf_status s = check_compress_qk(desc);
+  if (s != MF_OK) return s;
+  const size_t need = mfi::compress_qk_ws_layout(*desc, nullptr, nullptr, nullptr);
+  if (!workspace || workspace_bytes < need)
+    return fail(MF_ERR_INVALID, "workspace missing or smaller than mf_compress_qk_workspace_size");
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(MF_ERR_INVALID, "workspace must be 256-byte aligned");
+  uint32_t* st = status_ptr();
+  if (!st) return fail(MF_ERR_CUDA, "cannot resolve the device status word");
+  mfi::CompressWs ws;
+  mfi::QkWs q;
+  mfi::compress_qk_ws_layout(*desc, &ws, &q, workspace);
+  std::string err;
+  if (!mfi::launch_compress_qk(*desc, ws, q, st, static_cast<cudaStream_t>(stream), &err))
+    return fail(MF_ERR_CUDA, "mf_compress_qk: " + err);
   return MF_OK;
 }
 

@@ -37,6 +37,25 @@ size_t compress_ws_layout(const mf_compress_desc& d, CompressWs* ws, void* base)
 cudaError_t launch_compress(const mf_compress_desc& d, const CompressWs& ws, uint32_t* status,
                             cudaStream_t st);
 
+// the geometry pass of compression (per-sequence meta; off may be NULL: no map offsets)
+cudaError_t launch_meta(const int32_t* cu, const int64_t* off, int nseq, int max_seqlen, int B,
+                        int elem_bytes, const CompressWs& ws, uint32_t* status, int32_t* row_ptr,
+                        int32_t* nnz_out, cudaStream_t st);
+// selection and BSR index build from the masses of every causal block
+cudaError_t launch_select(const CompressWs& ws, int nseq, int max_seqlen, int B, const double* mass,
+                          double tau, int32_t* row_ptr, int32_t* col_idx, int32_t* nnz_out,
+                          int64_t capacity, uint32_t* status, cudaStream_t st);
+
+// scratch of mf_compress_qk beyond CompressWs
+struct QkWs {
+  float2* ml;         // [h_s][cb_stride][B] per-block max and exp-sum of each row
+  float* lse2;        // [h_s][T] row log2-sum-exp
+  int64_t cb_stride;  // causal-block capacity of the pack
+};
+size_t compress_qk_ws_layout(const mf_compress_qk_desc& d, CompressWs* ws, QkWs* q, void* base);
+bool launch_compress_qk(const mf_compress_qk_desc& d, const CompressWs& ws, const QkWs& q,
+                        uint32_t* status, cudaStream_t st, std::string* err);
+
 // one receiver layer's pointers
 struct RetrieveLayer {
   const int32_t* row_ptr;

@@ -140,6 +140,57 @@ mf_status mf_compress(const mf_compress_desc* desc, void* workspace, size_t work
 mf_status mf_compress_static(const mf_compress_desc* desc, void* stream);
 
 /* ------------------------------------------------------------------------------
+ * mf_compress_qk: compression straight from the sender's queries and keys, with no
+ * dense map anywhere (MapFlow page "MapFlow开源:大模型换班,Prefill为何能快20%?",
+ * section "存不下、读得慢?三个工程优化手段", subsection 1: block statistics are
+ * computed first, then the kept blocks, without assembling the dense matrix).
+ * The map of sender head s is its causal attention distribution
+ *   A_s[i][j] = exp(scale q_{i,s} . k_{j,g}) / sum_{j' <= i} exp(scale q_{i,s} . k_{j',g}),
+ * j <= i < L, g = floor(s * h_kv / h_s).  Three passes over the causal key blocks:
+ *   1. per (row, key block, head): the block's max scaled score and exp-sum (tensor cores
+ *      for q.k), to a scratch buffer;
+ *   2. per row: the log-sum-exp; per causal block: the head-summed mass (float64, fixed
+ *      order); then selection and row_ptr / col_idx exactly as mf_compress does;
+ *   3. the kept blocks only: A recomputed and written as bfloat16 values.
+ * Output layout, capacity handling and block_mass_out are those of mf_compress (values
+ * bfloat16).  lse_out (optional, float device [h_s][T]) receives each row's log2-sum-exp
+ * of the scores scaled by scale * log2(e).
+ * Requirements: dtype MF_BF16; d = 128; B = 64; h_s a multiple of h_kv; Q and K
+ * 16-byte aligned.  Q: [T][h_s][d], K: [T][h_kv][d] (varlen pack by cu_seqlens, T = total
+ * tokens, HOST value), both bfloat16 device.
+ * ------------------------------------------------------------------------------ */
+typedef struct {
+  const void* Q;                   /* device [T][h_s][d] bf16 */
+  const void* K;                   /* device [T][h_kv][d] bf16 */
+  mf_dtype dtype;                  /* MF_BF16 */
+  const int32_t* cu_seqlens;       /* device [nseq + 1] */
+  int32_t nseq;                    /* >= 1 */
+  int32_t max_seqlen;              /* host bound: every L_s <= max_seqlen */
+  int64_t T;                       /* host: total tokens (cu_seqlens[nseq]) */
+  int32_t h_s, h_kv, d;            /* sender query heads, key heads, head dim */
+  float scale;                     /* softmax scale; 0 means 1 / sqrt(d) */
+  int32_t B;                       /* block size (64) */
+  double tau;                      /* cumulative-mass threshold */
+  int32_t* row_ptr;                /* device out [R + 1] */
+  int32_t* col_idx;                /* device out [capacity_blocks] */
+  void* values;                    /* device out [capacity_blocks][h_s][B][B] bf16 */
+  int64_t capacity_blocks;
+  int32_t* nnz_out;                /* device out [1] */
+  double* block_mass_out;          /* device out, optional (NULL) */
+  float* lse_out;                  /* device out, optional (NULL) [h_s][T] */
+} mf_compress_qk_desc;
+
+/* Scratch bytes of mf_compress_qk (an upper bound from nseq, max_seqlen, T, h_s and
+ * capacity_blocks; the per-block statistics take h_s * causal blocks * B * 8 bytes). */
+mf_status mf_compress_qk_workspace_size(const mf_compress_qk_desc* desc, size_t* bytes);
+
+/* Enqueue compression from Q and K.  workspace as for mf_compress.  Errors: MF_ERR_INVALID
+ * for a bad descriptor, MF_ERR_UNSUPPORTED outside the requirements, MF_ERR_CUDA for a
+ * launch failure; device-side conditions through mf_get_status. */
+mf_status mf_compress_qk(const mf_compress_qk_desc* desc, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* ------------------------------------------------------------------------------
  * Fused retrieval for receiver layers l = l_r_begin .. l_r_end-1.
  *
  * Receiver layer l reads sender layer layer_map[l] (a BSR from mf_compress).  For
@@ -289,7 +340,7 @@ const char* mf_version(void);
 
 /* sizeof of this header's structs as the library was compiled, for bindings that
  * mirror them: which = 0 mf_compress_desc, 1 mf_bsr, 2 mf_retrieve_desc,
- * 3 mf_calib_desc.
+ * 3 mf_calib_desc, 4 mf_compress_qk_desc.
  * Returns 0 for any other value. */
 size_t mf_abi_struct_size(int which);
 

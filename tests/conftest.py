@@ -10,6 +10,9 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    # (re)build libmf.so before any test imports the package, which loads it
+    import __graft_entry__
+    __graft_entry__.load_builder().build()
 
 
 def pytest_collection_modifyitems(config, items):

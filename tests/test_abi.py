@@ -11,8 +11,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def mf():
-    from cross_model_attention_mf_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.load_builder().build()
     import cross_model_attention_mf_b200 as mf
     return mf
 
@@ -180,3 +180,28 @@ def test_retrieve_multi_fusing_rules(mf):
     assert mf._lib.mf_map_retrieve_multi(many(base), 0, None) == mf.MF_ERR_INVALID
     assert mf._lib.mf_map_retrieve_multi(many(base, _retrieve_desc(mf, arr, lm, d=0)), 2,
                                          None) == mf.MF_ERR_INVALID
+
+
+def test_compress_qk_descriptor_and_validation(mf):
+    """The binding fills every field of mf_compress_qk_desc; the host checks reject what the
+    kernels do not take, before any launch."""
+    import torch
+    Q = torch.zeros(100, 8, 128, dtype=torch.bfloat16)
+    K = torch.zeros(100, 2, 128, dtype=torch.bfloat16)
+    cu = torch.tensor([0, 60, 100], dtype=torch.int32)
+    out = mf.alloc_bsr(2, 4, 8, 64, torch.bfloat16, "cpu", n_causal=4)
+    d = mf._compress_qk_desc(Q, K, cu, 60, 64, 0.9, out)
+    assert (d.Q, d.K, d.cu_seqlens) == (Q.data_ptr(), K.data_ptr(), cu.data_ptr())
+    assert (d.nseq, d.max_seqlen, d.T, d.h_s, d.h_kv, d.d, d.B) == (2, 60, 100, 8, 2, 128, 64)
+    assert d.dtype == mf.MF_BF16 and d.capacity_blocks == 4 and d.block_mass_out == out.block_mass.data_ptr()
+    n = ctypes.c_size_t(0)
+    assert mf._lib.mf_compress_qk_workspace_size(ctypes.byref(d), ctypes.byref(n)) == mf.MF_OK
+    assert n.value >= 8 * 2 * 64 * 8  # (m, l) of every (head, causal block, row)
+    for field, value, rc in [("d", 64, mf.MF_ERR_UNSUPPORTED), ("B", 32, mf.MF_ERR_UNSUPPORTED),
+                             ("dtype", mf.MF_F32, mf.MF_ERR_UNSUPPORTED), ("h_kv", 3, mf.MF_ERR_INVALID),
+                             ("tau", 1.5, mf.MF_ERR_INVALID), ("nseq", 0, mf.MF_ERR_INVALID),
+                             ("scale", -1.0, mf.MF_ERR_INVALID)]:
+        bad = mf._compress_qk_desc(Q, K, cu, 60, 64, 0.9, out)
+        setattr(bad, field, value)
+        assert mf._lib.mf_compress_qk(ctypes.byref(bad), ctypes.c_void_p(4096), 1 << 30, None) == rc, field
+    assert mf._lib.mf_abi_struct_size(4) == ctypes.sizeof(mf.CompressQkDesc)
