@@ -222,6 +222,10 @@ def run_ours(args, rank, world, dev):
     if rank == 0 and not args.no_e2e:
         e2e = run_e2e(args, w, mf, pack, W, V, bsr, ws, O, qbase, dev)
 
+    cqk = None
+    if rank == 0 and not args.no_qk:
+        cqk = run_compress_qk(w, mf, dev, qk_len=args.qk_len)
+
     multi = None
     if rank == 0 and not args.no_multi:
         multi = run_multi(w, mf, bsr, nnz, qbase, dev)
@@ -231,7 +235,7 @@ def run_ours(args, rank, world, dev):
         calib = run_calib(w, mf, pack, dev, args.calib_len)
 
     return dict(w=w, nnz=nnz, elapsed=elapsed, t_comp=t_comp, t_ret=t_ret, clocks=clk.summary(),
-                e2e=e2e, calib=calib, multi=multi)
+                e2e=e2e, calib=calib, multi=multi, cqk=cqk)
 
 
 def run_calib(w, mf, pack, dev, calib_len=0, reps=5):
@@ -330,6 +334,59 @@ def run_multi(w, mf, bsr, nnz, qbase, dev, reps=20):
             "GB/s": b_shared / t_sh / 1e9, "reps": reps}
 
 
+MUFU_PER_SM_CLK = 16  # exp2 results per SM per clock (special-function units)
+
+
+def run_compress_qk(w, mf, dev, reps=5, qk_len=0):
+    """Compression from the sender's Q, K (no dense map) on the workload's sequence lengths,
+    sender heads h_s over h_kv key heads, d = 128, tau of the workload; CUDA events around the
+    whole call (stats, reduce, selection, gather).  Work: the Q.K^T products of every causal
+    64-key tile (2 d flops per score) and one exponential per causal score; both passes of the
+    kept blocks are counted separately."""
+    from synth.qk import gen_qk
+    if qk_len:
+        w = w.with_(lens=(qk_len,))
+    Q, K = gen_qk(w.lens, w.h_s, w.h_kv, 128, w.n_heavy, w.seed)
+    Q, K = Q.to(dev), K.to(dev)
+    cu = torch.tensor([0] + list(np.cumsum(w.lens)), dtype=torch.int32, device=dev)
+    out = mf.alloc_bsr(sum(w.nqb), w.causal_blocks, w.h_s, w.B, torch.bfloat16, dev)
+    need = mf.mf_compress_qk_workspace_size(len(w.lens), max(w.lens), w.tokens, w.h_s, w.h_kv,
+                                            w.causal_blocks)
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+    for _ in range(2):
+        mf.mf_compress_qk(Q, K, cu, max(w.lens), w.B, w.tau, out, workspace=ws)
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        mf.mf_compress_qk(Q, K, cu, max(w.lens), w.B, w.tau, out, workspace=ws)
+        e1.record(st)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e-3)
+    rc, bits = mf.mf_get_status()
+    if rc != mf.MF_OK:
+        raise RuntimeError(f"compress_qk status {rc} bits {bits:#x}")
+    nnz = int(out.nnz.cpu()[0])
+    t = statistics.median(ts)
+    # causal 64-key tiles of the stats pass: per 128-row query tile qt, key blocks 0 .. 2qt+1
+    tiles = 0
+    for n in w.nqb:
+        for qt in range(-(-n // 2)):
+            tiles += min(2 * qt + 2, n)
+    flops_stats = tiles * w.h_s * 2.0 * 128 * 64 * 128
+    flops_gather = nnz * w.h_s * 2.0 * 64 * 64 * 128 * 2  # the 128-row tile covers two blocks
+    scores = w.h_s * sum(L * (L + 1) // 2 for L in w.lens)
+    del Q, K, ws, out
+    torch.cuda.empty_cache()
+    return {"kernel": "mf_compress_qk (k_qk stats + k_qk_reduce + selection + k_qk gather)",
+            "workload": f"lens={list(w.lens)} h_s={w.h_s} h_kv={w.h_kv} d=128 B={w.B} tau={w.tau}",
+            "ms": t * 1e3, "nnz": nnz, "density": nnz / w.causal_blocks, "reps": reps,
+            "tokens_per_s_layer": w.tokens / t,
+            "flops": flops_stats + flops_gather, "TFLOP/s": (flops_stats + flops_gather) / t / 1e12,
+            "exp": scores + nnz * w.h_s * 64 * 64, "exp/s": (scores + nnz * w.h_s * 64 * 64) / t}
+
+
 def run_e2e(args, w, mf, pack, W, V, bsr, ws, O, qbase, dev):
     h_maps = torch.empty(pack.maps.shape, dtype=pack.maps.dtype, pin_memory=True)
     h_maps.copy_(pack.maps)
@@ -419,6 +476,11 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-qk", action="store_true", help="skip the compression-from-Q,K line")
+    ap.add_argument("--qk-len", type=int, default=0,
+                    help="sequence length of the compression-from-Q,K line (0: the workload's)")
+    ap.add_argument("--qk-only", action="store_true",
+                    help="print only the compression-from-Q,K measurement (profiling runs)")
     ap.add_argument("--no-multi", action="store_true", help="skip the several-receivers line")
     ap.add_argument("--no-calib", action="store_true", help="skip the head-map calibration line")
     ap.add_argument("--calib-len", type=int, default=0,
@@ -468,6 +530,10 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
+    if args.qk_only:
+        import cross_model_attention_mf_b200 as mf
+        print(json.dumps({"compress_qk": run_compress_qk(w, mf, dev, qk_len=args.qk_len)}), flush=True)
+        return
     res = run_ours(args, rank, world, dev)
     if rank == 0:
         hbm, tf_burst, tf_sus, src = peaks()
@@ -513,6 +579,16 @@ def main():
         }
         if res["e2e"] is not None:
             line["e2e"] = res["e2e"]
+        if res["cqk"] is not None:
+            c = res["cqk"]
+            sm_mhz = (res["clocks"] or {}).get("sm_mhz") or 1965.0
+            mufu = MUFU_PER_SM_CLK * torch.cuda.get_device_properties(0).multi_processor_count * sm_mhz * 1e6
+            c.update({"bound": "alu", "unit": "exp/s", "achieved": c["exp/s"], "peak": mufu,
+                      "frac": c["exp/s"] / mufu,
+                      "peak_source": f"{MUFU_PER_SM_CLK} exp2 per SM per clock x SMs x median SM clock",
+                      "tensor_frac": c["TFLOP/s"] / tf_burst,
+                      "tensor_peak_source": f"{src} (bf16_tflops burst)"})
+            line["compress_qk"] = c
         if res["multi"] is not None:
             m = res["multi"]
             m.update({"bound": "hbm", "peak": hbm, "unit": "GB/s", "frac": m["GB/s"] / hbm,

@@ -14,9 +14,9 @@
 //                         (tcgen05, M=128 N=64 K=16 x 8, Q and K tiles by TMA, 128-byte
 //                         swizzle, S double-buffered in TMEM), then one thread per row takes
 //                         the block's max m and exp-sum l = sum 2^(x - m) (causal mask on the
-//                         diagonal block) and stores (m, l).
-//   k_qk_reduce           one CTA per query block: lse per (head, row) from its (m, l) pairs,
-//                         then every causal block's head-summed mass
+//                         diagonal block), stores (m, l) and folds it into the row's running
+//                         lse, stored once the item has walked all the row's blocks.
+//   k_qk_mass             one CTA per causal block: the head-summed mass
 //                         sum_{s, i} l 2^(m - lse) in float64, fixed order.  Selection and
 //                         row_ptr / col_idx then run exactly as for dense maps.
 //   k_qk<true> (gather)   the same item walk over the kept blocks of the item's two query
@@ -161,6 +161,12 @@ __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t bdesc, uint
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
       "l"(a), "l"(bdesc), "r"(idesc), "r"(acc)
       : "memory");
+}
+// 2^x on the special-function unit (ex2.approx.ftz: results below 2^-126 flush to 0; 2^-inf = 0)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 // K-major operand, 128-byte swizzle: 8-row groups 1024 bytes apart
 __device__ __forceinline__ uint64_t kmajor_sw128(uint32_t addr) {
@@ -415,9 +421,11 @@ __global__ void __launch_bounds__(QT, 2)
       const QItem it = qdecode(p, idx);
       if (!it.valid) continue;
       const int i = QROWS * it.qt + r, qb = it.qb0 + (r >> 6), ii = r & 63;
-      const bool row_ok = i < it.L && it.t0 + i < p.T;  // (cu_seqlens beyond T: ST_INDEX below)
+      const bool row_ok = i < it.L && it.t0 + i < p.T;
+      if (!GATHER && i < it.L && !row_ok) atomicOr(p.status, ST_INDEX);  // cu_seqlens past T
       float lse = 0.0f;
       if (GATHER && row_ok) lse = p.lse2[(int64_t)it.head * p.T + it.t0 + i];
+      float run_m = -INFINITY, run_s = 0.0f;  // stats: the row's running max and exp-sum
       TileIt ti;
       tiles_begin<GATHER>(p, it, ti);
       int kb;
@@ -438,22 +446,33 @@ __global__ void __launch_bounds__(QT, 2)
         if (lane == 0) bar_arrive(bar(B_SEMPTY + b));
         ++tc;
         const bool diag = kb == qb;
+        float sv[64];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          sv[c] = __uint_as_float(v0[c]);
+          sv[c + 32] = __uint_as_float(v1[c]);
+        }
+        if (diag || !row_ok) {  // keys j > i (and every key of a row past the sequence) drop out
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (!row_ok || c > ii) sv[c] = -INFINITY;
+        }
         if (!GATHER) {
           if (row_ok && kb <= qb) {
-            float mx = -INFINITY;
+            // max of the raw scores (scaling by c2 > 0 keeps the order), four chains
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (!diag || c <= ii) mx = fmaxf(mx, __uint_as_float(v0[c]) * p.c2);
-              if (!diag || c + 32 <= ii) mx = fmaxf(mx, __uint_as_float(v1[c]) * p.c2);
-            }
-            float l = 0.0f;
+            for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
+            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.c2;
+            float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (!diag || c <= ii) l += exp2f(__uint_as_float(v0[c]) * p.c2 - mx);
-              if (!diag || c + 32 <= ii) l += exp2f(__uint_as_float(v1[c]) * p.c2 - mx);
-            }
+            for (int c = 0; c < 64; ++c) l4[c & 3] += ex2(fmaf(sv[c], p.c2, -mx));
+            const float l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
             const int64_t cb = it.cb0 + (int64_t)qb * (qb + 1) / 2 + kb;
             p.ml[((int64_t)it.head * p.cb_stride + cb) * KB + ii] = make_float2(mx, l);
+            const float nm = fmaxf(run_m, mx);
+            run_s = run_s * ex2(run_m - nm) + l * ex2(mx - nm);
+            run_m = nm;
           }
         } else {
           const int64_t n = r < 64 ? n0 : n1;
@@ -465,14 +484,9 @@ __global__ void __launch_bounds__(QT, 2)
               uint32_t w[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                float a[2];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                  const int c = 8 * c8 + 2 * e + h;
-                  const float sv = __uint_as_float(c < 32 ? v0[c & 31] : v1[c & 31]);
-                  a[h] = (row_ok && (!diag || c <= ii)) ? exp2f(sv * p.c2 - lse) : 0.0f;
-                }
-                const __nv_bfloat162 pk = __floats2bfloat162_rn(a[0], a[1]);
+                const int c = 8 * c8 + 2 * e;
+                const __nv_bfloat162 pk = __floats2bfloat162_rn(ex2(fmaf(sv[c], p.c2, -lse)),
+                                                                ex2(fmaf(sv[c + 1], p.c2, -lse)));
                 w[e] = *reinterpret_cast<const uint32_t*>(&pk);
               }
               dst[c8] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -480,6 +494,8 @@ __global__ void __launch_bounds__(QT, 2)
           }
         }
       }
+      // the item walked every causal key block of its rows: the row's log2-sum-exp
+      if (!GATHER && ok && row_ok) p.lse2[(int64_t)it.head * p.T + it.t0 + i] = run_m + log2f(run_s);
     }
   }
   fence_before();
@@ -491,63 +507,52 @@ __global__ void __launch_bounds__(QT, 2)
   }
 }
 
-// ------------------------------------------------------------------ lse and masses
-__device__ inline int find_row_seq(const int64_t* meta, int nseq, int64_t row) {
-  int lo = 0, hi = nseq - 1;  // last s whose first row is <= row
+// ------------------------------------------------------------------ masses
+__device__ inline int find_cb_seq(const int64_t* meta, int nseq, int64_t cb) {
+  int lo = 0, hi = nseq - 1;  // last s whose first causal block is <= cb
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (meta[META_HDR + 4 * mid + 2] <= row) lo = mid; else hi = mid - 1;
+    if (meta[META_HDR + 4 * mid + 3] <= cb) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
+__device__ inline int tri_row_of(int64_t c) {  // q with q (q + 1) / 2 <= c < (q + 1) (q + 2) / 2
+  int q = (int)((sqrt(8.0 * (double)c + 1.0) - 1.0) * 0.5);
+  while ((int64_t)(q + 1) * (q + 2) / 2 <= c) ++q;
+  while ((int64_t)q * (q + 1) / 2 > c) --q;
+  return q;
+}
 
-// One CTA per query block.  lse of every (head, row) from the row's (m, l) pairs, then the
-// mass of every causal block of the row: sum over heads and rows of l 2^(m - lse), float64,
-// each lane in a fixed order and the lanes combined by a fixed shuffle tree.
+// One CTA per causal block (qb, kb): mass = sum over heads s and rows i of the block of
+// l 2^(m - lse_i), float64; each thread sums its (head, row) pairs in a fixed order, then a
+// fixed shuffle tree and a fixed pass over the warps.
 constexpr int RT = 256;
-__global__ void __launch_bounds__(RT) k_qk_reduce(const __grid_constant__ QkParams p) {
-  extern __shared__ float s_lse[];  // [h_s][64]
-  const int64_t row = blockIdx.x;
-  if (row >= p.meta[0]) return;
-  const int s = find_row_seq(p.meta, p.nseq, row);
+__global__ void __launch_bounds__(RT) k_qk_mass(const __grid_constant__ QkParams p) {
+  __shared__ double red[RT / 32];
+  const int64_t cb = blockIdx.x;
+  if (cb >= p.meta[1]) return;
+  const int s = find_cb_seq(p.meta, p.nseq, cb);
   const int64_t* m = p.meta + META_HDR + 4 * s;
   const int L = (int)m[0];
-  const int qb = (int)(row - m[2]);
-  const int64_t cb0 = m[3] + (int64_t)qb * (qb + 1) / 2;
-  const int64_t t0 = p.cu[s];
+  const int64_t c = cb - m[3];
+  const int qb = tri_row_of(c);
+  const int64_t t0 = p.cu[s] + (int64_t)KB * qb;
   const int nv = min(KB, L - KB * qb);
-  for (int e = threadIdx.x; e < p.h_s * KB; e += RT) {
-    const int hs = e / KB, ii = e % KB;
-    float lse = -INFINITY;
-    if (ii < nv && t0 + (int64_t)KB * qb + ii >= p.T) {
-      atomicOr(p.status, ST_INDEX);  // cu_seqlens reaches past T
-    } else if (ii < nv) {
-      const float2* src = p.ml + ((int64_t)hs * p.cb_stride + cb0) * KB + ii;
-      float M = -INFINITY;
-      for (int kb = 0; kb <= qb; ++kb) M = fmaxf(M, src[(int64_t)kb * KB].x);
-      double sum = 0.0;
-      for (int kb = 0; kb <= qb; ++kb) {
-        const float2 v = src[(int64_t)kb * KB];
-        sum += (double)v.y * (double)exp2f(v.x - M);
-      }
-      lse = M + (float)log2(sum);
-      p.lse2[(int64_t)hs * p.T + t0 + (int64_t)KB * qb + ii] = lse;
-    }
-    s_lse[e] = lse;
+  double acc = 0.0;
+  for (int e = threadIdx.x; e < p.h_s * nv; e += RT) {
+    const int hs = e / nv, ii = e - hs * nv;
+    if (t0 + ii >= p.T) continue;  // cu_seqlens past T: reported by the stats pass
+    const float2 v = p.ml[((int64_t)hs * p.cb_stride + cb) * KB + ii];
+    acc += (double)v.y * (double)exp2f(v.x - p.lse2[(int64_t)hs * p.T + t0 + ii]);
   }
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pairs = p.h_s * nv;
-  for (int kb = warp; kb <= qb; kb += RT / 32) {
-    double acc = 0.0;
-    for (int e = lane; e < pairs; e += 32) {
-      const int hs = e / nv, ii = e - hs * nv;
-      const float2 v = p.ml[((int64_t)hs * p.cb_stride + cb0 + kb) * KB + ii];
-      acc += (double)v.y * (double)exp2f(v.x - s_lse[hs * KB + ii]);
-    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) p.mass[cb0 + kb] = acc;
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < RT / 32; ++w) t += red[w];
+    p.mass[cb] = t;
   }
 }
 
@@ -653,13 +658,8 @@ bool launch_compress_qk(const mf_compress_qk_desc& d, const CompressWs& ws, cons
   if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
   // 1. (m, l) of every (head, causal block, row)
   k_qk<false><<<grid, QT, QK_SMEM, st>>>(tmQ, tmK, p);
-  // 2. lse and masses, then selection
-  const size_t smem_r = sizeof(float) * (size_t)d.h_s * KB;
-  if (smem_r > 48 * 1024) {
-    e = cudaFuncSetAttribute(k_qk_reduce, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_r);
-    if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
-  }
-  k_qk_reduce<<<(unsigned)ws.max_rows, RT, smem_r, st>>>(p);
+  // 2. masses of every causal block, then selection
+  k_qk_mass<<<(unsigned)ws.max_cb, RT, 0, st>>>(p);
   e = launch_select(ws, d.nseq, d.max_seqlen, d.B, p.mass, d.tau, d.row_ptr, d.col_idx, d.nnz_out,
                     d.capacity_blocks, status, st);
   if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
