@@ -319,46 +319,57 @@ __global__ void __launch_bounds__(QT, 2)
 
   if (warp == 0) {
     // ================================================================ TMA producer
-    if (lane == 0) {
-      bool ok = true;
-      int64_t tc = 0, qi = 0;
-      for (int64_t idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
-        const QItem it = qdecode(p, idx);
-        if (!it.valid) continue;
-        TileIt ti;
-        tiles_begin<GATHER>(p, it, ti);
-        int kb;
-        int64_t n0, n1;
-        bool first = true;
-        const int g = it.head / gq;
-        while (ok && tiles_next<GATHER>(p, it, ti, &kb, &n0, &n1)) {
-          if (first) {
-            if (!(ok = bar_wait(bar(B_QEMPTY), (uint32_t)(qi & 1) ^ 1u, abort_flag, p.status))) break;
+    // the whole warp waits (a warp waiting with all lanes is suspended by the hardware; a lone
+    // polling lane would take issue slots from the row threads); lane 0 issues the copies
+    bool ok = true;
+    int64_t tc = 0, qi = 0;
+    for (int64_t idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
+      const QItem it = qdecode(p, idx);
+      if (!it.valid) continue;
+      TileIt ti;
+      tiles_begin<GATHER>(p, it, ti);
+      int kb;
+      int64_t n0, n1;
+      bool first = true;
+      const int g = it.head / gq;
+      while (ok && tiles_next<GATHER>(p, it, ti, &kb, &n0, &n1)) {
+        if (first) {
+          ok = __all_sync(0xffffffffu, bar_wait(bar(B_QEMPTY), (uint32_t)(qi & 1) ^ 1u, abort_flag,
+                                                p.status));
+          if (!ok) break;
+          if (lane == 0) {
             bar_expect(bar(B_QFULL), Q_BYTES);
             const int row = (int)(it.t0 + (int64_t)QROWS * it.qt);
             tma3(sb + OFF_Q, &tmQ, bar(B_QFULL), 0, it.head, row);
             tma3(sb + OFF_Q + Q_BYTES / 2, &tmQ, bar(B_QFULL), 64, it.head, row);
-            first = false;
-            ++qi;
           }
-          const int st = (int)(tc % KS);
-          if (!(ok = bar_wait(bar(B_KEMPTY + st), (uint32_t)((tc / KS) & 1) ^ 1u, abort_flag,
-                              p.status)))
-            break;
+          __syncwarp();
+          first = false;
+          ++qi;
+        }
+        const int st = (int)(tc % KS);
+        ok = __all_sync(0xffffffffu, bar_wait(bar(B_KEMPTY + st), (uint32_t)((tc / KS) & 1) ^ 1u,
+                                              abort_flag, p.status));
+        if (!ok) break;
+        if (lane == 0) {
           bar_expect(bar(B_KFULL + st), K_BYTES);
           const int key = (int)(it.t0 + (int64_t)KB * kb);
           tma3(sb + OFF_K + st * K_BYTES, &tmK, bar(B_KFULL + st), 0, g, key);
           tma3(sb + OFF_K + st * K_BYTES + K_BYTES / 2, &tmK, bar(B_KFULL + st), 64, g, key);
-          ++tc;
         }
+        __syncwarp();
+        ++tc;
       }
-      // drain: the last copies issued into every stage and into Q
+    }
+    // drain: the last copies issued into every stage and into Q
+    if (lane == 0) {
       for (int s = 0; s < KS; ++s) {
         const int64_t cnt = tc > s ? (tc - s - 1) / KS + 1 : 0;
         if (cnt) bar_drain(bar(B_KFULL + s), (uint32_t)((cnt - 1) & 1));
       }
       if (qi) bar_drain(bar(B_QFULL), (uint32_t)((qi - 1) & 1));
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ================================================================ MMA issue
     bool ok = true;
@@ -459,15 +470,20 @@ __global__ void __launch_bounds__(QT, 2)
         }
         if (!GATHER) {
           if (row_ok && kb <= qb) {
-            // max of the raw scores (scaling by c2 > 0 keeps the order), four chains
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            // max of the raw scores (scaling by c2 > 0 keeps the order), eight chains
+            float m8[8];
 #pragma unroll
-            for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
-            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.c2;
-            float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            for (int k = 0; k < 8; ++k) m8[k] = sv[k];
 #pragma unroll
-            for (int c = 0; c < 64; ++c) l4[c & 3] += ex2(fmaf(sv[c], p.c2, -mx));
-            const float l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], sv[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * p.c2;
+            float l8[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) l8[k] = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) l8[c & 7] += ex2(fmaf(sv[c], p.c2, -mx));
+            const float l = ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
             const int64_t cb = it.cb0 + (int64_t)qb * (qb + 1) / 2 + kb;
             p.ml[((int64_t)it.head * p.cb_stride + cb) * KB + ii] = make_float2(mx, l);
             const float nm = fmaxf(run_m, mx);
@@ -538,12 +554,21 @@ __global__ void __launch_bounds__(RT) k_qk_mass(const __grid_constant__ QkParams
   const int qb = tri_row_of(c);
   const int64_t t0 = p.cu[s] + (int64_t)KB * qb;
   const int nv = min(KB, L - KB * qb);
+  // warp w takes heads w, w + 8, ...; lane l rows 2l and 2l + 1 (one 16-byte load of the two
+  // (m, l) pairs); the loop is unrolled so several heads' loads are in flight
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i0 = 2 * lane;
   double acc = 0.0;
-  for (int e = threadIdx.x; e < p.h_s * nv; e += RT) {
-    const int hs = e / nv, ii = e - hs * nv;
-    if (t0 + ii >= p.T) continue;  // cu_seqlens past T: reported by the stats pass
-    const float2 v = p.ml[((int64_t)hs * p.cb_stride + cb) * KB + ii];
-    acc += (double)v.y * (double)exp2f(v.x - p.lse2[(int64_t)hs * p.T + t0 + ii]);
+  if (t0 + nv > p.T) {  // cu_seqlens past T: reported by the stats pass
+    if (threadIdx.x == 0) p.mass[cb] = 0.0;
+    return;
+  }
+#pragma unroll 4
+  for (int hs = warp; hs < p.h_s; hs += RT / 32) {
+    const float4 v = *reinterpret_cast<const float4*>(p.ml + ((int64_t)hs * p.cb_stride + cb) * KB + i0);
+    const float* lr = p.lse2 + (int64_t)hs * p.T + t0;
+    if (i0 < nv) acc += (double)v.y * (double)ex2(v.x - lr[i0]);
+    if (i0 + 1 < nv) acc += (double)v.w * (double)ex2(v.z - lr[i0 + 1]);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
