@@ -222,6 +222,10 @@ def run_ours(args, rank, world, dev):
     if rank == 0 and not args.no_e2e:
         e2e = run_e2e(args, w, mf, pack, W, V, bsr, ws, O, qbase, dev)
 
+    pcache = None
+    if rank == 0 and not args.no_cache:
+        pcache = run_prefix_cache(w, mf, bsr, nnz, dev)
+
     cqk = None
     if rank == 0 and not args.no_qk:
         cqk = run_compress_qk(w, mf, dev, qk_len=args.qk_len)
@@ -235,7 +239,7 @@ def run_ours(args, rank, world, dev):
         calib = run_calib(w, mf, pack, dev, args.calib_len)
 
     return dict(w=w, nnz=nnz, elapsed=elapsed, t_comp=t_comp, t_ret=t_ret, clocks=clk.summary(),
-                e2e=e2e, calib=calib, multi=multi, cqk=cqk)
+                e2e=e2e, calib=calib, multi=multi, cqk=cqk, pcache=pcache)
 
 
 def run_calib(w, mf, pack, dev, calib_len=0, reps=5):
@@ -387,6 +391,71 @@ def run_compress_qk(w, mf, dev, reps=5, qk_len=0):
             "exp": scores + nnz * w.h_s * 64 * 64, "exp/s": (scores + nnz * w.h_s * 64 * 64) / t}
 
 
+def run_prefix_cache(w, mf, bsr, nnz, dev, reps=20):
+    """Prefix-hash block cache: every row of the compressed sender layer cached, then the whole
+    request assembled from the cache on a side stream (CUDA events).  Bytes: the kept blocks
+    read from the pool and written to the request's BSR.  Overlap: the assembly beside a bf16
+    GEMM standing in for the receiver's own first-layer compute (8192 x 4096 x 4096) on the main
+    stream; hidden = (t_gemm + t_get - t_both) / t_get."""
+    blk = w.h_s * w.B * w.B * 2
+    pool = torch.empty(max(nnz, 1) * blk, dtype=torch.uint8, device=dev)
+    cache = mf.BlockCache(pool, w.h_s, w.B)
+    toks = np.random.default_rng(w.seed).integers(0, 150000, size=w.tokens).astype(np.int32)
+    h = mf.mf_prefix_hashes(toks, w.B)
+    cache.put(0, bsr, h)
+    out = mf.alloc_bsr(len(h), max(nnz, 1), w.h_s, w.B, torch.bfloat16, dev)
+    main, side = torch.cuda.current_stream(), torch.cuda.Stream(device=dev)
+    a = torch.randn(8192, 4096, device=dev, dtype=torch.bfloat16)
+    b = torch.randn(4096, 4096, device=dev, dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(main)
+            fn()
+            e1.record(main)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e-3)
+        return statistics.median(ts)
+
+    def get():
+        side.wait_stream(main)
+        hit = cache.get(0, h, out, stream=side)
+        assert hit == len(h)
+        main.wait_stream(side)
+
+    def gemm():
+        torch.matmul(a, b)
+
+    def both():
+        side.wait_stream(main)
+        cache.get(0, h, out, stream=side)
+        torch.matmul(a, b)
+        main.wait_stream(side)
+
+    t_get, t_mm, t_both = timed(get), timed(gemm), timed(both)
+    rc, bits = mf.mf_get_status()
+    if rc != mf.MF_OK:
+        raise RuntimeError(f"prefix cache status {rc} bits {bits:#x}")
+    ok = torch.equal(out.values[:nnz], bsr.values[:nnz])
+    st = cache.stats()
+    cache.close()
+    del pool, out, a, b
+    torch.cuda.empty_cache()
+    moved = 2 * nnz * blk
+    return {"kernel": "mf_cache_get (k_cache_copy + k_cache_row_ptr)",
+            "workload": f"{len(h)} query-block rows, {nnz} kept blocks ({nnz * blk / 1e6:.1f} MB)",
+            "ms": t_get * 1e3, "GB/s": moved / t_get / 1e9, "bytes": moved,
+            "gemm_ms": t_mm * 1e3, "both_ms": t_both * 1e3,
+            "hidden_frac": (t_mm + t_get - t_both) / t_get, "bitwise_equal": ok, "reps": reps,
+            "cache": st}
+
+
 def run_e2e(args, w, mf, pack, W, V, bsr, ws, O, qbase, dev):
     h_maps = torch.empty(pack.maps.shape, dtype=pack.maps.dtype, pin_memory=True)
     h_maps.copy_(pack.maps)
@@ -476,6 +545,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-cache", action="store_true", help="skip the prefix-cache line")
     ap.add_argument("--no-qk", action="store_true", help="skip the compression-from-Q,K line")
     ap.add_argument("--qk-len", type=int, default=0,
                     help="sequence length of the compression-from-Q,K line (0: the workload's)")
@@ -579,6 +649,11 @@ def main():
         }
         if res["e2e"] is not None:
             line["e2e"] = res["e2e"]
+        if res["pcache"] is not None:
+            c = res["pcache"]
+            c.update({"bound": "hbm", "peak": hbm, "unit": "GB/s", "frac": c["GB/s"] / hbm,
+                      "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)"})
+            line["prefix_cache"] = c
         if res["cqk"] is not None:
             c = res["cqk"]
             sm_mhz = (res["clocks"] or {}).get("sm_mhz") or 1965.0

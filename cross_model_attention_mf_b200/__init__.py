@@ -9,6 +9,7 @@ Functions mirror the C entry points:
     mf_compress_qk(...)     -> BSR, straight from the sender's Q and K (no dense map)
     mf_map_retrieve(...)    -> O
     mf_map_retrieve_multi(...) -> [O]   (one sender, several receivers)
+    mf_prefix_hashes(...), BlockCache(...).put / get / stats   (prefix-hash block cache)
     mf_get_status()         -> (status, bits)
     mf_compress_workspace_size(...), mf_retrieve_path(...), mf_version()
     mf_calib_gram(...), mf_calib_solve(...), mf_calib_path(...)   (head-map calibration)
@@ -55,6 +56,11 @@ class CompressQkDesc(ctypes.Structure):
                 ("nnz_out", _P), ("block_mass_out", _P), ("lse_out", _P)]
 
 
+class CacheDesc(ctypes.Structure):
+    _fields_ = [("pool", _P), ("pool_bytes", ctypes.c_size_t), ("h_s", _I32), ("B", _I32),
+                ("dtype", ctypes.c_int)]
+
+
 class BsrDesc(ctypes.Structure):
     _fields_ = [("row_ptr", _P), ("col_idx", _P), ("values", _P), ("capacity_blocks", _I64)]
 
@@ -87,6 +93,19 @@ _lib.mf_compress_qk_workspace_size.argtypes = [ctypes.POINTER(CompressQkDesc), c
 _lib.mf_compress_qk_workspace_size.restype = ctypes.c_int
 _lib.mf_compress_qk.argtypes = [ctypes.POINTER(CompressQkDesc), _P, ctypes.c_size_t, _P]
 _lib.mf_compress_qk.restype = ctypes.c_int
+_lib.mf_prefix_hashes.argtypes = [_P, _I64, _I32, _P]
+_lib.mf_prefix_hashes.restype = ctypes.c_int
+_lib.mf_cache_create.argtypes = [ctypes.POINTER(CacheDesc), ctypes.POINTER(_P)]
+_lib.mf_cache_create.restype = ctypes.c_int
+_lib.mf_cache_destroy.argtypes = [_P]
+_lib.mf_cache_destroy.restype = None
+_lib.mf_cache_put.argtypes = [_P, _I32, ctypes.POINTER(BsrDesc), _P, _P, _I64, _I32, _P,
+                              ctypes.POINTER(_I64), _P]
+_lib.mf_cache_put.restype = ctypes.c_int
+_lib.mf_cache_get.argtypes = [_P, _I32, _P, _I32, _P, _P, _P, _I64, ctypes.POINTER(_I32), _P]
+_lib.mf_cache_get.restype = ctypes.c_int
+_lib.mf_cache_stats.argtypes = [_P, _P]
+_lib.mf_cache_stats.restype = ctypes.c_int
 _lib.mf_map_retrieve.argtypes = [ctypes.POINTER(RetrieveDesc), _P]
 _lib.mf_map_retrieve.restype = ctypes.c_int
 _lib.mf_map_retrieve_multi.argtypes = [ctypes.POINTER(RetrieveDesc), ctypes.c_int, _P]
@@ -374,6 +393,71 @@ def mf_retrieve_path(layers, layer_map, W, V, cu_seqlens_q, cu_seqlens_k, qblock
                              cu_seqlens_k, qblock_base, max_seqlen_q, h_s, B, h_r, h_kv, 0, 0,
                              paged, MF_RETRIEVE_FORCE_SIMT if force_simt else 0)
     return _lib.mf_retrieve_path(ctypes.byref(d))
+
+
+def mf_prefix_hashes(tokens, B: int):
+    """uint64 [ceil(L / B)]: FNV-1a 64 of the token bytes of each prefix ending a query block."""
+    import numpy as np
+    t = np.ascontiguousarray(np.asarray(tokens, dtype=np.int32))
+    n = -(-t.size // B)
+    out = np.zeros(n, dtype=np.uint64)
+    _check(_lib.mf_prefix_hashes(t.ctypes.data_as(_P), t.size, int(B), out.ctypes.data_as(_P)))
+    return out
+
+
+class BlockCache:
+    """Prefix-hash cache of compressed query-block rows in a caller-owned device pool
+    (include/mf.h, mf_cache_*)."""
+
+    def __init__(self, pool: torch.Tensor, h_s: int, B: int, dtype=torch.bfloat16):
+        self.pool = pool  # keeps the memory alive
+        d = CacheDesc(_ptr(pool), pool.numel() * pool.element_size(), int(h_s), int(B),
+                      MF_BF16 if dtype == torch.bfloat16 else MF_F32)
+        h = _P()
+        _check(_lib.mf_cache_create(ctypes.byref(d), ctypes.byref(h)))
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _lib.mf_cache_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+    def put(self, layer: int, bsr: BSR, hashes, row0: int = 0, nrows: Optional[int] = None,
+            row_ptr_host=None, col_idx_host=None, stream=None) -> int:
+        """Insert rows [row0, row0 + nrows) of a compressed layer; returns the rows added.
+        The BSR's index arrays are read back to the host when not given."""
+        import numpy as np
+        rp = np.ascontiguousarray(row_ptr_host if row_ptr_host is not None
+                                  else bsr.row_ptr.cpu().numpy(), dtype=np.int32)
+        ci = np.ascontiguousarray(col_idx_host if col_idx_host is not None
+                                  else bsr.col_idx.cpu().numpy(), dtype=np.int32)
+        hs = np.ascontiguousarray(hashes, dtype=np.uint64)
+        n = len(hs) if nrows is None else nrows
+        got = _I64(0)
+        d = bsr.desc()
+        _check(_lib.mf_cache_put(self._h, int(layer), ctypes.byref(d), rp.ctypes.data_as(_P),
+                                 ci.ctypes.data_as(_P), int(row0), int(n), hs.ctypes.data_as(_P),
+                                 ctypes.byref(got), _stream(stream)))
+        return got.value
+
+    def get(self, layer: int, hashes, out: BSR, stream=None) -> int:
+        """Assemble the longest cached prefix of the rows into `out`; returns the rows found."""
+        import numpy as np
+        hs = np.ascontiguousarray(hashes, dtype=np.uint64)
+        hit = _I32(0)
+        _check(_lib.mf_cache_get(self._h, int(layer), hs.ctypes.data_as(_P), len(hs),
+                                 _ptr(out.row_ptr), _ptr(out.col_idx), _ptr(out.values),
+                                 out.capacity, ctypes.byref(hit), _stream(stream)))
+        return hit.value
+
+    def stats(self) -> dict:
+        import numpy as np
+        o = np.zeros(6, dtype=np.int64)
+        _check(_lib.mf_cache_stats(self._h, o.ctypes.data_as(_P)))
+        return dict(zip(("rows", "used", "free", "hits", "misses", "evicted"), o.tolist()))
 
 
 def mf_get_status(stream=None):

@@ -4,6 +4,7 @@
 
 #include <cstdio>
 #include <mutex>
+#include <algorithm>
 #include <cmath>
 #include <string>
 
@@ -294,6 +295,86 @@ mf_status mf_compress_qk(const mf_compress_qk_desc* desc, void* workspace, size_
   std::string err;
   if (!mfi::launch_compress_qk(*desc, ws, q, st, static_cast<cudaStream_t>(stream), &err))
     return fail(MF_ERR_CUDA, "mf_compress_qk: " + err);
+  return MF_OK;
+}
+
+mf_status mf_prefix_hashes(const int32_t* tokens, int64_t L, int32_t B, uint64_t* out) {
+  if ((!tokens && L > 0) || L < 0 || B < 1 || (!out && L > 0)) return fail(MF_ERR_INVALID, "bad tokens / L / B / out");
+  uint64_t h = 0xcbf29ce484222325ull;  // FNV-1a 64: offset basis, prime 2^40 + 2^8 + 0xb3
+  const int64_t nqb = (L + B - 1) / B;
+  for (int64_t k = 0; k < nqb; ++k) {
+    const int64_t e = std::min<int64_t>((k + 1) * B, L);
+    for (int64_t t = k * B; t < e; ++t) {
+      const uint32_t v = (uint32_t)tokens[t];
+      for (int b = 0; b < 4; ++b) {
+        h ^= (v >> (8 * b)) & 0xFFu;
+        h *= 0x100000001b3ull;
+      }
+    }
+    out[k] = h;
+  }
+  return MF_OK;
+}
+
+struct mf_block_cache {
+  mfi::BlockCache* c;
+  mf_cache_desc d;
+};
+
+mf_status mf_cache_create(const mf_cache_desc* desc, mf_block_cache** out) {
+  if (!desc || !out) return fail(MF_ERR_INVALID, "desc or out is NULL");
+  if (!desc->pool || reinterpret_cast<uintptr_t>(desc->pool) % 16) return fail(MF_ERR_INVALID, "pool must be a 16-byte aligned device pointer");
+  if (!is_dtype(desc->dtype) || desc->h_s < 1 || desc->h_s > 256 || !(desc->B == 32 || desc->B == 64 || desc->B == 128))
+    return fail(MF_ERR_INVALID, "bad dtype / h_s / B");
+  const size_t slot = (size_t)desc->h_s * desc->B * desc->B * (desc->dtype == MF_F32 ? 4 : 2);
+  if (desc->pool_bytes < slot) return fail(MF_ERR_INVALID, "pool smaller than one block");
+  if (desc->pool_bytes / slot >= ((size_t)1 << 31)) return fail(MF_ERR_UNSUPPORTED, "too many slots");
+  *out = new mf_block_cache{mfi::cache_create(*desc), *desc};
+  return MF_OK;
+}
+
+void mf_cache_destroy(mf_block_cache* cache) {
+  if (!cache) return;
+  mfi::cache_destroy(cache->c);
+  delete cache;
+}
+
+mf_status mf_cache_put(mf_block_cache* cache, int32_t layer, const mf_bsr* bsr,
+                       const int32_t* row_ptr_host, const int32_t* col_idx_host, int64_t row0,
+                       int32_t nrows, const uint64_t* hashes, int64_t* inserted, void* stream) {
+  if (!cache || !bsr || !row_ptr_host || !hashes || row0 < 0 || nrows < 0)
+    return fail(MF_ERR_INVALID, "bad cache / bsr / row_ptr_host / hashes / rows");
+  if (!bsr->values || reinterpret_cast<uintptr_t>(bsr->values) % 16) return fail(MF_ERR_INVALID, "bsr values must be 16-byte aligned");
+  for (int32_t r = 0; r < nrows; ++r) {
+    const int32_t b0 = row_ptr_host[row0 + r], b1 = row_ptr_host[row0 + r + 1];
+    if (b0 < 0 || b1 < b0) return fail(MF_ERR_INVALID, "row_ptr_host is not non-decreasing");
+    if (b1 > b0 && !col_idx_host) return fail(MF_ERR_INVALID, "col_idx_host is NULL");
+  }
+  const int64_t n = mfi::cache_put(cache->c, layer, *bsr, row_ptr_host, col_idx_host, row0, nrows,
+                                   hashes, static_cast<cudaStream_t>(stream));
+  if (n < 0) return fail(MF_ERR_CUDA, "mf_cache_put: copy launch failed");
+  if (inserted) *inserted = n;
+  return MF_OK;
+}
+
+mf_status mf_cache_get(mf_block_cache* cache, int32_t layer, const uint64_t* hashes, int32_t nrows,
+                       int32_t* row_ptr, int32_t* col_idx, void* values, int64_t capacity_blocks,
+                       int32_t* hit, void* stream) {
+  if (!cache || (!hashes && nrows > 0) || nrows < 0 || !row_ptr || !hit || capacity_blocks < 0 ||
+      (capacity_blocks > 0 && (!col_idx || !values)))
+    return fail(MF_ERR_INVALID, "bad cache / hashes / outputs");
+  if (values && reinterpret_cast<uintptr_t>(values) % 16) return fail(MF_ERR_INVALID, "values must be 16-byte aligned");
+  int h = 0;
+  if (!mfi::cache_get(cache->c, layer, hashes, nrows, row_ptr, col_idx, values, capacity_blocks, &h,
+                      static_cast<cudaStream_t>(stream)))
+    return fail(MF_ERR_CUDA, "mf_cache_get: copy launch failed");
+  *hit = h;
+  return MF_OK;
+}
+
+mf_status mf_cache_stats(mf_block_cache* cache, int64_t* out6) {
+  if (!cache || !out6) return fail(MF_ERR_INVALID, "cache or out is NULL");
+  mfi::cache_stats(cache->c, out6);
   return MF_OK;
 }
 

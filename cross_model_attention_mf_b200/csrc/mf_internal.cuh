@@ -77,6 +77,17 @@ bool tc_supported(const mf_retrieve_desc& d);
 bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* ls, int n,
                         uint32_t* status, cudaStream_t st, std::string* err);
 
+// prefix-hash block cache
+struct BlockCache;
+BlockCache* cache_create(const mf_cache_desc& d);
+void cache_destroy(BlockCache* c);
+int64_t cache_put(BlockCache* c, int layer, const mf_bsr& bsr, const int32_t* row_ptr_host,
+                  const int32_t* col_idx_host, int64_t row0, int nrows, const uint64_t* hashes,
+                  cudaStream_t st);
+bool cache_get(BlockCache* c, int layer, const uint64_t* hashes, int nrows, int32_t* row_ptr,
+               int32_t* col_idx, void* values, int64_t capacity, int* hit, cudaStream_t st);
+void cache_stats(BlockCache* c, int64_t* out6);
+
 // head-map calibration
 size_t calib_ws_bytes(const mf_calib_desc& d);
 int calib_path(const mf_calib_desc& d);

@@ -325,6 +325,51 @@ mf_status mf_calib_solve(const double* gram, int h_s, int h_r, double ridge, flo
 /* Which Gram kernel mf_calib_gram launches: 0 = SIMT, 1 = tcgen05; -1 invalid. */
 int mf_calib_path(const mf_calib_desc* desc);
 
+/* ------------------------------------------------------------------------------
+ * Prefix-hash cache of compressed blocks (MapFlow page "MapFlow开源:大模型换班,Prefill为何
+ * 能快20%?", section "存不下、读得慢?三个工程优化手段", subsection 2: the kept blocks are
+ * indexed by a prefix hash that carries the preceding context, the receiver finds its blocks
+ * through it, and fetching them may overlap the receiver's first layers).
+ *
+ * mf_prefix_hashes: out[k] (k < ceil(L / B)) = 64-bit FNV-1a of the little-endian bytes of
+ * tokens[0 .. min((k + 1) B, L)), i.e. of the whole prefix up to the end of query block k, so
+ * equal hashes mean equal preceding context.  Host only.
+ *
+ * The cache: the caller gives one device buffer (pool, pool_bytes, 16-byte aligned) that the
+ * cache cuts into slots of one kept block (h_s * B * B elements of dtype); the index, free list
+ * and least-recently-used order live on the host (thread-safe).  An entry is one query-block
+ * row of one sender layer, keyed by (layer, prefix hash).
+ *   mf_cache_put: copies rows [row0, row0 + nrows) of a compressed layer into the pool (rows
+ *     already present only move to the front of the LRU order; rows that do not fit evict the
+ *     least recently used rows; a row larger than the pool is skipped).  row_ptr_host and
+ *     col_idx_host are host copies of the BSR's index arrays.  *inserted (optional) = rows added.
+ *   mf_cache_get: assembles the longest cached prefix of a request's rows (hashes[0 .. nrows))
+ *     into a BSR: row_ptr [hit + 1], col_idx, values (device, capacity blocks).  *hit (host) =
+ *     rows found; the prefix ends at the first miss or where capacity runs out.
+ *   Both enqueue copies on `stream` and return at once; a get may run on a side stream while
+ *   the receiver computes its first layers (order the retrieval after it with an event).  The
+ *   caller orders a put after the gets that precede it (a put may evict and overwrite slots).
+ *   mf_cache_stats: rows, used slots, free slots, hits, misses, evictions (int64[6]).
+ * ------------------------------------------------------------------------------ */
+typedef struct mf_block_cache mf_block_cache;
+typedef struct {
+  void* pool;          /* device, owned by the caller, alive until mf_cache_destroy */
+  size_t pool_bytes;
+  int32_t h_s, B;
+  mf_dtype dtype;
+} mf_cache_desc;
+
+mf_status mf_prefix_hashes(const int32_t* tokens, int64_t L, int32_t B, uint64_t* out);
+mf_status mf_cache_create(const mf_cache_desc* desc, mf_block_cache** out);
+void mf_cache_destroy(mf_block_cache* cache);
+mf_status mf_cache_put(mf_block_cache* cache, int32_t layer, const mf_bsr* bsr,
+                       const int32_t* row_ptr_host, const int32_t* col_idx_host, int64_t row0,
+                       int32_t nrows, const uint64_t* hashes, int64_t* inserted, void* stream);
+mf_status mf_cache_get(mf_block_cache* cache, int32_t layer, const uint64_t* hashes, int32_t nrows,
+                       int32_t* row_ptr, int32_t* col_idx, void* values, int64_t capacity_blocks,
+                       int32_t* hit, void* stream);
+mf_status mf_cache_stats(mf_block_cache* cache, int64_t* out6);
+
 /* Synchronise `stream`, then read and clear this device's status word.  *bits
  * (optional) receives the raw bits: 1 index out of range, 2 capacity, 4 wait
  * timeout, 8 misaligned input, 16 page id out of range, 32 singular

@@ -1,0 +1,135 @@
+"""Prefix-hash block cache on the GPU: a request that shares a prefix with a cached one gets,
+bit for bit, the cached rows of that prefix; retrieval over the assembled BSR equals retrieval
+over the original rows; eviction follows least-recent use; assembly on a side stream overlaps
+work on the main stream and is ordered by an event (MapFlow page "MapFlow开源:大模型换班,Prefill
+为何能快20%?", section "存不下、读得慢?三个工程优化手段", subsection 2)."""
+import numpy as np
+import pytest
+import torch
+
+import cross_model_attention_mf_b200 as mf
+import synth
+from synth import device as sdev
+from tests.gpu_common import run_compress
+
+pytestmark = pytest.mark.gpu
+
+
+def _status_ok():
+    rc, bits = mf.mf_get_status()
+    assert rc == mf.MF_OK and bits == 0, (rc, bits)
+
+
+def _request(L, seed=0):
+    w = synth.Workload("cache", (L,), B=64, h_s=32, h_r=32, h_kv=8, d=128, dtype="bf16",
+                       tau=0.95, n_heavy=16, reading=3, seed=seed)
+    pack = sdev.fill_maps(sdev.alloc_maps(w), w, 0)
+    return w, pack, run_compress(w, pack)
+
+
+def _pool(blocks, h_s=32, B=64):
+    return torch.empty(blocks * h_s * B * B * 2, dtype=torch.uint8, device="cuda")
+
+
+def test_shared_prefix_gets_cached_rows_bitwise():
+    w, pack, bsr = _request(700)
+    rng = np.random.default_rng(1)
+    toks = rng.integers(0, 50000, size=700).astype(np.int32)
+    cache = mf.BlockCache(_pool(400), 32, 64)
+    hA = mf.mf_prefix_hashes(toks, 64)
+    assert cache.put(0, bsr, hA) == len(hA)
+    # request B: the same first 5 blocks (320 tokens), then other tokens
+    toksB = np.concatenate([toks[:320], rng.integers(0, 50000, size=200).astype(np.int32)])
+    hB = mf.mf_prefix_hashes(toksB, 64)
+    out = mf.alloc_bsr(len(hB), 200, 32, 64, torch.bfloat16, "cuda")
+    hit = cache.get(0, hB, out)
+    torch.cuda.synchronize()
+    assert hit == 5
+    rp = bsr.row_ptr.cpu().numpy()
+    n = rp[5]
+    assert out.row_ptr[:6].cpu().tolist() == rp[:6].tolist()
+    assert torch.equal(out.col_idx[:n], bsr.col_idx[:n])
+    assert torch.equal(out.values[:n], bsr.values[:n])
+    # retrieval over the assembled rows equals retrieval over the original rows
+    W = sdev.w_weights(w)
+    V = sdev.v_contiguous(w, 0)
+    qb = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cu_a = torch.tensor([0, 700], dtype=torch.int32, device="cuda")
+    cu_b = torch.tensor([0, 320], dtype=torch.int32, device="cuda")
+    O_a = mf.mf_map_retrieve([bsr], [0], W, V, cu_a, cu_a, qb, 700, 32, 8, total_q=700)[0]
+    O_b = mf.mf_map_retrieve([out], [0], W, V[:320].contiguous(), cu_b, cu_b, qb, 320, 32, 8,
+                             total_q=320)[0]
+    assert torch.equal(O_b, O_a[:320])
+    st = cache.stats()
+    assert st["rows"] == 11 and st["hits"] == 5 and st["misses"] == 1 and st["evicted"] == 0
+    _status_ok()
+
+
+def test_layers_are_separate_and_eviction_is_lru():
+    w, pack, bsr = _request(640)
+    rp = bsr.row_ptr.cpu().numpy()
+    sizes = np.diff(rp)
+    toks = np.arange(640, dtype=np.int32)
+    h = mf.mf_prefix_hashes(toks, 64)
+    need = int(sizes[:4].sum())
+    cache = mf.BlockCache(_pool(need), 32, 64)     # room for rows 0-3 only
+    assert cache.put(0, bsr, h[:4], row0=0, nrows=4) == 4
+    out = mf.alloc_bsr(10, 64, 32, 64, torch.bfloat16, "cuda")
+    assert cache.get(1, h, out) == 0               # another layer: nothing
+    assert cache.get(0, h[:2], out) == 2           # rows 0, 1 become the most recent
+    # row 4 needs room: the least recently used rows (3, then 2) go first
+    assert cache.put(0, bsr, h[4:5], row0=4, nrows=1) == 1
+    st = cache.stats()
+    assert st["evicted"] >= 1 and st["rows"] == 5 - st["evicted"]
+    hit = cache.get(0, h, out)
+    assert hit == 2                                # rows 0, 1 survive; the prefix breaks at 2
+    torch.cuda.synchronize()
+    n = rp[2]
+    assert torch.equal(out.values[:n], bsr.values[:n])
+    _status_ok()
+
+
+def test_assembly_on_a_side_stream_is_ordered_by_an_event():
+    w, pack, bsr = _request(1000, seed=3)
+    toks = np.arange(1000, dtype=np.int32) * 7
+    h = mf.mf_prefix_hashes(toks, 64)
+    cache = mf.BlockCache(_pool(600), 32, 64)
+    cache.put(0, bsr, h)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    out = mf.alloc_bsr(len(h), 600, 32, 64, torch.bfloat16, "cuda")
+    out.values.zero_()
+    torch.cuda.synchronize()
+    a = torch.randn(4096, 4096, device="cuda", dtype=torch.bfloat16)
+    busy = a @ a  # the receiver's own first layers stand here  # noqa: F841
+    with torch.cuda.stream(side):
+        hit = cache.get(0, h, out, stream=side)
+        ev = torch.cuda.Event()
+        ev.record(side)
+    torch.cuda.current_stream().wait_event(ev)
+    n = int(bsr.row_ptr[-1].item())
+    assert hit == len(h)
+    assert torch.equal(out.values[:n], bsr.values[:n])
+    assert torch.equal(out.row_ptr, bsr.row_ptr)
+    _status_ok()
+
+
+def test_one_put_larger_than_the_pool_keeps_the_latest_rows_intact():
+    """Rows evicted inside one put must not leave their data in the slots of later rows."""
+    w, pack, bsr = _request(900, seed=5)
+    rp = bsr.row_ptr.cpu().numpy()
+    sizes = np.diff(rp)
+    h = mf.mf_prefix_hashes(np.arange(900, dtype=np.int32) + 11, 64)
+    cap = int(sizes[-3:].sum())                    # room for about the last three rows
+    cache = mf.BlockCache(_pool(cap), 32, 64)
+    cache.put(0, bsr, h)
+    st = cache.stats()
+    assert st["evicted"] > 0 and st["used"] <= cap
+    out = mf.alloc_bsr(1, 64, 32, 64, torch.bfloat16, "cuda")
+    last = len(h) - 1
+    assert cache.get(0, h[last:], out) == 1
+    torch.cuda.synchronize()
+    n0, n1 = rp[last], rp[last + 1]
+    assert torch.equal(out.values[:n1 - n0], bsr.values[n0:n1])
+    assert torch.equal(out.col_idx[:n1 - n0], bsr.col_idx[n0:n1])
+    _status_ok()
