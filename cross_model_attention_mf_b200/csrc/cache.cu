@@ -32,7 +32,7 @@
 namespace mfi {
 namespace {
 
-constexpr int CHUNK = 192;
+constexpr int CHUNK = 1024;  // copies per launch (12 KB of kernel parameters)
 
 struct CopyChunk {
   const uint4* src;   // block k of the source at src + src_blk[k] * blk_vecs

@@ -2,7 +2,7 @@
 // over causal positions (tcgen05 + TMA + TMEM for bf16, SIMT otherwise), and the
 // least-squares solve for the head-mapping weights.
 //
-// MapFlow page "MapFlow开源:大模型换班,Prefill为何能快20%?", section "MapFlow 的核心思路":
+// MapFlow page "MapFlow开源:大模型换班,Prefill为何能快20%?", section "不传 KV Cache,改传“注意力关系”":
 // the weights that combine sender heads into receiver heads are learned once, offline, with
 // both models frozen; the page gives no objective.  Reading taken: least squares of every
 // receiver head's map Y_r on the sender heads' maps X_s over the causal positions

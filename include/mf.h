@@ -277,9 +277,9 @@ int mf_retrieve_path(const mf_retrieve_desc* desc);
 
 /* ------------------------------------------------------------------------
  * Head-map calibration (offline).  MapFlow page "MapFlow开源:大模型换班,Prefill为何能快20%?",
- * section "MapFlow 的核心思路": the weights that map sender heads onto receiver heads are
- * learned once, offline, with both models frozen ("头映射:学习一组线性组合权重",
- * "这些映射关系离线校准一次"); the page states no objective.  Reading taken: least squares of
+ * section "不传 KV Cache,改传“注意力关系”" (head and layer mapping): the weights that map
+ * sender heads onto receiver heads are learned once, offline, with both models frozen; the
+ * page states no objective.  Reading taken: least squares of
  * every receiver head's map on the sender heads' maps over the causal positions (i < L,
  * j <= i) of the calibration sequences, with an optional ridge term.  The layer map is then
  * chosen by the smallest residual (caller side: one Gram per candidate sender layer).

@@ -213,8 +213,8 @@ void mfo_retrieve_block(const void* vals, int dtype, const int32_t* kb, int n, i
 /*
  * Head-map calibration (offline step of the head mapping).  The pages say the linear-
  * combination weights that map sender heads onto receiver heads are learned once, offline,
- * with both models frozen ("头映射:学习一组线性组合权重" and "这些映射关系离线校准一次",
- * section "MapFlow 的核心思路"), but give no objective.  Reading taken: ordinary least squares
+ * with both models frozen (page "MapFlow开源:大模型换班,Prefill为何能快20%?", section
+ * "不传 KV Cache,改传“注意力关系”", head and layer mapping), but give no objective.  Reading taken: ordinary least squares
  * of each receiver head's map on the sender heads' maps over the causal positions of the
  * calibration sequences, with an optional ridge term:
  *   w_r = argmin_w  sum_{i < L, j <= i} (Y_r[i, j] - sum_s w[s] X_s[i, j])^2 + ridge * |w|^2.
