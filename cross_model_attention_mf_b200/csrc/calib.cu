@@ -186,9 +186,15 @@ __global__ void __launch_bounds__(GT, 1)
   const uint32_t DONE = bar0 + 8u * (2 * G_STAGES);
   const uint32_t tile_bytes = (uint32_t)p.F8 * 128u;
 
-  // this CTA's contiguous tile range, in stages of p.tps tiles
-  const int64_t t0 = p.n_tiles * blockIdx.x / gridDim.x, t1 = p.n_tiles * (blockIdx.x + 1) / gridDim.x;
-  const int n_st = (int)((t1 - t0 + p.tps - 1) / p.tps);
+  // stages of p.tps consecutive tiles, dealt round-robin: global stage g goes to CTA
+  // g % gridDim.x, so the CTAs work on neighbouring rows at the same time (the rows of all head
+  // planes they touch share pages: far fewer translation misses than one contiguous range per CTA)
+  const int64_t n_stages = (p.n_tiles + p.tps - 1) / p.tps;
+  const int n_st = blockIdx.x < n_stages ? (int)((n_stages - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+  auto stage_tiles = [&](int st, int64_t* ta, int* n) {
+    *ta = ((int64_t)blockIdx.x + (int64_t)st * gridDim.x) * p.tps;
+    *n = (int)(p.n_tiles - *ta < (int64_t)p.tps ? p.n_tiles - *ta : (int64_t)p.tps);
+  };
 
   if (threadIdx.x == 0) {
     s_abort = 0;
@@ -218,14 +224,18 @@ __global__ void __launch_bounds__(GT, 1)
 
   if (warp == 0) {
     // ================================================================ TMA producer
-    if (lane == 0) {
-      bool ok = true;
-      int issued = 0;
-      for (int st = 0; st < n_st && ok; ++st) {
-        const int s = st % G_STAGES;
-        if (!(ok = bar_wait(EMPTY(s), ((st / G_STAGES) & 1) ^ 1, abort_flag, p.status))) break;
-        const int64_t ta = t0 + (int64_t)st * p.tps;
-        const int n = (int)(t1 - ta < (int64_t)p.tps ? t1 - ta : (int64_t)p.tps);
+    // the whole warp waits (suspended by the hardware, where a lone polling lane would spin);
+    // lane 0 issues the copies
+    bool ok = true;
+    int issued = 0;
+    for (int st = 0; st < n_st && ok; ++st) {
+      const int s = st % G_STAGES;
+      ok = __all_sync(0xffffffffu, bar_wait(EMPTY(s), ((st / G_STAGES) & 1) ^ 1, abort_flag, p.status));
+      if (!ok) break;
+      int64_t ta;
+      int n;
+      stage_tiles(st, &ta, &n);
+      if (lane == 0) {
         bar_expect(FULL(s), (uint32_t)(n * (p.h_s + p.h_r) * 128));
         for (int k = 0; k < n; ++k) {
           int i, c;
@@ -234,9 +244,12 @@ __global__ void __launch_bounds__(GT, 1)
           tma3(dst, &tmX, FULL(s), c * KEYS, 0, i);
           tma3(dst + p.h_s * 128u, &tmY, FULL(s), c * KEYS, 0, i);
         }
-        ++issued;
       }
-      // drain: wait (bounded) for the last copies issued into every stage
+      __syncwarp();
+      ++issued;
+    }
+    // drain: wait (bounded) for the last copies issued into every stage
+    if (lane == 0)
       for (int s = 0; s < G_STAGES; ++s) {
         const int cnt = issued > s ? (issued - s - 1) / G_STAGES + 1 : 0;
         if (cnt) {
@@ -244,7 +257,7 @@ __global__ void __launch_bounds__(GT, 1)
           while (!bar_try(FULL(s), (cnt - 1) & 1) && gtimer() - w0 < G_TIMEOUT_NS) {}
         }
       }
-    }
+    __syncwarp();
   } else if (warp == 1) {
     // ================================================================ mask + MMA issue
     // D[f][g] += sum_k T[f][k] T[g][k]: M=128 (rows past F are ignored), N=Fn, K=16
@@ -255,8 +268,9 @@ __global__ void __launch_bounds__(GT, 1)
       const int s = st % G_STAGES;
       ok = __all_sync(0xffffffffu, bar_wait(FULL(s), (st / G_STAGES) & 1, abort_flag, p.status));
       if (!ok) break;
-      const int64_t ta = t0 + (int64_t)st * p.tps;
-      const int n = (int)(t1 - ta < (int64_t)p.tps ? t1 - ta : (int64_t)p.tps);
+      int64_t ta;
+      int n;
+      stage_tiles(st, &ta, &n);
       // keys j > i of a diagonal tile do not count: zero them in every feature row
       for (int k = 0; k < n; ++k) {
         int i, c;
