@@ -264,7 +264,8 @@ mf_status mf_map_retrieve(const mf_retrieve_desc* desc, void* stream);
  * pointers, nseq, max_seqlen_q) and the number of receiver layers, up to four receivers share
  * each launch: the CTAs of all receivers walk the same query blocks together, so the kept
  * map tiles are read from HBM once per step and reused from L2.  Otherwise the receivers run
- * one after another.  Errors as for mf_map_retrieve (the first failing descriptor). */
+ * one after another.  The receivers' O regions must not overlap.  Errors as for
+ * mf_map_retrieve (the first failing descriptor). */
 mf_status mf_map_retrieve_multi(const mf_retrieve_desc* descs, int n, void* stream);
 
 /* 1 when mf_map_retrieve_multi would share launches among descs, 0 when it would run them
