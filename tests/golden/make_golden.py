@@ -1,10 +1,14 @@
-"""Writes tests/golden/tiny_oracle.json from the oracle alone.
+"""Writes tests/golden/tiny_oracle.json and tests/golden/tiny_qk_oracle.json from the oracle alone.
 
 The MapFlow pages print no worked example with numbers, so the stored values here are the
 oracle's own result on the tiny workload (one sequence of 256 tokens, B=32, 4 sender heads,
 2 receiver heads, 1 KV head, d=64, f32, tau=0.9, 3 heavy columns, seed 0; the recipe of
 synth.maps).  The file pins the oracle against silent drift and gives the GPU tests a second,
 stored reference.  It calls nothing but `synth` (inputs) and `oracle/`.
+
+The second file is compression straight from Q, K on a small case (two sequences of 150 and
+70 tokens, 4 query heads over 2 key heads, d = 128, B = 64, tau = 0.9, the recipe of synth.qk,
+seed 0): block masses, kept sets and sampled kept values of the oracle's float64 maps.
 
     python tests/golden/make_golden.py
 """
@@ -52,7 +56,33 @@ def compute():
     }
 
 
+QK_LENS, QK_HS, QK_HKV, QK_D, QK_B, QK_TAU = (150, 70), 4, 2, 128, 64, 0.9
+
+
+def qk_case():
+    from synth.qk import gen_qk
+    return gen_qk(QK_LENS, QK_HS, QK_HKV, QK_D, 4, 0)
+
+
+def compute_qk():
+    Q, K = qk_case()
+    start, rows = 0, []
+    for L in QK_LENS:
+        Qs, Ks = Q[start:start + L], K[start:start + L]
+        for qb in range(-(-L // QK_B)):
+            m, kept, info, vals = oracle.compress_qk_row(Qs, Ks, L, QK_B, qb, QK_TAU, QK_D ** -0.5)
+            rows.append({"mass": [float("%.15g" % x) for x in m], "kept": kept.tolist(),
+                         "vals_sum": float(vals.sum()),
+                         "vals_sampled": [float("%.12g" % x) for x in vals.reshape(-1)[::997]]})
+        start += L
+    return {"workload": "qk: lens=(150, 70) h_s=4 h_kv=2 d=128 B=64 tau=0.9 seed=0 (synth.qk)",
+            "rows": rows}
+
+
 if __name__ == "__main__":
+    with open(os.path.join(HERE, "tiny_qk_oracle.json"), "w") as f:
+        json.dump(compute_qk(), f, indent=None, separators=(",", ":"))
+        f.write("\n")
     out = compute()
     with open(os.path.join(HERE, "tiny_oracle.json"), "w") as f:
         json.dump(out, f, indent=None, separators=(",", ":"))

@@ -74,3 +74,54 @@ def test_cuda_path_matches_stored_tiny_values():
     np.testing.assert_allclose(mass, flat, rtol=2e-6, atol=1e-12)
     got = O[0].cpu().numpy()[want["O_rows"]].reshape(-1)
     assert_O_close(got, np.asarray(want["O_sampled"]), "f32", "tiny vs stored")
+
+
+GOLD_QK = os.path.join(HERE, "golden", "tiny_qk_oracle.json")
+
+
+def _stored_qk():
+    with open(GOLD_QK) as f:
+        return json.load(f)
+
+
+def test_oracle_reproduces_stored_qk_values():
+    import make_golden
+    got, want = make_golden.compute_qk(), _stored_qk()
+    assert len(got["rows"]) == len(want["rows"])
+    for a, b in zip(got["rows"], want["rows"]):
+        assert a["kept"] == b["kept"]
+        np.testing.assert_allclose(a["mass"], b["mass"], rtol=1e-13, atol=0)
+        np.testing.assert_allclose(a["vals_sampled"], b["vals_sampled"], rtol=1e-11, atol=1e-15)
+        np.testing.assert_allclose(a["vals_sum"], b["vals_sum"], rtol=1e-12)
+
+
+@pytest.mark.gpu
+def test_gpu_compress_qk_matches_stored_values():
+    import torch
+    import cross_model_attention_mf_b200 as mf
+    import make_golden
+    import oracle
+    want = _stored_qk()["rows"]
+    Q, K = make_golden.qk_case()
+    lens, B, tau = make_golden.QK_LENS, make_golden.QK_B, make_golden.QK_TAU
+    nqb = [-(-L // B) for L in lens]
+    causal = sum(n * (n + 1) // 2 for n in nqb)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device="cuda")
+    out = mf.alloc_bsr(sum(nqb), causal, make_golden.QK_HS, B, torch.bfloat16, "cuda", n_causal=causal)
+    mf.mf_compress_qk(Q.cuda(), K.cuda(), cu, max(lens), B, tau, out)
+    rc, bits = mf.mf_get_status()
+    assert bits == 0
+    rp, ci = out.row_ptr.cpu().numpy(), out.col_idx.cpu().numpy()
+    mass = out.block_mass.cpu().numpy()
+    row, cb = 0, 0
+    for n in nqb:
+        for qb in range(n):
+            w = want[row]
+            np.testing.assert_allclose(mass[cb:cb + qb + 1], w["mass"], rtol=1e-5, atol=1e-9)
+            _, info = oracle.select(np.array(w["mass"]), qb, tau)
+            if not oracle.is_boundary(info, tau):
+                assert ci[rp[row]:rp[row + 1]].tolist() == w["kept"]
+                gsum = out.values[rp[row]:rp[row + 1]].double().sum().item()
+                np.testing.assert_allclose(gsum, w["vals_sum"], rtol=2e-3)
+            row += 1
+            cb += qb + 1
