@@ -205,3 +205,28 @@ def test_compress_qk_descriptor_and_validation(mf):
         setattr(bad, field, value)
         assert mf._lib.mf_compress_qk(ctypes.byref(bad), ctypes.c_void_p(4096), 1 << 30, None) == rc, field
     assert mf._lib.mf_abi_struct_size(4) == ctypes.sizeof(mf.CompressQkDesc)
+
+
+def test_multi_receiver_binding_descriptors(mf):
+    """The binding's several-receiver descriptors carry each receiver's own W, V, O, heads and
+    paging, and the shared packing; the host fusing decision follows from them (no launch)."""
+    import torch
+    layers = [mf.BSR(torch.zeros(3, dtype=torch.int32), torch.zeros(4, dtype=torch.int32),
+                     torch.zeros(4, 8, 64, 64, dtype=torch.bfloat16), torch.zeros(1, dtype=torch.int32))]
+    cu = torch.tensor([0, 100], dtype=torch.int32)
+    qb = torch.zeros(1, dtype=torch.int32)
+    rs = [mf.Receiver([0], torch.zeros(1, 8, 8), torch.zeros(1, 100, 2, 128, dtype=torch.bfloat16), 8, 2,
+                      O=torch.zeros(1, 100, 8, 128, dtype=torch.bfloat16)),
+          mf.Receiver([0], torch.zeros(1, 4, 8), torch.zeros(1, 100, 1, 128, dtype=torch.bfloat16), 4, 1,
+                      O=torch.zeros(1, 100, 4, 128, dtype=torch.bfloat16))]
+    arr, keep, outs = mf._multi_descs(layers, rs, cu, cu, qb, 100, 100, None)
+    assert [d.h_r for d in arr] == [8, 4] and [d.h_kv for d in arr] == [2, 1]
+    assert arr[0].W == rs[0].W.data_ptr() and arr[1].V == rs[1].V.data_ptr()
+    assert arr[0].O == outs[0].data_ptr() and arr[1].O == outs[1].data_ptr()
+    assert arr[0].cu_seqlens_q == arr[1].cu_seqlens_q == cu.data_ptr()
+    assert mf._lib.mf_retrieve_multi_fused(arr, 2) == 1
+    # a receiver whose GQA group exceeds 4 heads takes the SIMT kernel: no shared launch
+    rs.append(mf.Receiver([0], torch.zeros(1, 16, 8), torch.zeros(1, 100, 2, 128, dtype=torch.bfloat16),
+                          16, 2, O=torch.zeros(1, 100, 16, 128, dtype=torch.bfloat16)))
+    arr, keep, outs = mf._multi_descs(layers, rs, cu, cu, qb, 100, 100, None)
+    assert mf._lib.mf_retrieve_multi_fused(arr, 3) == 0
