@@ -10,10 +10,11 @@ Recipe, for one layer of a varlen pack (T tokens; per sequence, positions restar
 with g = s * h_kv // h_s, rope(pos) = a (cos(w_k pos), sin(w_k pos)), k < P = 16,
 w_k = 10000^(-k / P), a = sqrt(RECENCY * sqrt(d) / P), u_g a random unit vector (one per key
 head) in the non-positional dims, z ~ N(0, 1).  With the scale 1 / sqrt(d) the scaled score of
-query i and key j is about RECENCY * mean_k cos(w_k (i - j)) + SINK / HEAVY bonuses + noise:
-a recency peak, sinks and heavy columns as in the map recipe.  At L = 8192, tau = 0.95 this
-keeps about 11% of the causal blocks on average (1-2% in the longest rows).  Rounded to the
-requested dtype.  Nothing here computes a softmax, a mass or a selection.
+query i and key j is about RECENCY * mean_k cos(w_k (i - j)) + SINK / HEAVY bonuses + noise.
+The recency peak dominates (the last 8 keys hold 60-99% of a row's mass at 300-1000 tokens);
+sinks and heavy keys take a few percent.  At L = 8192 and tau = 0.95, about 3% of the causal
+blocks are kept (11% at 4096).  Rounded to the requested dtype.  Nothing here computes a
+softmax, a mass or a selection.
 """
 import numpy as np
 import torch

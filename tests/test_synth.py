@@ -99,3 +99,26 @@ def test_page_table_is_a_permutation():
     assert total == sum(-(-L // w.page_size) for L in w.lens)
     assert sorted(used.tolist()) == list(range(total))
     assert (np.diff(used) != 1).any()  # shuffled
+
+
+def test_qk_recipe_is_seeded_and_structured():
+    """synth.qk: same seed, same bytes; another seed, other bytes; the causal attention it
+    induces is concentrated (a recency peak, with sinks and heavy keys taking the rest), the
+    structure that makes block selection keep few blocks."""
+    import math
+
+    import numpy as np
+    import torch
+
+    import oracle
+    from synth.qk import gen_qk
+    Q, K = gen_qk((1000,), 4, 2, 128, 8, seed=0)
+    Q2, K2 = gen_qk((1000,), 4, 2, 128, 8, seed=0)
+    Q3, _ = gen_qk((1000,), 4, 2, 128, 8, seed=1)
+    assert Q.dtype == torch.bfloat16 and Q.shape == (1000, 4, 128) and K.shape == (1000, 2, 128)
+    assert torch.equal(Q, Q2) and torch.equal(K, K2) and not torch.equal(Q, Q3)
+    A = oracle.qk_maps(Q, K, 1000, 64, 1.0 / math.sqrt(128))
+    for i in (299, 600, 999):
+        row = A[0, i, :i + 1]
+        assert np.sort(row)[::-1][:10].sum() > 0.9      # ten keys hold most of the mass
+        assert row[i - 7:i + 1].sum() > 0.5             # the recency peak
