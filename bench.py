@@ -15,7 +15,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -61,66 +60,91 @@ REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_c
            0x100: "display_clock_setting"}
 
 
-def gpu_id(dev):
-    """nvidia-smi id of a CUDA device: its PCI bus id when torch reports it."""
+def _nvml_handle(dev):
+    """NVML handle of a CUDA device, matched by PCI location (CUDA_VISIBLE_DEVICES may renumber
+    devices, so the CUDA ordinal is not NVML's)."""
+    import pynvml
+    pynvml.nvmlInit()
     p = torch.cuda.get_device_properties(dev)
-    try:
-        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
-    except AttributeError:
-        return str(dev.index)
+    want = (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+    for k in range(pynvml.nvmlDeviceGetCount()):
+        h = pynvml.nvmlDeviceGetHandleByIndex(k)
+        pi = pynvml.nvmlDeviceGetPciInfo(h)
+        if (pi.domain, pi.bus, pi.device) == want:
+            return h
+    return None
 
 
 class ClockSampler:
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    """SM clock, its maximum and the clock-event reasons of one GPU, read through NVML (the
+    library nvidia-smi reports from) every `period` seconds on a background thread.  Start it
+    before the warm-up; `mark(True)` / `mark(False)` bracket the timed region, and `sample()`
+    takes one extra reading on demand (call it before the closing synchronize, while the GPU
+    is still busy), so even a timed region of a few milliseconds has readings of its own."""
+
+    def __init__(self, dev, period=0.005):
+        self.period = period
+        self.samples = []        # (time, sm_mhz, max_mhz, reason bits)
+        self.t_lo = self.t_hi = None
+        self.h = None
+        self.stop = threading.Event()
+        self.err = None
+        try:
+            self.h = _nvml_handle(dev)
+        except Exception as e:  # NVML missing: no clock record (reported as such)
+            self.err = f"{type(e).__name__}: {e}"
+
+    def sample(self):
+        if self.h is None:
+            return
+        import pynvml
+        try:
+            sm = pynvml.nvmlDeviceGetClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            bits = pynvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception as e:
+            self.err = f"{type(e).__name__}: {e}"
+            return
+        self.samples.append((time.perf_counter(), float(sm), float(mx), int(bits)))
+
+    def _run(self):
+        while not self.stop.is_set():
+            self.sample()
+            self.stop.wait(self.period)
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index),
-                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+        if self.h is not None:
+            self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
-        except OSError:
-            self.proc = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self.stop.set()
+        if self.h is not None:
             self.t.join(timeout=2)
 
+    def mark(self, start):
+        if start:
+            self.t_lo = time.perf_counter()
+        else:
+            self.t_hi = time.perf_counter()
+
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 4:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-                bits = int(parts[3], 16)
-            except ValueError:
-                continue
+        lo = self.t_lo if self.t_lo is not None else -1e300
+        hi = self.t_hi if self.t_hi is not None else 1e300
+        timed = [x for x in self.samples if lo <= x[0] <= hi]
+        if not timed:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": "nvml", "error": self.err or "no reading inside the timed region"}
+        reasons = set()
+        for x in timed:
             for b, name in REASONS.items():
-                if bits & b and name != "gpu_idle":
+                if x[3] & b and name != "gpu_idle":
                     reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(x[1] for x in timed),
+                "sm_max_mhz": max(x[2] for x in timed), "reasons": sorted(reasons),
+                "samples": len(timed), "samples_total": len(self.samples),
+                "sm_mhz_min": min(x[1] for x in timed), "source": "nvml"}
 
 
 # ------------------------------------------------------------------------ workload
@@ -137,7 +161,9 @@ def describe(w):
 
 
 def algorithmic(w, nnz):
-    """Algorithmic bytes / FLOPs of one compress and one retrieve launch."""
+    """Algorithmic bytes / FLOPs of one compress and one retrieve launch: what the method must
+    move once (every causal block read and the kept blocks written by compression; the kept
+    blocks, V, O and the indices read or written by retrieval) and the mixing + P.V products."""
     e = 4 if w.dtype == "f32" else 2
     blk = w.h_s * w.B * w.B * e
     rows = sum(w.nqb)
@@ -178,6 +204,7 @@ def run_ours(args, rank, world, dev):
         if ev is not None:
             ev[2].record(st)
 
+    clk = ClockSampler(dev).__enter__()  # runs from the warm-up to the end of the timed region
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -202,12 +229,15 @@ def run_ours(args, rank, world, dev):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(gpu_id(dev)) as clk:
-        t0.record(st)
-        for _ in range(args.steps):
-            step()
-        t1.record(st)
-        torch.cuda.synchronize()
+    clk.mark(True)
+    t0.record(st)
+    for _ in range(args.steps):
+        step()
+    t1.record(st)
+    clk.sample()  # one more reading while the queued steps still run
+    torch.cuda.synchronize()
+    clk.mark(False)
+    clk.__exit__(None, None, None)
     elapsed = t0.elapsed_time(t1) * 1e-3
     if world > 1:
         from cross_model_attention_mf_b200 import replicas

@@ -147,7 +147,8 @@ BlockCache* cache_create(const mf_cache_desc& d) {
 void cache_destroy(BlockCache* c) { delete c; }
 
 // Inserts rows [row0, row0 + nrows) of a compressed layer (row_ptr on the host).  Rows already
-// cached are refreshed in the LRU order only; a row larger than the whole pool is skipped.
+// cached are refreshed in the LRU order only; a row larger than the whole pool, or one that
+// reaches past the BSR's capacity (incomplete), is skipped.
 // Returns the number of rows inserted, or -1 on a launch failure.
 int64_t cache_put(BlockCache* c, int layer, const mf_bsr& bsr, const int32_t* row_ptr_host,
                   const int32_t* col_idx_host, int64_t row0, int nrows, const uint64_t* hashes,
@@ -163,7 +164,10 @@ int64_t cache_put(BlockCache* c, int layer, const mf_bsr& bsr, const int32_t* ro
       continue;
     }
     const int32_t b0 = row_ptr_host[row0 + r], b1 = row_ptr_host[row0 + r + 1];
-    const int64_t need = std::min<int64_t>(b1, bsr.capacity_blocks) - b0;
+    // a row that runs past the BSR's capacity (a compression that overflowed) lost some of its
+    // kept blocks: caching it would hand a short row to every later request with this prefix
+    if (b1 > bsr.capacity_blocks) continue;
+    const int64_t need = (int64_t)b1 - b0;
     if (need <= 0 || need > c->n_slots) continue;
     if ((int64_t)c->free_slots.size() < need && !src.empty()) {
       // a slot freed below may be the target of a copy gathered earlier in this call: launch

@@ -466,6 +466,7 @@ cudaError_t launch_compress(const mf_compress_desc& d, const CompressWs& ws, uin
   cudaError_t e = launch_meta(d.cu_seqlens, d.map_seq_offset, d.nseq, d.max_seqlen, d.B, elem, ws,
                               status, d.row_ptr, d.nnz_out, st);
   if (e != cudaSuccess) return e;
+  if (ws.max_cb == 0) return cudaSuccess;  // no query block (max_seqlen 0): k_meta wrote the empty BSR
   if (d.dtype == MF_F32) {
     if (d.B == 32) return launch_typed<float, 32>(d, ws, status, st, sms);
     if (d.B == 64) return launch_typed<float, 64>(d, ws, status, st, sms);

@@ -342,7 +342,9 @@ int mf_calib_path(const mf_calib_desc* desc);
  * row of one sender layer, keyed by (layer, prefix hash).
  *   mf_cache_put: copies rows [row0, row0 + nrows) of a compressed layer into the pool (rows
  *     already present only move to the front of the LRU order; rows that do not fit evict the
- *     least recently used rows; a row larger than the pool is skipped).  row_ptr_host and
+ *     least recently used rows; a row larger than the pool is skipped, and so is a row that
+ *     reaches past bsr->capacity_blocks, whose blocks an overflowed compression did not all
+ *     write).  row_ptr_host and
  *     col_idx_host are host copies of the BSR's index arrays.  *inserted (optional) = rows added.
  *   mf_cache_get: assembles the longest cached prefix of a request's rows (hashes[0 .. nrows))
  *     into a BSR: row_ptr [hit + 1], col_idx, values (device, capacity blocks).  *hit (host) =

@@ -133,3 +133,32 @@ def test_one_put_larger_than_the_pool_keeps_the_latest_rows_intact():
     assert torch.equal(out.values[:n1 - n0], bsr.values[n0:n1])
     assert torch.equal(out.col_idx[:n1 - n0], bsr.col_idx[n0:n1])
     _status_ok()
+
+
+def test_put_from_an_overflowed_bsr_caches_no_short_row():
+    """A compression that ran out of capacity wrote only the first capacity_blocks blocks; the
+    rows that reach past that point are incomplete and must not be cached (a later hit would
+    return a short row with no error)."""
+    w, pack, full = _request(700)
+    rp = full.row_ptr.cpu().numpy()
+    cap = int(rp[6]) - 1  # rows 0-4 fit; row 5 loses its last block
+    bsr = run_compress(w, pack, capacity=cap)
+    rc, bits = mf.mf_get_status()
+    assert rc == mf.MF_ERR_CAPACITY and bits == 2, (rc, bits)
+    assert bsr.row_ptr.cpu().tolist() == rp.tolist()  # row_ptr holds the true counts
+    toks = np.random.default_rng(3).integers(0, 50000, size=700).astype(np.int32)
+    h = mf.mf_prefix_hashes(toks, 64)
+    cache = mf.BlockCache(_pool(400), 32, 64)
+    assert cache.put(0, bsr, h) == 5
+    out = mf.alloc_bsr(len(h), 400, 32, 64, torch.bfloat16, "cuda")
+    assert cache.get(0, h, out) == 5
+    torch.cuda.synchronize()
+    n = int(rp[5])
+    assert out.row_ptr[:6].cpu().tolist() == rp[:6].tolist()
+    assert torch.equal(out.values[:n], full.values[:n])
+    # the complete rows, put from the full BSR, then fill the rest of the request
+    assert cache.put(0, full, h) == len(h) - 5
+    assert cache.get(0, h, out) == len(h)
+    torch.cuda.synchronize()
+    assert torch.equal(out.values[:int(rp[-1])], full.values[:int(rp[-1])])
+    _status_ok()

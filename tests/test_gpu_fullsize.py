@@ -11,7 +11,8 @@ import torch
 import cross_model_attention_mf_b200 as mf
 import synth
 from synth import device as sdev
-from tests.gpu_common import assert_O_close, check_rows, host_bsr, oracle_O_rows, run_compress
+from tests.gpu_common import (assert_O_close, check_rows, compare_rows, host_bsr, oracle_O_rows,
+                              oracle_pool, run_compress)
 
 pytestmark = pytest.mark.gpu
 
@@ -61,18 +62,51 @@ def test_ministral_pair_full():
     print(f"ministral_pair nnz={nnz} density={nnz / w.causal_blocks:.4f}")
 
 
-@pytest.mark.parametrize("tau,heavy,reading", [(0.95, 8, 1), (0.8, 8, 3)])
+# The long-context sweep: tau x heavy-column count under both map readings.  Points that share
+# (reading, heavy) share one 68.7 GB map fill, so they are listed next to each other.
+LONG_POINTS = [(tau, heavy, reading) for reading in (1, 3) for heavy in (8, 64)
+               for tau in (0.8, 0.9, 0.95, 0.99)]
+# query blocks whose kept sets are compared (row 0, the last row and rows around the middle),
+# and the blocks whose O rows are compared, on a few rows of each block
+LONG_ROWS = [0, 1, 2, 31, 64, 127, 128, 129, 191, 254, 255]
+LONG_O_BLOCKS = [0, 1, 128, 254, 255]
+LONG_O_ROWS = [(0, 4), (60, 68), (120, 128)]
+# most rows whose kept set may differ from the oracle's on one sweep point (only rows in the
+# near-tie band may differ at all); the expectation is 0
+LONG_MAX_MISMATCHED = 1
+
+_long_maps = {}
+
+
+def _long_pack(w):
+    key = (w.n_heavy, w.reading)
+    if key not in _long_maps:
+        _long_maps.clear()
+        torch.cuda.empty_cache()
+        _long_maps[key] = sdev.fill_maps(sdev.alloc_maps(w), w, 0)
+    return _long_maps[key]
+
+
+@pytest.mark.parametrize("tau,heavy,reading", LONG_POINTS,
+                         ids=[f"tau{t}-heavy{h}-R{r}" for t, h, r in LONG_POINTS])
 def test_long_context_full(tau, heavy, reading):
     w = synth.ALL["long_context"].with_(tau=tau, n_heavy=heavy, reading=reading)
-    pack = sdev.fill_maps(sdev.alloc_maps(w), w, 0)
-    bsr = run_compress(w, pack, capacity=w.causal_blocks // 2)
+    pack = _long_pack(w)
+    bsr = run_compress(w, pack, capacity=w.causal_blocks)
     _status_ok()
     nnz = _valid_sets(w, bsr)
-    rows = [(0, qb) for qb in _spread(w.nqb[0], 6)]
-    orows, nb = check_rows(w, pack, bsr, rows)
-    # near-tie rows (the walk ends within 1e-5 of tau, or two ranked masses within 1e-5 of
-    # the total) are allowed to differ; reading 1 has none, the denser reading 3 a few
-    assert nb == 0 or reading == 3
+    rows = [(0, qb) for qb in LONG_ROWS]
+    res = compare_rows(w, pack, bsr, rows)
+    orows, flagged, mism = res["orows"], res["flagged"], res["mismatched"]
+    print(f"long_context tau={tau} heavy={heavy} R{reading} nnz={nnz} "
+          f"density={nnz / w.causal_blocks:.4f} near-tie rows {flagged}/{len(rows)} "
+          f"differing rows {mism}/{len(rows)}")
+    # reading 1 has no near-tie row at all; under reading 3 the close-masses condition flags
+    # rows, but the GPU's masses are far closer to the oracle's than the band, so the kept
+    # sets are expected to match there as well
+    if reading == 1:
+        assert flagged == 0
+    assert mism <= LONG_MAX_MISMATCHED
     W = sdev.w_weights(w)
     V = sdev.v_contiguous(w, 0)
     cu = pack.cu_seqlens
@@ -80,13 +114,16 @@ def test_long_context_full(tau, heavy, reading):
                            w.h_kv, total_q=w.tokens)[0]
     _status_ok()
     Wl, Vh = W[0].cpu().numpy(), V.cpu()
-    for (_, qb) in rows[::2] + [rows[-1]]:
-        want, (lo, hi) = oracle_O_rows(w, orows, 0, qb, Wl, Vh, 0)
-        got = O[qb * w.B + lo:qb * w.B + hi].float().cpu().numpy()
-        assert_O_close(got, want, "bf16", f"long qb={qb}")
-    print(f"long_context tau={tau} heavy={heavy} R{reading} nnz={nnz} density={nnz / w.causal_blocks:.4f} "
-          f"near-tie rows {nb}/{len(rows)}")
-    del pack, bsr, O
+    with oracle_pool() as pool:
+        jobs = [(qb, rr, pool.submit(oracle_O_rows, w, orows, 0, qb, Wl, Vh, 0, row_range=rr))
+                for qb in LONG_O_BLOCKS for rr in LONG_O_ROWS]
+        for qb, rr, f in jobs:
+            want, (lo, hi) = f.result()
+            got = O[qb * w.B + lo:qb * w.B + hi].float().cpu().numpy()
+            assert_O_close(got, want, "bf16", f"long tau={tau} heavy={heavy} R{reading} qb={qb} rows {lo}-{hi}")
+    del bsr, O
+    if (tau, heavy, reading) == LONG_POINTS[-1] or tau == 0.99:
+        _long_maps.clear()
     torch.cuda.empty_cache()
 
 

@@ -292,3 +292,31 @@ def test_bad_page_reported():
                        w.h_r, w.h_kv, total_q=200, paged=(table, 16))
     rc, bits = mf.mf_get_status()
     assert rc == mf.MF_ERR_DEVICE_INDEX and bits & 16
+
+
+@pytest.mark.parametrize("entry", ["mf_compress", "mf_compress_static"])
+def test_empty_batch(entry):
+    """A batch with no query block (max_seqlen 0, an empty sequence) is valid input: an empty
+    BSR (row_ptr [0], nnz 0) and nothing else; retrieval over it writes nothing."""
+    import ctypes
+    dev = "cuda"
+    maps = torch.zeros(8, dtype=torch.bfloat16, device=dev)
+    off = torch.zeros(1, dtype=torch.int64, device=dev)
+    cu = torch.zeros(2, dtype=torch.int32, device=dev)
+    out = mf.alloc_bsr(0, 4, 4, 64, torch.bfloat16, dev)
+    out.row_ptr.fill_(-7)
+    out.nnz.fill_(-7)
+    if entry == "mf_compress":
+        mf.mf_compress(maps, off, cu, 0, 4, 64, 0.9, out)
+    else:
+        d = mf._compress_desc(maps, off, cu, 0, 4, 64, 0.9, out)
+        assert mf._lib.mf_compress_static(ctypes.byref(d), torch.cuda.current_stream().cuda_stream) == mf.MF_OK
+    _status_ok()
+    assert out.row_ptr.cpu().tolist() == [0] and int(out.nnz.cpu()[0]) == 0
+    W = torch.zeros((1, 4, 4), dtype=torch.float32, device=dev)
+    V = torch.zeros((1, 1, 128), dtype=torch.bfloat16, device=dev)
+    O = torch.full((1, 1, 4, 128), 3.0, dtype=torch.bfloat16, device=dev)
+    qb = torch.zeros(1, dtype=torch.int32, device=dev)
+    mf.mf_map_retrieve([out], [0], W, V, cu, cu, qb, 0, 4, 1, O=O)
+    _status_ok()
+    assert (O == 3.0).all()
