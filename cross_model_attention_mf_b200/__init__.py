@@ -11,6 +11,7 @@ Functions mirror the C entry points:
     mf_map_retrieve_multi(...) -> [O]   (one sender, several receivers)
     mf_prefix_hashes(...), BlockCache(...).put / get / stats   (prefix-hash block cache)
     mf_get_status()         -> (status, bits)
+    mf_set_wait_limit(...)  bounded-wait limit (and a test stall) of the tensor-core kernels
     mf_compress_workspace_size(...), mf_retrieve_path(...), mf_version()
     mf_calib_gram(...), mf_calib_solve(...), mf_calib_path(...)   (head-map calibration)
 """
@@ -114,6 +115,8 @@ _lib.mf_retrieve_multi_fused.argtypes = [ctypes.POINTER(RetrieveDesc), ctypes.c_
 _lib.mf_retrieve_multi_fused.restype = ctypes.c_int
 _lib.mf_retrieve_path.argtypes = [ctypes.POINTER(RetrieveDesc)]
 _lib.mf_retrieve_path.restype = ctypes.c_int
+_lib.mf_set_wait_limit.argtypes = [ctypes.c_uint64, ctypes.c_int]
+_lib.mf_set_wait_limit.restype = ctypes.c_int
 _lib.mf_get_status.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
 _lib.mf_get_status.restype = ctypes.c_int
 _lib.mf_last_error.argtypes = []
@@ -458,6 +461,13 @@ class BlockCache:
         o = np.zeros(6, dtype=np.int64)
         _check(_lib.mf_cache_stats(self._h, o.ctypes.data_as(_P)))
         return dict(zip(("rows", "used", "free", "hits", "misses", "evicted"), o.tolist()))
+
+
+def mf_set_wait_limit(limit_ns: int = 0, stall: bool = False) -> None:
+    """Limit of every pipeline wait of the tensor-core kernels for later launches (0: the
+    default, 2 s); stall=True makes those launches wait on a barrier nothing arrives at, so the
+    limit runs out and MF_ERR_TIMEOUT is reported (a test of the timeout path)."""
+    _check(_lib.mf_set_wait_limit(int(limit_ns), 1 if stall else 0))
 
 
 def mf_get_status(stream=None):

@@ -45,7 +45,6 @@ constexpr uint32_t G_STAGE_BYTES = 64 * 1024;
 constexpr uint32_t G_PAD_BYTES = 128 * 128;  // rows an M=128 operand may read past the last tile
 constexpr uint32_t G_OFF_BAR = G_STAGES * G_STAGE_BYTES + G_PAD_BYTES;
 constexpr uint32_t G_SMEM = G_OFF_BAR + 256 + 1024;  // + alignment slack
-constexpr uint64_t G_TIMEOUT_NS = 2000000000ull;
 constexpr int FMAX_TC = 128, FMAX_SIMT = 64, HMAX = 64;
 
 struct GramParams {
@@ -54,6 +53,8 @@ struct GramParams {
   int64_t n_tiles;             // sum over rows i < L of (floor(i / 64) + 1)
   double* partial;             // [gridDim.x][F][F]
   uint32_t* status;
+  uint64_t wait_ns;            // limit of every pipeline wait
+  int stall;                   // test: the MMA warp first waits on a barrier nothing arrives at
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -83,17 +84,17 @@ __device__ __forceinline__ bool bar_try(uint32_t b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// bounded wait: false (and ST_TIMEOUT, abort flag) after G_TIMEOUT_NS or once another role
-// has given up
+// bounded wait: false (and ST_TIMEOUT, abort flag) after limit_ns or once another role has
+// given up
 __device__ __forceinline__ bool bar_wait(uint32_t b, uint32_t parity, volatile int* abort_flag,
-                                         uint32_t* status) {
+                                         uint32_t* status, uint64_t limit_ns) {
   if (bar_try(b, parity)) return true;
   const uint64_t t0 = gtimer();
   for (uint32_t it = 1;; ++it) {
     if (bar_try(b, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort_flag) return false;
-      if (gtimer() - t0 > G_TIMEOUT_NS) {
+      if (gtimer() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicOr(status, ST_TIMEOUT);
         return false;
@@ -184,6 +185,7 @@ __global__ void __launch_bounds__(GT, 1)
   auto FULL = [&](int s) { return bar0 + 8u * (uint32_t)s; };
   auto EMPTY = [&](int s) { return bar0 + 8u * (uint32_t)(G_STAGES + s); };
   const uint32_t DONE = bar0 + 8u * (2 * G_STAGES);
+  const uint32_t NEVER = bar0 + 8u * (2 * G_STAGES + 1);  // test stall: nothing arrives here
   const uint32_t tile_bytes = (uint32_t)p.F8 * 128u;
 
   // stages of p.tps consecutive tiles, dealt round-robin: global stage g goes to CTA
@@ -203,6 +205,7 @@ __global__ void __launch_bounds__(GT, 1)
       bar_init(EMPTY(s), 1);
     }
     bar_init(DONE, 1);
+    bar_init(NEVER, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   // the pad an M=128 operand may read past the last tile of the last stage
@@ -230,7 +233,7 @@ __global__ void __launch_bounds__(GT, 1)
     int issued = 0;
     for (int st = 0; st < n_st && ok; ++st) {
       const int s = st % G_STAGES;
-      ok = __all_sync(0xffffffffu, bar_wait(EMPTY(s), ((st / G_STAGES) & 1) ^ 1, abort_flag, p.status));
+      ok = __all_sync(0xffffffffu, bar_wait(EMPTY(s), ((st / G_STAGES) & 1) ^ 1, abort_flag, p.status, p.wait_ns));
       if (!ok) break;
       int64_t ta;
       int n;
@@ -254,7 +257,7 @@ __global__ void __launch_bounds__(GT, 1)
         const int cnt = issued > s ? (issued - s - 1) / G_STAGES + 1 : 0;
         if (cnt) {
           const uint64_t w0 = gtimer();
-          while (!bar_try(FULL(s), (cnt - 1) & 1) && gtimer() - w0 < G_TIMEOUT_NS) {}
+          while (!bar_try(FULL(s), (cnt - 1) & 1) && gtimer() - w0 < DRAIN_NS) {}
         }
       }
     __syncwarp();
@@ -264,9 +267,11 @@ __global__ void __launch_bounds__(GT, 1)
     const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(p.Fn >> 3) << 17) |
                            ((128u >> 4) << 24);
     bool ok = true;
+    // test stall: a wait that can only run out (the whole CTA then stops as on any timeout)
+    if (p.stall) ok = __all_sync(0xffffffffu, bar_wait(NEVER, 0, abort_flag, p.status, p.wait_ns));
     for (int st = 0; st < n_st && ok; ++st) {
       const int s = st % G_STAGES;
-      ok = __all_sync(0xffffffffu, bar_wait(FULL(s), (st / G_STAGES) & 1, abort_flag, p.status));
+      ok = __all_sync(0xffffffffu, bar_wait(FULL(s), (st / G_STAGES) & 1, abort_flag, p.status, p.wait_ns));
       if (!ok) break;
       int64_t ta;
       int n;
@@ -306,12 +311,12 @@ __global__ void __launch_bounds__(GT, 1)
     if (lane == 0) {
       commit(DONE);
       const uint64_t w0 = gtimer();
-      while (!bar_try(DONE, 0) && gtimer() - w0 < G_TIMEOUT_NS) {}
+      while (!bar_try(DONE, 0) && gtimer() - w0 < DRAIN_NS) {}
     }
     __syncwarp();
   } else {
     // ================================================================ read D
-    bool ok = __all_sync(0xffffffffu, bar_wait(DONE, 0, abort_flag, p.status));
+    bool ok = __all_sync(0xffffffffu, bar_wait(DONE, 0, abort_flag, p.status, p.wait_ns));
     if (ok) {
       fence_after();
       const int q = warp & 3;  // TMEM lane quarter of this warp
@@ -553,6 +558,8 @@ bool launch_calib_gram(const mf_calib_desc& d, void* ws, uint32_t* status, cudaS
     p.n_tiles = tiles_of_length(L);
     p.partial = static_cast<double*>(ws);
     p.status = status;
+    p.wait_ns = wait_limit_ns();
+    p.stall = wait_stall();
     const char* X = static_cast<const char*>(d.sender_maps) + d.sender_seq_offset[s] * esz;
     const char* Y = static_cast<const char*>(d.receiver_maps) + d.receiver_seq_offset[s] * esz;
     int grid;

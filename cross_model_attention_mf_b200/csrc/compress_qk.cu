@@ -53,11 +53,12 @@ constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
 constexpr uint32_t OFF_BAR = OFF_K + KS * K_BYTES;
 constexpr uint32_t QK_SMEM = OFF_BAR + 256 + 1024;  // + alignment slack
-constexpr uint64_t QK_TIMEOUT_NS = 2000000000ull;
 constexpr int META_HDR = 4;                    // CompressWs::meta header words
 enum {
   B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_KEMPTY = B_KFULL + KS, B_SFULL = B_KEMPTY + KS,
-  B_SEMPTY = B_SFULL + 2, B_DONE = B_SEMPTY + 2, B_COUNT = B_DONE + 1
+  B_SEMPTY = B_SFULL + 2, B_DONE = B_SEMPTY + 2,
+  B_NEVER = B_DONE + 1,  // test stall: nothing ever arrives here
+  B_COUNT = B_NEVER + 1
 };
 static_assert(B_COUNT * 8 <= 256, "barrier area");
 static_assert(2 * QK_SMEM <= 232448, "two CTAs per SM");
@@ -81,6 +82,8 @@ struct QkParams {
   __nv_bfloat16* values;
   double* mass;
   uint32_t* status;
+  uint64_t wait_ns;  // limit of every pipeline wait
+  int stall;         // test: the MMA warp first waits on B_NEVER
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -113,17 +116,17 @@ __device__ __forceinline__ bool bar_try(uint32_t b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// bounded wait: false (and ST_TIMEOUT, abort flag) after QK_TIMEOUT_NS or once another role
-// has given up
+// bounded wait: false (and ST_TIMEOUT, abort flag) after limit_ns or once another role has
+// given up
 __device__ __forceinline__ bool bar_wait(uint32_t b, uint32_t parity, volatile int* abort_flag,
-                                         uint32_t* status) {
+                                         uint32_t* status, uint64_t limit_ns) {
   if (bar_try(b, parity)) return true;
   const uint64_t t0 = gtimer();
   for (uint32_t it = 1;; ++it) {
     if (bar_try(b, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort_flag) return false;
-      if (gtimer() - t0 > QK_TIMEOUT_NS) {
+      if (gtimer() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicOr(status, ST_TIMEOUT);
         return false;
@@ -133,7 +136,7 @@ __device__ __forceinline__ bool bar_wait(uint32_t b, uint32_t parity, volatile i
 }
 __device__ __forceinline__ void bar_drain(uint32_t b, uint32_t parity) {
   const uint64_t t0 = gtimer();
-  while (!bar_try(b, parity) && gtimer() - t0 < QK_TIMEOUT_NS) {}
+  while (!bar_try(b, parity) && gtimer() - t0 < DRAIN_NS) {}
 }
 __device__ __forceinline__ void tma3(uint32_t dst, const CUtensorMap* tm, uint32_t b, int c0,
                                      int c1, int c2) {
@@ -302,6 +305,7 @@ __global__ void __launch_bounds__(QT, 2)
       bar_init(bar(B_SEMPTY + b), 4);
     }
     bar_init(bar(B_DONE), 1);
+    bar_init(bar(B_NEVER), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -335,7 +339,7 @@ __global__ void __launch_bounds__(QT, 2)
       while (ok && tiles_next<GATHER>(p, it, ti, &kb, &n0, &n1)) {
         if (first) {
           ok = __all_sync(0xffffffffu, bar_wait(bar(B_QEMPTY), (uint32_t)(qi & 1) ^ 1u, abort_flag,
-                                                p.status));
+                                                p.status, p.wait_ns));
           if (!ok) break;
           if (lane == 0) {
             bar_expect(bar(B_QFULL), Q_BYTES);
@@ -349,7 +353,7 @@ __global__ void __launch_bounds__(QT, 2)
         }
         const int st = (int)(tc % KS);
         ok = __all_sync(0xffffffffu, bar_wait(bar(B_KEMPTY + st), (uint32_t)((tc / KS) & 1) ^ 1u,
-                                              abort_flag, p.status));
+                                              abort_flag, p.status, p.wait_ns));
         if (!ok) break;
         if (lane == 0) {
           bar_expect(bar(B_KFULL + st), K_BYTES);
@@ -374,6 +378,9 @@ __global__ void __launch_bounds__(QT, 2)
     // ================================================================ MMA issue
     bool ok = true;
     int64_t tc = 0, qi = 0;
+    // test stall: a wait that can only run out (the whole CTA then stops as on any timeout)
+    if (p.stall)
+      ok = __all_sync(0xffffffffu, bar_wait(bar(B_NEVER), 0, abort_flag, p.status, p.wait_ns));
     for (int64_t idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
       const QItem it = qdecode(p, idx);
       if (!it.valid) continue;
@@ -385,16 +392,16 @@ __global__ void __launch_bounds__(QT, 2)
       while (ok && tiles_next<GATHER>(p, it, ti, &kb, &n0, &n1)) {
         if (first) {
           ok = __all_sync(0xffffffffu,
-                          bar_wait(bar(B_QFULL), (uint32_t)(qi & 1), abort_flag, p.status));
+                          bar_wait(bar(B_QFULL), (uint32_t)(qi & 1), abort_flag, p.status, p.wait_ns));
           if (!ok) break;
           first = false;
         }
         const int st = (int)(tc % KS), b = (int)(tc & 1);
         ok = __all_sync(0xffffffffu, bar_wait(bar(B_KFULL + st), (uint32_t)((tc / KS) & 1),
-                                              abort_flag, p.status));
+                                              abort_flag, p.status, p.wait_ns));
         if (ok)
           ok = __all_sync(0xffffffffu, bar_wait(bar(B_SEMPTY + b), (uint32_t)((tc >> 1) & 1) ^ 1u,
-                                                abort_flag, p.status));
+                                                abort_flag, p.status, p.wait_ns));
         if (!ok) break;
         if (lane == 0) {
           fence_after();
@@ -444,7 +451,7 @@ __global__ void __launch_bounds__(QT, 2)
       while (tiles_next<GATHER>(p, it, ti, &kb, &n0, &n1)) {
         const int b = (int)(tc & 1);
         ok = __all_sync(0xffffffffu, bar_wait(bar(B_SFULL + b), (uint32_t)((tc >> 1) & 1),
-                                              abort_flag, p.status));
+                                              abort_flag, p.status, p.wait_ns));
         if (!ok) break;
         fence_after();
         uint32_t v0[32], v1[32];
@@ -673,6 +680,8 @@ bool launch_compress_qk(const mf_compress_qk_desc& d, const CompressWs& ws, cons
   p.values = static_cast<__nv_bfloat16*>(d.values);
   p.mass = d.block_mass_out ? d.block_mass_out : ws.mass;
   p.status = status;
+  p.wait_ns = wait_limit_ns();
+  p.stall = wait_stall();
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -2,6 +2,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <cstdio>
 #include <mutex>
 #include <algorithm>
@@ -112,7 +113,18 @@ mf_status static_ws_ptr(void** out) {
   return MF_OK;
 }
 
+std::atomic<uint64_t> g_wait_ns{0};  // 0: the default limit
+std::atomic<int> g_stall{0};
+
 }  // namespace
+
+namespace mfi {
+uint64_t wait_limit_ns() {
+  const uint64_t v = g_wait_ns.load(std::memory_order_relaxed);
+  return v ? v : DRAIN_NS;
+}
+int wait_stall() { return g_stall.load(std::memory_order_relaxed); }
+}  // namespace mfi
 
 namespace {
 // receiver layer l of a retrieval descriptor
@@ -481,6 +493,12 @@ mf_status mf_calib_solve(const double* gram, int h_s, int h_r, double ridge, flo
   cudaError_t e = mfi::launch_calib_solve(gram, h_s, h_r, ridge, W, residual, st,
                                           static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(MF_ERR_CUDA, std::string("calib solve launch: ") + cudaGetErrorString(e));
+  return MF_OK;
+}
+
+mf_status mf_set_wait_limit(uint64_t limit_ns, int stall) {
+  g_wait_ns.store(limit_ns, std::memory_order_relaxed);
+  g_stall.store(stall ? 1 : 0, std::memory_order_relaxed);
   return MF_OK;
 }
 

@@ -20,6 +20,12 @@ enum : uint32_t {
   ST_SINGULAR = 32u, // a calibration Gram that is not positive definite
 };
 
+// limit of every pipeline wait in the tensor-core kernels (ns) and the test stall flag, as set
+// by mf_set_wait_limit (read at each launch)
+uint64_t wait_limit_ns();
+int wait_stall();
+constexpr uint64_t DRAIN_NS = 2000000000ull;  // bound of the waits for work already issued
+
 // scratch of mf_compress (carved out of the caller's workspace)
 struct CompressWs {
   int64_t* meta;      // [4 + 4 * nseq]: total rows, total causal blocks, -, -, then per

@@ -40,9 +40,9 @@
 // 0-1, 2-3), so P.V of one half overlaps the conversion of the other.  Consumer warps
 // wait with all 32 lanes (the hardware suspends such a warp; a lone polling lane would
 // spin) and signal once per warp (lane 0 after __syncwarp).  TMEM: D2 in columns
-// [0, 256), D1 in [256, 512).  Every mbarrier wait is bounded by a timer: on expiry the
-// CTA records ST_TIMEOUT, all roles stop, in-flight copies and MMAs are drained (bounded)
-// and TMEM is freed.
+// [0, 256), D1 in [256, 512).  Every mbarrier wait is bounded by a timer (mf_set_wait_limit,
+// default 2 s): on expiry the CTA records ST_TIMEOUT, all roles stop, in-flight copies and
+// MMAs are drained (bounded) and TMEM is freed.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -93,14 +93,15 @@ constexpr uint32_t OFF_ITEMS = OFF_W + W_BYTES_MAX;
 constexpr uint32_t OFF_BAR = OFF_ITEMS + ITEMS_MAX * ITEM_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "dynamic shared memory of one CTA");
-constexpr uint64_t TIMEOUT_NS = 2000000000ull;
 
 // barrier slots (8 bytes each)
 enum {
   B_AFULL = 0, B_AEMPTY = B_AFULL + A_STAGES, B_HFULL = B_AEMPTY + A_STAGES,
   B_HEMPTY = B_HFULL + HS, B_D1FULL = B_HEMPTY + HS, B_D1EMPTY = B_D1FULL + 1,
   B_OFULL = B_D1EMPTY + 1,
-  B_OEMPTY = B_OFULL + 1, B_DRAIN1 = B_OEMPTY + 2, B_DRAIN2 = B_DRAIN1 + 1, B_COUNT = B_DRAIN2 + 1
+  B_OEMPTY = B_OFULL + 1, B_DRAIN1 = B_OEMPTY + 2, B_DRAIN2 = B_DRAIN1 + 1,
+  B_NEVER = B_DRAIN2 + 1,  // test stall: nothing ever arrives here
+  B_COUNT = B_NEVER + 1
 };
 static_assert(B_COUNT * 8 <= 512, "barrier area");
 
@@ -136,6 +137,8 @@ struct TcParams {
   int h_s, nsc, B;
   RecvParams rv[NRMAX];
   uint32_t* status;
+  uint64_t wait_ns;  // limit of every pipeline wait
+  int stall;         // test: the mixing issuer first waits on B_NEVER
 };
 struct VMaps {
   CUtensorMap m[NRMAX];
@@ -171,16 +174,16 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: false if the CTA aborted or the wait ran out of time.
+// Bounded wait: false if the CTA aborted or the wait ran out of time (limit_ns).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status) {
+                                          uint32_t* status, uint64_t limit_ns) {
   if (mbar_try(bar, parity)) return true;
   uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > TIMEOUT_NS) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicOr(status, ST_TIMEOUT);
         return false;
@@ -369,6 +372,7 @@ __global__ void __launch_bounds__(NT, 1)
     mbar_init(bar(B_OFULL), 1);
     mbar_init(bar(B_DRAIN1), 1);
     mbar_init(bar(B_DRAIN2), 1);
+    mbar_init(bar(B_NEVER), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -436,7 +440,7 @@ __global__ void __launch_bounds__(NT, 1)
           }
           if (is_a) {
             for (int c = 0; c < p.nsc && ok; ++c) {
-              if (!(ok = mbar_wait(bar(B_AEMPTY + as), aph ^ 1, abort_flag, p.status))) break;
+              if (!(ok = mbar_wait(bar(B_AEMPTY + as), aph ^ 1, abort_flag, p.status, p.wait_ns))) break;
               TRACE(0, 3);
               mbar_expect_tx(bar(B_AFULL + as), A_BYTES);
               tma_load_4d(sb + OFF_A + as * A_BYTES, &tmA, bar(B_AFULL + as), half * KT, c * SC,
@@ -452,7 +456,7 @@ __global__ void __launch_bounds__(NT, 1)
           if (!kb_ok) atomicOr(p.status, ST_INDEX);
           const int tok0 = kb * p.B + half * KT;
           for (int h = 0; h < NG / PH && ok; ++h) {
-            if (!(ok = mbar_wait(bar(B_HEMPTY + vs), vph ^ 1, abort_flag, p.status))) break;
+            if (!(ok = mbar_wait(bar(B_HEMPTY + vs), vph ^ 1, abort_flag, p.status, p.wait_ns))) break;
             TRACE(5, 4);
             mbar_expect_tx(bar(B_HFULL + vs), V_BYTES);
             for (int gl = 0; gl < PH; ++gl) {
@@ -489,7 +493,7 @@ __global__ void __launch_bounds__(NT, 1)
         const int cnt = a_issued > k ? (a_issued - k - 1) / A_STAGES + 1 : 0;
         if (cnt) {
           const uint64_t t0 = globaltimer();
-          while (!mbar_try(bar(B_AFULL + k), (cnt - 1) & 1) && globaltimer() - t0 < TIMEOUT_NS) {}
+          while (!mbar_try(bar(B_AFULL + k), (cnt - 1) & 1) && globaltimer() - t0 < DRAIN_NS) {}
         }
       }
       // (a V slot's phase also needs the converters' arrivals: after an abort this wait runs
@@ -498,7 +502,7 @@ __global__ void __launch_bounds__(NT, 1)
         const int cnt = v_issued > k ? (v_issued - k - 1) / HS + 1 : 0;
         if (cnt) {
           const uint64_t t0 = globaltimer();
-          while (!mbar_try(bar(B_HFULL + k), (cnt - 1) & 1) && globaltimer() - t0 < TIMEOUT_NS) {}
+          while (!mbar_try(bar(B_HFULL + k), (cnt - 1) & 1) && globaltimer() - t0 < DRAIN_NS) {}
         }
       }
     }
@@ -511,17 +515,19 @@ __global__ void __launch_bounds__(NT, 1)
       int T = 0;  // tiles processed so far
       const uint64_t wdesc0 = smem_desc(sb + OFF_W, 512u, 128u, 0u);
       const uint64_t adesc0 = smem_desc(sb + OFF_A, 2048u, 1024u, 2u);
+      // test stall: a wait that can only run out (the whole CTA then stops as on any timeout)
+      if (p.stall) ok = mbar_wait(bar(B_NEVER), 0, abort_flag, p.status, p.wait_ns);
       for (int idx = blockIdx.x, ik = 0; idx < p.n_items && ok; idx += gridDim.x, ++ik) {
         const Item it = item(ik, idx);
         if (!it.valid) continue;
         TRACE(1, 1);
         for (int t = 0; t < it.n_tiles && ok; ++t, ++T) {
           // D1 must have been read out by the previous tile's converters
-          if (!(ok = mbar_wait(bar(B_D1EMPTY), (T & 1) ^ 1, abort_flag, p.status))) break;
+          if (!(ok = mbar_wait(bar(B_D1EMPTY), (T & 1) ^ 1, abort_flag, p.status, p.wait_ns))) break;
           tc_fence_after();
           // chunk-major: each s-chunk is mixed into all eight M tiles, then its stage is freed
           for (int c = 0; c < p.nsc && ok; ++c) {
-            if (!(ok = mbar_wait(bar(B_AFULL + as), aph, abort_flag, p.status))) break;
+            if (!(ok = mbar_wait(bar(B_AFULL + as), aph, abort_flag, p.status, p.wait_ns))) break;
             tc_fence_after();
             if (c == 0) TRACE(1, 3);
             const uint64_t ad = adesc0 + (((uint32_t)as * A_BYTES) >> 4);
@@ -541,7 +547,7 @@ __global__ void __launch_bounds__(NT, 1)
       }
       tc_commit(bar(B_DRAIN1));
       const uint64_t t0 = globaltimer();
-      while (!mbar_try(bar(B_DRAIN1), 0) && globaltimer() - t0 < TIMEOUT_NS) {}
+      while (!mbar_try(bar(B_DRAIN1), 0) && globaltimer() - t0 < DRAIN_NS) {}
     }
   } else if (warp == 2) {
     // ================================================================ P.V MMA issuer
@@ -559,11 +565,11 @@ __global__ void __launch_bounds__(NT, 1)
         for (int t = 0; t < it.n_tiles && ok; ++t, ++T) {
           for (int h = 0; h < NG / PH && ok; ++h) {
             // the half's V tiles and P^T are in slot vs
-            if (!(ok = mbar_wait(bar(B_HFULL + vs), vph, abort_flag, p.status))) break;
+            if (!(ok = mbar_wait(bar(B_HFULL + vs), vph, abort_flag, p.status, p.wait_ns))) break;
             TRACE(4, 8);
             // the previous item's epilogue must have read this half of D2 out
             if (t == 0 && K > 0) {
-              if (!(ok = mbar_wait(bar(B_OEMPTY + h), (K - 1) & 1, abort_flag, p.status))) break;
+              if (!(ok = mbar_wait(bar(B_OEMPTY + h), (K - 1) & 1, abort_flag, p.status, p.wait_ns))) break;
               TRACE(4, 9);
             }
             tc_fence_after();
@@ -590,7 +596,7 @@ __global__ void __launch_bounds__(NT, 1)
         if (!ok) break;
         if (it.n_tiles == 0 && K > 0) {  // take the epilogue's phases in order all the same
           for (int h = 0; h < NG / PH && ok; ++h)
-            ok = mbar_wait(bar(B_OEMPTY + h), (K - 1) & 1, abort_flag, p.status);
+            ok = mbar_wait(bar(B_OEMPTY + h), (K - 1) & 1, abort_flag, p.status, p.wait_ns);
           if (!ok) break;
         }
         tc_commit(bar(B_OFULL));  // D2 of this item complete (immediate when it has no tile)
@@ -599,7 +605,7 @@ __global__ void __launch_bounds__(NT, 1)
       }
       tc_commit(bar(B_DRAIN2));
       const uint64_t t0 = globaltimer();
-      while (!mbar_try(bar(B_DRAIN2), 0) && globaltimer() - t0 < TIMEOUT_NS) {}
+      while (!mbar_try(bar(B_DRAIN2), 0) && globaltimer() - t0 < DRAIN_NS) {}
     }
   } else if (warp < 4 + 4 * CONV_SETS) {
     // ================================================================ convert P (hi + lo)
@@ -623,7 +629,7 @@ __global__ void __launch_bounds__(NT, 1)
       const Item q = item(ek, eidx);
       const bool have = q.n_tiles > 0;
       const int ilo = q.row_lo - q.i_begin, ihi = q.row_hi - q.i_begin;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_OFULL), K & 1, abort_flag, p.status)))
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_OFULL), K & 1, abort_flag, p.status, p.wait_ns)))
         return false;
       tc_fence_after();
       if (warp == 4 && lane == 0) TRACE(3, 1);
@@ -690,7 +696,7 @@ __global__ void __launch_bounds__(NT, 1)
         const bool kb_ok = kb >= 0 && kb <= it.qb;
         const int tok0 = kb * p.B + half * KT;
         // warp-uniform control flow: tcgen05.ld is a warp-collective instruction
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_D1FULL), T & 1, abort_flag, p.status));
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_D1FULL), T & 1, abort_flag, p.status, p.wait_ns));
         if (!ok) break;
         tc_fence_after();
         if (warp == 4 && lane == 0) TRACE(2, 1);
@@ -741,7 +747,7 @@ __global__ void __launch_bounds__(NT, 1)
           // this half of the P buffer must have been consumed by the previous tile's P.V
           const int hq = T * (NG / PH) + h, ps = hq % HS;  // half-tile count, slot
           ok = __all_sync(0xffffffffu, mbar_wait(bar(B_HEMPTY + ps), ((hq / HS) & 1) ^ 1,
-                                                 abort_flag, p.status));
+                                                 abort_flag, p.status, p.wait_ns));
           if (!ok) break;
           if (warp == 4 && lane == 0) TRACE(2, 4);
 #pragma unroll
@@ -854,6 +860,8 @@ bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* 
   p.h_s = d0.h_s; p.nsc = (d0.h_s + SC - 1) / SC; p.B = B;
   p.nrecv = n;
   p.status = status;
+  p.wait_ns = wait_limit_ns();
+  p.stall = wait_stall();
   int NH = 0;
   for (int k = 0; k < n; ++k) {
     const mf_retrieve_desc& d = *ds[k];

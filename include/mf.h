@@ -373,6 +373,22 @@ mf_status mf_cache_get(mf_block_cache* cache, int32_t layer, const uint64_t* has
                        int32_t* hit, void* stream);
 mf_status mf_cache_stats(mf_block_cache* cache, int64_t* out6);
 
+/* ------------------------------------------------------------------------------
+ * Bounded waits (a property of this library; the MapFlow pages have no counterpart).
+ * Every pipeline wait inside the tensor-core kernels (mf_map_retrieve and
+ * mf_map_retrieve_multi on the tcgen05 path, mf_compress_qk, mf_calib_gram on the tcgen05
+ * path) gives up after a time limit: the CTA then records MF_ERR_TIMEOUT in the status word,
+ * every role of the CTA stops, the copies and MMAs it already issued are waited for (bounded
+ * by 2 s) and its tensor memory is released, so the kernel returns and the context stays
+ * usable.  mf_set_wait_limit sets that limit, in nanoseconds, for the launches made after the
+ * call by any thread of this process; limit_ns = 0 restores the default of 2 s.  With
+ * stall != 0 those launches also make the MMA-issuing warp of every CTA first wait on a
+ * barrier that nothing arrives at, so the limit is certain to run out: a way to exercise the
+ * timeout path without a fault or a hang.  The outputs of a launch that timed out are
+ * undefined; a later call with stall = 0 computes normally.  Always returns MF_OK.
+ * ------------------------------------------------------------------------------ */
+mf_status mf_set_wait_limit(uint64_t limit_ns, int stall);
+
 /* Synchronise `stream`, then read and clear this device's status word.  *bits
  * (optional) receives the raw bits: 1 index out of range, 2 capacity, 4 wait
  * timeout, 8 misaligned input, 16 page id out of range, 32 singular

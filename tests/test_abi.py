@@ -230,3 +230,10 @@ def test_multi_receiver_binding_descriptors(mf):
                           16, 2, O=torch.zeros(1, 100, 16, 128, dtype=torch.bfloat16)))
     arr, keep, outs = mf._multi_descs(layers, rs, cu, cu, qb, 100, 100, None)
     assert mf._lib.mf_retrieve_multi_fused(arr, 3) == 0
+
+
+def test_wait_limit_setter(mf):
+    """The bounded-wait limit is host state read at each launch: setting and restoring it needs
+    no device (the GPU tests in test_gpu_timeout.py make a wait run out with it)."""
+    assert mf._lib.mf_set_wait_limit(5_000_000, 1) == mf.MF_OK
+    assert mf._lib.mf_set_wait_limit(0, 0) == mf.MF_OK
