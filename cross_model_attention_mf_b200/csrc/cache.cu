@@ -13,9 +13,10 @@
 // block copies run on the GPU.
 //
 // Copies.  k_cache_copy moves whole blocks (16-byte vector loads, each block split over 8 CTAs);
-// the list of (source block, destination block, column) triples travels as a kernel parameter in
-// chunks of CHUNK, so a put or a get needs no staging buffer and no synchronisation: it is
-// ordered on the caller's stream like any other launch.  Rows evicted by a put may still be read
+// the list of (source block, destination block, column) triples, and for a get the row
+// pointers, travel as a kernel parameter (in structs of 64, 256 or 1024 entries), so a put or a
+// get needs no staging buffer and no synchronisation: it is ordered on the caller's stream like
+// any other launch.  Rows evicted by a put may still be read
 // by an earlier get on another stream; the caller orders puts after the gets that precede them.
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -32,24 +33,32 @@
 namespace mfi {
 namespace {
 
-constexpr int CHUNK = 1024;  // copies per launch (12 KB of kernel parameters)
-
+// A launch carries its copy list as a kernel parameter: (source block, destination block,
+// column) triples and, for a get, the row pointers of the assembled rows.  The parameter
+// struct comes in three sizes so that a small request does not ship 12 KB of parameters.
+template <int N>
 struct CopyChunk {
   const uint4* src;   // block k of the source at src + src_blk[k] * blk_vecs
   uint4* dst;
   int32_t* col_dst;   // when not NULL: col_dst[dst_blk[k]] = col[k]
+  int32_t* row_ptr;   // when not NULL: row_ptr[rp_first + k] = rp[k], k < rp_n
   int64_t blk_vecs;   // 16-byte vectors per block
-  int n;
-  int32_t src_blk[CHUNK];
-  int32_t dst_blk[CHUNK];
-  int32_t col[CHUNK];
+  int n, rp_first, rp_n;
+  int32_t src_blk[N];
+  int32_t dst_blk[N];
+  int32_t col[N];
+  int32_t rp[N + 1];
 };
+constexpr int CHUNK_MAX = 1024;  // copies per launch (the largest parameter struct, 16 KB)
 
 // grid (blocks, SPLIT): CTA (k, part) copies part `part` of block k, four 16-byte vectors in
-// flight per thread
+// flight per thread; CTA (0, 0) also writes the row pointers the launch carries
 constexpr int SPLIT = 8;
-__global__ void __launch_bounds__(256) k_cache_copy(const __grid_constant__ CopyChunk c) {
+template <int N>
+__global__ void __launch_bounds__(256) k_cache_copy(const __grid_constant__ CopyChunk<N> c) {
   const int k = blockIdx.x;
+  if (c.row_ptr && k == 0 && blockIdx.y == 0)
+    for (int e = threadIdx.x; e < c.rp_n; e += 256) c.row_ptr[c.rp_first + e] = c.rp[e];
   if (k >= c.n) return;
   const uint4* s = c.src + (int64_t)c.src_blk[k] * c.blk_vecs;
   uint4* d = c.dst + (int64_t)c.dst_blk[k] * c.blk_vecs;
@@ -65,16 +74,6 @@ __global__ void __launch_bounds__(256) k_cache_copy(const __grid_constant__ Copy
       if (v + u * 256 < v1) d[v + u * 256] = r[u];
   }
   if (c.col_dst && blockIdx.y == 0 && threadIdx.x == 0) c.col_dst[c.dst_blk[k]] = c.col[k];
-}
-
-constexpr int RP_CHUNK = 512;
-struct RowPtrChunk {
-  int32_t* row_ptr;
-  int first, n;
-  int32_t v[RP_CHUNK];
-};
-__global__ void k_cache_row_ptr(const __grid_constant__ RowPtrChunk c) {
-  for (int k = threadIdx.x; k < c.n; k += blockDim.x) c.row_ptr[c.first + k] = c.v[k];
 }
 
 struct Key {
@@ -107,23 +106,50 @@ struct BlockCache {
 
 namespace {
 
+template <int N>
+bool launch_chunk(const char* src, char* dst, int32_t* col_dst, int64_t blk_bytes,
+                  const std::vector<int32_t>& s, const std::vector<int32_t>& d,
+                  const std::vector<int32_t>& col, size_t k0, int n, int32_t* row_ptr,
+                  const std::vector<int32_t>& rp, size_t r0, int rp_n, cudaStream_t st) {
+  CopyChunk<N> c;
+  c.src = reinterpret_cast<const uint4*>(src);
+  c.dst = reinterpret_cast<uint4*>(dst);
+  c.col_dst = col_dst;
+  c.row_ptr = rp_n > 0 ? row_ptr : nullptr;
+  c.blk_vecs = blk_bytes / 16;
+  c.n = n;
+  c.rp_first = (int)r0;
+  c.rp_n = rp_n;
+  for (int k = 0; k < n; ++k) {
+    c.src_blk[k] = s[k0 + k];
+    c.dst_blk[k] = d[k0 + k];
+    c.col[k] = col.empty() ? 0 : col[k0 + k];
+  }
+  for (int k = 0; k < rp_n; ++k) c.rp[k] = rp[r0 + k];
+  k_cache_copy<N><<<dim3((unsigned)std::max(n, 1), SPLIT), 256, 0, st>>>(c);
+  return cudaGetLastError() == cudaSuccess;
+}
+
+// Copies block s[k] of src to block d[k] of dst (and col[k] to col_dst[d[k]] when col_dst is
+// set), and writes rp[] to row_ptr[] when row_ptr is set, in as few launches as the parameter
+// limit allows.
 bool launch_copies(const char* src, char* dst, int32_t* col_dst, int64_t blk_bytes,
                    const std::vector<int32_t>& s, const std::vector<int32_t>& d,
-                   const std::vector<int32_t>& col, cudaStream_t st) {
-  for (size_t k0 = 0; k0 < s.size(); k0 += CHUNK) {
-    CopyChunk c;
-    c.src = reinterpret_cast<const uint4*>(src);
-    c.dst = reinterpret_cast<uint4*>(dst);
-    c.col_dst = col_dst;
-    c.blk_vecs = blk_bytes / 16;
-    c.n = (int)std::min<size_t>(CHUNK, s.size() - k0);
-    for (int k = 0; k < c.n; ++k) {
-      c.src_blk[k] = s[k0 + k];
-      c.dst_blk[k] = d[k0 + k];
-      c.col[k] = col.empty() ? 0 : col[k0 + k];
-    }
-    k_cache_copy<<<dim3((unsigned)c.n, SPLIT), 256, 0, st>>>(c);
-    if (cudaGetLastError() != cudaSuccess) return false;
+                   const std::vector<int32_t>& col, int32_t* row_ptr,
+                   const std::vector<int32_t>& rp, cudaStream_t st) {
+  size_t k0 = 0, r0 = 0;
+  const size_t n_rp = row_ptr ? rp.size() : 0;
+  while (k0 < s.size() || r0 < n_rp) {
+    const size_t left = std::max(s.size() - k0, n_rp - r0 > 0 ? n_rp - r0 - 1 : 0);
+    const int N = left <= 64 ? 64 : left <= 256 ? 256 : CHUNK_MAX;
+    const int n = (int)std::min<size_t>(N, s.size() - k0);
+    const int rp_n = (int)std::min<size_t>(N + 1, n_rp - r0);
+    bool ok = N == 64 ? launch_chunk<64>(src, dst, col_dst, blk_bytes, s, d, col, k0, n, row_ptr, rp, r0, rp_n, st)
+            : N == 256 ? launch_chunk<256>(src, dst, col_dst, blk_bytes, s, d, col, k0, n, row_ptr, rp, r0, rp_n, st)
+                       : launch_chunk<CHUNK_MAX>(src, dst, col_dst, blk_bytes, s, d, col, k0, n, row_ptr, rp, r0, rp_n, st);
+    if (!ok) return false;
+    k0 += n;
+    r0 += rp_n;
   }
   return true;
 }
@@ -173,7 +199,7 @@ int64_t cache_put(BlockCache* c, int layer, const mf_bsr& bsr, const int32_t* ro
       // a slot freed below may be the target of a copy gathered earlier in this call: launch
       // those copies first, so that stream order puts the new row's copy after them
       if (!launch_copies(static_cast<const char*>(bsr.values), c->pool, nullptr, c->slot_bytes, src,
-                         dst, {}, st))
+                         dst, {}, nullptr, {}, st))
         return -1;
       src.clear();
       dst.clear();
@@ -200,8 +226,8 @@ int64_t cache_put(BlockCache* c, int layer, const mf_bsr& bsr, const int32_t* ro
     c->index.emplace(key, std::move(e));
     ++inserted;
   }
-  if (!src.empty() &&
-      !launch_copies(static_cast<const char*>(bsr.values), c->pool, nullptr, c->slot_bytes, src, dst, {}, st))
+  if (!src.empty() && !launch_copies(static_cast<const char*>(bsr.values), c->pool, nullptr,
+                                     c->slot_bytes, src, dst, {}, nullptr, {}, st))
     return -1;
   return inserted;
 }
@@ -213,6 +239,7 @@ bool cache_get(BlockCache* c, int layer, const uint64_t* hashes, int nrows, int3
                int32_t* col_idx, void* values, int64_t capacity, int* hit, cudaStream_t st) {
   std::lock_guard<std::mutex> g(c->mu);
   std::vector<int32_t> src, dst, col, rp{0};
+  src.reserve(256); dst.reserve(256); col.reserve(256); rp.reserve((size_t)nrows + 1);
   int h = 0;
   for (int r = 0; r < nrows; ++r) {
     auto it = c->index.find(Key{layer, hashes[r]});
@@ -230,19 +257,9 @@ bool cache_get(BlockCache* c, int layer, const uint64_t* hashes, int nrows, int3
     ++h;
   }
   *hit = h;
-  if (!src.empty() &&
-      !launch_copies(c->pool, static_cast<char*>(values), col_idx, c->slot_bytes, src, dst, col, st))
-    return false;
-  for (size_t k0 = 0; k0 < rp.size(); k0 += RP_CHUNK) {
-    RowPtrChunk q;
-    q.row_ptr = row_ptr;
-    q.first = (int)k0;
-    q.n = (int)std::min<size_t>(RP_CHUNK, rp.size() - k0);
-    for (int k = 0; k < q.n; ++k) q.v[k] = rp[k0 + k];
-    k_cache_row_ptr<<<1, 256, 0, st>>>(q);
-    if (cudaGetLastError() != cudaSuccess) return false;
-  }
-  return true;
+  // one launch (for requests of up to 1024 blocks) copies the blocks and writes row_ptr
+  return launch_copies(c->pool, static_cast<char*>(values), col_idx, c->slot_bytes, src, dst, col,
+                       row_ptr, rp, st);
 }
 
 void cache_stats(BlockCache* c, int64_t* out6) {

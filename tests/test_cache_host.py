@@ -9,6 +9,8 @@ import ctypes
 import numpy as np
 import pytest
 
+from oracle.cache_model import prefix_hashes
+
 
 @pytest.fixture(scope="module")
 def mf():
@@ -18,22 +20,11 @@ def mf():
     return mf
 
 
-def _fnv1a_prefixes(tokens, B):
-    """FNV-1a 64 of every block-ending prefix, from the published definition."""
-    h, out, mask = 0xcbf29ce484222325, [], (1 << 64) - 1
-    for k in range(-(-len(tokens) // B)):
-        for t in tokens[k * B:(k + 1) * B]:
-            for byte in int(t).to_bytes(4, "little", signed=True):
-                h = ((h ^ byte) * 0x100000001b3) & mask
-        out.append(h)
-    return out
-
-
 def test_prefix_hashes_definition_and_prefix_property(mf):
     rng = np.random.default_rng(0)
     toks = rng.integers(-5, 150000, size=333).astype(np.int32)
     h = mf.mf_prefix_hashes(toks, 64)
-    assert h.tolist() == _fnv1a_prefixes(toks.tolist(), 64)
+    assert h.tolist() == prefix_hashes(toks, 64)  # the oracle's FNV-1a, pinned to published vectors
     assert len(h) == 6
     # a shared prefix gives shared hashes up to the first differing block, then none
     other = toks.copy()

@@ -162,3 +162,72 @@ def test_put_from_an_overflowed_bsr_caches_no_short_row():
     torch.cuda.synchronize()
     assert torch.equal(out.values[:int(rp[-1])], full.values[:int(rp[-1])])
     _status_ok()
+
+
+def test_matches_the_host_model():
+    """A sequence of puts and gets over two layers and three requests (two sharing a prefix),
+    in a pool small enough to evict: after every operation the library's return value, its
+    counters and every assembled row (row_ptr, col_idx, values, bit for bit) equal those of
+    the plain host model of the cache (oracle/cache_model.py)."""
+    import oracle
+    from oracle.cache_model import PrefixCacheModel, prefix_hashes
+
+    rng = np.random.default_rng(7)
+    toks_a = rng.integers(0, 50000, size=700).astype(np.int32)
+    toks_b = np.concatenate([toks_a[:320], rng.integers(0, 50000, size=380).astype(np.int32)])
+    toks_c = rng.integers(0, 50000, size=700).astype(np.int32)
+    hashes = {}
+    for name, toks in (("A", toks_a), ("B", toks_b), ("C", toks_c)):
+        h = mf.mf_prefix_hashes(toks, 64)
+        assert h.tolist() == prefix_hashes(toks, 64)
+        hashes[name] = h
+    # compressed layers: layer 0 from request A's maps (its rows serve every request in this
+    # test: only the keys differ), layer 1 from another map layer
+    w, pack, bsr0 = _request(700)
+    sdev.fill_maps(pack, w, 1)
+    bsr1 = run_compress(w, pack)
+    _status_ok()
+    src = {}
+    for layer, b in ((0, bsr0), (1, bsr1)):
+        raw, _ = oracle.as_raw(b.values[:int(b.nnz.cpu()[0])].cpu())
+        src[layer] = (b, b.row_ptr.cpu().numpy(), b.col_idx.cpu().numpy(), raw)
+    n_slots = 60
+    cache = mf.BlockCache(_pool(n_slots), 32, 64)
+    model = PrefixCacheModel(n_slots)
+    out = mf.alloc_bsr(11, 200, 32, 64, torch.bfloat16, "cuda")
+
+    def put(layer, req, row0, n):
+        b, rp, ci, raw = src[layer]
+        h = hashes[req][row0:row0 + n]
+        got = cache.put(layer, b, h, row0=row0, nrows=n)
+        want = model.put(layer, rp, ci, raw, b.capacity, row0, h.tolist())
+        assert got == want, ("put", layer, req, row0, n, got, want)
+
+    def get(layer, req, capacity=200):
+        out.row_ptr.fill_(-1)
+        o = mf.BSR(out.row_ptr, out.col_idx, out.values[:capacity], out.nnz)
+        got = cache.get(layer, hashes[req], o)
+        want, rp, ci, vals = model.get(layer, hashes[req].tolist(), capacity)
+        assert got == want, ("get", layer, req, got, want)
+        torch.cuda.synchronize()
+        assert out.row_ptr[:got + 1].cpu().tolist() == rp
+        n = rp[-1]
+        assert out.col_idx[:n].cpu().tolist() == ci
+        if n:
+            raw, _ = oracle.as_raw(out.values[:n].cpu())
+            assert raw.tobytes() == vals.tobytes()
+
+    ops = [("put", 0, "A", 0, 11), ("get", 0, "B"), ("put", 1, "A", 0, 6), ("put", 0, "C", 0, 11),
+           ("get", 0, "A"), ("get", 1, "B"), ("put", 0, "B", 0, 11), ("get", 0, "C"),
+           ("get", 0, "A", 30), ("put", 1, "C", 3, 8), ("get", 1, "A"), ("get", 0, "B"),
+           ("put", 0, "A", 5, 6), ("get", 0, "A")]
+    for op in ops:
+        if op[0] == "put":
+            put(*op[1:])
+        else:
+            get(*op[1:])
+        st = cache.stats()
+        ms = model.stats()
+        assert st == ms, (op, st, ms)
+    assert cache.stats()["evicted"] > 0
+    _status_ok()
