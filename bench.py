@@ -268,8 +268,13 @@ def run_ours(args, rank, world, dev):
     if rank == 0 and not args.no_calib:
         calib = run_calib(w, mf, pack, dev, args.calib_len)
 
+    cold = None
+    if rank == 0 and not args.no_configs:
+        hbm, tf_burst, _, _ = peaks()
+        cold = run_cold_retrieve(w, mf, bsr, nnz, W, V, O, qbase, dev, hbm, tf_burst)
+
     return dict(w=w, nnz=nnz, elapsed=elapsed, t_comp=t_comp, t_ret=t_ret, clocks=clk.summary(),
-                e2e=e2e, calib=calib, multi=multi, cqk=cqk, pcache=pcache)
+                e2e=e2e, calib=calib, multi=multi, cqk=cqk, pcache=pcache, cold=cold)
 
 
 def run_calib(w, mf, pack, dev, calib_len=0, reps=5):
@@ -534,17 +539,307 @@ def run_e2e(args, w, mf, pack, W, V, bsr, ws, O, qbase, dev):
             "d2h_bytes_per_step": int(d2h), "steps": n}
 
 
+# ------------------------------------------------------------------------ the other workloads
+L2_FLUSH_BYTES = 256 << 20  # written between timed repetitions: twice the 126 MB L2
+
+
+def _timed(fn, st, reps, warm=3, flush=None):
+    """Median device time of fn over reps repetitions (CUDA events on stream st), after warm
+    untimed runs; when flush is given it is overwritten before every repetition, outside the
+    timed interval, so no input is still in L2."""
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        fn()
+        e1.record(st)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e-3)
+    return statistics.median(ts)
+
+
+def retrieve_algorithmic(w, nnz, rows, T_q, T_k, layers=1):
+    """Algorithmic bytes / FLOPs of retrieval over `rows` query blocks holding nnz kept blocks
+    (all layers together): kept blocks, V of T_k keys, O of T_q queries and the indices, once;
+    mixing and P.V products of every kept block."""
+    e = 4 if w.dtype == "f32" else 2
+    blk = w.h_s * w.B * w.B * e
+    b = (nnz * blk + layers * (T_k * w.h_kv * w.d * e + T_q * w.h_r * w.d * e + 4 * (rows + 1)
+                                + 4 * w.h_r * w.h_s) + 4 * nnz)
+    f = nnz * (2 * w.h_r * w.h_s * w.B * w.B + 2 * w.h_r * w.B * w.B * w.d)
+    return b, f
+
+
+def _ret_line(w, t, b, f, hbm, tf, tokens, layers=1):
+    t_roof = max(b / (hbm * 1e9), f / (tf * 1e12))
+    return {"ms": t * 1e3, "GB/s": b / t / 1e9, "TFLOP/s": f / t / 1e12, "bytes": b, "flops": f,
+            "tokens_per_s_layer": tokens * layers / t, "roofline_frac": t_roof / t,
+            "bound": "hbm" if b / (hbm * 1e9) >= f / (tf * 1e12) else "tensor"}
+
+
+def _comp_line(w, t, nnz, hbm, causal=None, rows=None):
+    e = 4 if w.dtype == "f32" else 2
+    blk = w.h_s * w.B * w.B * e
+    causal = w.causal_blocks if causal is None else causal
+    rows = sum(w.nqb) if rows is None else rows
+    b = causal * blk + nnz * blk + 4 * nnz + 4 * (rows + 1)
+    return {"ms": t * 1e3, "GB/s": b / t / 1e9, "bytes": b, "roofline_frac": b / (hbm * 1e9) / t,
+            "tokens_per_s_layer": w.tokens / t}
+
+
+def run_long_context(mf, dev, hbm, tf, points, reps=3):
+    """Long-context workload (L = 32768, B = 128, 32 -> 24 / 8 heads) at the given
+    (tau, heavy columns, map reading) points: compression of the 68.7 GB dense layer (larger
+    than L2 by itself) and retrieval of the compressed layer (L2 flushed before each
+    repetition)."""
+    from synth import device as sdev
+    base = synth_all()["long_context"]
+    st = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out, pack, key = [], None, None
+    for tau, heavy, reading in points:
+        w = base.with_(tau=tau, n_heavy=heavy, reading=reading)
+        if key != (heavy, reading):
+            pack = None
+            torch.cuda.empty_cache()
+            pack = sdev.fill_maps(sdev.alloc_maps(w, dev), w, 0)
+            key = (heavy, reading)
+        cap = w.causal_blocks
+        bsr = mf.alloc_bsr(sum(w.nqb), cap, w.h_s, w.B, pack.maps.dtype, dev)
+        ws = torch.empty(mf.mf_compress_workspace_size(1, w.lens[0], w.B, cap), dtype=torch.uint8,
+                         device=dev)
+        cu = pack.cu_seqlens
+        t_c = _timed(lambda: mf.mf_compress(pack.maps, pack.map_seq_offset, cu, w.lens[0], w.h_s,
+                                            w.B, w.tau, bsr, ws), st, reps, warm=1)
+        nnz = int(bsr.nnz.cpu()[0])
+        W, V = sdev.w_weights(w, dev), sdev.v_contiguous(w, 0, dev)
+        O = torch.empty((1, w.tokens, w.h_r, w.d), dtype=V.dtype, device=dev)
+        qb = sdev.qblock_base(w, dev)
+        t_r = _timed(lambda: mf.mf_map_retrieve([bsr], [0], W, V, cu, cu, qb, w.lens[0], w.h_r,
+                                                w.h_kv, O=O), st, reps, warm=1, flush=flush)
+        _status_or_raise(mf, "long_context")
+        b, f = retrieve_algorithmic(w, nnz, sum(w.nqb), w.tokens, w.tokens)
+        out.append({"tau": tau, "heavy": heavy, "reading": reading, "nnz": nnz,
+                    "density": nnz / w.causal_blocks,
+                    "compress": _comp_line(w, t_c, nnz, hbm),
+                    "retrieve": _ret_line(w, t_r, b, f, hbm, tf, w.tokens)})
+        del bsr, ws, W, V, O
+    del pack, flush
+    torch.cuda.empty_cache()
+    return {"workload": "long_context: L=32768, B=128, h_s=32 -> h_r=24, h_kv=8, d=128, bf16",
+            "points": out, "reps": reps, "l2": "retrieval: L2 flushed before every repetition"}
+
+
+def run_qwen(mf, dev, hbm, tf, reps=3):
+    """Qwen-like pair: 40 sender layers compressed one by one (each layer's dense maps, 6 GB,
+    generated into one reused buffer; compression timed per layer), then the 36 receiver layers
+    retrieved (layer map l_s = round(l_r 39 / 35)): each layer alone, all 36 in one call, and
+    the 36 per-layer launches captured once in a CUDA graph and replayed."""
+    from synth import device as sdev
+    w = synth_all()["qwen_pair"]
+    lm = w.layer_map()
+    st = torch.cuda.current_stream()
+    pack = sdev.alloc_maps(w, dev)
+    cap = 2048
+    ws = torch.empty(mf.mf_compress_workspace_size(len(w.lens), max(w.lens), w.B, cap),
+                     dtype=torch.uint8, device=dev)
+    bsrs, t_comp, nnzs = [], [], []
+    cu = pack.cu_seqlens
+    for l in range(w.n_sender_layers):
+        sdev.fill_maps(pack, w, l)
+        b = mf.alloc_bsr(sum(w.nqb), cap, w.h_s, w.B, pack.maps.dtype, dev)
+        t_comp.append(_timed(lambda: mf.mf_compress(pack.maps, pack.map_seq_offset, cu, max(w.lens),
+                                                    w.h_s, w.B, w.tau, b, ws), st, 2, warm=1))
+        bsrs.append(b)
+        nnzs.append(int(b.nnz.cpu()[0]))
+    _status_or_raise(mf, "qwen compress")
+    del pack
+    torch.cuda.empty_cache()
+    W = sdev.w_weights(w, dev)
+    T = w.tokens
+    V = torch.empty((w.n_receiver_layers, T, w.h_kv, w.d), dtype=torch.bfloat16, device=dev)
+    for l in range(w.n_receiver_layers):
+        V[l] = sdev.v_contiguous(w, l, dev)
+    O = torch.empty((w.n_receiver_layers, T, w.h_r, w.d), dtype=torch.bfloat16, device=dev)
+    qb = sdev.qblock_base(w, dev)
+    maxlen = max(w.lens)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def layer(l):
+        mf.mf_map_retrieve(bsrs, lm, W, V, cu, cu, qb, maxlen, w.h_r, w.h_kv, O=O[l:l + 1],
+                           l_r_range=(l, l + 1), v_layer_stride=V[0].numel())
+
+    def all_layers():
+        mf.mf_map_retrieve(bsrs, lm, W, V, cu, cu, qb, maxlen, w.h_r, w.h_kv, O=O,
+                           v_layer_stride=V[0].numel())
+
+    t_layer = [_timed(lambda: layer(l), st, reps, warm=1, flush=flush) for l in range(w.n_receiver_layers)]
+    t_all = _timed(all_layers, st, reps, warm=1, flush=flush)
+    g = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream(device=dev)
+    cs.wait_stream(st)
+    with torch.cuda.graph(g, stream=cs):
+        for l in range(w.n_receiver_layers):
+            mf.mf_map_retrieve(bsrs, lm, W, V, cu, cu, qb, maxlen, w.h_r, w.h_kv, O=O[l:l + 1],
+                               l_r_range=(l, l + 1), v_layer_stride=V[0].numel(), stream=cs)
+    torch.cuda.synchronize()
+    t_graph = _timed(g.replay, st, reps, warm=1, flush=flush)
+    _status_or_raise(mf, "qwen retrieve")
+    nnz_r = [nnzs[lm[l]] for l in range(w.n_receiver_layers)]
+    rows = sum(w.nqb)
+    per = [_ret_line(w, t, *retrieve_algorithmic(w, n, rows, T, T), hbm, tf, T)
+           for t, n in zip(t_layer, nnz_r)]
+    b_all, f_all = retrieve_algorithmic(w, sum(nnz_r), rows, T, T, layers=w.n_receiver_layers)
+    comp = [_comp_line(w, t, n, hbm) for t, n in zip(t_comp, nnzs)]
+    del g, bsrs, V, O, flush
+    torch.cuda.empty_cache()
+
+    def summary(lines, key):
+        v = sorted(x[key] for x in lines)
+        return {"median": v[len(v) // 2], "min": v[0], "max": v[-1]}
+
+    return {"workload": "qwen_pair: 40 sender layers h_s=40 -> 36 receiver layers h_r=32, h_kv=8, "
+                        "d=128, varlen 2048/4096/6144/4096, B=64, tau=0.95, bf16",
+            "density_per_sender_layer": summary([{"d": n / w.causal_blocks} for n in nnzs], "d"),
+            "compress_per_sender_layer": {k: summary(comp, k) for k in ("ms", "GB/s", "roofline_frac")},
+            "retrieve_per_receiver_layer": {k: summary(per, k) for k in
+                                            ("ms", "GB/s", "TFLOP/s", "tokens_per_s_layer", "roofline_frac")},
+            "retrieve_36_layers_one_call": _ret_line(w, t_all, b_all, f_all, hbm, tf, T,
+                                                     layers=w.n_receiver_layers),
+            "retrieve_36_layers_graph": _ret_line(w, t_graph, b_all, f_all, hbm, tf, T,
+                                                  layers=w.n_receiver_layers),
+            "reps": reps, "l2": "retrieval: L2 flushed before every repetition"}
+
+
+def run_routing(mf, dev, hbm, tf, reps=3):
+    """Multi-turn routing batch: 16 varlen sequences (1k-8k tokens) compressed in one call, then
+    retrieved by chunked prefill (2048-token query chunks against the whole prefix) over a paged
+    V (16-token pages, shuffled block table): every chunk step timed, and the sum."""
+    from synth import device as sdev
+    w = synth_all()["routing_batch"]
+    st = torch.cuda.current_stream()
+    pack = sdev.fill_maps(sdev.alloc_maps(w, dev), w, 0)
+    cap = 8192
+    bsr = mf.alloc_bsr(sum(w.nqb), cap, w.h_s, w.B, pack.maps.dtype, dev)
+    ws = torch.empty(mf.mf_compress_workspace_size(len(w.lens), max(w.lens), w.B, cap),
+                     dtype=torch.uint8, device=dev)
+    cu = pack.cu_seqlens
+    t_c = _timed(lambda: mf.mf_compress(pack.maps, pack.map_seq_offset, cu, max(w.lens), w.h_s,
+                                        w.B, w.tau, bsr, ws), st, reps, warm=1)
+    nnz = int(bsr.nnz.cpu()[0])
+    rp = bsr.row_ptr.cpu().numpy()
+    del pack
+    torch.cuda.empty_cache()
+    W = sdev.w_weights(w, dev)
+    V = sdev.v_contiguous(w, 0, dev)
+    Vp, table = sdev.v_paged(w, V)
+    del V
+    qb = sdev.qblock_base(w, dev)
+    qbase = np.concatenate([[0], np.cumsum(w.nqb)[:-1]])
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    steps = []
+    for step in synth_chunks(w):
+        cu_q, cu_k, mq = sdev.step_tensors(step, dev)
+        Tq = int(cu_q[-1])
+        O = torch.empty((1, Tq, w.h_r, w.d), dtype=torch.bfloat16, device=dev)
+        t = _timed(lambda: mf.mf_map_retrieve([bsr], [0], W, Vp, cu_q, cu_k, qb, mq, w.h_r, w.h_kv,
+                                              O=O, paged=(table, w.page_size)), st, reps, warm=1,
+                   flush=flush)
+        rows = n_step = 0
+        for s, (q_len, k_len) in enumerate(step):
+            if q_len == 0:
+                continue
+            q0 = k_len - q_len
+            r0, r1 = qbase[s] + q0 // w.B, qbase[s] + -(-k_len // w.B)
+            rows += r1 - r0
+            n_step += int(rp[r1] - rp[r0])
+        b, f = retrieve_algorithmic(w, n_step, rows, Tq, sum(k for _, k in step))
+        line = _ret_line(w, t, b, f, hbm, tf, Tq)
+        line.update({"queries": Tq, "nnz": n_step})
+        steps.append(line)
+    _status_or_raise(mf, "routing")
+    t_tot = sum(x["ms"] for x in steps) * 1e-3
+    b_tot = sum(x["bytes"] for x in steps)
+    f_tot = sum(x["flops"] for x in steps)
+    del bsr, Vp, flush
+    torch.cuda.empty_cache()
+    return {"workload": "routing_batch: 16 sequences 1k-8k tokens, chunk 2048, paged V (16-token "
+                        "pages, shuffled), h_s=32 -> h_r=32, h_kv=8, d=128, B=64, tau=0.95, bf16",
+            "nnz": nnz, "density": nnz / w.causal_blocks,
+            "compress": _comp_line(w, t_c, nnz, hbm),
+            "retrieve_per_chunk_step": steps,
+            "retrieve_all_steps": _ret_line(w, t_tot, b_tot, f_tot, hbm, tf, w.tokens),
+            "reps": reps, "l2": "retrieval: L2 flushed before every repetition"}
+
+
+def run_cold_retrieve(w, mf, bsr, nnz, W, V, O, qb, dev, hbm, tf, reps=20):
+    """Retrieval of the main workload with L2 flushed (a 256 MB write) before every repetition:
+    in the timed step the kept blocks were written by the compression just before and partly sit
+    in L2."""
+    st = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    cu = torch.tensor([0] + list(np.cumsum(w.lens)), dtype=torch.int32, device=dev)
+    t = _timed(lambda: mf.mf_map_retrieve([bsr], [0], W, V, cu, cu, qb, max(w.lens), w.h_r, w.h_kv,
+                                          O=O), st, reps, flush=flush)
+    del flush
+    torch.cuda.empty_cache()
+    b, f = retrieve_algorithmic(w, nnz, sum(w.nqb), w.tokens, w.tokens)
+    line = _ret_line(w, t, b, f, hbm, tf, w.tokens)
+    line["l2"] = "flushed before every repetition"
+    return line
+
+
+def _status_or_raise(mf, what):
+    rc, bits = mf.mf_get_status()
+    if rc != mf.MF_OK:
+        raise RuntimeError(f"{what}: device status {rc} bits {bits:#x}")
+
+
+def mf_mod():
+    import cross_model_attention_mf_b200 as mf
+    return mf
+
+
+def synth_all():
+    import synth
+    return synth.ALL
+
+
+def synth_chunks(w):
+    import synth
+    return synth.chunks(w)
+
+
 # ------------------------------------------------------------------------ oracle (CPU baseline)
-def oracle_sample(w, pack_host_rows, W_l, V_host, rows):
-    """Oracle compress + retrieve of the sampled query blocks (whole sequences)."""
+def _oracle_row(w, qb, slab, W_l, V_host):
+    """Oracle compression + retrieval of one query block (whole rows of sequence 0)."""
     import oracle
+    m = oracle.row_masses(slab, w.lens[0], w.B, qb)
+    kept, _ = oracle.select(m, qb, w.tau)
+    vals = np.stack([oracle.gather_block(slab, w.lens[0], w.B, qb, int(kb)) for kb in kept])
+    lo, hi = 0, min(w.lens[0], (qb + 1) * w.B) - qb * w.B
+    oracle.retrieve_block(vals, kept, qb, w.B, W_l, V_host, w.h_kv, (lo, hi))
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, slabs, W_l, V_host, rows, threads):
+    """Wall time of the oracle on the sampled query blocks, one block per task on `threads`
+    host threads (the C oracle runs with the GIL released)."""
+    from concurrent.futures import ThreadPoolExecutor
     t0 = time.perf_counter()
-    for (qb, slab) in zip(rows, pack_host_rows):
-        m = oracle.row_masses(slab, w.lens[0], w.B, qb)
-        kept, _ = oracle.select(m, qb, w.tau)
-        vals = np.stack([oracle.gather_block(slab, w.lens[0], w.B, qb, int(kb)) for kb in kept])
-        lo, hi = 0, min(w.lens[0], (qb + 1) * w.B) - qb * w.B
-        oracle.retrieve_block(vals, kept, qb, w.B, W_l, V_host, w.h_kv, (lo, hi))
+    with ThreadPoolExecutor(max_workers=threads) as pool:
+        list(pool.map(lambda a: _oracle_row(w, a[0], a[1], W_l, V_host), zip(rows, slabs)))
     return time.perf_counter() - t0
 
 
@@ -566,11 +861,13 @@ def cpu_sample_inputs(w, n_rows, dev):
 
 def cpu_baseline(w, dev, n_rows):
     rows, slabs, W_l, V_host = cpu_sample_inputs(w, n_rows, dev)
-    dt = oracle_sample(w, slabs, W_l, V_host, rows)
+    cores = host_cores()
+    dt = oracle_sample(w, slabs, W_l, V_host, rows, cores)
     toks = sum(min(w.lens[0], (qb + 1) * w.B) - qb * w.B for qb in rows)
-    return {"value": toks / dt, "unit": "tokens/s/layer", "cores": 1, "kind": "oracle",
+    return {"value": toks / dt, "unit": "tokens/s/layer", "cores": cores, "kind": "oracle",
             "sample": f"{len(rows)} of {w.nqb[0]} query blocks ({toks} tokens) of sequence 0, "
-                      f"compress + retrieve, single-threaded C oracle, {dt:.1f} s"}
+                      f"compress + retrieve, float64 C oracle on {cores} host threads (one query "
+                      f"block per task), {dt:.2f} s wall"}
 
 
 # ------------------------------------------------------------------------ main
@@ -597,6 +894,10 @@ def main():
     ap.add_argument("--no-calib", action="store_true", help="skip the head-map calibration line")
     ap.add_argument("--calib-len", type=int, default=0,
                     help="calibrate on a sequence of this many tokens (0: the workload's own)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads (long context, Qwen-like, routing batch, cold L2)")
+    ap.add_argument("--long-points", default="0.95:8:1,0.8:8:3,0.99:64:3",
+                    help="long-context points tau:heavy:reading, comma separated")
     ap.add_argument("--capacity", type=int, default=0,
                     help="BSR capacity in blocks (0: every causal block, which never overflows)")
     args = ap.parse_args()
@@ -611,28 +912,33 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        # each step: the oracle on one query block of the workload (cycling over 8 blocks
-        # spread along the sequence); the run stops early after ~60 s of CPU time
-        rows, slabs, W_l, V_host = cpu_sample_inputs(w, 8, dev)
-        one = lambda t: oracle_sample(w, [slabs[t % len(rows)]], W_l, V_host, [rows[t % len(rows)]])
+        # each step: the oracle on one batch of query blocks (one per host thread, cycling over
+        # blocks spread along the sequence); the run stops early after ~60 s of wall time
+        cores = host_cores()
+        rows, slabs, W_l, V_host = cpu_sample_inputs(w, max(8, cores), dev)
+
+        def one(t):
+            idx = [(t * cores + k) % len(rows) for k in range(cores)]
+            dt = oracle_sample(w, [slabs[i] for i in idx], W_l, V_host, [rows[i] for i in idx], cores)
+            return dt, sum(min(w.lens[0], (rows[i] + 1) * w.B) - rows[i] * w.B for i in idx)
+
         warm = min(args.warmup, 2)
         for t in range(warm):
             one(t)
         spent, k, toks = 0.0, 0, 0
         while k < max(args.steps, 1) and (spent < 60.0 or k == 0):
-            spent += one(k)
-            qb = rows[k % len(rows)]
-            toks += min(w.lens[0], (qb + 1) * w.B) - qb * w.B
+            dt, n = one(warm + k)
+            spent += dt
+            toks += n
             k += 1
-        dt = spent / k
         v = toks / spent
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s/layer",
-                "n_gpus": args.gpus, "steps": k, "warmup": warm, "ms_per_step": dt * 1e3,
+                "n_gpus": args.gpus, "steps": k, "warmup": warm, "ms_per_step": spent / k * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": {"workload": describe(w)},
-                "cpu_baseline": {"value": v, "unit": "tokens/s/layer", "cores": 1, "kind": "oracle",
-                                 "sample": f"{k} steps of one query block each ({toks} tokens), "
-                                           f"compress + retrieve, single-threaded C oracle"},
+                "cpu_baseline": {"value": v, "unit": "tokens/s/layer", "cores": cores, "kind": "oracle",
+                                 "sample": f"{k} steps of {cores} query blocks each ({toks} tokens), "
+                                           f"compress + retrieve, float64 C oracle on {cores} host threads"},
                 "e2e": {"value": v, "unit": "tokens/s/layer", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -686,7 +992,9 @@ def main():
                 "tensor_TFLOP/s": ret_tf, "tensor_peak": tf_burst,
                 "traffic": measured_traffic("mf_map_retrieve", w.name),
                 "peak_source": f"{src} (hbm_gbs; bf16_tflops burst for the tensor side)"},
-            "gpu_launches": 6 * args.steps,
+            # per step: k_meta, k_stats (with the fused selection), k_scan_compact, k_gather,
+            # k_retrieve_tc
+            "gpu_launches": 5 * args.steps,
             "clocks": res["clocks"],
         }
         if res["e2e"] is not None:
@@ -716,6 +1024,16 @@ def main():
             c.update({"bound": "hbm", "peak": hbm, "unit": "GB/s", "frac": c["GB/s"] / hbm,
                       "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)"})
             line["calibration"] = c
+        if res["cold"] is not None:
+            line["retrieve_cold_l2"] = res["cold"]
+        if not args.no_configs:
+            pts = [tuple(float(x) if i == 0 else int(x) for i, x in enumerate(p.split(":")))
+                   for p in args.long_points.split(",") if p]
+            line["configs"] = {
+                "qwen_pair": run_qwen(mf_mod(), dev, hbm, tf_burst),
+                "long_context": run_long_context(mf_mod(), dev, hbm, tf_burst, pts),
+                "routing_batch": run_routing(mf_mod(), dev, hbm, tf_burst),
+            }
         if not args.no_cpu and world == 1:
             line["cpu_baseline"] = cpu_baseline(w, dev, args.cpu_rows)
         print(json.dumps(line), flush=True)

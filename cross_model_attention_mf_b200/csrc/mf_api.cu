@@ -80,6 +80,8 @@ mf_status check_retrieve(const mf_retrieve_desc* d) {
     if (!b.row_ptr || !b.col_idx || !b.values || b.capacity_blocks < 0)
       return fail(MF_ERR_INVALID, "incomplete BSR for a mapped sender layer");
   }
+  if (mfi::tc_supported(*d) && reinterpret_cast<uintptr_t>(d->V) % 16)
+    return fail(MF_ERR_INVALID, "V must be 16-byte aligned");
   if (!mfi::tc_supported(*d) && (int64_t)d->B * d->d > 16384)
     return fail(MF_ERR_UNSUPPORTED, "B * d > 16384 needs the tensor-core path");
   return MF_OK;
@@ -518,7 +520,8 @@ mf_status mf_get_status(void* stream, uint32_t* bits) {
   if (v & mfi::ST_TIMEOUT) return fail(MF_ERR_TIMEOUT, "device: pipeline wait timed out");
   if (v & mfi::ST_ALIGN) return fail(MF_ERR_INVALID, "device: misaligned map offset");
   if (v & mfi::ST_PAGE) return fail(MF_ERR_DEVICE_INDEX, "device: page id out of range");
-  return fail(MF_ERR_INVALID, "device: calibration Gram is not positive definite");
+  if (v & mfi::ST_SINGULAR) return fail(MF_ERR_INVALID, "device: calibration Gram is not positive definite");
+  return fail(MF_ERR_RANGE, "device: V or the mixed map P outside the float16 range (|x| > 65504)");
 }
 
 }  // extern "C"
