@@ -36,6 +36,7 @@ MF_OK, MF_ERR_INVALID, MF_ERR_UNSUPPORTED, MF_ERR_CAPACITY, MF_ERR_CUDA, MF_ERR_
     MF_ERR_DEVICE_INDEX, MF_ERR_RANGE = range(8)
 MF_F32, MF_BF16 = 0, 1
 MF_RETRIEVE_FORCE_SIMT = 1
+MF_RETRIEVE_O_F32 = 2
 
 _P = ctypes.c_void_p
 _I32 = ctypes.c_int32
@@ -313,9 +314,10 @@ def mf_map_retrieve(layers: Sequence[BSR], layer_map: Sequence[int], W: torch.Te
                     qblock_base: torch.Tensor, max_seqlen_q: int, h_r: int, h_kv: int,
                     O: Optional[torch.Tensor] = None, l_r_range=None, total_q: Optional[int] = None,
                     paged=None, v_layer_stride: int = 0, force_simt: bool = False,
-                    stream=None) -> torch.Tensor:
+                    o_f32: bool = False, stream=None) -> torch.Tensor:
     """Enqueue fused retrieval for receiver layers l_r_range (default: all of layer_map).
-    O: [n_layers, T_q, h_r, d] (allocated when None).  paged = (block_table, page_size)."""
+    O: [n_layers, T_q, h_r, d] (allocated when None; float32 with o_f32, else V's dtype).
+    paged = (block_table, page_size)."""
     if l_r_range is None:
         l_r_range = (0, len(layer_map))
     n_l = l_r_range[1] - l_r_range[0]
@@ -323,10 +325,12 @@ def mf_map_retrieve(layers: Sequence[BSR], layer_map: Sequence[int], W: torch.Te
     if O is None:
         if total_q is None:
             raise ValueError("total_q is needed to allocate O")
-        O = torch.empty((n_l, total_q, h_r, V.shape[-1]), dtype=V.dtype, device=V.device)
+        O = torch.empty((n_l, total_q, h_r, V.shape[-1]), dtype=torch.float32 if o_f32 else V.dtype,
+                        device=V.device)
+    flags = (MF_RETRIEVE_FORCE_SIMT if force_simt else 0) | (MF_RETRIEVE_O_F32 if o_f32 else 0)
     d, keep = _retrieve_desc(layers, layer_map, l_r_range, W, V, O, cu_seqlens_q, cu_seqlens_k,
                              qblock_base, max_seqlen_q, h_s, B, h_r, h_kv, v_layer_stride,
-                             0, paged, MF_RETRIEVE_FORCE_SIMT if force_simt else 0)
+                             0, paged, flags)
     _check(_lib.mf_map_retrieve(ctypes.byref(d), _stream(stream)))
     del keep
     return O

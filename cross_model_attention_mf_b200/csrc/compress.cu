@@ -6,16 +6,19 @@
 // first, then the blocks to keep are chosen by cumulative attention probability,
 // and only those are written -- no second dense matrix is assembled.
 //
-// Kernels (one launch each, all on the caller's stream):
+// Kernels (all on the caller's stream):
 //   k_meta          per-sequence geometry of the varlen pack (one thread)
 //   k_stats         head-summed mass of every causal block: a streaming reduction
 //                   with 16-byte loads, float32 partials of 8 (bf16) or 4 (f32)
 //                   elements combined in float64, fixed order (deterministic)
-//   k_select        per query block: sort candidates (mass desc, kb asc), walk
+//   selection       per query block: sort candidates (mass desc, kb asc), walk
 //                   the running float64 sum until it reaches tau * total, write the
-//                   row's kept indices in ascending order to a per-row list
-//   k_scan_compact  row_ptr by exclusive scan of the counts, then copy the per-row
-//                   lists into col_idx
+//                   row's kept indices in ascending order to a per-row list; done by
+//                   the k_stats CTA that writes the row's last mass (rows of up to
+//                   1024 candidates; longer rows: a k_select launch)
+//   scan/compact    row_ptr by exclusive scan of the counts, then copy the per-row
+//                   lists into col_idx; done by the k_stats CTA that selects the last
+//                   row (after a k_select launch: k_scan_compact)
 //   k_gather        copy each kept block with the causal/length mask applied, one
 //                   (block, sender head) unit per CTA iteration
 #include <cuda_bf16.h>
@@ -50,6 +53,8 @@ __device__ inline int tri_row(int64_t c) {
 __global__ void k_meta(const int32_t* cu, const int64_t* off, int nseq, int max_seqlen, int B,
                        int elem_bytes, int64_t* meta, uint32_t* status, int32_t* row_ptr,
                        int32_t* nnz_out, int32_t* row_done, int64_t max_rows) {
+  // the next kernel (k_stats) may launch now; it waits for this grid before reading anything
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (row_done)  // per-row counters of the fused selection start at zero on every call
     for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < max_rows;
          r += (int64_t)gridDim.x * blockDim.x)
@@ -203,25 +208,105 @@ __device__ void select_row(const int64_t* __restrict__ meta, int nseq, const dou
   __syncthreads();
 }
 
+// Exclusive scan of the counts into row_ptr by all NT threads of one CTA (independent loads,
+// so their latencies overlap), then each row's list is copied into col_idx (warp per row).
+// part: NT int64 of shared scratch.  Counts and lists are read through L2 (other CTAs may have
+// written them moments ago).
+constexpr int SCAN_PER = 8;
+template <int NT>
+__device__ void scan_compact(const int64_t* __restrict__ meta, int nseq, const int32_t* counts,
+                             const int32_t* kept_local, int32_t* __restrict__ row_ptr,
+                             int32_t* __restrict__ col_idx, int32_t* __restrict__ kept_row,
+                             int32_t* __restrict__ nnz_out, int64_t capacity, uint32_t* status,
+                             int64_t* part, int64_t* carry) {
+  const int64_t R = meta[0];
+  const int t = threadIdx.x;
+  if (t == 0) *carry = 0;
+  __syncthreads();
+  for (int64_t base = 0; base < R; base += (int64_t)NT * SCAN_PER) {
+    const int64_t r0 = base + (int64_t)t * SCAN_PER;
+    int32_t c[SCAN_PER];
+#pragma unroll
+    for (int k = 0; k < SCAN_PER; ++k) c[k] = r0 + k < R ? __ldcg(counts + r0 + k) : 0;
+    int64_t sum = 0;
+#pragma unroll
+    for (int k = 0; k < SCAN_PER; ++k) sum += c[k];
+    part[t] = sum;
+    __syncthreads();
+    for (int o = 1; o < NT; o <<= 1) {  // inclusive Hillis-Steele scan
+      const int64_t v = t >= o ? part[t - o] : 0;
+      __syncthreads();
+      part[t] += v;
+      __syncthreads();
+    }
+    int64_t run = *carry + part[t] - sum;
+#pragma unroll
+    for (int k = 0; k < SCAN_PER; ++k)
+      if (r0 + k < R) {
+        row_ptr[r0 + k] = (int32_t)run;
+        run += c[k];
+      }
+    __syncthreads();
+    if (t == NT - 1) *carry += part[NT - 1];
+    __syncthreads();
+  }
+  const int64_t nnz = *carry;
+  if (t == 0) {
+    row_ptr[R] = (int32_t)nnz;
+    *nnz_out = (int32_t)nnz;
+    if (nnz > capacity) atomicOr(status, ST_CAPACITY);
+  }
+  __syncthreads();
+  const int warp = t >> 5, lane = t & 31;
+  for (int64_t row = warp; row < R; row += NT / 32) {
+    const int s = find_seq(meta, nseq, row, 2);
+    const int64_t* m = meta + META_HDR + 4 * s;
+    const int qb = (int)(row - m[2]);
+    const int32_t* kl = kept_local + m[3] + (int64_t)qb * (qb + 1) / 2;
+    const int64_t n0 = row_ptr[row];
+    const int cnt = __ldcg(counts + row);
+    for (int k = lane; k < cnt; k += 32)
+      if (n0 + k < capacity) {
+        col_idx[n0 + k] = __ldcg(kl + k);
+        kept_row[n0 + k] = (int32_t)row;
+      }
+  }
+}
+
 // rows with at most this many candidates are selected inside k_stats (its shared scratch)
 constexpr int SEL_FUSED_MAX = 1024;
 
 // Masses of every causal block.  Item = (sequence, qb, kb) over all sender heads.  With
 // row_done set, the CTA that writes the last mass of a row (a per-row counter reaches qb + 1)
 // also selects that row, so selection overlaps the rest of the stream.
+struct FusedTail {             // selection and BSR index build inside k_stats
+  int32_t* row_done;           // [rows] masses written per row
+  unsigned long long* rows_selected;  // rows whose selection is done
+  double tau;
+  int32_t* counts;
+  int32_t* kept_local;
+  int32_t* row_ptr;
+  int32_t* col_idx;
+  int32_t* kept_row;
+  int32_t* nnz_out;
+  int64_t capacity;
+  uint32_t* status;
+};
+
 template <typename T, int B, int NT>
 __global__ void __launch_bounds__(NT) k_stats(const T* __restrict__ maps,
                                               const int64_t* __restrict__ seq_off,
                                               const int64_t* __restrict__ meta, int nseq,
-                                              int h_s, double* mass, int32_t* row_done,
-                                              double tau, int32_t* __restrict__ counts,
-                                              int32_t* __restrict__ kept_local) {
+                                              int h_s, double* mass, const FusedTail ft) {
   constexpr int EPV = Vec<T>::EPV, VPR = B / EPV, VPB = B * VPR;  // vectors per row / per head
   constexpr int U = 4;
   __shared__ double red[NT / 32];
   __shared__ uint64_t sel[SEL_FUSED_MAX * 3 / 2];  // keys and indices of one row's candidates
   __shared__ int misc[NT / 32 + 2];
-  __shared__ int s_last;
+  __shared__ int s_last, s_all;
+  __shared__ int64_t part[NT], carry;
+  // launched while k_meta may still run (programmatic dependent launch): wait for it
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t total = meta[1];
   const int64_t nv = (int64_t)h_s * VPB;
   for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
@@ -276,14 +361,26 @@ __global__ void __launch_bounds__(NT) k_stats(const T* __restrict__ maps,
     }
     const double t = block_sum_f64<NT>(acc, red);
     if (threadIdx.x == 0) mass[item] = t;
-    if (row_done) {
+    if (ft.row_done) {
       if (threadIdx.x == 0) {
         __threadfence();  // this mass is visible before the count that announces it
-        s_last = atomicAdd(&row_done[m[2] + qb], 1) == qb ? 1 : 0;
+        s_last = atomicAdd(&ft.row_done[m[2] + qb], 1) == qb ? 1 : 0;
         __threadfence();
       }
       __syncthreads();
-      if (s_last) select_row<NT>(meta, nseq, mass, tau, m[2] + qb, counts, kept_local, sel, misc);
+      if (s_last) {
+        select_row<NT>(meta, nseq, mass, ft.tau, m[2] + qb, ft.counts, ft.kept_local, sel, misc);
+        // the CTA that selects the last row also builds row_ptr and col_idx
+        if (threadIdx.x == 0) {
+          __threadfence();
+          s_all = atomicAdd(ft.rows_selected, 1ull) == (unsigned long long)(meta[0] - 1) ? 1 : 0;
+          __threadfence();
+        }
+        __syncthreads();
+        if (s_all)
+          scan_compact<NT>(meta, nseq, ft.counts, ft.kept_local, ft.row_ptr, ft.col_idx,
+                           ft.kept_row, ft.nnz_out, ft.capacity, ft.status, part, &carry);
+      }
     }
   }
 }
@@ -302,9 +399,8 @@ __global__ void __launch_bounds__(NT) k_select(const int64_t* __restrict__ meta,
   select_row<NT>(meta, nseq, mass, tau, row, counts, kept_local, sm, misc);
 }
 
-// One CTA: exclusive scan of the counts into row_ptr (independent loads, so their
-// latencies overlap), then each row's list is copied into col_idx (warp per row).
-constexpr int SCAN_NT = 1024, SCAN_PER = 8;
+// The scan as its own launch (after a separate selection launch).
+constexpr int SCAN_NT = 1024;
 __global__ void __launch_bounds__(SCAN_NT) k_scan_compact(
     const int64_t* __restrict__ meta, int nseq, const int32_t* __restrict__ counts,
     const int32_t* __restrict__ kept_local, int32_t* __restrict__ row_ptr,
@@ -312,58 +408,8 @@ __global__ void __launch_bounds__(SCAN_NT) k_scan_compact(
     int64_t capacity, uint32_t* status) {
   __shared__ int64_t part[SCAN_NT];
   __shared__ int64_t carry;
-  const int64_t R = meta[0];
-  const int t = threadIdx.x;
-  if (t == 0) carry = 0;
-  __syncthreads();
-  for (int64_t base = 0; base < R; base += (int64_t)SCAN_NT * SCAN_PER) {
-    const int64_t r0 = base + (int64_t)t * SCAN_PER;
-    int32_t c[SCAN_PER];
-#pragma unroll
-    for (int k = 0; k < SCAN_PER; ++k) c[k] = r0 + k < R ? counts[r0 + k] : 0;
-    int64_t sum = 0;
-#pragma unroll
-    for (int k = 0; k < SCAN_PER; ++k) sum += c[k];
-    part[t] = sum;
-    __syncthreads();
-    for (int o = 1; o < SCAN_NT; o <<= 1) {  // inclusive Hillis-Steele scan
-      const int64_t v = t >= o ? part[t - o] : 0;
-      __syncthreads();
-      part[t] += v;
-      __syncthreads();
-    }
-    int64_t run = carry + part[t] - sum;
-#pragma unroll
-    for (int k = 0; k < SCAN_PER; ++k)
-      if (r0 + k < R) {
-        row_ptr[r0 + k] = (int32_t)run;
-        run += c[k];
-      }
-    __syncthreads();
-    if (t == SCAN_NT - 1) carry += part[SCAN_NT - 1];
-    __syncthreads();
-  }
-  const int64_t nnz = carry;
-  if (t == 0) {
-    row_ptr[R] = (int32_t)nnz;
-    *nnz_out = (int32_t)nnz;
-    if (nnz > capacity) atomicOr(status, ST_CAPACITY);
-  }
-  __syncthreads();
-  const int warp = t >> 5, lane = t & 31;
-  for (int64_t row = warp; row < R; row += SCAN_NT / 32) {
-    const int s = find_seq(meta, nseq, row, 2);
-    const int64_t* m = meta + META_HDR + 4 * s;
-    const int qb = (int)(row - m[2]);
-    const int32_t* kl = kept_local + m[3] + (int64_t)qb * (qb + 1) / 2;
-    const int64_t n0 = row_ptr[row];
-    const int cnt = counts[row];
-    for (int k = lane; k < cnt; k += 32)
-      if (n0 + k < capacity) {
-        col_idx[n0 + k] = kl[k];
-        kept_row[n0 + k] = (int32_t)row;
-      }
-  }
+  scan_compact<SCAN_NT>(meta, nseq, counts, kept_local, row_ptr, col_idx, kept_row, nnz_out,
+                        capacity, status, part, &carry);
 }
 
 template <typename T, int B, int NT>
@@ -375,6 +421,8 @@ __global__ void __launch_bounds__(NT) k_gather(const T* __restrict__ maps,
                                                const int32_t* __restrict__ col_idx,
                                                const int32_t* __restrict__ kept_row,
                                                T* __restrict__ values) {
+  // launched while k_stats may still run (programmatic dependent launch): wait for it
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int EPV = Vec<T>::EPV, VPR = B / EPV, VPB = B * VPR;  // vectors per row / per head
   constexpr int U = (VPB + NT - 1) / NT;
   const int64_t nnz = min((int64_t)*nnz_in, capacity);
@@ -421,6 +469,26 @@ __global__ void __launch_bounds__(NT) k_gather(const T* __restrict__ maps,
   }
 }
 
+// A launch that may start while the previous kernel on the stream still runs (programmatic
+// dependent launch); the kernel itself waits for that kernel (griddepcontrol.wait) before it
+// touches memory.  Saves the launch gap between the passes of one compression.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), int grid, int threads, cudaStream_t st,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3((unsigned)threads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  return e == cudaSuccess ? cudaGetLastError() : e;
+}
+
 template <typename T, int B>
 cudaError_t launch_typed(const mf_compress_desc& d, const CompressWs& ws, uint32_t* status,
                          cudaStream_t st, int sms) {
@@ -429,20 +497,32 @@ cudaError_t launch_typed(const mf_compress_desc& d, const CompressWs& ws, uint32
   double* mass = d.block_mass_out ? d.block_mass_out : ws.mass;
   const int grid_stats = (int)std::min<int64_t>(ws.max_cb, (int64_t)sms * 8);
   const bool fused = (d.max_seqlen + B - 1) / B <= SEL_FUSED_MAX;
-  k_stats<T, B, NT><<<grid_stats, NT, 0, st>>>(maps, d.map_seq_offset, ws.meta, d.nseq, d.h_s,
-                                                mass, fused ? ws.row_done : nullptr, d.tau,
-                                                ws.counts, ws.kept_local);
-  cudaError_t e = fused ? launch_scan(ws, d.nseq, d.row_ptr, d.col_idx, d.nnz_out,
-                                      d.capacity_blocks, status, st)
-                        : launch_select(ws, d.nseq, d.max_seqlen, B, mass, d.tau, d.row_ptr,
-                                        d.col_idx, d.nnz_out, d.capacity_blocks, status, st);
+  FusedTail ft;
+  ft.row_done = fused ? ws.row_done : nullptr;
+  ft.rows_selected = reinterpret_cast<unsigned long long*>(ws.meta + 2);
+  ft.tau = d.tau;
+  ft.counts = ws.counts;
+  ft.kept_local = ws.kept_local;
+  ft.row_ptr = d.row_ptr;
+  ft.col_idx = d.col_idx;
+  ft.kept_row = ws.kept_row;
+  ft.nnz_out = d.nnz_out;
+  ft.capacity = d.capacity_blocks;
+  ft.status = status;
+  cudaError_t e = launch_dependent(k_stats<T, B, NT>, grid_stats, NT, st, maps, d.map_seq_offset,
+                                   (const int64_t*)ws.meta, d.nseq, d.h_s, mass, ft);
   if (e != cudaSuccess) return e;
+  if (!fused) {
+    e = launch_select(ws, d.nseq, d.max_seqlen, B, mass, d.tau, d.row_ptr, d.col_idx, d.nnz_out,
+                      d.capacity_blocks, status, st);
+    if (e != cudaSuccess) return e;
+  }
   const int grid_g = (int)std::max<int64_t>(
       1, std::min<int64_t>(std::max<int64_t>(d.capacity_blocks, 1) * d.h_s, (int64_t)sms * 8));
-  k_gather<T, B, NT><<<grid_g, NT, 0, st>>>(maps, d.map_seq_offset, ws.meta, d.nseq, d.h_s,
-                                            d.nnz_out, d.capacity_blocks, d.col_idx, ws.kept_row,
-                                            static_cast<T*>(d.values));
-  return cudaGetLastError();
+  return launch_dependent(k_gather<T, B, NT>, grid_g, NT, st, maps, d.map_seq_offset,
+                          (const int64_t*)ws.meta, d.nseq, d.h_s, (const int32_t*)d.nnz_out,
+                          d.capacity_blocks, (const int32_t*)d.col_idx,
+                          (const int32_t*)ws.kept_row, static_cast<T*>(d.values));
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }

@@ -82,6 +82,8 @@ mf_status check_retrieve(const mf_retrieve_desc* d) {
   }
   if (mfi::tc_supported(*d) && reinterpret_cast<uintptr_t>(d->V) % 16)
     return fail(MF_ERR_INVALID, "V must be 16-byte aligned");
+  if ((d->flags & MF_RETRIEVE_O_F32) && !mfi::tc_supported(*d))
+    return fail(MF_ERR_UNSUPPORTED, "float32 O (MF_RETRIEVE_O_F32) needs the tensor-core path");
   if (!mfi::tc_supported(*d) && (int64_t)d->B * d->d > 16384)
     return fail(MF_ERR_UNSUPPORTED, "B * d > 16384 needs the tensor-core path");
   return MF_OK;
@@ -132,6 +134,7 @@ namespace {
 // receiver layer l of a retrieval descriptor
 mfi::RetrieveLayer layer_of(const mf_retrieve_desc& d, int l) {
   const int64_t ve = d.v_dtype == MF_F32 ? 4 : 2;
+  const int64_t oe = (d.flags & MF_RETRIEVE_O_F32) ? 4 : ve;
   const int64_t o_stride = d.o_layer_stride ? d.o_layer_stride : (int64_t)d.total_q * d.h_r * d.d;
   const mf_bsr& b = d.layers[d.layer_map[l]];
   mfi::RetrieveLayer L;
@@ -141,7 +144,7 @@ mfi::RetrieveLayer layer_of(const mf_retrieve_desc& d, int l) {
   L.capacity = b.capacity_blocks;
   L.W = d.W + (int64_t)l * d.h_r * d.h_s;
   L.V = static_cast<const char*>(d.V) + (int64_t)l * d.v_layer_stride * ve;
-  L.O = static_cast<char*>(d.O) + (int64_t)(l - d.l_r_begin) * o_stride * ve;
+  L.O = static_cast<char*>(d.O) + (int64_t)(l - d.l_r_begin) * o_stride * oe;
   return L;
 }
 

@@ -120,7 +120,8 @@ constexpr int NRMAX = 4;  // receivers served by one launch (one BSR, several W 
 // one receiver: its head map, V and O (and its V paging)
 struct RecvParams {
   const float* W;  // [h_r][h_s]
-  __nv_bfloat16* O;
+  void* O;         // bf16, or float32 when o_f32
+  int o_f32;
   const __nv_bfloat16* V;
   const int32_t* block_table;
   int paged, page_size, n_pages, max_pages;
@@ -590,6 +591,36 @@ __global__ void __launch_bounds__(NT, 1)
         return false;
       tc_fence_after();
       for (int gl = 0; gl < GO; ++gl) {
+        const int G = hc * NGC + rank * GO + gl;
+        if (q_r.o_f32) {
+          // float32 O: each lane stores its own head dim (a warp writes 128 contiguous bytes);
+          // D2 is released only after the last column is stored
+          float* of = static_cast<float*>(q_r.O) + u.o_row0 * rs + (int64_t)G * q_r.gq * D + d;
+#pragma unroll
+          for (int c32 = 0; c32 < NPV / 32; ++c32) {
+            uint32_t o[32];
+            if (have) {
+              tmem_ld32(tl + 128u * gl + 32u * c32, o);
+              tmem_wait_ld();
+              reg_fence(o);
+            } else {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] = 0u;
+            }
+#pragma unroll
+            for (int cc = 0; cc < 32; ++cc) {
+              const int n = 32 * c32 + cc;
+              const int c = n >> 3, pp = (n >> 2) & 1, h = n & 3;
+              const int r = 8 * (c >> 2) + 4 * ((c >> 1) & 1) + 2 * pp + (c & 1);
+              if (G < q_r.h_kv && h < q_r.gq && r >= ilo && r < ihi)
+                of[(int64_t)r * rs + h * D] = __uint_as_float(o[cc]);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_OEMPTY + gl));
+          continue;
+        }
         uint32_t pk[NPV / 2];  // columns (2u, 2u + 1) rounded to bf16
 #pragma unroll
         for (int c32 = 0; c32 < NPV / 32; ++c32) {
@@ -610,10 +641,10 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_OEMPTY + gl));
-        const int G = hc * NGC + rank * GO + gl;
         if (G < q_r.h_kv) {
           const bool odd = lane & 1;
-          __nv_bfloat16* ob = q_r.O + u.o_row0 * rs + (int64_t)G * q_r.gq * D + (d & ~1);
+          __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(q_r.O) + u.o_row0 * rs +
+                              (int64_t)G * q_r.gq * D + (d & ~1);
 #pragma unroll
           for (int u2 = 0; u2 < NPV / 2; ++u2) {
             // columns n = 2 u2 (head h even) and n + 1 (head h + 1) of the same row
@@ -907,7 +938,8 @@ bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* 
     const mf_retrieve_desc& d = *ds[k];
     const RetrieveLayer& l = ls[k];
     RecvParams& r = p.rv[k];
-    r.W = l.W; r.O = static_cast<__nv_bfloat16*>(l.O);
+    r.W = l.W; r.O = l.O;
+    r.o_f32 = (d.flags & MF_RETRIEVE_O_F32) ? 1 : 0;
     r.V = static_cast<const __nv_bfloat16*>(l.V);
     r.block_table = d.block_table; r.paged = d.paged; r.page_size = d.page_size;
     r.n_pages = d.n_pages; r.max_pages = d.max_pages; r.total_k = d.total_k;

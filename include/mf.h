@@ -207,8 +207,9 @@ mf_status mf_compress_qk(const mf_compress_qk_desc* desc, void* workspace, size_
  *   contiguous: [T_k][h_kv][d], key j of sequence s at token cu_seqlens_k[s] + j;
  *   paged:      [n_pages][page_size][h_kv][d], key j at page
  *               block_table[s * max_pages + j / page_size], row j % page_size.
- * O (dtype v_dtype) is [l_r_end - l_r_begin][T_q][h_r][d] with layer stride
- * o_layer_stride elements (0 = T_q * h_r * d).
+ * O (dtype v_dtype, or float32 with flag MF_RETRIEVE_O_F32) is
+ * [l_r_end - l_r_begin][T_q][h_r][d] with layer stride o_layer_stride elements
+ * (0 = T_q * h_r * d).
  * Arithmetic: MF_F32 maps/V run in float32 throughout.  MF_BF16 maps and V run on
  * tcgen05 tensor cores: W is split into a bf16 pair (hi + lo, ~16 bits), the mixed
  * map P is accumulated in float32 and rounded to float16, V is converted to float16
@@ -229,6 +230,9 @@ typedef struct {
 } mf_bsr;
 
 #define MF_RETRIEVE_FORCE_SIMT 1   /* flags: run the SIMT kernel even where tensor cores apply */
+#define MF_RETRIEVE_O_F32 2        /* flags: O is float32 (the unrounded float32 accumulators);
+                                      tensor-core path only (bf16 maps and V), else
+                                      MF_ERR_UNSUPPORTED */
 
 typedef struct {
   const mf_bsr* layers;            /* host [n_sender_layers] */

@@ -320,3 +320,77 @@ def test_empty_batch(entry):
     mf.mf_map_retrieve([out], [0], W, V, cu, cu, qb, 0, 4, 1, O=O)
     _status_ok()
     assert (O == 3.0).all()
+
+
+def _raw_close(got, want, amax, rl2, what):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    err = float(np.abs(got - want).max())
+    rel = float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30))
+    print(f"[O f32] {what}: raw max-abs {err:.3e}, rel-L2 {rel:.3e}")
+    assert err <= amax and rel <= rl2, f"{what}: raw max-abs {err:.3e} (<= {amax}), rel-L2 {rel:.3e} (<= {rl2})"
+
+
+@pytest.mark.parametrize("name,lens,B,h_s,h_r,h_kv,reading", [
+    ("f32out_varlen", (300, 129, 64), 64, 32, 32, 8, 3),
+    ("f32out_b128_gq3", (400,), 128, 32, 24, 8, 3),
+    ("f32out_hs40", (257,), 64, 40, 32, 8, 1),
+])
+def test_float32_output_meets_the_literal_bounds(name, lens, B, h_s, h_r, h_kv, reading):
+    """With float32 O (MF_RETRIEVE_O_F32) the tensor-core kernel's accumulators are compared
+    with the oracle unrounded: raw max-abs 2e-2 and relative L2 1e-2, every row; its bf16 output
+    is that float32 output rounded to nearest even."""
+    w = synth.Workload(name, lens, B=B, h_s=h_s, h_r=h_r, h_kv=h_kv, d=128, dtype="bf16", tau=0.95,
+                       n_heavy=16, reading=reading)
+    pack = sdev.fill_maps(sdev.alloc_maps(w), w, 0)
+    bsr = run_compress(w, pack)
+    _status_ok()
+    orows, _ = check_rows(w, pack, bsr, _all_rows(w))
+    W = sdev.w_weights(w)
+    V = sdev.v_contiguous(w, 0)
+    qbase, cu = sdev.qblock_base(w), pack.cu_seqlens
+    O32 = mf.mf_map_retrieve([bsr], [0], W, V, cu, cu, qbase, max(w.lens), w.h_r, w.h_kv,
+                             total_q=w.tokens, o_f32=True)[0]
+    O16 = mf.mf_map_retrieve([bsr], [0], W, V, cu, cu, qbase, max(w.lens), w.h_r, w.h_kv,
+                             total_q=w.tokens)[0]
+    _status_ok()
+    assert O32.dtype == torch.float32
+    assert torch.equal(O32.to(torch.bfloat16), O16)
+    want = _oracle_O_all(w, orows, W[0].cpu().numpy(), V.cpu())
+    _raw_close(O32.cpu().numpy(), want, 2e-2, 1e-2, name)
+
+
+def test_float32_output_full_size_sampled():
+    """The Ministral-like pair with float32 O: sampled query blocks held to the literal bounds."""
+    w = synth.ALL["ministral_pair"]
+    pack = sdev.fill_maps(sdev.alloc_maps(w), w, 0)
+    bsr = run_compress(w, pack)
+    _status_ok()
+    rows = [(0, qb) for qb in (0, 1, 63, 64, 126, 127)]
+    orows, nb = check_rows(w, pack, bsr, rows)
+    assert nb == 0
+    W = sdev.w_weights(w)
+    V = sdev.v_contiguous(w, 0)
+    cu = pack.cu_seqlens
+    O = mf.mf_map_retrieve([bsr], [0], W, V, cu, cu, sdev.qblock_base(w), w.lens[0], w.h_r,
+                           w.h_kv, total_q=w.tokens, o_f32=True)[0]
+    _status_ok()
+    Wl, Vh = W[0].cpu().numpy(), V.cpu()
+    for _, qb in rows:
+        want, (lo, hi) = oracle_O_rows(w, orows, 0, qb, Wl, Vh, 0)
+        _raw_close(O[qb * w.B + lo:qb * w.B + hi].cpu().numpy(), want, 2e-2, 1e-2, f"ministral qb={qb}")
+    del pack, bsr, O
+    torch.cuda.empty_cache()
+
+
+def test_float32_output_refused_on_the_simt_path():
+    w = synth.ALL["tiny"]
+    pack = sdev.fill_maps(sdev.alloc_maps(w), w, 0)
+    bsr = run_compress(w, pack)
+    W, V = sdev.w_weights(w), sdev.v_contiguous(w, 0)
+    cu = pack.cu_seqlens
+    with pytest.raises(mf.MFError) as e:
+        mf.mf_map_retrieve([bsr], [0], W, V, cu, cu, sdev.qblock_base(w), w.lens[0], w.h_r, w.h_kv,
+                           total_q=w.tokens, o_f32=True)
+    assert e.value.status == mf.MF_ERR_UNSUPPORTED
+    _status_ok()
