@@ -755,7 +755,7 @@ def run_routing(mf, dev, hbm, tf, reps=3):
             if q_len == 0:
                 continue
             q0 = k_len - q_len
-            r0, r1 = qbase[s] + q0 // w.B, qbase[s] + -(-k_len // w.B)
+            r0, r1 = int(qbase[s]) + q0 // w.B, int(qbase[s]) + -(-k_len // w.B)
             rows += r1 - r0
             n_step += int(rp[r1] - rp[r0])
         b, f = retrieve_algorithmic(w, n_step, rows, Tq, sum(k for _, k in step))
@@ -798,6 +798,13 @@ def _status_or_raise(mf, what):
     rc, bits = mf.mf_get_status()
     if rc != mf.MF_OK:
         raise RuntimeError(f"{what}: device status {rc} bits {bits:#x}")
+
+
+def _json_default(o):
+    """numpy scalars (and anything else with .item()) as plain numbers"""
+    if hasattr(o, "item"):
+        return o.item()
+    raise TypeError(f"not JSON serialisable: {type(o).__name__}")
 
 
 def mf_mod():
@@ -1029,14 +1036,17 @@ def main():
         if not args.no_configs:
             pts = [tuple(float(x) if i == 0 else int(x) for i, x in enumerate(p.split(":")))
                    for p in args.long_points.split(",") if p]
-            line["configs"] = {
-                "qwen_pair": run_qwen(mf_mod(), dev, hbm, tf_burst),
-                "long_context": run_long_context(mf_mod(), dev, hbm, tf_burst, pts),
-                "routing_batch": run_routing(mf_mod(), dev, hbm, tf_burst),
-            }
+            line["configs"] = {}
+            for name, fn in (("qwen_pair", lambda: run_qwen(mf_mod(), dev, hbm, tf_burst)),
+                             ("long_context", lambda: run_long_context(mf_mod(), dev, hbm, tf_burst, pts)),
+                             ("routing_batch", lambda: run_routing(mf_mod(), dev, hbm, tf_burst))):
+                line["configs"][name] = fn()
+                # each workload's figures also go to stderr as soon as they exist
+                print(json.dumps({name: line["configs"][name]}, default=_json_default), file=sys.stderr,
+                      flush=True)
         if not args.no_cpu and world == 1:
             line["cpu_baseline"] = cpu_baseline(w, dev, args.cpu_rows)
-        print(json.dumps(line), flush=True)
+        print(json.dumps(line, default=_json_default), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
 
