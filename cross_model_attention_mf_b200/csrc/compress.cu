@@ -114,6 +114,10 @@ __device__ inline uint64_t order_key(double x) {
   const uint64_t b = (uint64_t)__double_as_longlong(x);
   return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
 }
+// the mass back from its key (exact: the key is a bijection of the float64 bits)
+__device__ inline double key_mass(uint64_t k) {
+  return __longlong_as_double((long long)((k >> 63) ? (k & 0x7fffffffffffffffull) : ~k));
+}
 
 // Selection of one query block (row) by all NT threads of the calling CTA.  Candidates kb < qb
 // sorted by (mass desc, kb asc) in shared memory (bitonic), then one thread walks the float64
@@ -161,18 +165,21 @@ __device__ void select_row(const int64_t* __restrict__ meta, int nseq, const dou
       __syncthreads();
     }
   if (threadIdx.x == 0) {
+    // the walk reads the sorted masses back from their keys in shared memory (a serial loop of
+    // global loads would pay the L2 latency per candidate)
+    const double m_diag = __ldcg(mr + qb);
     double total = 0.0;
-    total += __ldcg(mr + qb);
-    for (int t = 0; t < n; ++t) total += __ldcg(mr + idx[t]);
+    total += m_diag;
+    for (int t = 0; t < n; ++t) total += key_mass(key[t]);
     const double target = tau * total;
     double S = 0.0;
     int nk = n + 1;
-    S += __ldcg(mr + qb);
+    S += m_diag;
     if (S >= target) {
       nk = 1;
     } else {
       for (int t = 0; t < n; ++t) {
-        S += __ldcg(mr + idx[t]);
+        S += key_mass(key[t]);
         if (S >= target) { nk = t + 2; break; }
       }
     }

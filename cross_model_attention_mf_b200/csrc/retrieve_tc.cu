@@ -166,26 +166,37 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-// try_wait with cluster-scope acquire: data written by peer CTAs (st.async) before they
-// completed the phase is visible after it returns true
+// try_wait; with CL, cluster-scope acquire (for the barriers peer CTAs signal: data a peer
+// wrote before completing the phase is visible once it returns true)
+template <bool CL = false>
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
+  if (CL)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
   return ok != 0;
 }
 // Bounded wait: false if the CTA aborted or the wait ran out of time (limit_ns).
+template <bool CL = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           uint32_t* status, uint64_t limit_ns) {
-  if (mbar_try(bar, parity)) return true;
+  if (mbar_try<CL>(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try(bar, parity)) return true;
+    if (mbar_try<CL>(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > limit_ns) {
@@ -196,9 +207,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
   }
 }
+template <bool CL = false>
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer();
-  while (!mbar_try(bar, parity) && globaltimer() - t0 < DRAIN_NS) {}
+  while (!mbar_try<CL>(bar, parity) && globaltimer() - t0 < DRAIN_NS) {}
 }
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
                                             int c0, int c1, int c2, int c3) {
@@ -344,12 +356,36 @@ __device__ __forceinline__ Unit decode(const TcParams& p, int idx) {
   return u;
 }
 
+// Optional timeline trace (compile with -DMF_TRACE): for the first TRACE_CTAS CTAs, per role,
+// SM-clock stamps of pipeline events kept in shared memory and copied out at the end, read back
+// with mf_trace_dump().  Each role has a single writing thread.  Roles: 0 map producer, 1 mixing
+// issuer, 2 P.V issuer, 3 first converter warp, 4 first V loader warp.
+#ifdef MF_TRACE
+constexpr int TRACE_CTAS = 16, TRACE_N = 512, TRACE_ROLES = 5;
+__device__ uint64_t g_trace[TRACE_CTAS][TRACE_ROLES][TRACE_N];
+#define TRACE(role, code)                                                                  \
+  do {                                                                                     \
+    const int n_ = s_tn[role];                                                             \
+    if (n_ < TRACE_N - 1) {                                                                \
+      s_tr[role][1 + n_] = ((uint64_t)(code) << 56) | ((uint64_t)clock64() & ((1ull << 56) - 1)); \
+      s_tn[role] = n_ + 1;                                                                 \
+    }                                                                                      \
+  } while (0)
+#else
+#define TRACE(role, code)
+#endif
+
 // ------------------------------------------------------------------ kernel
 __global__ void __launch_bounds__(NT, 1)
     k_retrieve_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
+#ifdef MF_TRACE
+  __shared__ uint64_t s_tr[TRACE_ROLES][TRACE_N];
+  __shared__ volatile int s_tn[TRACE_ROLES];
+  if (threadIdx.x < TRACE_ROLES) s_tn[threadIdx.x] = 0;
+#endif
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -442,6 +478,7 @@ __global__ void __launch_bounds__(NT, 1)
           ok = __all_sync(0xffffffffu, mbar_wait(bar(B_AEMPTY + as), aph ^ 1, abort_flag, p.status, p.wait_ns));
           if (!ok) break;
           if (lane == 0) {
+            TRACE(0, 1);
             mbar_expect_tx(bar(B_AFULL + as), A_BYTES);
             tma_load_4d(sb + OFF_A + as * A_BYTES, &tmA, bar(B_AFULL + as), half * KT, c * SC,
                         w * WR + rank * RM, (int)e);
@@ -478,12 +515,14 @@ __global__ void __launch_bounds__(NT, 1)
         for (int hf = 0; hf < 2 && ok; ++hf) {
           ok = __all_sync(0xffffffffu, mbar_wait(bar(B_D1EMPTY + hf), (T & 1) ^ 1, abort_flag, p.status, p.wait_ns));
           if (!ok) break;
+          if (lane == 0) TRACE(1, 2 + hf);
           int st = as;
           uint32_t ph = aph;
           for (int c = 0; c < p.nsc && ok; ++c) {
             if (hf == 0) {
               ok = __all_sync(0xffffffffu, mbar_wait(bar(B_AFULL + st), ph, abort_flag, p.status, p.wait_ns));
               if (!ok) break;
+              if (lane == 0) TRACE(1, 4);
             }
             if (lane == 0) {
               tc_fence_after();
@@ -528,8 +567,11 @@ __global__ void __launch_bounds__(NT, 1)
         // the owner announces the bytes its peers will complete on the slot's barrier
         if (lane == 0) mbar_expect_tx(bar(B_PFULL + ps), PSLOT_BYTES);
         __syncwarp();
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PFULL + ps), (T / PSLOTS) & 1, abort_flag, p.status, p.wait_ns));
+        if (lane == 0) TRACE(2, 5);
+        ok = __all_sync(0xffffffffu, mbar_wait<true>(bar(B_PFULL + ps), (T / PSLOTS) & 1, abort_flag, p.status, p.wait_ns));
+        if (lane == 0) TRACE(2, 6);
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_VFULL + vs), (T / VSLOTS) & 1, abort_flag, p.status, p.wait_ns));
+        if (lane == 0) TRACE(2, 7);
         // the previous unit's epilogue must have read D2 out
         for (int gl = 0; gl < GO && ok && t == 0 && K > 0; ++gl)
           ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OEMPTY + gl), (K - 1) & 1, abort_flag, p.status, p.wait_ns));
@@ -547,6 +589,7 @@ __global__ void __launch_bounds__(NT, 1)
           }
           tc_commit(bar(B_VEMPTY + vs));
           tc_commit_mc(bar(B_PEMPTY + ps), (uint16_t)((1u << CS) - 1u));  // the slot is free in all four CTAs
+          TRACE(2, 8);
         }
         __syncwarp();
       }
@@ -587,8 +630,10 @@ __global__ void __launch_bounds__(NT, 1)
       const Unit u = unit(ek, eidx);
       const bool have = u.n_tiles > 0;
       const int ilo = u.row_lo - u.i_begin, ihi = u.row_hi - u.i_begin;
+      if (warp == 4 && lane == 0) TRACE(3, 15);
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_OFULL), Ke & 1, abort_flag, p.status, p.wait_ns)))
         return false;
+      if (warp == 4 && lane == 0) TRACE(3, 16);
       tc_fence_after();
       for (int gl = 0; gl < GO; ++gl) {
         const int G = hc * NGC + rank * GO + gl;
@@ -660,6 +705,7 @@ __global__ void __launch_bounds__(NT, 1)
           }
         }
       }
+      if (warp == 4 && lane == 0) TRACE(3, 17);
       return true;
     };
     bool ok = true;
@@ -686,8 +732,10 @@ __global__ void __launch_bounds__(NT, 1)
         const bool full = kb_ok && tok0 + KT - 1 <= u.i_begin + rank * RM;
         uint32_t pkA[HV / 2], pkB[HV / 2];
         for (int pair = 0; pair < 2 && ok; ++pair) {
+          if (warp == 4 && lane == 0) TRACE(3, 9 + pair);
           ok = __all_sync(0xffffffffu, mbar_wait(bar(B_D1FULL + pair), T & 1, abort_flag, p.status, p.wait_ns));
           if (!ok) break;
+          if (warp == 4 && lane == 0) TRACE(3, 11 + pair);
           tc_fence_after();
 #pragma unroll
           for (int mm = 0; mm < 2; ++mm) {
@@ -716,10 +764,11 @@ __global__ void __launch_bounds__(NT, 1)
           }
           // the slot must have been consumed by all four owners (tile T - PSLOTS)
           if (pair == 0 && T >= PSLOTS) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PEMPTY + ps), ((T / PSLOTS) & 1) ^ 1,
-                                                   abort_flag, p.status, p.wait_ns));
+            ok = __all_sync(0xffffffffu, mbar_wait<true>(bar(B_PEMPTY + ps), ((T / PSLOTS) & 1) ^ 1,
+                                                         abort_flag, p.status, p.wait_ns));
             if (!ok) break;
           }
+          if (warp == 4 && lane == 0) TRACE(3, 13 + pair);
           // one 16-byte chunk per group: rows (2*(2 pair) + rb, 2*(2 pair + 1) + rb), 4 heads each
           const uint32_t c = 4u * (uint32_t)rank + 2u * (uint32_t)pair + (uint32_t)rb;
           const uint32_t off = OFF_P + (uint32_t)ps * PSLOT_BYTES + (c >> 3) * 8192u +
@@ -749,72 +798,97 @@ __global__ void __launch_bounds__(NT, 1)
     if (lane == 0)
       for (int k = 0; k < PSLOTS; ++k) {
         const int cnt = T > k ? (T - k - 1) / PSLOTS + 1 : 0;
-        if (cnt) mbar_drain(bar(B_PEMPTY + k), (cnt - 1) & 1);
+        if (cnt) mbar_drain<true>(bar(B_PEMPTY + k), (cnt - 1) & 1);
       }
     __syncwarp();
   } else if (warp >= 8) {
     // ================================================================ V loaders
     // 128 threads; per tile 2 groups x 64 keys x 16 vectors of 8 dims: 16 vectors per thread.
-    // Loads for a tile are issued before the wait for its slot, so their latency overlaps it.
+    // A cursor runs one tile ahead: the loads of the next tile are in flight while this one is
+    // converted and stored.
     const int tid = threadIdx.x - 8 * 32;
     bool ok = true;
     int T = 0;
     float amax = 0.0f;
-    for (int idx = cl, ik = 0; idx < p.n_units && ok; idx += ncl, ++ik) {
-      const Unit u = unit(ik, idx);
-      if (!u.valid) continue;
-      int kb = u.kb0;
-      for (int t = 0; t < u.n_tiles && ok; ++t, ++T) {
-        const int half = t % tpb;
-        if (t > 0 && half == 0) kb = p.col_idx[u.rp0 + t / tpb];
-        const bool kb_ok = kb >= 0 && kb <= u.qb;
-        if (!kb_ok && rank == 0 && tid == 0) atomicOr(p.status, ST_INDEX);
-        const int tok0 = kb * p.B + half * KT;
-        const int vs = T % VSLOTS;
-        uint4 r[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int v = tid + 128 * i;
-          const int gl = v >> 10, key = (v >> 4) & 63, ch = v & 15;
-          const int G = hc * NGC + rank * GO + gl;
-          const int tok = tok0 + key;
-          r[i] = make_uint4(0u, 0u, 0u, 0u);
-          if (kb_ok && tok < u.k_len && G < q_r.h_kv) {
-            int64_t row = -1;
-            if (!q_r.paged) {
-              row = (int64_t)u.k0 + tok;
-              if (row >= q_r.total_k) row = -1;
-            } else {
-              const int slot = tok / q_r.page_size;
-              if (slot < q_r.max_pages) {
-                const int pg = q_r.block_table[(int64_t)u.s * q_r.max_pages + slot];
-                if (pg >= 0 && pg < q_r.n_pages) row = (int64_t)pg * q_r.page_size + tok % q_r.page_size;
-                else atomicOr(p.status, ST_PAGE);
-              }
-            }
-            if (row >= 0)
-              r[i] = __ldg(reinterpret_cast<const uint4*>(q_r.V + (row * q_r.h_kv + G) * D + ch * 8));
-          }
-        }
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_VEMPTY + vs), ((T / VSLOTS) & 1) ^ 1, abort_flag,
-                                               p.status, p.wait_ns));
-        if (!ok) break;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int v = tid + 128 * i;
-          const int gl = v >> 10, key = (v >> 4) & 63, ch = v & 15;
-          const uint32_t dst = sb + OFF_V + (uint32_t)vs * VSLOT_BYTES + (uint32_t)gl * VG_BYTES +
-                               ((uint32_t)ch >> 3) * 8192u + (uint32_t)key * 128u +
-                               ((((uint32_t)ch & 7u) ^ ((uint32_t)key & 7u)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
-                       "r"(bf2_to_h2(r[i].x, amax)), "r"(bf2_to_h2(r[i].y, amax)),
-                       "r"(bf2_to_h2(r[i].z, amax)), "r"(bf2_to_h2(r[i].w, amax))
-                       : "memory");
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_VFULL + vs));
+    // cursor over this cluster's tiles in order (units without tiles are skipped)
+    int c_ik = -1, c_idx = cl - ncl, c_t = 0, c_kb = -1;
+    Unit c_u;
+    c_u.n_tiles = 0;
+    auto advance = [&]() -> bool {  // to the next tile; false when none is left
+      ++c_t;
+      while (c_t >= c_u.n_tiles) {
+        ++c_ik;
+        c_idx += ncl;
+        if (c_idx >= p.n_units) return false;
+        c_u = unit(c_ik, c_idx);
+        if (!c_u.valid) c_u.n_tiles = 0;
+        c_t = 0;
       }
+      if (c_t % tpb == 0) c_kb = c_t == 0 ? c_u.kb0 : p.col_idx[c_u.rp0 + c_t / tpb];
+      return true;
+    };
+    auto issue = [&](uint4 (&r)[16]) {
+      const int half = c_t % tpb;
+      const bool kb_ok = c_kb >= 0 && c_kb <= c_u.qb;
+      if (!kb_ok && rank == 0 && tid == 0) atomicOr(p.status, ST_INDEX);
+      const int tok0 = c_kb * p.B + half * KT;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int v = tid + 128 * i;
+        const int gl = v >> 10, key = (v >> 4) & 63, ch = v & 15;
+        const int G = hc * NGC + rank * GO + gl;
+        const int tok = tok0 + key;
+        r[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (kb_ok && tok < c_u.k_len && G < q_r.h_kv) {
+          int64_t row = -1;
+          if (!q_r.paged) {
+            row = (int64_t)c_u.k0 + tok;
+            if (row >= q_r.total_k) row = -1;
+          } else {
+            const int slot = tok / q_r.page_size;
+            if (slot < q_r.max_pages) {
+              const int pg = q_r.block_table[(int64_t)c_u.s * q_r.max_pages + slot];
+              if (pg >= 0 && pg < q_r.n_pages) row = (int64_t)pg * q_r.page_size + tok % q_r.page_size;
+              else atomicOr(p.status, ST_PAGE);
+            }
+          }
+          if (row >= 0)
+            r[i] = __ldg(reinterpret_cast<const uint4*>(q_r.V + (row * q_r.h_kv + G) * D + ch * 8));
+        }
+      }
+    };
+    uint4 ra[16], rb[16];
+    bool have = advance();
+    if (have) issue(ra);
+    while (have && ok) {
+      const bool more = advance();
+      if (more) issue(rb);
+      const int vs = T % VSLOTS;
+      if (warp == 8 && lane == 0) TRACE(4, 18);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_VEMPTY + vs), ((T / VSLOTS) & 1) ^ 1, abort_flag,
+                                             p.status, p.wait_ns));
+      if (!ok) break;
+      if (warp == 8 && lane == 0) TRACE(4, 19);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int v = tid + 128 * i;
+        const int gl = v >> 10, key = (v >> 4) & 63, ch = v & 15;
+        const uint32_t dst = sb + OFF_V + (uint32_t)vs * VSLOT_BYTES + (uint32_t)gl * VG_BYTES +
+                             ((uint32_t)ch >> 3) * 8192u + (uint32_t)key * 128u +
+                             ((((uint32_t)ch & 7u) ^ ((uint32_t)key & 7u)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
+                     "r"(bf2_to_h2(ra[i].x, amax)), "r"(bf2_to_h2(ra[i].y, amax)),
+                     "r"(bf2_to_h2(ra[i].z, amax)), "r"(bf2_to_h2(ra[i].w, amax))
+                     : "memory");
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_VFULL + vs));
+      if (warp == 8 && lane == 0) TRACE(4, 20);
+      ++T;
+      have = more;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) ra[i] = rb[i];
     }
     if (amax > F16_MAX) atomicOr(p.status, ST_RANGE);
   }
@@ -826,6 +900,13 @@ __global__ void __launch_bounds__(NT, 1)
     const uint64_t t0 = globaltimer();
     while (globaltimer() - t0 < GRACE_NS) {}
   }
+#ifdef MF_TRACE
+  if (blockIdx.x < TRACE_CTAS)
+    for (int e = threadIdx.x; e < TRACE_ROLES * TRACE_N; e += NT) {
+      const int r = e / TRACE_N, k = e % TRACE_N;
+      g_trace[blockIdx.x][r][k] = k == 0 ? (uint64_t)s_tn[r] : s_tr[r][k];
+    }
+#endif
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
@@ -978,3 +1059,13 @@ bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* 
 }
 
 }  // namespace mfi
+
+#ifdef MF_TRACE
+extern "C" __attribute__((visibility("default"))) int mf_trace_dump(void* host, size_t bytes) {
+  if (bytes < sizeof(mfi::g_trace)) return -1;
+  if (cudaMemcpyFromSymbol(host, mfi::g_trace, sizeof(mfi::g_trace)) != cudaSuccess) return -2;
+  static uint64_t zero[mfi::TRACE_CTAS][mfi::TRACE_ROLES][mfi::TRACE_N];
+  if (cudaMemcpyToSymbol(mfi::g_trace, zero, sizeof(zero)) != cudaSuccess) return -3;
+  return 0;
+}
+#endif
