@@ -33,7 +33,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 MF_OK, MF_ERR_INVALID, MF_ERR_UNSUPPORTED, MF_ERR_CAPACITY, MF_ERR_CUDA, MF_ERR_TIMEOUT, \
-    MF_ERR_DEVICE_INDEX, MF_ERR_RANGE = range(8)
+    MF_ERR_DEVICE_INDEX = range(7)
 MF_F32, MF_BF16 = 0, 1
 MF_RETRIEVE_FORCE_SIMT = 1
 MF_RETRIEVE_O_F32 = 2

@@ -6,19 +6,16 @@
 // first, then the blocks to keep are chosen by cumulative attention probability,
 // and only those are written -- no second dense matrix is assembled.
 //
-// Kernels (all on the caller's stream):
+// Kernels (one launch each, all on the caller's stream):
 //   k_meta          per-sequence geometry of the varlen pack (one thread)
 //   k_stats         head-summed mass of every causal block: a streaming reduction
 //                   with 16-byte loads, float32 partials of 8 (bf16) or 4 (f32)
 //                   elements combined in float64, fixed order (deterministic)
-//   selection       per query block: sort candidates (mass desc, kb asc), walk
+//   k_select        per query block: sort candidates (mass desc, kb asc), walk
 //                   the running float64 sum until it reaches tau * total, write the
-//                   row's kept indices in ascending order to a per-row list; done by
-//                   the k_stats CTA that writes the row's last mass (rows of up to
-//                   1024 candidates; longer rows: a k_select launch)
-//   scan/compact    row_ptr by exclusive scan of the counts, then copy the per-row
-//                   lists into col_idx; done by the k_stats CTA that selects the last
-//                   row (after a k_select launch: k_scan_compact)
+//                   row's kept indices in ascending order to a per-row list
+//   k_scan_compact  row_ptr by exclusive scan of the counts, then copy the per-row
+//                   lists into col_idx
 //   k_gather        copy each kept block with the causal/length mask applied, one
 //                   (block, sender head) unit per CTA iteration
 #include <cuda_bf16.h>
@@ -52,13 +49,7 @@ __device__ inline int tri_row(int64_t c) {
 
 __global__ void k_meta(const int32_t* cu, const int64_t* off, int nseq, int max_seqlen, int B,
                        int elem_bytes, int64_t* meta, uint32_t* status, int32_t* row_ptr,
-                       int32_t* nnz_out, int32_t* row_done, int64_t max_rows) {
-  // the next kernel (k_stats) may launch now; it waits for this grid before reading anything
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (row_done)  // per-row counters of the fused selection start at zero on every call
-    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < max_rows;
-         r += (int64_t)gridDim.x * blockDim.x)
-      row_done[r] = 0;
+                       int32_t* nnz_out) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   int64_t rows = 0, cb = 0;
   uint32_t st = 0;
@@ -109,211 +100,15 @@ __device__ inline double block_sum_f64(double v, double* red) {
   return t;  // valid in thread 0
 }
 
-__device__ inline uint64_t order_key(double x) {
-  if (x == 0.0) x = 0.0;  // -0 sorts with +0
-  const uint64_t b = (uint64_t)__double_as_longlong(x);
-  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
-}
-// the mass back from its key (exact: the key is a bijection of the float64 bits)
-__device__ inline double key_mass(uint64_t k) {
-  return __longlong_as_double((long long)((k >> 63) ? (k & 0x7fffffffffffffffull) : ~k));
-}
-
-// Selection of one query block (row) by all NT threads of the calling CTA.  Candidates kb < qb
-// sorted by (mass desc, kb asc) in shared memory (bitonic), then one thread walks the float64
-// running sum from the diagonal block until it reaches tau * total; the row's kept indices go
-// to kept_local in ascending order, their count to counts[row].  sm holds at least
-// n2 = (next power of two >= qb) keys and indices (12 n2 bytes); misc holds NT / 32 + 2 ints.
-// Masses are read through L2 (another CTA may have written them moments ago).
-template <int NT>
-__device__ void select_row(const int64_t* __restrict__ meta, int nseq, const double* mass,
-                           double tau, int64_t row, int32_t* __restrict__ counts,
-                           int32_t* __restrict__ kept_local, uint64_t* sm, int* misc) {
-  int& s_nkeep = misc[0];
-  int& s_base = misc[1];
-  int* s_warp = misc + 2;
-  const int s = find_seq(meta, nseq, row, 2);
-  const int64_t* m = meta + META_HDR + 4 * s;
-  const int qb = (int)(row - m[2]);
-  const int64_t tri = m[3] + (int64_t)qb * (qb + 1) / 2;
-  const double* mr = mass + tri;
-  const int n = qb;
-  int n2 = 1;
-  while (n2 < n) n2 <<= 1;
-  uint64_t* key = sm;
-  int* idx = reinterpret_cast<int*>(sm + n2);
-  for (int t = threadIdx.x; t < n2; t += NT) {
-    if (t < n) { key[t] = order_key(__ldcg(mr + t)); idx[t] = t; }
-    else { key[t] = 0ull; idx[t] = 0x7fffffff; }
-  }
-  __syncthreads();
-  // bitonic sort into (key desc, idx asc)
-  for (int k = 2; k <= n2; k <<= 1)
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int t = threadIdx.x; t < n2; t += NT) {
-        const int p = t ^ j;
-        if (p > t) {
-          const bool up = (t & k) == 0;  // this run sorts into the target order
-          const uint64_t ka = key[t], kb2 = key[p];
-          const int ia = idx[t], ib = idx[p];
-          const bool a_first = ka > kb2 || (ka == kb2 && ia < ib);
-          if (up != a_first) {
-            key[t] = kb2; key[p] = ka; idx[t] = ib; idx[p] = ia;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  if (threadIdx.x == 0) {
-    // the walk reads the sorted masses back from their keys in shared memory (a serial loop of
-    // global loads would pay the L2 latency per candidate)
-    const double m_diag = __ldcg(mr + qb);
-    double total = 0.0;
-    total += m_diag;
-    for (int t = 0; t < n; ++t) total += key_mass(key[t]);
-    const double target = tau * total;
-    double S = 0.0;
-    int nk = n + 1;
-    S += m_diag;
-    if (S >= target) {
-      nk = 1;
-    } else {
-      for (int t = 0; t < n; ++t) {
-        S += key_mass(key[t]);
-        if (S >= target) { nk = t + 2; break; }
-      }
-    }
-    s_nkeep = nk;
-    counts[row] = nk;
-  }
-  __syncthreads();
-  // kept flags by key-block index (reusing the key array), then an ordered compaction:
-  // the row's kept indices in ascending order at kept_local[tri ...]
-  const int nk = s_nkeep;
-  uint8_t* kept = reinterpret_cast<uint8_t*>(key);
-  for (int t = threadIdx.x; t <= n; t += NT) kept[t] = 0;
-  __syncthreads();
-  for (int t = threadIdx.x; t < nk - 1; t += NT) kept[idx[t]] = 1;
-  if (threadIdx.x == 0) kept[qb] = 1;
-  if (threadIdx.x == 0) s_base = 0;
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int k0 = 0; k0 <= n; k0 += NT) {
-    const int kb = k0 + threadIdx.x;
-    const bool f = kb <= n && kept[kb];
-    const uint32_t bal = __ballot_sync(0xffffffffu, f);
-    __syncthreads();
-    if (lane == 0) s_warp[warp] = __popc(bal);
-    __syncthreads();
-    int before = s_base;
-    for (int w = 0; w < warp; ++w) before += s_warp[w];
-    if (f) kept_local[tri + before + __popc(bal & ((1u << lane) - 1u))] = kb;
-    __syncthreads();
-    if (threadIdx.x == 0)
-      for (int w = 0; w < NT / 32; ++w) s_base += s_warp[w];
-  }
-  __syncthreads();
-}
-
-// Exclusive scan of the counts into row_ptr by all NT threads of one CTA (independent loads,
-// so their latencies overlap), then each row's list is copied into col_idx (warp per row).
-// part: NT int64 of shared scratch.  Counts and lists are read through L2 (other CTAs may have
-// written them moments ago).
-constexpr int SCAN_PER = 8;
-template <int NT>
-__device__ void scan_compact(const int64_t* __restrict__ meta, int nseq, const int32_t* counts,
-                             const int32_t* kept_local, int32_t* __restrict__ row_ptr,
-                             int32_t* __restrict__ col_idx, int32_t* __restrict__ kept_row,
-                             int32_t* __restrict__ nnz_out, int64_t capacity, uint32_t* status,
-                             int64_t* part, int64_t* carry) {
-  const int64_t R = meta[0];
-  const int t = threadIdx.x;
-  if (t == 0) *carry = 0;
-  __syncthreads();
-  for (int64_t base = 0; base < R; base += (int64_t)NT * SCAN_PER) {
-    const int64_t r0 = base + (int64_t)t * SCAN_PER;
-    int32_t c[SCAN_PER];
-#pragma unroll
-    for (int k = 0; k < SCAN_PER; ++k) c[k] = r0 + k < R ? __ldcg(counts + r0 + k) : 0;
-    int64_t sum = 0;
-#pragma unroll
-    for (int k = 0; k < SCAN_PER; ++k) sum += c[k];
-    part[t] = sum;
-    __syncthreads();
-    for (int o = 1; o < NT; o <<= 1) {  // inclusive Hillis-Steele scan
-      const int64_t v = t >= o ? part[t - o] : 0;
-      __syncthreads();
-      part[t] += v;
-      __syncthreads();
-    }
-    int64_t run = *carry + part[t] - sum;
-#pragma unroll
-    for (int k = 0; k < SCAN_PER; ++k)
-      if (r0 + k < R) {
-        row_ptr[r0 + k] = (int32_t)run;
-        run += c[k];
-      }
-    __syncthreads();
-    if (t == NT - 1) *carry += part[NT - 1];
-    __syncthreads();
-  }
-  const int64_t nnz = *carry;
-  if (t == 0) {
-    row_ptr[R] = (int32_t)nnz;
-    *nnz_out = (int32_t)nnz;
-    if (nnz > capacity) atomicOr(status, ST_CAPACITY);
-  }
-  __syncthreads();
-  const int warp = t >> 5, lane = t & 31;
-  for (int64_t row = warp; row < R; row += NT / 32) {
-    const int s = find_seq(meta, nseq, row, 2);
-    const int64_t* m = meta + META_HDR + 4 * s;
-    const int qb = (int)(row - m[2]);
-    const int32_t* kl = kept_local + m[3] + (int64_t)qb * (qb + 1) / 2;
-    const int64_t n0 = row_ptr[row];
-    const int cnt = __ldcg(counts + row);
-    for (int k = lane; k < cnt; k += 32)
-      if (n0 + k < capacity) {
-        col_idx[n0 + k] = __ldcg(kl + k);
-        kept_row[n0 + k] = (int32_t)row;
-      }
-  }
-}
-
-// rows with at most this many candidates are selected inside k_stats (its shared scratch)
-constexpr int SEL_FUSED_MAX = 1024;
-
-// Masses of every causal block.  Item = (sequence, qb, kb) over all sender heads.  With
-// row_done set, the CTA that writes the last mass of a row (a per-row counter reaches qb + 1)
-// also selects that row, so selection overlaps the rest of the stream.
-struct FusedTail {             // selection and BSR index build inside k_stats
-  int32_t* row_done;           // [rows] masses written per row
-  unsigned long long* rows_selected;  // rows whose selection is done
-  double tau;
-  int32_t* counts;
-  int32_t* kept_local;
-  int32_t* row_ptr;
-  int32_t* col_idx;
-  int32_t* kept_row;
-  int32_t* nnz_out;
-  int64_t capacity;
-  uint32_t* status;
-};
-
+// Masses of every causal block.  Item = (sequence, qb, kb) over all sender heads.
 template <typename T, int B, int NT>
 __global__ void __launch_bounds__(NT) k_stats(const T* __restrict__ maps,
                                               const int64_t* __restrict__ seq_off,
                                               const int64_t* __restrict__ meta, int nseq,
-                                              int h_s, double* mass, const FusedTail ft) {
+                                              int h_s, double* __restrict__ mass) {
   constexpr int EPV = Vec<T>::EPV, VPR = B / EPV, VPB = B * VPR;  // vectors per row / per head
   constexpr int U = 4;
   __shared__ double red[NT / 32];
-  __shared__ uint64_t sel[SEL_FUSED_MAX * 3 / 2];  // keys and indices of one row's candidates
-  __shared__ int misc[NT / 32 + 2];
-  __shared__ int s_last, s_all;
-  __shared__ int64_t part[NT], carry;
-  // launched while k_meta may still run (programmatic dependent launch): wait for it
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t total = meta[1];
   const int64_t nv = (int64_t)h_s * VPB;
   for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
@@ -368,46 +163,110 @@ __global__ void __launch_bounds__(NT) k_stats(const T* __restrict__ maps,
     }
     const double t = block_sum_f64<NT>(acc, red);
     if (threadIdx.x == 0) mass[item] = t;
-    if (ft.row_done) {
-      if (threadIdx.x == 0) {
-        __threadfence();  // this mass is visible before the count that announces it
-        s_last = atomicAdd(&ft.row_done[m[2] + qb], 1) == qb ? 1 : 0;
-        __threadfence();
-      }
-      __syncthreads();
-      if (s_last) {
-        select_row<NT>(meta, nseq, mass, ft.tau, m[2] + qb, ft.counts, ft.kept_local, sel, misc);
-        // the CTA that selects the last row also builds row_ptr and col_idx
-        if (threadIdx.x == 0) {
-          __threadfence();
-          s_all = atomicAdd(ft.rows_selected, 1ull) == (unsigned long long)(meta[0] - 1) ? 1 : 0;
-          __threadfence();
-        }
-        __syncthreads();
-        if (s_all)
-          scan_compact<NT>(meta, nseq, ft.counts, ft.kept_local, ft.row_ptr, ft.col_idx,
-                           ft.kept_row, ft.nnz_out, ft.capacity, ft.status, part, &carry);
-      }
-    }
   }
 }
 
-// One CTA per query block (row): the selection as its own launch (rows with more than
-// SEL_FUSED_MAX candidates, and compression from Q, K).
+__device__ inline uint64_t order_key(double x) {
+  if (x == 0.0) x = 0.0;  // -0 sorts with +0
+  const uint64_t b = (uint64_t)__double_as_longlong(x);
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+// One CTA per query block (row).  Candidates kb < qb sorted by (mass desc, kb asc);
+// the walk starts from the diagonal block.
 template <int NT>
 __global__ void __launch_bounds__(NT) k_select(const int64_t* __restrict__ meta, int nseq,
                                                const double* __restrict__ mass, double tau,
                                                int32_t* __restrict__ counts,
                                                int32_t* __restrict__ kept_local) {
   extern __shared__ uint64_t sm[];
-  __shared__ int misc[NT / 32 + 2];
+  __shared__ int s_nkeep;
   const int64_t row = blockIdx.x;
   if (row >= meta[0]) return;
-  select_row<NT>(meta, nseq, mass, tau, row, counts, kept_local, sm, misc);
+  const int s = find_seq(meta, nseq, row, 2);
+  const int64_t* m = meta + META_HDR + 4 * s;
+  const int qb = (int)(row - m[2]);
+  const int64_t tri = m[3] + (int64_t)qb * (qb + 1) / 2;
+  const double* mr = mass + tri;
+  const int n = qb;
+  int n2 = 1;
+  while (n2 < n) n2 <<= 1;
+  uint64_t* key = sm;
+  int* idx = reinterpret_cast<int*>(sm + n2);
+  for (int t = threadIdx.x; t < n2; t += NT) {
+    if (t < n) { key[t] = order_key(mr[t]); idx[t] = t; }
+    else { key[t] = 0ull; idx[t] = 0x7fffffff; }
+  }
+  __syncthreads();
+  // bitonic sort into (key desc, idx asc)
+  for (int k = 2; k <= n2; k <<= 1)
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int t = threadIdx.x; t < n2; t += NT) {
+        const int p = t ^ j;
+        if (p > t) {
+          const bool up = (t & k) == 0;  // this run sorts into the target order
+          const uint64_t ka = key[t], kb2 = key[p];
+          const int ia = idx[t], ib = idx[p];
+          const bool a_first = ka > kb2 || (ka == kb2 && ia < ib);
+          if (up != a_first) {
+            key[t] = kb2; key[p] = ka; idx[t] = ib; idx[p] = ia;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  if (threadIdx.x == 0) {
+    double total = 0.0;
+    total += mr[qb];
+    for (int t = 0; t < n; ++t) total += mr[idx[t]];
+    const double target = tau * total;
+    double S = 0.0;
+    int nk = n + 1;
+    S += mr[qb];
+    if (S >= target) {
+      nk = 1;
+    } else {
+      for (int t = 0; t < n; ++t) {
+        S += mr[idx[t]];
+        if (S >= target) { nk = t + 2; break; }
+      }
+    }
+    s_nkeep = nk;
+    counts[row] = nk;
+  }
+  __syncthreads();
+  // kept flags by key-block index (reusing the key array), then an ordered compaction:
+  // the row's kept indices in ascending order at kept_local[tri ...]
+  const int nk = s_nkeep;
+  uint8_t* kept = reinterpret_cast<uint8_t*>(key);
+  for (int t = threadIdx.x; t <= n; t += NT) kept[t] = 0;
+  __syncthreads();
+  for (int t = threadIdx.x; t < nk - 1; t += NT) kept[idx[t]] = 1;
+  if (threadIdx.x == 0) kept[qb] = 1;
+  __syncthreads();
+  __shared__ int s_warp[NT / 32];
+  __shared__ int s_base;
+  if (threadIdx.x == 0) s_base = 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int k0 = 0; k0 <= n; k0 += NT) {
+    const int kb = k0 + threadIdx.x;
+    const bool f = kb <= n && kept[kb];
+    const uint32_t bal = __ballot_sync(0xffffffffu, f);
+    __syncthreads();
+    if (lane == 0) s_warp[warp] = __popc(bal);
+    __syncthreads();
+    int before = s_base;
+    for (int w = 0; w < warp; ++w) before += s_warp[w];
+    if (f) kept_local[tri + before + __popc(bal & ((1u << lane) - 1u))] = kb;
+    __syncthreads();
+    if (threadIdx.x == 0)
+      for (int w = 0; w < NT / 32; ++w) s_base += s_warp[w];
+  }
 }
 
-// The scan as its own launch (after a separate selection launch).
-constexpr int SCAN_NT = 1024;
+// One CTA: exclusive scan of the counts into row_ptr (independent loads, so their
+// latencies overlap), then each row's list is copied into col_idx (warp per row).
+constexpr int SCAN_NT = 1024, SCAN_PER = 8;
 __global__ void __launch_bounds__(SCAN_NT) k_scan_compact(
     const int64_t* __restrict__ meta, int nseq, const int32_t* __restrict__ counts,
     const int32_t* __restrict__ kept_local, int32_t* __restrict__ row_ptr,
@@ -415,8 +274,58 @@ __global__ void __launch_bounds__(SCAN_NT) k_scan_compact(
     int64_t capacity, uint32_t* status) {
   __shared__ int64_t part[SCAN_NT];
   __shared__ int64_t carry;
-  scan_compact<SCAN_NT>(meta, nseq, counts, kept_local, row_ptr, col_idx, kept_row, nnz_out,
-                        capacity, status, part, &carry);
+  const int64_t R = meta[0];
+  const int t = threadIdx.x;
+  if (t == 0) carry = 0;
+  __syncthreads();
+  for (int64_t base = 0; base < R; base += (int64_t)SCAN_NT * SCAN_PER) {
+    const int64_t r0 = base + (int64_t)t * SCAN_PER;
+    int32_t c[SCAN_PER];
+#pragma unroll
+    for (int k = 0; k < SCAN_PER; ++k) c[k] = r0 + k < R ? counts[r0 + k] : 0;
+    int64_t sum = 0;
+#pragma unroll
+    for (int k = 0; k < SCAN_PER; ++k) sum += c[k];
+    part[t] = sum;
+    __syncthreads();
+    for (int o = 1; o < SCAN_NT; o <<= 1) {  // inclusive Hillis-Steele scan
+      const int64_t v = t >= o ? part[t - o] : 0;
+      __syncthreads();
+      part[t] += v;
+      __syncthreads();
+    }
+    int64_t run = carry + part[t] - sum;
+#pragma unroll
+    for (int k = 0; k < SCAN_PER; ++k)
+      if (r0 + k < R) {
+        row_ptr[r0 + k] = (int32_t)run;
+        run += c[k];
+      }
+    __syncthreads();
+    if (t == SCAN_NT - 1) carry += part[SCAN_NT - 1];
+    __syncthreads();
+  }
+  const int64_t nnz = carry;
+  if (t == 0) {
+    row_ptr[R] = (int32_t)nnz;
+    *nnz_out = (int32_t)nnz;
+    if (nnz > capacity) atomicOr(status, ST_CAPACITY);
+  }
+  __syncthreads();
+  const int warp = t >> 5, lane = t & 31;
+  for (int64_t row = warp; row < R; row += SCAN_NT / 32) {
+    const int s = find_seq(meta, nseq, row, 2);
+    const int64_t* m = meta + META_HDR + 4 * s;
+    const int qb = (int)(row - m[2]);
+    const int32_t* kl = kept_local + m[3] + (int64_t)qb * (qb + 1) / 2;
+    const int64_t n0 = row_ptr[row];
+    const int cnt = counts[row];
+    for (int k = lane; k < cnt; k += 32)
+      if (n0 + k < capacity) {
+        col_idx[n0 + k] = kl[k];
+        kept_row[n0 + k] = (int32_t)row;
+      }
+  }
 }
 
 template <typename T, int B, int NT>
@@ -428,8 +337,6 @@ __global__ void __launch_bounds__(NT) k_gather(const T* __restrict__ maps,
                                                const int32_t* __restrict__ col_idx,
                                                const int32_t* __restrict__ kept_row,
                                                T* __restrict__ values) {
-  // launched while k_stats may still run (programmatic dependent launch): wait for it
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int EPV = Vec<T>::EPV, VPR = B / EPV, VPB = B * VPR;  // vectors per row / per head
   constexpr int U = (VPB + NT - 1) / NT;
   const int64_t nnz = min((int64_t)*nnz_in, capacity);
@@ -476,26 +383,6 @@ __global__ void __launch_bounds__(NT) k_gather(const T* __restrict__ maps,
   }
 }
 
-// A launch that may start while the previous kernel on the stream still runs (programmatic
-// dependent launch); the kernel itself waits for that kernel (griddepcontrol.wait) before it
-// touches memory.  Saves the launch gap between the passes of one compression.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_dependent(void (*kern)(KArgs...), int grid, int threads, cudaStream_t st,
-                             Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid, 1, 1);
-  cfg.blockDim = dim3((unsigned)threads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
-  return e == cudaSuccess ? cudaGetLastError() : e;
-}
-
 template <typename T, int B>
 cudaError_t launch_typed(const mf_compress_desc& d, const CompressWs& ws, uint32_t* status,
                          cudaStream_t st, int sms) {
@@ -503,33 +390,17 @@ cudaError_t launch_typed(const mf_compress_desc& d, const CompressWs& ws, uint32
   const T* maps = static_cast<const T*>(d.maps);
   double* mass = d.block_mass_out ? d.block_mass_out : ws.mass;
   const int grid_stats = (int)std::min<int64_t>(ws.max_cb, (int64_t)sms * 8);
-  const bool fused = (d.max_seqlen + B - 1) / B <= SEL_FUSED_MAX;
-  FusedTail ft;
-  ft.row_done = fused ? ws.row_done : nullptr;
-  ft.rows_selected = reinterpret_cast<unsigned long long*>(ws.meta + 2);
-  ft.tau = d.tau;
-  ft.counts = ws.counts;
-  ft.kept_local = ws.kept_local;
-  ft.row_ptr = d.row_ptr;
-  ft.col_idx = d.col_idx;
-  ft.kept_row = ws.kept_row;
-  ft.nnz_out = d.nnz_out;
-  ft.capacity = d.capacity_blocks;
-  ft.status = status;
-  cudaError_t e = launch_dependent(k_stats<T, B, NT>, grid_stats, NT, st, maps, d.map_seq_offset,
-                                   (const int64_t*)ws.meta, d.nseq, d.h_s, mass, ft);
+  k_stats<T, B, NT><<<grid_stats, NT, 0, st>>>(maps, d.map_seq_offset, ws.meta, d.nseq, d.h_s,
+                                                mass);
+  cudaError_t e = launch_select(ws, d.nseq, d.max_seqlen, B, mass, d.tau, d.row_ptr, d.col_idx,
+                                d.nnz_out, d.capacity_blocks, status, st);
   if (e != cudaSuccess) return e;
-  if (!fused) {
-    e = launch_select(ws, d.nseq, d.max_seqlen, B, mass, d.tau, d.row_ptr, d.col_idx, d.nnz_out,
-                      d.capacity_blocks, status, st);
-    if (e != cudaSuccess) return e;
-  }
   const int grid_g = (int)std::max<int64_t>(
       1, std::min<int64_t>(std::max<int64_t>(d.capacity_blocks, 1) * d.h_s, (int64_t)sms * 8));
-  return launch_dependent(k_gather<T, B, NT>, grid_g, NT, st, maps, d.map_seq_offset,
-                          (const int64_t*)ws.meta, d.nseq, d.h_s, (const int32_t*)d.nnz_out,
-                          d.capacity_blocks, (const int32_t*)d.col_idx,
-                          (const int32_t*)ws.kept_row, static_cast<T*>(d.values));
+  k_gather<T, B, NT><<<grid_g, NT, 0, st>>>(maps, d.map_seq_offset, ws.meta, d.nseq, d.h_s,
+                                            d.nnz_out, d.capacity_blocks, d.col_idx, ws.kept_row,
+                                            static_cast<T*>(d.values));
+  return cudaGetLastError();
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -539,16 +410,8 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 cudaError_t launch_meta(const int32_t* cu, const int64_t* off, int nseq, int max_seqlen, int B,
                         int elem_bytes, const CompressWs& ws, uint32_t* status, int32_t* row_ptr,
                         int32_t* nnz_out, cudaStream_t st) {
-  const int grid = (int)std::min<int64_t>(64, std::max<int64_t>(1, (ws.max_rows + 255) / 256));
-  k_meta<<<grid, 256, 0, st>>>(cu, off, nseq, max_seqlen, B, elem_bytes, ws.meta, status, row_ptr,
-                               nnz_out, ws.row_done, ws.max_rows);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_scan(const CompressWs& ws, int nseq, int32_t* row_ptr, int32_t* col_idx,
-                        int32_t* nnz_out, int64_t capacity, uint32_t* status, cudaStream_t st) {
-  k_scan_compact<<<1, SCAN_NT, 0, st>>>(ws.meta, nseq, ws.counts, ws.kept_local, row_ptr, col_idx,
-                                        ws.kept_row, nnz_out, capacity, status);
+  k_meta<<<1, 32, 0, st>>>(cu, off, nseq, max_seqlen, B, elem_bytes, ws.meta, status, row_ptr,
+                           nnz_out);
   return cudaGetLastError();
 }
 
@@ -566,9 +429,9 @@ cudaError_t launch_select(const CompressWs& ws, int nseq, int max_seqlen, int B,
   }
   k_select<128><<<(unsigned)ws.max_rows, 128, smem_sel, st>>>(ws.meta, nseq, mass, tau, ws.counts,
                                                               ws.kept_local);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  return launch_scan(ws, nseq, row_ptr, col_idx, nnz_out, capacity, status, st);
+  k_scan_compact<<<1, SCAN_NT, 0, st>>>(ws.meta, nseq, ws.counts, ws.kept_local, row_ptr, col_idx,
+                                        ws.kept_row, nnz_out, capacity, status);
+  return cudaGetLastError();
 }
 
 size_t compress_ws_layout(const mf_compress_desc& d, CompressWs* ws, void* base) {
@@ -581,7 +444,6 @@ size_t compress_ws_layout(const mf_compress_desc& d, CompressWs* ws, void* base)
   const size_t o_kept_local = off; off = align_up(off + sizeof(int32_t) * (size_t)max_cb, 256);
   const size_t o_counts = off; off = align_up(off + sizeof(int32_t) * (size_t)max_rows, 256);
   const size_t o_kept = off; off = align_up(off + sizeof(int32_t) * (size_t)std::max<int64_t>(d.capacity_blocks, 1), 256);
-  const size_t o_done = off; off = align_up(off + sizeof(int32_t) * (size_t)max_rows, 256);
   if (ws) {
     char* b = static_cast<char*>(base);
     ws->meta = reinterpret_cast<int64_t*>(b + o_meta);
@@ -589,7 +451,6 @@ size_t compress_ws_layout(const mf_compress_desc& d, CompressWs* ws, void* base)
     ws->kept_local = reinterpret_cast<int32_t*>(b + o_kept_local);
     ws->counts = reinterpret_cast<int32_t*>(b + o_counts);
     ws->kept_row = reinterpret_cast<int32_t*>(b + o_kept);
-    ws->row_done = reinterpret_cast<int32_t*>(b + o_done);
     ws->max_cb = max_cb;
     ws->max_rows = max_rows;
   }

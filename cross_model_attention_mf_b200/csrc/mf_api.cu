@@ -523,8 +523,7 @@ mf_status mf_get_status(void* stream, uint32_t* bits) {
   if (v & mfi::ST_TIMEOUT) return fail(MF_ERR_TIMEOUT, "device: pipeline wait timed out");
   if (v & mfi::ST_ALIGN) return fail(MF_ERR_INVALID, "device: misaligned map offset");
   if (v & mfi::ST_PAGE) return fail(MF_ERR_DEVICE_INDEX, "device: page id out of range");
-  if (v & mfi::ST_SINGULAR) return fail(MF_ERR_INVALID, "device: calibration Gram is not positive definite");
-  return fail(MF_ERR_RANGE, "device: V or the mixed map P outside the float16 range (|x| > 65504)");
+  return fail(MF_ERR_INVALID, "device: calibration Gram is not positive definite");
 }
 
 }  // extern "C"

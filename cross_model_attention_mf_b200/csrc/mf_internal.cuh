@@ -18,7 +18,6 @@ enum : uint32_t {
   ST_ALIGN = 8u,     // a sequence's map offset is not 16-byte aligned
   ST_PAGE = 16u,     // a page id out of range
   ST_SINGULAR = 32u, // a calibration Gram that is not positive definite
-  ST_RANGE = 64u,    // a tensor-core operand outside the float16 range (|V| or |P| > 65504)
 };
 
 // limit of every pipeline wait in the tensor-core kernels (ns) and the test stall flag, as set
@@ -35,8 +34,6 @@ struct CompressWs {
   int32_t* kept_local;  // [max_cb] each row's kept key blocks, ascending, at its causal base
   int32_t* counts;    // [max_rows] kept blocks per row
   int32_t* kept_row;  // [capacity] BSR row of each kept block
-  int32_t* row_done;  // [max_rows] blocks of each row whose mass is written (NULL: selection
-                      // runs as its own launch)
   int64_t max_cb, max_rows;
 };
 
@@ -50,9 +47,6 @@ cudaError_t launch_compress(const mf_compress_desc& d, const CompressWs& ws, uin
 cudaError_t launch_meta(const int32_t* cu, const int64_t* off, int nseq, int max_seqlen, int B,
                         int elem_bytes, const CompressWs& ws, uint32_t* status, int32_t* row_ptr,
                         int32_t* nnz_out, cudaStream_t st);
-// BSR index build (row_ptr by scan, col_idx) from the per-row kept lists
-cudaError_t launch_scan(const CompressWs& ws, int nseq, int32_t* row_ptr, int32_t* col_idx,
-                        int32_t* nnz_out, int64_t capacity, uint32_t* status, cudaStream_t st);
 // selection and BSR index build from the masses of every causal block
 cudaError_t launch_select(const CompressWs& ws, int nseq, int max_seqlen, int B, const double* mass,
                           double tau, int32_t* row_ptr, int32_t* col_idx, int32_t* nnz_out,

@@ -1,5 +1,4 @@
-// Fused map retrieval on sm_100a tensor cores: clusters of four CTAs (tcgen05 + TMA + TMEM +
-// distributed shared memory).
+// Fused map retrieval on sm_100a tensor cores (tcgen05 + TMA + TMEM).
 //
 // MapFlow page "MapFlow开源:大模型换班,Prefill为何能快20%?" (aitest123.com),
 // section "存不下、读得慢?三个工程优化手段", subsection 3 "算得省的:融合内核执行":
@@ -8,43 +7,44 @@
 // receiver's dense map.  The pages' kernel is Triton on A800; this one is a
 // new design for B200.
 //
-// Work unit = (sequence, query block, 32-row window, head chunk of 8 KV groups x 4 virtual
-// receiver heads; a group of gq <= 4 heads is padded to 4).  One cluster of four CTAs takes a
-// unit at a time (persistent: the clusters walk the units, largest query blocks first); every
-// CTA of the cluster walks the same units and tiles.  CTA k of the cluster, for each kept
-// 64-key tile of the unit:
+// Work item = (sequence, query block, 16-row chunk, 4 KV groups = 16 virtual
+// receiver heads; a group of gq <= 4 heads is padded to 4).  The kernel is
+// persistent: each CTA walks items blockIdx.x, blockIdx.x + gridDim.x, ... (the grid
+// is a multiple of the head-chunk count, so a CTA keeps one head chunk and one W^T),
+// and every ring runs across item boundaries, so the loads and the mixing of the
+// next item overlap the tail of the current one.  For each kept 64-key tile:
 //
-//   mixing   D1[pos][(part, v)] = sum_s A_s[pos] W_part[v][s]      tcgen05 M=128 N=64 K=16
-//            for its own 8 rows [8k, 8k+8) of the window and all 32 virtual heads:
-//            pos = (row, key) of 2 rows x 64 keys (4 M tiles), A MN-major SW128 straight from
-//            TMA; W split into bf16 hi and lo parts stacked along N (~16 bits of W);
-//   convert  P = hi + lo (float32), causal mask, P rounded to float16; the part of each KV
-//            group is sent to the CTA that owns the group (CTA g owns groups 2g, 2g+1 of the
-//            chunk) with st.async into its shared memory, completing bytes on its barrier;
-//   P.V      for its two groups and all 32 rows of the window, D2 in TMEM:
-//            D2[dim][(row, head)] += V^T[dim][key] P^T[key][(row, head)]   M=128 N=128 K=16,
-//            float16 operands, float32 accumulation; V of the group is read from global
-//            memory by four loader warps, converted bf16 -> float16 (exact within the float16
-//            range) and stored in the MN-major SW128 operand layout;
-//   epilogue once the unit's last tile is done: D2 rounded to bf16 and stored as O rows.
-// So every kept map tile is read once from HBM, the mixing has every receiver head in one
-// MMA, and P.V runs at N = 128 with V read once per 32 rows.  A P.V commit is multicast to
-// all four CTAs' "P slot free" barriers; the owner of a slot announces the bytes it expects.
+//   mixing  D1[pos][(part, r)] = sum_s A_s[pos] * W_part[r][s]   tcgen05 M=128 N=32 K=16
+//           pos = (row, key) of 2 rows x 64 keys (one M tile), A tile MN-major SW128
+//           from TMA; B = W^T with W split into bf16 hi and lo parts stacked along N,
+//           so one MMA per M tile and s-chunk keeps ~16 bits of W.  D1 holds the eight
+//           32-column M tiles of one key tile in TMEM.
+//   convert 16 warps read D1 (lane = position), form P = hi part + lo part (float32),
+//           apply the causal mask and split P into bf16 hi + lo (P = hi + lo to ~16
+//           bits), written as P^T[key][(row, head)] (MN-major SW128) per group.
+//   P.V     D2[dim][(row, head)] += V^T[dim][key] * (P^T_hi + P^T_lo)[key][(row, head)]
+//           tcgen05 M=128 (d) N=64 K=16 per group, two MMAs per K step; V tile
+//           MN-major SW128 by TMA (contiguous or paged).  D2 stays in TMEM for the
+//           whole row chunk.
+// The hi/lo splits leave the final bf16 rounding of O as the only rounding that
+// matters.
 //
-// Arithmetic: W ~16 bits (hi + lo bf16), P float32 rounded to float16 (relative 2^-11), V
-// float16 (exact for |V| <= 65504), float32 accumulation, O rounded to bf16.  A |V| or |P|
-// above the float16 range sets status bit ST_RANGE.
-//
-// Warp roles (12 warps): 0 TMA producer of the map tiles; 1 mixing MMA issuer + TMEM owner;
-// 2 P.V MMA issuer; 3 idle; 4-7 converters (one per TMEM lane quarter) and the O epilogue;
-// 8-11 V loaders.  TMEM: D2 (two groups x 128 columns) in [0, 256), D1 (4 M tiles x 64
-// columns, two halves with their own barriers) in [256, 512).  Every mbarrier wait is bounded
-// (mf_set_wait_limit, default 2 s): on expiry the CTA records ST_TIMEOUT and every role
-// stops; issued copies and MMAs are drained (bounded), the cluster meets once more so that no
-// CTA leaves while a peer may still write into it, and TMEM is freed.
+// Warp roles: 0 TMA producer of the map tiles; 1 mixing MMA issuer (+ TMEM owner);
+// 2 P.V MMA issuer; 3 TMA producer of the V tiles (separate producers and issuers, so
+// no stream waits behind another); 4-19 convert (four sets of four warps, one warp per
+// TMEM lane quarter; set k converts the M tiles m = k, k + 4 for all 16 heads) and, once
+// per item, run the O epilogue (set k reads D2 group k, releases it for the next item's
+// P.V and stores O).  Barriers are tile- or half-tile-granular: a barrier operation costs
+// hundreds of cycles.  Converters release D1 as soon as it is in registers, so the next
+// tile's mixing overlaps the conversion; P^T and the V ring work in half tiles (groups
+// 0-1, 2-3), so P.V of one half overlaps the conversion of the other.  Consumer warps
+// wait with all 32 lanes (the hardware suspends such a warp; a lone polling lane would
+// spin) and signal once per warp (lane 0 after __syncwarp).  TMEM: D2 in columns
+// [0, 256), D1 in [256, 512).  Every mbarrier wait is bounded by a timer (mf_set_wait_limit,
+// default 2 s): on expiry the CTA records ST_TIMEOUT, all roles stop, in-flight copies and
+// MMAs are drained (bounded) and TMEM is freed.
 #include <cuda.h>
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 #include <stdint.h>
 
@@ -57,63 +57,59 @@
 namespace mfi {
 namespace {
 
-constexpr int CS = 4;             // CTAs per cluster
-constexpr int WR = 32;            // query rows per unit
-constexpr int RM = WR / CS;       // rows mixed by each CTA: 8
-constexpr int KT = 64;            // keys per tile
-constexpr int NGC = 8;            // KV groups per head chunk
-constexpr int GO = NGC / CS;      // groups owned by each CTA: 2
-constexpr int GQP = 4;            // virtual heads per group
-constexpr int HV = NGC * GQP;     // virtual heads per chunk: 32
-constexpr int D = 128;            // head dim
-constexpr int SC = 16;            // sender heads per A chunk (one MMA K step)
-constexpr int NPV = WR * GQP;     // P.V N of one group: 128
-constexpr int NT = 384;           // 12 warps
-constexpr int A_STAGES = 4;       // >= sender-head chunks of a tile (h_s <= 64)
-constexpr int PSLOTS = 2, VSLOTS = 2;
-constexpr uint32_t A_BYTES = RM * SC * KT * 2;     // 16 KB: 8 rows x 16 heads x 64 keys
-constexpr uint32_t PG_BYTES = NPV * KT * 2;        // 16 KB: one group's P^T of a tile
-constexpr uint32_t PSLOT_BYTES = GO * PG_BYTES;    // 32 KB
-constexpr uint32_t VG_BYTES = D * KT * 2;          // 16 KB: one group's V tile
-constexpr uint32_t VSLOT_BYTES = GO * VG_BYTES;    // 32 KB
-constexpr uint32_t W_CHUNK = 2 * HV * SC * 2;      // 2 KB: W^T (hi and lo rows) of 16 sender heads
+constexpr int NT = 640;        // 20 warps
+constexpr int CONV_SETS = 4;   // convert warp sets
+constexpr int R = 16;          // query rows per CTA
+constexpr int KT = 64;         // keys per tile
+constexpr int NG = 4;          // KV groups per CTA
+constexpr int GQP = 4;         // virtual heads per group
+constexpr int HV = NG * GQP;   // virtual receiver heads per CTA
+constexpr int D = 128;         // head dim
+constexpr int SC = 16;         // sender heads per A chunk (one MMA K step)
+constexpr int MT = R * KT / 128;  // M tiles (of 128 positions) per tile: 8
+#ifndef MF_TC_A_STAGES
+#define MF_TC_A_STAGES 2
+#endif
+constexpr int A_STAGES = MF_TC_A_STAGES;
+// Half tiles (KV groups 2h, 2h + 1) flow through a ring of HS slots; a slot holds the half's
+// V tiles (loaded by TMA) and its P^T (written by the converters), filled and freed together.
+constexpr int PH = 2;   // groups per half tile
+constexpr int HS = 2;   // half-tile slots: one key tile
+constexpr uint32_t A_BYTES = R * SC * KT * 2;   // 32 KB
+constexpr uint32_t VGRP_BYTES = KT * D * 2;     // 16 KB: one group's V tile
+constexpr uint32_t V_BYTES = PH * VGRP_BYTES;   // 32 KB: V of one half tile
+constexpr uint32_t PT_BYTES = KT * 64 * 2;      // 8 KB: one group's P^T (hi or lo)
+constexpr uint32_t PSLOT_BYTES = 2 * PT_BYTES;  // hi + lo of one group
 constexpr uint32_t OFF_A = 0;
-constexpr uint32_t OFF_P = OFF_A + A_STAGES * A_BYTES;
-constexpr uint32_t OFF_V = OFF_P + PSLOTS * PSLOT_BYTES;
-constexpr uint32_t OFF_W = OFF_V + VSLOTS * VSLOT_BYTES;
-constexpr int ITEMS_MAX = 32;                      // units per CTA decoded up front
+constexpr uint32_t OFF_V = OFF_A + A_STAGES * A_BYTES;
+constexpr uint32_t OFF_P = OFF_V + HS * V_BYTES;
+constexpr uint32_t PHALF_BYTES = PH * PSLOT_BYTES;  // 32 KB
+constexpr uint32_t OFF_W = OFF_P + HS * PHALF_BYTES;
+constexpr uint32_t W_CHUNK = 1024;              // W^T (32 rows = hi, lo) per s-chunk
+constexpr uint32_t W_BYTES_MAX = 4 * W_CHUNK;   // up to 4 chunks (h_s <= 64)
+constexpr int ITEMS_MAX = 64;                     // work items per CTA decoded up front
 constexpr uint32_t ITEM_BYTES = 64;
-constexpr uint32_t OFF_ITEMS = OFF_W + 4 * W_CHUNK;
+constexpr uint32_t OFF_ITEMS = OFF_W + W_BYTES_MAX;
 constexpr uint32_t OFF_BAR = OFF_ITEMS + ITEMS_MAX * ITEM_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "dynamic shared memory of one CTA");
-static_assert(OFF_P % 1024 == 0 && OFF_V % 1024 == 0 && OFF_W % 1024 == 0, "operand alignment");
-constexpr float F16_MAX = 65504.0f;
-constexpr uint64_t GRACE_NS = 100000;  // after an abort: time for peers' stores still in flight
 
 // barrier slots (8 bytes each)
 enum {
-  B_AFULL = 0, B_AEMPTY = B_AFULL + A_STAGES,
-  B_D1FULL = B_AEMPTY + A_STAGES,  // [2]: halves of D1 (M tiles 0-1, 2-3)
-  B_D1EMPTY = B_D1FULL + 2,        // [2]
-  B_PFULL = B_D1EMPTY + 2,         // [PSLOTS]: st.async bytes of all four CTAs + the owner's expect
-  B_PEMPTY = B_PFULL + PSLOTS,     // [PSLOTS]: P.V commits of the four owners (multicast)
-  B_VFULL = B_PEMPTY + PSLOTS,     // [VSLOTS]: the four V loader warps
-  B_VEMPTY = B_VFULL + VSLOTS,     // [VSLOTS]: this CTA's P.V commit
-  B_OFULL = B_VEMPTY + VSLOTS,     // D2 of a unit complete
-  B_OEMPTY = B_OFULL + 1,          // [GO]: a group's D2 read by the epilogue
-  B_DRAIN1 = B_OEMPTY + GO, B_DRAIN2 = B_DRAIN1 + 1,
-  B_NEVER = B_DRAIN2 + 1,          // test stall: nothing ever arrives here
+  B_AFULL = 0, B_AEMPTY = B_AFULL + A_STAGES, B_HFULL = B_AEMPTY + A_STAGES,
+  B_HEMPTY = B_HFULL + HS, B_D1FULL = B_HEMPTY + HS, B_D1EMPTY = B_D1FULL + 1,
+  B_OFULL = B_D1EMPTY + 1,
+  B_OEMPTY = B_OFULL + 1, B_DRAIN1 = B_OEMPTY + 2, B_DRAIN2 = B_DRAIN1 + 1,
+  B_NEVER = B_DRAIN2 + 1,  // test stall: nothing ever arrives here
   B_COUNT = B_NEVER + 1
 };
 static_assert(B_COUNT * 8 <= 512, "barrier area");
 
-// instruction descriptors (kind::f16): D f32 (bit 4), A / B type at bits 7 / 10 (0 f16,
-// 1 bf16), A / B major at bits 15 / 16 (1 = MN-major), N >> 3 at bit 17, M >> 4 at bit 24
+// instruction descriptors (kind::f16): D f32, A/B bf16, majors, N >> 3, M >> 4
 constexpr uint32_t IDESC_MIX = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (0u << 16) |
-                               ((64u >> 3) << 17) | ((128u >> 4) << 24);
-constexpr uint32_t IDESC_PV = (1u << 4) | (0u << 7) | (0u << 10) | (1u << 15) | (1u << 16) |
-                              ((128u >> 3) << 17) | ((128u >> 4) << 24);
+                               ((32u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t IDESC_PV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                              ((64u >> 3) << 17) | ((128u >> 4) << 24);
 
 constexpr int NRMAX = 4;  // receivers served by one launch (one BSR, several W / V / O)
 
@@ -122,10 +118,9 @@ struct RecvParams {
   const float* W;  // [h_r][h_s]
   void* O;         // bf16, or float32 when o_f32
   int o_f32;
-  const __nv_bfloat16* V;
   const int32_t* block_table;
   int paged, page_size, n_pages, max_pages;
-  int64_t total_k;  // rows of a contiguous V
+  int total_k;     // V rows (contiguous V): the out-of-range row that reads zeros
   int h_r, h_kv, gq, hcs;
 };
 struct TcParams {
@@ -135,16 +130,19 @@ struct TcParams {
   const int32_t* cu_q;
   const int32_t* cu_k;
   const int32_t* qblock_base;
-  int nseq, nqbq, wcs;     // sequences, query blocks per sequence (bound), windows per block
-  int NH;                  // head chunks of all receivers together
+  int nqbq, rcs;    // query blocks, row chunks per block
+  int NH;           // head chunks of all receivers together
   int hh_base[NRMAX + 1];  // first head chunk of each receiver
   int nrecv;
-  int n_units;
+  int n_items;
   int h_s, nsc, B;
   RecvParams rv[NRMAX];
   uint32_t* status;
   uint64_t wait_ns;  // limit of every pipeline wait
   int stall;         // test: the mixing issuer first waits on B_NEVER
+};
+struct VMaps {
+  CUtensorMap m[NRMAX];
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -166,37 +164,24 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-// try_wait; with CL, cluster-scope acquire (for the barriers peer CTAs signal: data a peer
-// wrote before completing the phase is visible once it returns true)
-template <bool CL = false>
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-  if (CL)
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-  else
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
   return ok != 0;
 }
 // Bounded wait: false if the CTA aborted or the wait ran out of time (limit_ns).
-template <bool CL = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           uint32_t* status, uint64_t limit_ns) {
-  if (mbar_try<CL>(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
+  if (mbar_try(bar, parity)) return true;
+  uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try<CL>(bar, parity)) return true;
+    if (mbar_try(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > limit_ns) {
@@ -207,10 +192,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
   }
 }
-template <bool CL = false>
-__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try<CL>(bar, parity) && globaltimer() - t0 < DRAIN_NS) {}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
 }
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
                                             int c0, int c1, int c2, int c3) {
@@ -219,23 +207,6 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm,
       " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
-}
-__device__ __forceinline__ uint32_t cluster_map(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-// 16 bytes into a peer CTA's shared memory, completing 16 bytes on its barrier
-__device__ __forceinline__ void st_async16(uint32_t raddr, uint32_t rbar, uint32_t a, uint32_t b,
-                                           uint32_t c, uint32_t d) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::
-          "r"(raddr), "r"(a), "r"(b), "r"(c), "r"(d), "r"(rbar)
-      : "memory");
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -246,14 +217,6 @@ __device__ __forceinline__ void tc_fence_after() {
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
-}
-// commit whose barrier arrival goes to the barrier at the same offset in every CTA of `mask`
-__device__ __forceinline__ void tc_commit_mc(uint32_t bar, uint16_t mask) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(bar),
-      "h"(mask)
-      : "memory");
 }
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate) {
@@ -287,7 +250,8 @@ __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 // Register fence: the compiler sees v redefined here, so no use of v moves above this point
-// (above the tcgen05.wait::ld that makes v valid).
+// (above the tcgen05.wait::ld that makes v valid, or above a barrier signal that should go
+// out before the arithmetic on v).
 __device__ __forceinline__ void reg_fence(uint32_t (&v)[32]) {
   asm volatile(""
                : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
@@ -297,87 +261,76 @@ __device__ __forceinline__ void reg_fence(uint32_t (&v)[32]) {
                  "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]), "+r"(v[29]),
                  "+r"(v[30]), "+r"(v[31]));
 }
-__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
-  __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
-// two bf16 (one 32-bit word) -> two float16 (one word); |x| is folded into amax
-__device__ __forceinline__ uint32_t bf2_to_h2(uint32_t w, float& amax) {
-  const float a = __uint_as_float(w << 16), b = __uint_as_float(w & 0xFFFF0000u);
-  amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
-  return pack_h2(a, b);
-}
 
-// ------------------------------------------------------------------ work units
-struct Unit {
-  int s, qb, i_begin, row_lo, row_hi, k_len, n_tiles, k0, kb0;
-  int64_t rp0;
-  int64_t o_row0;  // O row of window row 0 (cu_seqlens_q[s] + i_begin - q0)
-  bool valid, bsr_ok;
-};
-static_assert(sizeof(Unit) <= ITEM_BYTES, "unit table slot");
-
-// unit idx = ((qbr * nseq + s) * wcs + w) * NH + hh: qbr counts query blocks back from the
-// last one of the sequence's chunk, so the largest units (most kept blocks) come first;
-// hh = a receiver's head chunk.  Identical in every role and every CTA of the cluster.
-__device__ __forceinline__ Unit decode(const TcParams& p, int idx) {
-  Unit u;
-  u.valid = false;
-  u.bsr_ok = true;
-  u.n_tiles = 0;
-  idx /= p.NH;
-  const int w = idx % p.wcs;
-  idx /= p.wcs;
-  const int s = idx % p.nseq;
-  const int qbr = idx / p.nseq;
-  const int q_len = p.cu_q[s + 1] - p.cu_q[s];
-  const int k_len = p.cu_k[s + 1] - p.cu_k[s];
-  const int q0 = k_len - q_len;
-  if (q_len <= 0 || q0 < 0) return u;
-  const int qb_first = q0 / p.B, qb_last = (k_len - 1) / p.B;
-  const int qb = qb_last - qbr;
-  if (qb < qb_first) return u;
-  const int i_begin = qb * p.B + w * WR;
-  const int row_lo = max(q0, i_begin), row_hi = min(k_len, i_begin + WR);
-  if (row_lo >= row_hi) return u;
-  const int64_t brow = (int64_t)p.qblock_base[s] + qb;
-  const int64_t rp0 = p.row_ptr[brow], rp1 = p.row_ptr[brow + 1];
-  u.bsr_ok = rp0 >= 0 && rp1 >= rp0 && rp1 <= p.capacity && rp1 - rp0 <= qb + 1;
-  u.n_tiles = u.bsr_ok ? (int)(rp1 - rp0) * (p.B / KT) : 0;
-  u.s = s; u.qb = qb; u.i_begin = i_begin; u.row_lo = row_lo; u.row_hi = row_hi;
-  u.k_len = k_len; u.rp0 = rp0; u.k0 = p.cu_k[s];
-  u.kb0 = u.n_tiles > 0 ? p.col_idx[rp0] : -1;
-  u.o_row0 = (int64_t)p.cu_q[s] + (i_begin - q0);
-  u.valid = true;
-  return u;
-}
-
-// Optional timeline trace (compile with -DMF_TRACE): for the first TRACE_CTAS CTAs, per role,
-// SM-clock stamps of pipeline events kept in shared memory and copied out at the end, read back
-// with mf_trace_dump().  Each role has a single writing thread.  Roles: 0 map producer, 1 mixing
-// issuer, 2 P.V issuer, 3 first converter warp, 4 first V loader warp.
+// Optional timeline trace (compile with -DMF_TRACE): per CTA and role, SM-clock stamps of
+// pipeline events kept in shared memory and copied out at the end, read back with
+// mf_trace_dump().  Each role has a single writing thread.
 #ifdef MF_TRACE
-constexpr int TRACE_CTAS = 16, TRACE_N = 512, TRACE_ROLES = 5;
+constexpr int TRACE_CTAS = 160, TRACE_N = 256, TRACE_ROLES = 6;
 __device__ uint64_t g_trace[TRACE_CTAS][TRACE_ROLES][TRACE_N];
-#define TRACE(role, code)                                                                  \
-  do {                                                                                     \
-    const int n_ = s_tn[role];                                                             \
-    if (n_ < TRACE_N - 1) {                                                                \
+#define TRACE(role, code)                                                            \
+  do {                                                                               \
+    const int n_ = s_tn[role];                                                       \
+    if (n_ < TRACE_N - 1) {                                                          \
       s_tr[role][1 + n_] = ((uint64_t)(code) << 56) | ((uint64_t)clock64() & ((1ull << 56) - 1)); \
-      s_tn[role] = n_ + 1;                                                                 \
-    }                                                                                      \
+      s_tn[role] = n_ + 1;                                                           \
+    }                                                                                \
   } while (0)
 #else
 #define TRACE(role, code)
 #endif
 
 // ------------------------------------------------------------------ kernel
+struct Item {
+  int s, qb, q0, i_begin, row_lo, row_hi, k_len, n_tiles;
+  int k0;   // first key row of the sequence (cu_seqlens_k[s])
+  int kb0;  // key block of the row's first kept block (col_idx[rp0]), -1 without tiles
+  int64_t rp0;
+  int64_t o_row0;  // O row of query position i_begin (cu_seqlens_q[s] + i_begin - q0)
+  bool valid, bsr_ok;
+};
+static_assert(sizeof(Item) <= ITEM_BYTES, "item table slot");
+
+// item idx = ((s * nqbq + qbl) * rcs + rc) * NH + hh, hh = a receiver's head chunk;
+// identical in every role
+__device__ __forceinline__ Item decode(const TcParams& p, int idx) {
+  Item it;
+  it.valid = false;
+  it.bsr_ok = true;
+  it.n_tiles = 0;
+  idx /= p.NH;
+  const int rc = idx % p.rcs;
+  idx /= p.rcs;
+  const int qbl = idx % p.nqbq;
+  const int s = idx / p.nqbq;
+  const int q_len = p.cu_q[s + 1] - p.cu_q[s];
+  const int k_len = p.cu_k[s + 1] - p.cu_k[s];
+  const int q0 = k_len - q_len;
+  if (q_len <= 0 || q0 < 0) return it;
+  const int qb = q0 / p.B + qbl;
+  if ((int64_t)qb * p.B >= k_len) return it;
+  const int i_begin = qb * p.B + rc * R;
+  const int row_lo = max(q0, i_begin), row_hi = min(k_len, i_begin + R);
+  if (row_lo >= row_hi) return it;
+  const int64_t brow = (int64_t)p.qblock_base[s] + qb;
+  const int64_t rp0 = p.row_ptr[brow], rp1 = p.row_ptr[brow + 1];
+  it.bsr_ok = rp0 >= 0 && rp1 >= rp0 && rp1 <= p.capacity && rp1 - rp0 <= qb + 1;
+  it.n_tiles = it.bsr_ok ? (int)(rp1 - rp0) * (p.B / KT) : 0;
+  it.s = s; it.qb = qb; it.q0 = q0; it.i_begin = i_begin; it.row_lo = row_lo;
+  it.row_hi = row_hi; it.k_len = k_len; it.rp0 = rp0; it.k0 = p.cu_k[s];
+  it.kb0 = it.n_tiles > 0 ? p.col_idx[rp0] : -1;
+  it.o_row0 = (int64_t)p.cu_q[s] + (i_begin - q0);
+  it.valid = true;
+  return it;
+}
+
 __global__ void __launch_bounds__(NT, 1)
-    k_retrieve_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ TcParams p) {
+    k_retrieve_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ VMaps tmVs,
+                  const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
@@ -389,33 +342,35 @@ __global__ void __launch_bounds__(NT, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rank = (int)(blockIdx.x % CS);     // rank in the cluster (cluster dims (4, 1, 1))
-  const int cl = (int)(blockIdx.x / CS), ncl = (int)(gridDim.x / CS);
-  // receiver and head chunk: constant per cluster (the cluster count is a multiple of NH)
-  const int hh = cl % p.NH;
+  // receiver and head chunk: constant per CTA (gridDim.x is a multiple of NH)
+  const int hh = blockIdx.x % p.NH;
   int ri = 0;
   while (ri + 1 < p.nrecv && hh >= p.hh_base[ri + 1]) ++ri;
   const RecvParams& q_r = p.rv[ri];
+  const CUtensorMap* tmV = &tmVs.m[ri];
   const int hc = hh - p.hh_base[ri];
   const int tpb = p.B / KT;
 
   const uint32_t sb = smem_u32(smem);
   const uint32_t bar0 = sb + OFF_BAR;
   auto bar = [&](int k) { return bar0 + 8u * (uint32_t)k; };
-  // unit k of this cluster (idx = cl + k * ncl): the first ITEMS_MAX from the table decoded
-  // once below, later ones decoded where they are needed
-  Unit* s_units = reinterpret_cast<Unit*>(smem + OFF_ITEMS);
-  auto unit = [&](int k, int idx) -> Unit { return k < ITEMS_MAX ? s_units[k] : decode(p, idx); };
+  // item k of this CTA (idx = blockIdx.x + k * gridDim.x): the first ITEMS_MAX come from the
+  // table decoded once below, later ones are decoded where they are needed
+  Item* s_items = reinterpret_cast<Item*>(smem + OFF_ITEMS);
+  auto item = [&](int k, int idx) -> Item { return k < ITEMS_MAX ? s_items[k] : decode(p, idx); };
 
   // ---- setup
   if (threadIdx.x == 0) {
     s_abort = 0;
     for (int k = 0; k < A_STAGES; ++k) { mbar_init(bar(B_AFULL + k), 1); mbar_init(bar(B_AEMPTY + k), 1); }
-    for (int h = 0; h < 2; ++h) { mbar_init(bar(B_D1FULL + h), 1); mbar_init(bar(B_D1EMPTY + h), 4); }
-    for (int k = 0; k < PSLOTS; ++k) { mbar_init(bar(B_PFULL + k), 1); mbar_init(bar(B_PEMPTY + k), CS); }
-    for (int k = 0; k < VSLOTS; ++k) { mbar_init(bar(B_VFULL + k), 4); mbar_init(bar(B_VEMPTY + k), 1); }
+    for (int k = 0; k < HS; ++k) {
+      mbar_init(bar(B_HFULL + k), 1 + 4 * CONV_SETS);  // V producer + converter warps
+      mbar_init(bar(B_HEMPTY + k), 1);
+    }
+    mbar_init(bar(B_D1FULL), 1);
+    mbar_init(bar(B_D1EMPTY), 4 * CONV_SETS);
+    for (int h = 0; h < NG / PH; ++h) mbar_init(bar(B_OEMPTY + h), 4 * PH);  // epilogue warps
     mbar_init(bar(B_OFULL), 1);
-    for (int g = 0; g < GO; ++g) mbar_init(bar(B_OEMPTY + g), 4);
     mbar_init(bar(B_DRAIN1), 1);
     mbar_init(bar(B_DRAIN2), 1);
     mbar_init(bar(B_NEVER), 1);
@@ -428,478 +383,433 @@ __global__ void __launch_bounds__(NT, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  // W^T of this chunk's 32 virtual heads, bf16, K-major without swizzle, 64 rows per s:
-  // row n < 32 is the hi part of virtual head n, row 32 + n its lo part.  Element (n, s) at
-  // (s/8)*1024 + (n/8)*128 + (n%8)*16 + (s%8)*2.
+  // W^T of this CTA's 16 virtual heads, bf16, K-major without swizzle, 32 rows per s:
+  // row n < 16 is the hi part of head n, row 16 + n its lo part.  Element (n, s) at
+  // (s/8)*512 + (n/8)*128 + (n%8)*16 + (s%8)*2.
   {
     const int ks = p.nsc * SC;
     uint16_t* wt = reinterpret_cast<uint16_t*>(smem + OFF_W);
     for (int e = threadIdx.x; e < HV * ks; e += NT) {
-      const int v = e / ks, hs = e % ks;
-      const int G = hc * NGC + v / GQP, q = v % GQP;
+      const int rv = e / ks, hs = e % ks;
+      const int G = hc * NG + rv / GQP, q = rv % GQP;
       float w = 0.0f;
       if (q < q_r.gq && G < q_r.h_kv && hs < p.h_s) w = q_r.W[(int64_t)(G * q_r.gq + q) * p.h_s + hs];
       __nv_bfloat16 hi = __float2bfloat16_rn(w);
       __nv_bfloat16 lo = __float2bfloat16_rn(w - __bfloat162float(hi));
-      const int base = (hs >> 3) * 1024 + (hs & 7) * 2;
-      wt[(base + (v >> 3) * 128 + (v & 7) * 16) >> 1] = *reinterpret_cast<uint16_t*>(&hi);
-      wt[(base + ((v + HV) >> 3) * 128 + (v & 7) * 16) >> 1] = *reinterpret_cast<uint16_t*>(&lo);
+      const int base = (hs >> 3) * 512 + (hs & 7) * 2;
+      wt[(base + (rv >> 3) * 128 + (rv & 7) * 16) >> 1] = *reinterpret_cast<uint16_t*>(&hi);
+      wt[(base + ((rv + 16) >> 3) * 128 + (rv & 7) * 16) >> 1] = *reinterpret_cast<uint16_t*>(&lo);
     }
   }
+  // the item table: one decode per item instead of one per item and role
   for (int k = threadIdx.x; k < ITEMS_MAX; k += NT) {
-    const int idx = cl + k * ncl;
-    if (idx < p.n_units) s_units[k] = decode(p, idx);
+    const int idx = blockIdx.x + k * gridDim.x;
+    if (idx < p.n_items) s_items[k] = decode(p, idx);
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   tc_fence_before();
   __syncthreads();
-  // every CTA of the cluster has initialised its barriers before any peer signals them
-  cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
   volatile int* abort_flag = &s_abort;
 
-  if (warp == 0) {
-    // ================================================================ TMA producer (map tiles)
-    // the whole warp waits (suspended by the hardware); lane 0 issues the copies
-    int as = 0;
-    uint32_t aph = 0;
-    int a_issued = 0;
-    bool ok = true;
-    for (int idx = cl, ik = 0; idx < p.n_units && ok; idx += ncl, ++ik) {
-      const Unit u = unit(ik, idx);
-      if (!u.valid) continue;
-      if (!u.bsr_ok && rank == 0 && lane == 0) atomicOr(p.status, ST_INDEX);
-      const int w = (idx / p.NH) % p.wcs;
-      for (int t = 0; t < u.n_tiles && ok; ++t) {
-        const int64_t e = u.rp0 + t / tpb;
-        const int half = t % tpb;
-        for (int c = 0; c < p.nsc && ok; ++c) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_AEMPTY + as), aph ^ 1, abort_flag, p.status, p.wait_ns));
-          if (!ok) break;
-          if (lane == 0) {
-            TRACE(0, 1);
-            mbar_expect_tx(bar(B_AFULL + as), A_BYTES);
-            tma_load_4d(sb + OFF_A + as * A_BYTES, &tmA, bar(B_AFULL + as), half * KT, c * SC,
-                        w * WR + rank * RM, (int)e);
+  if (warp == 0 || warp == 3) {
+    // ================================================================ TMA producers
+    // warp 0: map tiles (A chunks) in mixing order; warp 3: V tiles in P.V order (one stage
+    // per half tile = groups 2h, 2h + 1)
+    if (lane == 0) {
+      const bool is_a = warp == 0;
+      int as = 0, vs = 0;
+      uint32_t aph = 0, vph = 0;
+      int a_issued = 0, v_issued = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x, ik = 0; idx < p.n_items && ok; idx += gridDim.x, ++ik) {
+        const Item it = item(ik, idx);
+        if (!it.valid) continue;
+        if (is_a) TRACE(0, 1);
+        if (is_a && !it.bsr_ok) atomicOr(p.status, ST_INDEX);
+        const int rc = (idx / p.NH) % p.rcs;
+        // key block of the current kept block and, loaded one block ahead, of the next one
+        const int nblk = it.n_tiles / tpb;
+        int kb_cur = it.kb0, kb_nxt = (!is_a && nblk > 1) ? p.col_idx[it.rp0 + 1] : -1;
+        for (int t = 0; t < it.n_tiles && ok; ++t) {
+          const int64_t e = it.rp0 + t / tpb;
+          const int half = t % tpb;
+          if (!is_a && t > 0 && half == 0) {
+            kb_cur = kb_nxt;
+            if (t / tpb + 1 < nblk) kb_nxt = p.col_idx[e + 1];
           }
-          __syncwarp();
-          ++a_issued;
-          if (++as == A_STAGES) { as = 0; aph ^= 1; }
+          if (is_a) {
+            for (int c = 0; c < p.nsc && ok; ++c) {
+              if (!(ok = mbar_wait(bar(B_AEMPTY + as), aph ^ 1, abort_flag, p.status, p.wait_ns))) break;
+              TRACE(0, 3);
+              mbar_expect_tx(bar(B_AFULL + as), A_BYTES);
+              tma_load_4d(sb + OFF_A + as * A_BYTES, &tmA, bar(B_AFULL + as), half * KT, c * SC,
+                          rc * R, (int)e);
+              TRACE(0, 2);
+              ++a_issued;
+              if (++as == A_STAGES) { as = 0; aph ^= 1; }
+            }
+            continue;
+          }
+          const int kb = kb_cur;
+          const bool kb_ok = kb >= 0 && kb <= it.qb;
+          if (!kb_ok) atomicOr(p.status, ST_INDEX);
+          const int tok0 = kb * p.B + half * KT;
+          for (int h = 0; h < NG / PH && ok; ++h) {
+            if (!(ok = mbar_wait(bar(B_HEMPTY + vs), vph ^ 1, abort_flag, p.status, p.wait_ns))) break;
+            TRACE(5, 4);
+            mbar_expect_tx(bar(B_HFULL + vs), V_BYTES);
+            for (int gl = 0; gl < PH; ++gl) {
+              const uint32_t dst = sb + OFF_V + vs * V_BYTES + gl * VGRP_BYTES;
+              const int G = hc * NG + h * PH + gl;
+              if (!q_r.paged) {
+                const int row = kb_ok ? it.k0 + tok0 : q_r.total_k;  // out of range reads 0
+                tma_load_3d(dst, tmV, bar(B_HFULL + vs), 0, G, row);
+                tma_load_3d(dst + 8192, tmV, bar(B_HFULL + vs), 64, G, row);
+              } else {
+                const int ps = q_r.page_size;
+                for (int q = 0; q < KT / ps; ++q) {
+                  const int tok = tok0 + q * ps;
+                  const int slot = tok / ps;
+                  int page = q_r.n_pages;  // out of range: the copy reads zeros
+                  if (kb_ok && tok < it.k_len && slot < q_r.max_pages) {
+                    const int pg = q_r.block_table[(int64_t)it.s * q_r.max_pages + slot];
+                    if (pg >= 0 && pg < q_r.n_pages) page = pg;
+                    else atomicOr(p.status, ST_PAGE);
+                  }
+                  tma_load_4d(dst + q * ps * 128, tmV, bar(B_HFULL + vs), 0, G, 0, page);
+                  tma_load_4d(dst + 8192 + q * ps * 128, tmV, bar(B_HFULL + vs), 64, G, 0, page);
+                }
+              }
+            }
+            ++v_issued;
+            TRACE(5, 3);
+            if (++vs == HS) { vs = 0; vph ^= 1; }
+          }
         }
       }
-    }
-    // drain: wait (bounded) for the last copy issued into every stage
-    if (lane == 0)
+      // drain: wait (bounded) for the last copy issued into every stage
       for (int k = 0; k < A_STAGES; ++k) {
         const int cnt = a_issued > k ? (a_issued - k - 1) / A_STAGES + 1 : 0;
-        if (cnt) mbar_drain(bar(B_AFULL + k), (cnt - 1) & 1);
+        if (cnt) {
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try(bar(B_AFULL + k), (cnt - 1) & 1) && globaltimer() - t0 < DRAIN_NS) {}
+        }
       }
-    __syncwarp();
+      // (a V slot's phase also needs the converters' arrivals: after an abort this wait runs
+      // out its bounded time)
+      for (int k = 0; k < HS; ++k) {
+        const int cnt = v_issued > k ? (v_issued - k - 1) / HS + 1 : 0;
+        if (cnt) {
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try(bar(B_HFULL + k), (cnt - 1) & 1) && globaltimer() - t0 < DRAIN_NS) {}
+        }
+      }
+    }
   } else if (warp == 1) {
     // ================================================================ mixing MMA issuer
-    bool ok = true;
-    // test stall: a wait that can only run out (the whole cluster then stops as on any timeout)
-    if (p.stall) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_NEVER), 0, abort_flag, p.status, p.wait_ns));
-    int as = 0;
-    uint32_t aph = 0;
-    int T = 0;  // tiles processed so far
-    const uint64_t wdesc0 = smem_desc(sb + OFF_W, 1024u, 128u, 0u);
-    const uint64_t adesc0 = smem_desc(sb + OFF_A, 2048u, 1024u, 2u);
-    for (int idx = cl, ik = 0; idx < p.n_units && ok; idx += ncl, ++ik) {
-      const Unit u = unit(ik, idx);
-      if (!u.valid) continue;
-      for (int t = 0; t < u.n_tiles && ok; ++t, ++T) {
-        // half 0 (M tiles 0, 1) over all sender-head chunks, then half 1 (M tiles 2, 3); the
-        // tile's chunks stay in the A ring until half 1 has read them (A_STAGES >= chunks)
-        for (int hf = 0; hf < 2 && ok; ++hf) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_D1EMPTY + hf), (T & 1) ^ 1, abort_flag, p.status, p.wait_ns));
-          if (!ok) break;
-          if (lane == 0) TRACE(1, 2 + hf);
-          int st = as;
-          uint32_t ph = aph;
+    if (lane == 0) {
+      int as = 0;
+      uint32_t aph = 0;
+      bool ok = true;
+      int T = 0;  // tiles processed so far
+      const uint64_t wdesc0 = smem_desc(sb + OFF_W, 512u, 128u, 0u);
+      const uint64_t adesc0 = smem_desc(sb + OFF_A, 2048u, 1024u, 2u);
+      // test stall: a wait that can only run out (the whole CTA then stops as on any timeout)
+      if (p.stall) ok = mbar_wait(bar(B_NEVER), 0, abort_flag, p.status, p.wait_ns);
+      for (int idx = blockIdx.x, ik = 0; idx < p.n_items && ok; idx += gridDim.x, ++ik) {
+        const Item it = item(ik, idx);
+        if (!it.valid) continue;
+        TRACE(1, 1);
+        for (int t = 0; t < it.n_tiles && ok; ++t, ++T) {
+          // D1 must have been read out by the previous tile's converters
+          if (!(ok = mbar_wait(bar(B_D1EMPTY), (T & 1) ^ 1, abort_flag, p.status, p.wait_ns))) break;
+          tc_fence_after();
+          // chunk-major: each s-chunk is mixed into all eight M tiles, then its stage is freed
           for (int c = 0; c < p.nsc && ok; ++c) {
-            if (hf == 0) {
-              ok = __all_sync(0xffffffffu, mbar_wait(bar(B_AFULL + st), ph, abort_flag, p.status, p.wait_ns));
-              if (!ok) break;
-              if (lane == 0) TRACE(1, 4);
-            }
-            if (lane == 0) {
-              tc_fence_after();
-              const uint64_t ad = adesc0 + (((uint32_t)st * A_BYTES) >> 4);
-              const uint64_t wd = wdesc0 + ((c * W_CHUNK) >> 4);
+            if (!(ok = mbar_wait(bar(B_AFULL + as), aph, abort_flag, p.status, p.wait_ns))) break;
+            tc_fence_after();
+            if (c == 0) TRACE(1, 3);
+            const uint64_t ad = adesc0 + (((uint32_t)as * A_BYTES) >> 4);
+            const uint64_t wd = wdesc0 + ((c * W_CHUNK) >> 4);
 #pragma unroll
-              for (int mm = 0; mm < 2; ++mm) {
-                const int m = 2 * hf + mm;
-                tc_mma(tmem + 256u + 64u * (uint32_t)m, ad + ((m * 4096u) >> 4), wd, IDESC_MIX,
-                       c > 0 ? 1u : 0u);
-              }
-              if (hf == 1) tc_commit(bar(B_AEMPTY + st));
-            }
-            __syncwarp();
-            if (++st == A_STAGES) { st = 0; ph ^= 1; }
+            for (int m = 0; m < MT; ++m)
+              tc_mma(tmem + 256u + 32u * (uint32_t)m, ad + ((m * 4096u) >> 4), wd, IDESC_MIX,
+                     c > 0 ? 1u : 0u);
+            TRACE(1, 5);
+            tc_commit(bar(B_AEMPTY + as));
+            if (++as == A_STAGES) { as = 0; aph ^= 1; }
           }
           if (!ok) break;
-          if (lane == 0) tc_commit(bar(B_D1FULL + hf));
-          __syncwarp();
-          if (hf == 1) { as = st; aph = ph; }
+          tc_commit(bar(B_D1FULL));
+          TRACE(1, 4);
         }
       }
-    }
-    if (lane == 0) {
       tc_commit(bar(B_DRAIN1));
-      mbar_drain(bar(B_DRAIN1), 0);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try(bar(B_DRAIN1), 0) && globaltimer() - t0 < DRAIN_NS) {}
     }
-    __syncwarp();
   } else if (warp == 2) {
     // ================================================================ P.V MMA issuer
-    bool ok = true;
-    int T = 0, K = 0;  // tiles and units processed so far
-    const uint64_t vdesc0 = smem_desc(sb + OFF_V, 8192u, 1024u, 2u);
-    const uint64_t pdesc0 = smem_desc(sb + OFF_P, 8192u, 1024u, 2u);
-    int ng = 0;  // this CTA's real groups
-    for (int gl = 0; gl < GO; ++gl) ng += (hc * NGC + rank * GO + gl < q_r.h_kv) ? 1 : 0;
-    for (int idx = cl, ik = 0; idx < p.n_units && ok; idx += ncl, ++ik) {
-      const Unit u = unit(ik, idx);
-      if (!u.valid) continue;
-      for (int t = 0; t < u.n_tiles && ok; ++t, ++T) {
-        const int ps = T % PSLOTS, vs = T % VSLOTS;
-        // the owner announces the bytes its peers will complete on the slot's barrier
-        if (lane == 0) mbar_expect_tx(bar(B_PFULL + ps), PSLOT_BYTES);
-        __syncwarp();
-        if (lane == 0) TRACE(2, 5);
-        ok = __all_sync(0xffffffffu, mbar_wait<true>(bar(B_PFULL + ps), (T / PSLOTS) & 1, abort_flag, p.status, p.wait_ns));
-        if (lane == 0) TRACE(2, 6);
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_VFULL + vs), (T / VSLOTS) & 1, abort_flag, p.status, p.wait_ns));
-        if (lane == 0) TRACE(2, 7);
-        // the previous unit's epilogue must have read D2 out
-        for (int gl = 0; gl < GO && ok && t == 0 && K > 0; ++gl)
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OEMPTY + gl), (K - 1) & 1, abort_flag, p.status, p.wait_ns));
-        if (!ok) break;
-        if (lane == 0) {
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          tc_fence_after();
-          for (int gl = 0; gl < ng; ++gl) {
-            const uint64_t vd = vdesc0 + ((vs * VSLOT_BYTES + gl * VG_BYTES) >> 4);
-            const uint64_t pd = pdesc0 + ((ps * PSLOT_BYTES + gl * PG_BYTES) >> 4);
-#pragma unroll
-            for (int kk = 0; kk < KT / 16; ++kk)
-              tc_mma(tmem + 128u * (uint32_t)gl, vd + ((kk * 2048u) >> 4), pd + ((kk * 2048u) >> 4),
-                     IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(bar(B_VEMPTY + vs));
-          tc_commit_mc(bar(B_PEMPTY + ps), (uint16_t)((1u << CS) - 1u));  // the slot is free in all four CTAs
-          TRACE(2, 8);
-        }
-        __syncwarp();
-      }
-      if (!ok) break;
-      if (u.n_tiles == 0 && K > 0) {  // take the epilogue's phases in order all the same
-        for (int gl = 0; gl < GO && ok; ++gl)
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OEMPTY + gl), (K - 1) & 1, abort_flag, p.status, p.wait_ns));
-        if (!ok) break;
-      }
-      if (lane == 0) tc_commit(bar(B_OFULL));  // D2 of this unit complete (at once with no tile)
-      __syncwarp();
-      ++K;
-    }
     if (lane == 0) {
-      tc_commit(bar(B_DRAIN2));
-      mbar_drain(bar(B_DRAIN2), 0);
-    }
-    __syncwarp();
-  } else if (warp >= 4 && warp < 8) {
-    // ================================================================ convert P, epilogue
-    // Warp q owns TMEM lane quarter q: in every M tile its lane is position l = 32q + lane =
-    // (row 2m + rb, key j) with j = l % 64, rb = l / 64.  Rows 2m + rb of the pair of M tiles
-    // (0, 1) or (2, 3) at key j, 4 heads of a group each, make one 16-byte chunk of that
-    // group's P^T: n = 8c + 4p + h with c = 4 rank + 2 pair + rb, p = row within the pair.
-    const int q = warp & 3;
-    const int l = q * 32 + lane;
-    const int j = l & 63, rb = l >> 6;
-    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
-    // peers' shared-memory windows
-    uint32_t rbase[CS];
-#pragma unroll
-    for (int r = 0; r < CS; ++r) rbase[r] = cluster_map(sb, (uint32_t)r);
-    const int64_t rs = (int64_t)q_r.h_r * D;  // O row stride
-    const int d = q * 32 + lane;               // epilogue: this lane's head dim
-    // epilogue of a unit: D2 group gl -> O rows (bf16), lanes paired so that each store
-    // writes two adjacent head dims
-    auto epilogue = [&](int ek, int eidx, int Ke) -> bool {
-      const Unit u = unit(ek, eidx);
-      const bool have = u.n_tiles > 0;
-      const int ilo = u.row_lo - u.i_begin, ihi = u.row_hi - u.i_begin;
-      if (warp == 4 && lane == 0) TRACE(3, 15);
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_OFULL), Ke & 1, abort_flag, p.status, p.wait_ns)))
-        return false;
-      if (warp == 4 && lane == 0) TRACE(3, 16);
-      tc_fence_after();
-      for (int gl = 0; gl < GO; ++gl) {
-        const int G = hc * NGC + rank * GO + gl;
-        if (q_r.o_f32) {
-          // float32 O: each lane stores its own head dim (a warp writes 128 contiguous bytes);
-          // D2 is released only after the last column is stored
-          float* of = static_cast<float*>(q_r.O) + u.o_row0 * rs + (int64_t)G * q_r.gq * D + d;
-#pragma unroll
-          for (int c32 = 0; c32 < NPV / 32; ++c32) {
-            uint32_t o[32];
-            if (have) {
-              tmem_ld32(tl + 128u * gl + 32u * c32, o);
-              tmem_wait_ld();
-              reg_fence(o);
-            } else {
-#pragma unroll
-              for (int c = 0; c < 32; ++c) o[c] = 0u;
+      int vs = 0;
+      uint32_t vph = 0;
+      bool ok = true;
+      int T = 0, K = 0;  // tiles and items processed so far
+      const uint64_t vdesc0 = smem_desc(sb + OFF_V, 8192u, 1024u, 2u);
+      const uint64_t pdesc0 = smem_desc(sb + OFF_P, 8192u, 1024u, 2u);
+      for (int idx = blockIdx.x, ik = 0; idx < p.n_items && ok; idx += gridDim.x, ++ik) {
+        const Item it = item(ik, idx);
+        if (!it.valid) continue;
+        TRACE(4, 6);
+        for (int t = 0; t < it.n_tiles && ok; ++t, ++T) {
+          for (int h = 0; h < NG / PH && ok; ++h) {
+            // the half's V tiles and P^T are in slot vs
+            if (!(ok = mbar_wait(bar(B_HFULL + vs), vph, abort_flag, p.status, p.wait_ns))) break;
+            TRACE(4, 8);
+            // the previous item's epilogue must have read this half of D2 out
+            if (t == 0 && K > 0) {
+              if (!(ok = mbar_wait(bar(B_OEMPTY + h), (K - 1) & 1, abort_flag, p.status, p.wait_ns))) break;
+              TRACE(4, 9);
             }
+            tc_fence_after();
+            TRACE(4, 5);
+            // the MMAs of the half's two groups are interleaved, so consecutive MMAs accumulate
+            // into different D2 columns
+            const uint64_t pd = pdesc0 + ((vs * PHALF_BYTES) >> 4);
+            const uint64_t vd = vdesc0 + ((vs * V_BYTES) >> 4);
 #pragma unroll
-            for (int cc = 0; cc < 32; ++cc) {
-              const int n = 32 * c32 + cc;
-              const int c = n >> 3, pp = (n >> 2) & 1, h = n & 3;
-              const int r = 8 * (c >> 2) + 4 * ((c >> 1) & 1) + 2 * pp + (c & 1);
-              if (G < q_r.h_kv && h < q_r.gq && r >= ilo && r < ihi)
-                of[(int64_t)r * rs + h * D] = __uint_as_float(o[cc]);
-            }
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+              for (int part = 0; part < 2; ++part)
+#pragma unroll
+                for (int gl = 0; gl < PH; ++gl)
+                  tc_mma(tmem + 64u * (uint32_t)(h * PH + gl),
+                         vd + ((gl * VGRP_BYTES + k * 2048u) >> 4),
+                         pd + ((gl * PSLOT_BYTES + part * PT_BYTES + k * 2048u) >> 4), IDESC_PV,
+                         (t > 0 || k > 0 || part > 0) ? 1u : 0u);
+            TRACE(4, 10);
+            tc_commit(bar(B_HEMPTY + vs));  // V and P^T of the slot consumed
+            if (++vs == HS) { vs = 0; vph ^= 1; }
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_OEMPTY + gl));
-          continue;
         }
-        uint32_t pk[NPV / 2];  // columns (2u, 2u + 1) rounded to bf16
+        if (!ok) break;
+        if (it.n_tiles == 0 && K > 0) {  // take the epilogue's phases in order all the same
+          for (int h = 0; h < NG / PH && ok; ++h)
+            ok = mbar_wait(bar(B_OEMPTY + h), (K - 1) & 1, abort_flag, p.status, p.wait_ns);
+          if (!ok) break;
+        }
+        tc_commit(bar(B_OFULL));  // D2 of this item complete (immediate when it has no tile)
+        TRACE(4, 7);
+        ++K;
+      }
+      tc_commit(bar(B_DRAIN2));
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try(bar(B_DRAIN2), 0) && globaltimer() - t0 < DRAIN_NS) {}
+    }
+  } else if (warp < 4 + 4 * CONV_SETS) {
+    // ================================================================ convert P (hi + lo)
+    // Warp (set, quarter) owns TMEM lanes of its quarter in M tiles set and set + 4, i.e.
+    // key j of rows 2 set + rb and 2 set + 8 + rb, which is exactly one 16-byte chunk of the
+    // P^T row of key j (D2 column n = 8 (2 set + rb) + 4 mi + head): one conflict-free
+    // 16-byte store per group for the hi part and one for the lo part.
+    const int quarter = warp & 3;
+    const int set = (warp - 4) >> 2;
+    const int lrow = quarter * 32 + lane;  // TMEM lane = position in an M tile
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int j = lrow & 63, rb = lrow >> 6;
+    const uint32_t choff =
+        (uint32_t)j * 128u + ((((uint32_t)(2 * set + rb)) ^ ((uint32_t)j & 7u)) << 4);
+    // O epilogue of an item, shared by the 16 warps: warp (set, quarter) reads D2 group g = set
+    // (64 columns) for head dims [32 quarter, 32 quarter + 32), releases it and stores O
+    const int ng = min(NG, q_r.h_kv - hc * NG);  // real groups of this head chunk
+    const int64_t rs = (int64_t)q_r.h_r * D;     // O row stride
+    // the item (table slot ek, index eidx) is re-read from the item table here
+    auto epilogue = [&](int ek, int eidx, int K) -> bool {
+      const Item q = item(ek, eidx);
+      const bool have = q.n_tiles > 0;
+      const int ilo = q.row_lo - q.i_begin, ihi = q.row_hi - q.i_begin;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_OFULL), K & 1, abort_flag, p.status, p.wait_ns)))
+        return false;
+      tc_fence_after();
+      if (warp == 4 && lane == 0) TRACE(3, 1);
+      const int g = set;
+      if (q_r.o_f32) {
+        // float32 O: each lane stores its own head dim (a warp writes 128 contiguous bytes);
+        // D2 is released once every column is stored
+        float* of = static_cast<float*>(q_r.O) +
+                    (q.o_row0 * q_r.h_r + (int64_t)(hc * NG + g) * q_r.gq) * D + quarter * 32 + lane;
 #pragma unroll
-        for (int c32 = 0; c32 < NPV / 32; ++c32) {
+        for (int hh = 0; hh < 2; ++hh) {
           uint32_t o[32];
           if (have) {
-            tmem_ld32(tl + 128u * gl + 32u * c32, o);
+            tmem_ld32(tl + 64u * g + 32u * hh, o);
             tmem_wait_ld();
             reg_fence(o);
           } else {
 #pragma unroll
             for (int c = 0; c < 32; ++c) o[c] = 0u;
           }
+          // column n = 8 c + 4 mi + head holds row 2 (c / 2) + 8 mi + c % 2
 #pragma unroll
-          for (int u2 = 0; u2 < 16; ++u2)
-            pk[16 * c32 + u2] = pack_bf2(__uint_as_float(o[2 * u2]), __uint_as_float(o[2 * u2 + 1]));
+          for (int cc = 0; cc < 32; ++cc) {
+            const int n = 32 * hh + cc, c8 = n >> 3;
+            const int ii = 2 * (c8 >> 1) + 8 * ((n >> 2) & 1) + (c8 & 1), rv = n & 3;
+            if (g < ng && rv < q_r.gq && ii >= ilo && ii < ihi) of[ii * rs + rv * D] = __uint_as_float(o[cc]);
+          }
         }
-        // D2 of this group is read: the next unit's P.V may overwrite it
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_OEMPTY + gl));
-        if (G < q_r.h_kv) {
-          const bool odd = lane & 1;
-          __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(q_r.O) + u.o_row0 * rs +
-                              (int64_t)G * q_r.gq * D + (d & ~1);
+        if (lane == 0) mbar_arrive(bar(B_OEMPTY + g / PH));
+        return true;
+      }
+      uint32_t pr[32];  // the group's 64 columns rounded to bf16, as pairs (2u, 2u + 1)
 #pragma unroll
-          for (int u2 = 0; u2 < NPV / 2; ++u2) {
-            // columns n = 2 u2 (head h even) and n + 1 (head h + 1) of the same row
-            const uint32_t mine = pk[u2];
-            const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
-            // even lane: column n at dims (d, d + 1); odd lane: column n + 1 at (d - 1, d)
-            const uint32_t wv = odd ? __byte_perm(other, mine, 0x7632) : __byte_perm(mine, other, 0x5410);
-            const int n = 2 * u2 + (odd ? 1 : 0);
-            const int c = n >> 3, pp = (n >> 2) & 1, h = n & 3;
-            const int r = 8 * (c >> 2) + 4 * ((c >> 1) & 1) + 2 * pp + (c & 1);
-            if (h < q_r.gq && r >= ilo && r < ihi)
-              *reinterpret_cast<uint32_t*>(ob + (int64_t)r * rs + h * D) = wv;
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t o[32];
+        if (have) {
+          tmem_ld32(tl + 64u * g + 32u * hh, o);
+          tmem_wait_ld();
+          reg_fence(o);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          pr[16 * hh + u] = pack_bf16(__uint_as_float(o[2 * u]), __uint_as_float(o[2 * u + 1]));
+      }
+      // D2 of this group is read: the next item's P.V may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_OEMPTY + g / PH));
+      if (warp == 4 && lane == 0) TRACE(3, 2);
+      if (g < ng) {
+        __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(q_r.O) +
+                            (q.o_row0 * q_r.h_r + (int64_t)(hc * NG + g) * q_r.gq) * D + quarter * 32 + lane;
+        // column n = 8 c + 4 mi + head holds row 2 (c / 2) + 8 mi + c % 2
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            const int n = 2 * u + b, c8 = n >> 3;
+            const int ii = 2 * (c8 >> 1) + 8 * ((n >> 2) & 1) + (c8 & 1), rv = n & 3;
+            if (rv < q_r.gq && ii >= ilo && ii < ihi)
+              *reinterpret_cast<uint16_t*>(ob + ii * rs + rv * D) =
+                  (uint16_t)(b ? pr[u] >> 16 : pr[u] & 0xFFFFu);
           }
         }
       }
-      if (warp == 4 && lane == 0) TRACE(3, 17);
       return true;
     };
     bool ok = true;
-    int T = 0, K = 0;   // tiles converted, epilogues done
-    int pk_unit = -1, pidx = 0;  // a unit whose epilogue is still to run (after the next unit's first tile)
-    float amax = 0.0f;
-    for (int idx = cl, ik = 0; idx < p.n_units && ok; idx += ncl, ++ik) {
-      const Unit u = unit(ik, idx);
-      if (!u.valid) continue;
-      int kb = u.kb0;
-      for (int t = 0; t < u.n_tiles && ok; ++t, ++T) {
-        if (t == 1 && pk_unit >= 0) {
-          ok = epilogue(pk_unit, pidx, K++);
-          pk_unit = -1;
+    int T = 0, K = 0;     // tiles converted, epilogues done
+    // an item whose O epilogue is still to run (pk < 0: none): it runs after the next item's
+    // first tile is converted, so P.V never waits for the stores
+    int pk = -1, pidx = 0;
+    int kb_prev = -1;  // key block of the previous tile (tiles of one kept block share it)
+    for (int idx = blockIdx.x, ik = 0; idx < p.n_items && ok; idx += gridDim.x, ++ik) {
+      const Item it = item(ik, idx);
+      if (!it.valid) continue;
+      for (int t = 0; t < it.n_tiles && ok; ++t, ++T) {
+        // the previous item's epilogue, after this item's first tile
+        if (t == 1 && pk >= 0) {
+          ok = epilogue(pk, pidx, K++);
+          pk = -1;
           if (!ok) break;
         }
+        const int64_t e = it.rp0 + t / tpb;
         const int half = t % tpb;
-        if (t > 0 && half == 0) kb = p.col_idx[u.rp0 + t / tpb];
-        const bool kb_ok = kb >= 0 && kb <= u.qb;
+        const int kb = half == 0 && t == 0 ? it.kb0 : (half == 0 ? p.col_idx[e] : kb_prev);
+        kb_prev = kb;
+        const bool kb_ok = kb >= 0 && kb <= it.qb;
         const int tok0 = kb * p.B + half * KT;
-        const int ps = T % PSLOTS;
-        // rows of this thread: window row 8 rank + 2m + rb, query position i_begin + that
-        const int ibase = u.i_begin + rank * RM + rb;
-        const bool full = kb_ok && tok0 + KT - 1 <= u.i_begin + rank * RM;
-        uint32_t pkA[HV / 2], pkB[HV / 2];
-        for (int pair = 0; pair < 2 && ok; ++pair) {
-          if (warp == 4 && lane == 0) TRACE(3, 9 + pair);
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_D1FULL + pair), T & 1, abort_flag, p.status, p.wait_ns));
+        // warp-uniform control flow: tcgen05.ld is a warp-collective instruction
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_D1FULL), T & 1, abort_flag, p.status, p.wait_ns));
+        if (!ok) break;
+        tc_fence_after();
+        if (warp == 4 && lane == 0) TRACE(2, 1);
+        // both M tiles into registers first, so that D1 is released as early as possible
+        // (columns 0-15: A.W_hi of the 16 heads, 16-31: A.W_lo)
+        uint32_t v[MT / CONV_SETS][32];
+#pragma unroll
+        for (int mi = 0; mi < MT / CONV_SETS; ++mi)
+          tmem_ld32(tl + 256u + 32u * (uint32_t)(set + mi * CONV_SETS), v[mi]);
+        tmem_wait_ld();
+        if (warp == 4 && lane == 0) TRACE(2, 5);
+        // D1 is in registers: the next tile's mixing may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_D1EMPTY));
+#pragma unroll
+        for (int mi = 0; mi < MT / CONV_SETS; ++mi) reg_fence(v[mi]);
+        // P = hi + lo with hi = P truncated to bf16 and lo = bf16(P - hi); a tile wholly below
+        // the diagonal of every row needs no causal mask
+        const bool full = kb_ok && tok0 + KT - 1 <= it.i_begin;
+        uint32_t hw[NG][4], lw[NG][4];  // per group: the chunk's packed hi and lo words
+#pragma unroll
+        for (int mi = 0; mi < MT / CONV_SETS; ++mi) {
+          const int ii = 2 * (set + mi * CONV_SETS) + rb;
+          const float mk = kb_ok && tok0 + j <= it.i_begin + ii ? 1.0f : 0.0f;
+#pragma unroll
+          for (int g = 0; g < NG; ++g) {
+#pragma unroll
+            for (int c = 0; c < 4; c += 2) {
+              float x0 = __uint_as_float(v[mi][4 * g + c]) + __uint_as_float(v[mi][16 + 4 * g + c]);
+              float x1 =
+                  __uint_as_float(v[mi][4 * g + c + 1]) + __uint_as_float(v[mi][16 + 4 * g + c + 1]);
+              if (!full) {
+                x0 *= mk;
+                x1 *= mk;
+              }
+              const uint32_t b0 = __float_as_uint(x0) & 0xFFFF0000u;
+              const uint32_t b1 = __float_as_uint(x1) & 0xFFFF0000u;
+              hw[g][2 * mi + c / 2] = __byte_perm(b0, b1, 0x7632);
+              // P - hi is exact in f32; one rounding to bf16 for the pair
+              lw[g][2 * mi + c / 2] = pack_bf16(x0 - __uint_as_float(b0), x1 - __uint_as_float(b1));
+            }
+          }
+        }
+        if (warp == 4 && lane == 0) TRACE(2, 3);
+#pragma unroll
+        for (int h = 0; h < NG / PH; ++h) {
+          // this half of the P buffer must have been consumed by the previous tile's P.V
+          const int hq = T * (NG / PH) + h, ps = hq % HS;  // half-tile count, slot
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_HEMPTY + ps), ((hq / HS) & 1) ^ 1,
+                                                 abort_flag, p.status, p.wait_ns));
           if (!ok) break;
-          if (warp == 4 && lane == 0) TRACE(3, 11 + pair);
-          tc_fence_after();
+          if (warp == 4 && lane == 0) TRACE(2, 4);
 #pragma unroll
-          for (int mm = 0; mm < 2; ++mm) {
-            const int m = 2 * pair + mm;
-            uint32_t hi[32], lo[32];
-            tmem_ld32(tl + 256u + 64u * (uint32_t)m, hi);
-            tmem_ld32(tl + 256u + 64u * (uint32_t)m + 32u, lo);
-            tmem_wait_ld();
-            reg_fence(hi);
-            reg_fence(lo);
-            if (mm == 1) {  // both M tiles of the half are in registers: release D1
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(bar(B_D1EMPTY + pair));
-            }
-            const float mk = (kb_ok && tok0 + j <= ibase + 2 * m) ? 1.0f : 0.0f;
-            uint32_t* pk = mm == 0 ? pkA : pkB;
-#pragma unroll
-            for (int v = 0; v < HV; v += 2) {
-              float x0 = __uint_as_float(hi[v]) + __uint_as_float(lo[v]);
-              float x1 = __uint_as_float(hi[v + 1]) + __uint_as_float(lo[v + 1]);
-              if (!full) { x0 *= mk; x1 *= mk; }
-              amax = fmaxf(amax, fmaxf(fabsf(x0), fabsf(x1)));
-              pk[v / 2] = pack_h2(x0, x1);
-            }
+          for (int gl = 0; gl < PH; ++gl) {
+            const int g = h * PH + gl;
+            const uint32_t pt = sb + OFF_P + ps * PHALF_BYTES + gl * PSLOT_BYTES + choff;
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pt), "r"(hw[g][0]),
+                         "r"(hw[g][1]), "r"(hw[g][2]), "r"(hw[g][3])
+                         : "memory");
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pt + PT_BYTES),
+                         "r"(lw[g][0]), "r"(lw[g][1]), "r"(lw[g][2]), "r"(lw[g][3])
+                         : "memory");
           }
-          // the slot must have been consumed by all four owners (tile T - PSLOTS)
-          if (pair == 0 && T >= PSLOTS) {
-            ok = __all_sync(0xffffffffu, mbar_wait<true>(bar(B_PEMPTY + ps), ((T / PSLOTS) & 1) ^ 1,
-                                                         abort_flag, p.status, p.wait_ns));
-            if (!ok) break;
-          }
-          if (warp == 4 && lane == 0) TRACE(3, 13 + pair);
-          // one 16-byte chunk per group: rows (2*(2 pair) + rb, 2*(2 pair + 1) + rb), 4 heads each
-          const uint32_t c = 4u * (uint32_t)rank + 2u * (uint32_t)pair + (uint32_t)rb;
-          const uint32_t off = OFF_P + (uint32_t)ps * PSLOT_BYTES + (c >> 3) * 8192u +
-                               (uint32_t)j * 128u + (((c & 7u) ^ ((uint32_t)j & 7u)) << 4);
-#pragma unroll
-          for (int g = 0; g < NGC; ++g) {
-            const int owner = g / GO, gl = g % GO;
-            st_async16(rbase[owner] + off + (uint32_t)gl * PG_BYTES,
-                       rbase[owner] + OFF_BAR + 8u * (uint32_t)(B_PFULL + ps),
-                       pkA[2 * g], pkA[2 * g + 1], pkB[2 * g], pkB[2 * g + 1]);
-          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_HFULL + ps));
         }
         if (!ok) break;
+        if (warp == 4 && lane == 0) TRACE(2, 2);
       }
       if (!ok) break;
-      if (pk_unit >= 0) {
-        ok = epilogue(pk_unit, pidx, K++);
-        pk_unit = -1;
+      if (pk >= 0) {
+        ok = epilogue(pk, pidx, K++);
         if (!ok) break;
       }
-      pk_unit = ik;
+      pk = ik;
       pidx = idx;
     }
-    if (ok && pk_unit >= 0) ok = epilogue(pk_unit, pidx, K++);
-    if (amax > F16_MAX) atomicOr(p.status, ST_RANGE);
-    // every owner has consumed the slots this CTA filled last (their commits have arrived here)
-    if (lane == 0)
-      for (int k = 0; k < PSLOTS; ++k) {
-        const int cnt = T > k ? (T - k - 1) / PSLOTS + 1 : 0;
-        if (cnt) mbar_drain<true>(bar(B_PEMPTY + k), (cnt - 1) & 1);
-      }
-    __syncwarp();
-  } else if (warp >= 8) {
-    // ================================================================ V loaders
-    // 128 threads; per tile 2 groups x 64 keys x 16 vectors of 8 dims: 16 vectors per thread.
-    // A cursor runs one tile ahead: the loads of the next tile are in flight while this one is
-    // converted and stored.
-    const int tid = threadIdx.x - 8 * 32;
-    bool ok = true;
-    int T = 0;
-    float amax = 0.0f;
-    // cursor over this cluster's tiles in order (units without tiles are skipped)
-    int c_ik = -1, c_idx = cl - ncl, c_t = 0, c_kb = -1;
-    Unit c_u;
-    c_u.n_tiles = 0;
-    auto advance = [&]() -> bool {  // to the next tile; false when none is left
-      ++c_t;
-      while (c_t >= c_u.n_tiles) {
-        ++c_ik;
-        c_idx += ncl;
-        if (c_idx >= p.n_units) return false;
-        c_u = unit(c_ik, c_idx);
-        if (!c_u.valid) c_u.n_tiles = 0;
-        c_t = 0;
-      }
-      if (c_t % tpb == 0) c_kb = c_t == 0 ? c_u.kb0 : p.col_idx[c_u.rp0 + c_t / tpb];
-      return true;
-    };
-    auto issue = [&](uint4 (&r)[16]) {
-      const int half = c_t % tpb;
-      const bool kb_ok = c_kb >= 0 && c_kb <= c_u.qb;
-      if (!kb_ok && rank == 0 && tid == 0) atomicOr(p.status, ST_INDEX);
-      const int tok0 = c_kb * p.B + half * KT;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int v = tid + 128 * i;
-        const int gl = v >> 10, key = (v >> 4) & 63, ch = v & 15;
-        const int G = hc * NGC + rank * GO + gl;
-        const int tok = tok0 + key;
-        r[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (kb_ok && tok < c_u.k_len && G < q_r.h_kv) {
-          int64_t row = -1;
-          if (!q_r.paged) {
-            row = (int64_t)c_u.k0 + tok;
-            if (row >= q_r.total_k) row = -1;
-          } else {
-            const int slot = tok / q_r.page_size;
-            if (slot < q_r.max_pages) {
-              const int pg = q_r.block_table[(int64_t)c_u.s * q_r.max_pages + slot];
-              if (pg >= 0 && pg < q_r.n_pages) row = (int64_t)pg * q_r.page_size + tok % q_r.page_size;
-              else atomicOr(p.status, ST_PAGE);
-            }
-          }
-          if (row >= 0)
-            r[i] = __ldg(reinterpret_cast<const uint4*>(q_r.V + (row * q_r.h_kv + G) * D + ch * 8));
-        }
-      }
-    };
-    uint4 ra[16], rb[16];
-    bool have = advance();
-    if (have) issue(ra);
-    while (have && ok) {
-      const bool more = advance();
-      if (more) issue(rb);
-      const int vs = T % VSLOTS;
-      if (warp == 8 && lane == 0) TRACE(4, 18);
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_VEMPTY + vs), ((T / VSLOTS) & 1) ^ 1, abort_flag,
-                                             p.status, p.wait_ns));
-      if (!ok) break;
-      if (warp == 8 && lane == 0) TRACE(4, 19);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int v = tid + 128 * i;
-        const int gl = v >> 10, key = (v >> 4) & 63, ch = v & 15;
-        const uint32_t dst = sb + OFF_V + (uint32_t)vs * VSLOT_BYTES + (uint32_t)gl * VG_BYTES +
-                             ((uint32_t)ch >> 3) * 8192u + (uint32_t)key * 128u +
-                             ((((uint32_t)ch & 7u) ^ ((uint32_t)key & 7u)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
-                     "r"(bf2_to_h2(ra[i].x, amax)), "r"(bf2_to_h2(ra[i].y, amax)),
-                     "r"(bf2_to_h2(ra[i].z, amax)), "r"(bf2_to_h2(ra[i].w, amax))
-                     : "memory");
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_VFULL + vs));
-      if (warp == 8 && lane == 0) TRACE(4, 20);
-      ++T;
-      have = more;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) ra[i] = rb[i];
-    }
-    if (amax > F16_MAX) atomicOr(p.status, ST_RANGE);
+    if (ok && pk >= 0) ok = epilogue(pk, pidx, K++);
   }
   tc_fence_before();
   __syncthreads();
-  // no CTA leaves while a peer may still signal or write into it
-  cluster_sync_all();
-  if (*abort_flag) {  // stores a stopped peer issued may still be in flight towards this CTA
-    const uint64_t t0 = globaltimer();
-    while (globaltimer() - t0 < GRACE_NS) {}
-  }
 #ifdef MF_TRACE
   if (blockIdx.x < TRACE_CTAS)
     for (int e = threadIdx.x; e < TRACE_ROLES * TRACE_N; e += NT) {
@@ -942,41 +852,6 @@ bool encode(CUtensorMap* tm, const void* base, int rank, const uint64_t* dims,
   return true;
 }
 
-// clusters of four CTAs that can be resident at once on the current device (queried once per
-// device: the answer depends on the GPC layout, not on the launch)
-int max_clusters(std::string* err) {
-  static std::mutex mu;
-  static int cache[64];
-  int dev = 0;
-  cudaGetDevice(&dev);
-  std::lock_guard<std::mutex> g(mu);
-  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
-  cudaError_t e = cudaFuncSetAttribute(k_retrieve_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SMEM_BYTES);
-  if (e != cudaSuccess) { *err = cudaGetErrorString(e); return 0; }
-  int sms = 148;
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(sms / CS * CS), 1, 1);
-  cfg.blockDim = dim3(NT, 1, 1);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CS;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  e = cudaOccupancyMaxActiveClusters(&n, k_retrieve_tc, &cfg);
-  if (e != cudaSuccess || n < 1) {
-    *err = std::string("cudaOccupancyMaxActiveClusters: ") + cudaGetErrorString(e);
-    return 0;
-  }
-  if (dev >= 0 && dev < 64) cache[dev] = n;
-  return n;
-}
-
 }  // namespace
 
 bool tc_supported(const mf_retrieve_desc& d) {
@@ -985,7 +860,9 @@ bool tc_supported(const mf_retrieve_desc& d) {
   if (!(d.B == 64 || d.B == 128) || d.d != D) return false;
   if (d.h_kv <= 0 || d.h_r % d.h_kv != 0 || d.h_r / d.h_kv > GQP) return false;
   if (d.h_s <= 0 || d.h_s > 64) return false;
-  if (d.paged && d.page_size < 1) return false;
+  if (d.paged && !(d.page_size == 8 || d.page_size == 16 || d.page_size == 32 || d.page_size == 64))
+    return false;
+  if (!d.paged && d.total_k >= (int64_t)1 << 31) return false;
   return true;
 }
 
@@ -1000,15 +877,16 @@ bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* 
     const uint64_t dims[4] = {(uint64_t)B, (uint64_t)d0.h_s, (uint64_t)B,
                               (uint64_t)std::max<int64_t>(l0.capacity, 1)};
     const uint64_t strides[3] = {(uint64_t)B * B * 2, (uint64_t)B * 2, (uint64_t)d0.h_s * B * B * 2};
-    const uint32_t box[4] = {KT, SC, RM, 1};
+    const uint32_t box[4] = {KT, SC, R, 1};
     if (!encode(&tmA, l0.values, 4, dims, strides, box, err)) return false;
   }
+  VMaps vm;
+  memset(&vm, 0, sizeof vm);
   TcParams p{};
   p.row_ptr = l0.row_ptr; p.col_idx = l0.col_idx; p.capacity = l0.capacity;
   p.cu_q = d0.cu_seqlens_q; p.cu_k = d0.cu_seqlens_k; p.qblock_base = d0.qblock_base;
-  p.nseq = d0.nseq;
-  p.nqbq = (d0.max_seqlen_q + B - 1) / B + 1;  // a chunk may start inside a block
-  p.wcs = B / WR;
+  p.nqbq = (d0.max_seqlen_q + B - 1) / B;
+  p.rcs = B / R;
   p.h_s = d0.h_s; p.nsc = (d0.h_s + SC - 1) / SC; p.B = B;
   p.nrecv = n;
   p.status = status;
@@ -1018,42 +896,46 @@ bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* 
   for (int k = 0; k < n; ++k) {
     const mf_retrieve_desc& d = *ds[k];
     const RetrieveLayer& l = ls[k];
+    if (!d.paged) {  // V [T][h_kv][d]: dims (dim, kv head, token)
+      const uint64_t dims[3] = {(uint64_t)D, (uint64_t)d.h_kv, (uint64_t)std::max<int64_t>(d.total_k, 1)};
+      const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)d.h_kv * D * 2};
+      const uint32_t box[3] = {64, 1, KT};
+      if (!encode(&vm.m[k], l.V, 3, dims, strides, box, err)) return false;
+    } else {  // V [pages][page][h_kv][d]: dims (dim, kv head, row in page, page)
+      const uint64_t dims[4] = {(uint64_t)D, (uint64_t)d.h_kv, (uint64_t)d.page_size,
+                                (uint64_t)std::max(d.n_pages, 1)};
+      const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)d.h_kv * D * 2,
+                                   (uint64_t)d.page_size * d.h_kv * D * 2};
+      const uint32_t box[4] = {64, 1, (uint32_t)d.page_size, 1};
+      if (!encode(&vm.m[k], l.V, 4, dims, strides, box, err)) return false;
+    }
     RecvParams& r = p.rv[k];
     r.W = l.W; r.O = l.O;
     r.o_f32 = (d.flags & MF_RETRIEVE_O_F32) ? 1 : 0;
-    r.V = static_cast<const __nv_bfloat16*>(l.V);
     r.block_table = d.block_table; r.paged = d.paged; r.page_size = d.page_size;
-    r.n_pages = d.n_pages; r.max_pages = d.max_pages; r.total_k = d.total_k;
+    r.n_pages = d.n_pages; r.max_pages = d.max_pages; r.total_k = (int)d.total_k;
     r.h_r = d.h_r; r.h_kv = d.h_kv; r.gq = d.h_r / d.h_kv;
-    r.hcs = (d.h_kv + NGC - 1) / NGC;
+    r.hcs = (d.h_kv + NG - 1) / NG;
     p.hh_base[k] = NH;
     NH += r.hcs;
   }
   p.hh_base[n] = NH;
   p.NH = NH;
-  const int64_t n_units = (int64_t)p.nqbq * d0.nseq * p.wcs * NH;
-  if (n_units == 0 || d0.max_seqlen_q == 0) return true;
-  if (n_units >= ((int64_t)1 << 31)) { *err = "too many work units"; return false; }
-  p.n_units = (int)n_units;
-  const int mc = max_clusters(err);
-  if (mc < 1) return false;
-  // persistent clusters, a multiple of the head-chunk count (one receiver and one W^T each)
-  int64_t ncl = std::min<int64_t>(n_units, mc);
-  ncl = std::max<int64_t>(NH, ncl / NH * NH);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(ncl * CS), 1, 1);
-  cfg.blockDim = dim3(NT, 1, 1);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CS;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, k_retrieve_tc, tmA, p);
-  if (e == cudaSuccess) e = cudaGetLastError();
+  const int64_t n_items = (int64_t)d0.nseq * p.nqbq * p.rcs * NH;
+  if (n_items == 0) return true;
+  if (n_items >= ((int64_t)1 << 31)) { *err = "too many work items"; return false; }
+  p.n_items = (int)n_items;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // persistent grid, a multiple of the head-chunk count (one receiver and one W^T per CTA)
+  int64_t grid = std::min<int64_t>(n_items, sms);
+  grid = std::max<int64_t>(NH, grid / NH * NH);
+  cudaError_t e = cudaFuncSetAttribute(k_retrieve_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SMEM_BYTES);
+  if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
+  k_retrieve_tc<<<(unsigned)grid, NT, SMEM_BYTES, st>>>(tmA, vm, p);
+  e = cudaGetLastError();
   if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
   return true;
 }

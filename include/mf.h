@@ -59,8 +59,7 @@ typedef enum {
   MF_ERR_CAPACITY = 3,     /* device: more kept blocks than capacity_blocks */
   MF_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
   MF_ERR_TIMEOUT = 5,      /* device: a pipeline wait ran out of time */
-  MF_ERR_DEVICE_INDEX = 6, /* device: a BSR row/column or page id was out of range */
-  MF_ERR_RANGE = 7         /* device: a tensor-core operand outside the float16 range */
+  MF_ERR_DEVICE_INDEX = 6  /* device: a BSR row/column or page id was out of range */
 } mf_status;
 
 typedef enum { MF_F32 = 0, MF_BF16 = 1 } mf_dtype;
@@ -212,15 +211,15 @@ mf_status mf_compress_qk(const mf_compress_qk_desc* desc, void* workspace, size_
  * (0 = T_q * h_r * d).
  * Arithmetic: MF_F32 maps/V run in float32 throughout.  MF_BF16 maps and V run on
  * tcgen05 tensor cores: W is split into a bf16 pair (hi + lo, ~16 bits), the mixed
- * map P is accumulated in float32 and rounded to float16, V is converted to float16
- * (exact for |V| <= 65504), P.V is accumulated in float32 and O rounded to bf16
- * (round to nearest even).  A |V| or |P| above 65504 on this path is reported as
- * MF_ERR_RANGE by mf_get_status (the output is then undefined).  Each output row's
- * accumulation order depends only on its query block's kept blocks, so chunked,
- * paged and varlen layouts give bit-identical rows.
+ * map P is accumulated in float32 and split into a bf16 pair (hi truncated, lo the
+ * rounded remainder), P.V takes both parts with float32 accumulation, and O is rounded
+ * to bf16 (round to nearest even).  Each output row's accumulation order depends only
+ * on its query block's kept blocks, so chunked, paged and varlen layouts give
+ * bit-identical rows.
  * Requirements: h_r % h_kv == 0; layer_map[l] < n_sender_layers; d <= 256.
  * The tensor-core path needs MF_BF16 maps and V (V 16-byte aligned), B in {64, 128},
- * d = 128, h_r / h_kv <= 4 and h_s <= 64; other shapes run a float32 SIMT kernel.
+ * d = 128, h_r / h_kv <= 4, h_s <= 64 and (if paged) page_size in {8, 16, 32, 64};
+ * other shapes run a float32 SIMT kernel.
  * ------------------------------------------------------------------------------ */
 typedef struct {
   const int32_t* row_ptr;          /* device */
@@ -398,8 +397,8 @@ mf_status mf_set_wait_limit(uint64_t limit_ns, int stall);
 /* Synchronise `stream`, then read and clear this device's status word.  *bits
  * (optional) receives the raw bits: 1 index out of range, 2 capacity, 4 wait
  * timeout, 8 misaligned input, 16 page id out of range, 32 singular
- * calibration Gram, 64 a tensor-core operand outside the float16 range.  Returns
- * MF_OK when no bit was set, else the status of the lowest set bit. */
+ * calibration Gram.  Returns MF_OK when no bit was set, else the status of the lowest
+ * set bit. */
 mf_status mf_get_status(void* stream, uint32_t* bits);
 
 /* Message for the calling thread's last failed call ("" if none). */
