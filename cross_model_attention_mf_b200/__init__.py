@@ -37,6 +37,7 @@ MF_OK, MF_ERR_INVALID, MF_ERR_UNSUPPORTED, MF_ERR_CAPACITY, MF_ERR_CUDA, MF_ERR_
 MF_F32, MF_BF16 = 0, 1
 MF_RETRIEVE_FORCE_SIMT = 1
 MF_RETRIEVE_O_F32 = 2
+MF_RETRIEVE_P_SPLIT = 4
 
 _P = ctypes.c_void_p
 _I32 = ctypes.c_int32
@@ -314,10 +315,11 @@ def mf_map_retrieve(layers: Sequence[BSR], layer_map: Sequence[int], W: torch.Te
                     qblock_base: torch.Tensor, max_seqlen_q: int, h_r: int, h_kv: int,
                     O: Optional[torch.Tensor] = None, l_r_range=None, total_q: Optional[int] = None,
                     paged=None, v_layer_stride: int = 0, force_simt: bool = False,
-                    o_f32: bool = False, stream=None) -> torch.Tensor:
+                    o_f32: bool = False, p_split: bool = False, stream=None) -> torch.Tensor:
     """Enqueue fused retrieval for receiver layers l_r_range (default: all of layer_map).
     O: [n_layers, T_q, h_r, d] (allocated when None; float32 with o_f32, else V's dtype).
-    paged = (block_table, page_size)."""
+    paged = (block_table, page_size).  p_split: P.V takes P as a bf16 pair in every query
+    block (MF_RETRIEVE_P_SPLIT)."""
     if l_r_range is None:
         l_r_range = (0, len(layer_map))
     n_l = l_r_range[1] - l_r_range[0]
@@ -327,7 +329,8 @@ def mf_map_retrieve(layers: Sequence[BSR], layer_map: Sequence[int], W: torch.Te
             raise ValueError("total_q is needed to allocate O")
         O = torch.empty((n_l, total_q, h_r, V.shape[-1]), dtype=torch.float32 if o_f32 else V.dtype,
                         device=V.device)
-    flags = (MF_RETRIEVE_FORCE_SIMT if force_simt else 0) | (MF_RETRIEVE_O_F32 if o_f32 else 0)
+    flags = ((MF_RETRIEVE_FORCE_SIMT if force_simt else 0) | (MF_RETRIEVE_O_F32 if o_f32 else 0)
+             | (MF_RETRIEVE_P_SPLIT if p_split else 0))
     d, keep = _retrieve_desc(layers, layer_map, l_r_range, W, V, O, cu_seqlens_q, cu_seqlens_k,
                              qblock_base, max_seqlen_q, h_s, B, h_r, h_kv, v_layer_stride,
                              0, paged, flags)

@@ -82,6 +82,8 @@ mf_status check_retrieve(const mf_retrieve_desc* d) {
   }
   if (mfi::tc_supported(*d) && reinterpret_cast<uintptr_t>(d->V) % 16)
     return fail(MF_ERR_INVALID, "V must be 16-byte aligned");
+  if (d->flags & ~(MF_RETRIEVE_FORCE_SIMT | MF_RETRIEVE_O_F32 | MF_RETRIEVE_P_SPLIT))
+    return fail(MF_ERR_INVALID, "unknown retrieve flags");
   if ((d->flags & MF_RETRIEVE_O_F32) && !mfi::tc_supported(*d))
     return fail(MF_ERR_UNSUPPORTED, "float32 O (MF_RETRIEVE_O_F32) needs the tensor-core path");
   if (!mfi::tc_supported(*d) && (int64_t)d->B * d->d > 16384)

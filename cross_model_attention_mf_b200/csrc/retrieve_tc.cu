@@ -20,14 +20,18 @@
 //           so one MMA per M tile and s-chunk keeps ~16 bits of W.  D1 holds the eight
 //           32-column M tiles of one key tile in TMEM.
 //   convert 16 warps read D1 (lane = position), form P = hi part + lo part (float32),
-//           apply the causal mask and split P into bf16 hi + lo (P = hi + lo to ~16
-//           bits), written as P^T[key][(row, head)] (MN-major SW128) per group.
-//   P.V     D2[dim][(row, head)] += V^T[dim][key] * (P^T_hi + P^T_lo)[key][(row, head)]
-//           tcgen05 M=128 (d) N=64 K=16 per group, two MMAs per K step; V tile
-//           MN-major SW128 by TMA (contiguous or paged).  D2 stays in TMEM for the
-//           whole row chunk.
-// The hi/lo splits leave the final bf16 rounding of O as the only rounding that
-// matters.
+//           apply the causal mask and write P as P^T[key][(row, head)] (MN-major SW128)
+//           per group: split into bf16 hi + lo (P = hi + lo to ~16 bits) for float32
+//           O, on request, and in the first query block of a sequence (rows with at
+//           most B keys, where |P| is largest); rounded once to bf16 elsewhere, as a
+//           bf16 attention kernel rounds its P.
+//   P.V     D2[dim][(row, head)] += V^T[dim][key] * P^T[key][(row, head)]
+//           tcgen05 M=128 (d) N=64 K=16 per group, one MMA per K step and part of P;
+//           V tile MN-major SW128 by TMA (contiguous or paged).  D2 stays in TMEM for
+//           the whole row chunk.
+// Every tcgen05.mma with N <= 64 occupies the tensor pipe about as long as any other
+// (a fixed cost per instruction measured on B200), so the kernel's tensor time follows
+// its MMA count: 16 mixing + 16 P.V MMAs per tile with P in one part, 32 P.V with two.
 //
 // Warp roles: 0 TMA producer of the map tiles; 1 mixing MMA issuer (+ TMEM owner);
 // 2 P.V MMA issuer; 3 TMA producer of the V tiles (separate producers and issuers, so
@@ -51,6 +55,7 @@
 #include <algorithm>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "mf_internal.cuh"
 
@@ -118,6 +123,7 @@ struct RecvParams {
   const float* W;  // [h_r][h_s]
   void* O;         // bf16, or float32 when o_f32
   int o_f32;
+  int p_split;     // P in hi and lo parts in every item
   const int32_t* block_table;
   int paged, page_size, n_pages, max_pages;
   int total_k;     // V rows (contiguous V): the out-of-range row that reads zeros
@@ -350,6 +356,11 @@ __global__ void __launch_bounds__(NT, 1)
   const CUtensorMap* tmV = &tmVs.m[ri];
   const int hc = hh - p.hh_base[ri];
   const int tpb = p.B / KT;
+  // P.V multiplies P in bf16 hi and lo parts (P to ~16 bits) for float32 O, when the caller asks
+  // for it, and in the first query block of a sequence, whose rows see at most B keys and carry
+  // the largest |P|; elsewhere P is rounded once to bf16, as in a bf16 attention kernel
+  const bool split_all = q_r.o_f32 != 0 || q_r.p_split != 0;
+  auto split_p = [&](const Item& q) { return split_all || q.qb == 0; };
 
   const uint32_t sb = smem_u32(smem);
   const uint32_t bar0 = sb + OFF_BAR;
@@ -456,6 +467,43 @@ __global__ void __launch_bounds__(NT, 1)
           const bool kb_ok = kb >= 0 && kb <= it.qb;
           if (!kb_ok) atomicOr(p.status, ST_INDEX);
           const int tok0 = kb * p.B + half * KT;
+          if (!q_r.paged) {
+            const int row = kb_ok ? it.k0 + tok0 : q_r.total_k;  // out of range reads 0
+            for (int h = 0; h < NG / PH && ok; ++h) {
+              if (!(ok = mbar_wait(bar(B_HEMPTY + vs), vph ^ 1, abort_flag, p.status, p.wait_ns))) break;
+              TRACE(5, 4);
+              mbar_expect_tx(bar(B_HFULL + vs), V_BYTES);
+              for (int gl = 0; gl < PH; ++gl) {
+                const uint32_t dst = sb + OFF_V + vs * V_BYTES + gl * VGRP_BYTES;
+                const int G = hc * NG + h * PH + gl;
+                tma_load_3d(dst, tmV, bar(B_HFULL + vs), 0, G, row);
+                tma_load_3d(dst + 8192, tmV, bar(B_HFULL + vs), 64, G, row);
+              }
+              ++v_issued;
+              TRACE(5, 3);
+              if (++vs == HS) { vs = 0; vph ^= 1; }
+            }
+            continue;
+          }
+          // paged V: the tile's page ids, looked up once for all groups (independent loads)
+          const int ps = q_r.page_size;
+          int pages[KT / 8];
+          uint32_t looked = 0;  // bit q: page q's id comes from the block table
+#pragma unroll
+          for (int q = 0; q < KT / 8; ++q) {
+            const int tok = tok0 + q * ps, slot = tok / ps;
+            pages[q] = q_r.n_pages;  // out of range: the copy reads zeros
+            if (q * ps < KT && kb_ok && tok < it.k_len && slot < q_r.max_pages) {
+              pages[q] = q_r.block_table[(int64_t)it.s * q_r.max_pages + slot];
+              looked |= 1u << q;
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < KT / 8; ++q)
+            if (((looked >> q) & 1u) && (pages[q] < 0 || pages[q] >= q_r.n_pages)) {
+              atomicOr(p.status, ST_PAGE);
+              pages[q] = q_r.n_pages;
+            }
           for (int h = 0; h < NG / PH && ok; ++h) {
             if (!(ok = mbar_wait(bar(B_HEMPTY + vs), vph ^ 1, abort_flag, p.status, p.wait_ns))) break;
             TRACE(5, 4);
@@ -463,24 +511,11 @@ __global__ void __launch_bounds__(NT, 1)
             for (int gl = 0; gl < PH; ++gl) {
               const uint32_t dst = sb + OFF_V + vs * V_BYTES + gl * VGRP_BYTES;
               const int G = hc * NG + h * PH + gl;
-              if (!q_r.paged) {
-                const int row = kb_ok ? it.k0 + tok0 : q_r.total_k;  // out of range reads 0
-                tma_load_3d(dst, tmV, bar(B_HFULL + vs), 0, G, row);
-                tma_load_3d(dst + 8192, tmV, bar(B_HFULL + vs), 64, G, row);
-              } else {
-                const int ps = q_r.page_size;
-                for (int q = 0; q < KT / ps; ++q) {
-                  const int tok = tok0 + q * ps;
-                  const int slot = tok / ps;
-                  int page = q_r.n_pages;  // out of range: the copy reads zeros
-                  if (kb_ok && tok < it.k_len && slot < q_r.max_pages) {
-                    const int pg = q_r.block_table[(int64_t)it.s * q_r.max_pages + slot];
-                    if (pg >= 0 && pg < q_r.n_pages) page = pg;
-                    else atomicOr(p.status, ST_PAGE);
-                  }
-                  tma_load_4d(dst + q * ps * 128, tmV, bar(B_HFULL + vs), 0, G, 0, page);
-                  tma_load_4d(dst + 8192 + q * ps * 128, tmV, bar(B_HFULL + vs), 64, G, 0, page);
-                }
+#pragma unroll
+              for (int q = 0; q < KT / 8; ++q) {
+                if (q * ps >= KT) break;
+                tma_load_4d(dst + q * ps * 128, tmV, bar(B_HFULL + vs), 0, G, 0, pages[q]);
+                tma_load_4d(dst + 8192 + q * ps * 128, tmV, bar(B_HFULL + vs), 64, G, 0, pages[q]);
               }
             }
             ++v_issued;
@@ -579,16 +614,22 @@ __global__ void __launch_bounds__(NT, 1)
             // into different D2 columns
             const uint64_t pd = pdesc0 + ((vs * PHALF_BYTES) >> 4);
             const uint64_t vd = vdesc0 + ((vs * V_BYTES) >> 4);
+            // P in its hi and lo parts, or rounded to bf16 (the item's split rule)
+            auto issue = [&](auto parts) {
+              constexpr int NP = decltype(parts)::value;
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
+              for (int k = 0; k < 4; ++k)
 #pragma unroll
-              for (int part = 0; part < 2; ++part)
+                for (int part = 0; part < NP; ++part)
 #pragma unroll
-                for (int gl = 0; gl < PH; ++gl)
-                  tc_mma(tmem + 64u * (uint32_t)(h * PH + gl),
-                         vd + ((gl * VGRP_BYTES + k * 2048u) >> 4),
-                         pd + ((gl * PSLOT_BYTES + part * PT_BYTES + k * 2048u) >> 4), IDESC_PV,
-                         (t > 0 || k > 0 || part > 0) ? 1u : 0u);
+                  for (int gl = 0; gl < PH; ++gl)
+                    tc_mma(tmem + 64u * (uint32_t)(h * PH + gl),
+                           vd + ((gl * VGRP_BYTES + k * 2048u) >> 4),
+                           pd + ((gl * PSLOT_BYTES + part * PT_BYTES + k * 2048u) >> 4), IDESC_PV,
+                           (t > 0 || k > 0 || part > 0) ? 1u : 0u);
+            };
+            if (split_p(it)) issue(std::integral_constant<int, 2>{});
+            else issue(std::integral_constant<int, 1>{});
             TRACE(4, 10);
             tc_commit(bar(B_HEMPTY + vs));  // V and P^T of the slot consumed
             if (++vs == HS) { vs = 0; vph ^= 1; }
@@ -744,57 +785,74 @@ __global__ void __launch_bounds__(NT, 1)
         if (lane == 0) mbar_arrive(bar(B_D1EMPTY));
 #pragma unroll
         for (int mi = 0; mi < MT / CONV_SETS; ++mi) reg_fence(v[mi]);
-        // P = hi + lo with hi = P truncated to bf16 and lo = bf16(P - hi); a tile wholly below
-        // the diagonal of every row needs no causal mask
-        const bool full = kb_ok && tok0 + KT - 1 <= it.i_begin;
-        uint32_t hw[NG][4], lw[NG][4];  // per group: the chunk's packed hi and lo words
+        // Split items: P = hi + lo with hi = P truncated to bf16 and lo = bf16(P - hi), both
+        // written.  Other items: P rounded to bf16, one part.  Both variants are written out, so
+        // that neither carries the other's registers.  A tile wholly below the diagonal of every
+        // row needs no causal mask.
+        auto convert = [&](auto lo_parts) -> bool {
+          constexpr bool SPLIT = decltype(lo_parts)::value;
+          const bool full = kb_ok && tok0 + KT - 1 <= it.i_begin;
+          // per group: the chunk's packed hi (or only) words and lo words
+          uint32_t hw[NG][4], lw[SPLIT ? NG : 1][4];
 #pragma unroll
-        for (int mi = 0; mi < MT / CONV_SETS; ++mi) {
-          const int ii = 2 * (set + mi * CONV_SETS) + rb;
-          const float mk = kb_ok && tok0 + j <= it.i_begin + ii ? 1.0f : 0.0f;
+          for (int mi = 0; mi < MT / CONV_SETS; ++mi) {
+            const int ii = 2 * (set + mi * CONV_SETS) + rb;
+            const float mk = kb_ok && tok0 + j <= it.i_begin + ii ? 1.0f : 0.0f;
 #pragma unroll
-          for (int g = 0; g < NG; ++g) {
+            for (int g = 0; g < NG; ++g) {
 #pragma unroll
-            for (int c = 0; c < 4; c += 2) {
-              float x0 = __uint_as_float(v[mi][4 * g + c]) + __uint_as_float(v[mi][16 + 4 * g + c]);
-              float x1 =
-                  __uint_as_float(v[mi][4 * g + c + 1]) + __uint_as_float(v[mi][16 + 4 * g + c + 1]);
-              if (!full) {
-                x0 *= mk;
-                x1 *= mk;
+              for (int c = 0; c < 4; c += 2) {
+                float x0 =
+                    __uint_as_float(v[mi][4 * g + c]) + __uint_as_float(v[mi][16 + 4 * g + c]);
+                float x1 = __uint_as_float(v[mi][4 * g + c + 1]) +
+                           __uint_as_float(v[mi][16 + 4 * g + c + 1]);
+                if (!full) {
+                  x0 *= mk;
+                  x1 *= mk;
+                }
+                if constexpr (SPLIT) {
+                  const uint32_t b0 = __float_as_uint(x0) & 0xFFFF0000u;
+                  const uint32_t b1 = __float_as_uint(x1) & 0xFFFF0000u;
+                  hw[g][2 * mi + c / 2] = __byte_perm(b0, b1, 0x7632);
+                  // P - hi is exact in f32; one rounding to bf16 for the pair
+                  lw[SPLIT ? g : 0][2 * mi + c / 2] =
+                      pack_bf16(x0 - __uint_as_float(b0), x1 - __uint_as_float(b1));
+                } else {
+                  hw[g][2 * mi + c / 2] = pack_bf16(x0, x1);
+                }
               }
-              const uint32_t b0 = __float_as_uint(x0) & 0xFFFF0000u;
-              const uint32_t b1 = __float_as_uint(x1) & 0xFFFF0000u;
-              hw[g][2 * mi + c / 2] = __byte_perm(b0, b1, 0x7632);
-              // P - hi is exact in f32; one rounding to bf16 for the pair
-              lw[g][2 * mi + c / 2] = pack_bf16(x0 - __uint_as_float(b0), x1 - __uint_as_float(b1));
             }
           }
-        }
-        if (warp == 4 && lane == 0) TRACE(2, 3);
+          if (warp == 4 && lane == 0) TRACE(2, 3);
+          bool ok_ = true;
 #pragma unroll
-        for (int h = 0; h < NG / PH; ++h) {
-          // this half of the P buffer must have been consumed by the previous tile's P.V
-          const int hq = T * (NG / PH) + h, ps = hq % HS;  // half-tile count, slot
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_HEMPTY + ps), ((hq / HS) & 1) ^ 1,
-                                                 abort_flag, p.status, p.wait_ns));
-          if (!ok) break;
-          if (warp == 4 && lane == 0) TRACE(2, 4);
+          for (int h = 0; h < NG / PH; ++h) {
+            // this half of the P buffer must have been consumed by the previous tile's P.V
+            const int hq = T * (NG / PH) + h, ps = hq % HS;  // half-tile count, slot
+            ok_ = __all_sync(0xffffffffu, mbar_wait(bar(B_HEMPTY + ps), ((hq / HS) & 1) ^ 1,
+                                                    abort_flag, p.status, p.wait_ns));
+            if (!ok_) break;
+            if (warp == 4 && lane == 0) TRACE(2, 4);
 #pragma unroll
-          for (int gl = 0; gl < PH; ++gl) {
-            const int g = h * PH + gl;
-            const uint32_t pt = sb + OFF_P + ps * PHALF_BYTES + gl * PSLOT_BYTES + choff;
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pt), "r"(hw[g][0]),
-                         "r"(hw[g][1]), "r"(hw[g][2]), "r"(hw[g][3])
-                         : "memory");
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pt + PT_BYTES),
-                         "r"(lw[g][0]), "r"(lw[g][1]), "r"(lw[g][2]), "r"(lw[g][3])
-                         : "memory");
+            for (int gl = 0; gl < PH; ++gl) {
+              const int g = h * PH + gl;
+              const uint32_t pt = sb + OFF_P + ps * PHALF_BYTES + gl * PSLOT_BYTES + choff;
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pt), "r"(hw[g][0]),
+                           "r"(hw[g][1]), "r"(hw[g][2]), "r"(hw[g][3])
+                           : "memory");
+              if constexpr (SPLIT)
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pt + PT_BYTES),
+                             "r"(lw[SPLIT ? g : 0][0]), "r"(lw[SPLIT ? g : 0][1]),
+                             "r"(lw[SPLIT ? g : 0][2]), "r"(lw[SPLIT ? g : 0][3])
+                             : "memory");
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_HFULL + ps));
           }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_HFULL + ps));
-        }
+          return ok_;
+        };
+        ok = split_p(it) ? convert(std::true_type{}) : convert(std::false_type{});
         if (!ok) break;
         if (warp == 4 && lane == 0) TRACE(2, 2);
       }
@@ -912,6 +970,7 @@ bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* 
     RecvParams& r = p.rv[k];
     r.W = l.W; r.O = l.O;
     r.o_f32 = (d.flags & MF_RETRIEVE_O_F32) ? 1 : 0;
+    r.p_split = (d.flags & MF_RETRIEVE_P_SPLIT) ? 1 : 0;
     r.block_table = d.block_table; r.paged = d.paged; r.page_size = d.page_size;
     r.n_pages = d.n_pages; r.max_pages = d.max_pages; r.total_k = (int)d.total_k;
     r.h_r = d.h_r; r.h_kv = d.h_kv; r.gq = d.h_r / d.h_kv;

@@ -210,12 +210,16 @@ mf_status mf_compress_qk(const mf_compress_qk_desc* desc, void* workspace, size_
  * [l_r_end - l_r_begin][T_q][h_r][d] with layer stride o_layer_stride elements
  * (0 = T_q * h_r * d).
  * Arithmetic: MF_F32 maps/V run in float32 throughout.  MF_BF16 maps and V run on
- * tcgen05 tensor cores: W is split into a bf16 pair (hi + lo, ~16 bits), the mixed
- * map P is accumulated in float32 and split into a bf16 pair (hi truncated, lo the
- * rounded remainder), P.V takes both parts with float32 accumulation, and O is rounded
- * to bf16 (round to nearest even).  Each output row's accumulation order depends only
- * on its query block's kept blocks, so chunked, paged and varlen layouts give
- * bit-identical rows.
+ * tcgen05 tensor cores: W is split into a bf16 pair (hi + lo, ~16 bits) and the mixed
+ * map P is accumulated in float32.  P.V (float32 accumulation) then takes P either as
+ * a bf16 pair (hi truncated, lo the rounded remainder: P to ~16 bits) or rounded once
+ * to bf16 (round to nearest even, as a bf16 attention kernel rounds its P): the pair
+ * with float32 O (MF_RETRIEVE_O_F32), with flag MF_RETRIEVE_P_SPLIT, and in the first
+ * query block of every sequence (rows with at most B keys, where |P| is largest);
+ * one rounding elsewhere, which adds at most 2^-8 |P_r[i][j]| |V[j]| per key to the
+ * error of O.  A bf16 O is rounded to nearest even.  Each output row's accumulation
+ * order depends only on its query block's kept blocks, so chunked, paged and varlen
+ * layouts give bit-identical rows.
  * Requirements: h_r % h_kv == 0; layer_map[l] < n_sender_layers; d <= 256.
  * The tensor-core path needs MF_BF16 maps and V (V 16-byte aligned), B in {64, 128},
  * d = 128, h_r / h_kv <= 4, h_s <= 64 and (if paged) page_size in {8, 16, 32, 64};
@@ -232,6 +236,8 @@ typedef struct {
 #define MF_RETRIEVE_O_F32 2        /* flags: O is float32 (the unrounded float32 accumulators);
                                       tensor-core path only (bf16 maps and V), else
                                       MF_ERR_UNSUPPORTED */
+#define MF_RETRIEVE_P_SPLIT 4      /* flags: P.V takes P as a bf16 pair in every query block
+                                      (tensor-core path; the SIMT path is float32 anyway) */
 
 typedef struct {
   const mf_bsr* layers;            /* host [n_sender_layers] */

@@ -338,8 +338,10 @@ def _raw_close(got, want, amax, rl2, what):
 ])
 def test_float32_output_meets_the_literal_bounds(name, lens, B, h_s, h_r, h_kv, reading):
     """With float32 O (MF_RETRIEVE_O_F32) the tensor-core kernel's accumulators are compared
-    with the oracle unrounded: raw max-abs 2e-2 and relative L2 1e-2, every row; its bf16 output
-    is that float32 output rounded to nearest even."""
+    with the oracle unrounded: raw max-abs 2e-2 and relative L2 1e-2, every row.  With P as a
+    bf16 pair everywhere (MF_RETRIEVE_P_SPLIT) the bf16 output is that float32 output rounded
+    to nearest even, bit for bit; by default the same holds in the first query block of each
+    sequence (P split there), and every row meets the bf16 bounds."""
     w = synth.Workload(name, lens, B=B, h_s=h_s, h_r=h_r, h_kv=h_kv, d=128, dtype="bf16", tau=0.95,
                        n_heavy=16, reading=reading)
     pack = sdev.fill_maps(sdev.alloc_maps(w), w, 0)
@@ -354,10 +356,19 @@ def test_float32_output_meets_the_literal_bounds(name, lens, B, h_s, h_r, h_kv, 
     O16 = mf.mf_map_retrieve([bsr], [0], W, V, cu, cu, qbase, max(w.lens), w.h_r, w.h_kv,
                              total_q=w.tokens)[0]
     _status_ok()
+    O16s = mf.mf_map_retrieve([bsr], [0], W, V, cu, cu, qbase, max(w.lens), w.h_r, w.h_kv,
+                              total_q=w.tokens, p_split=True)[0]
+    _status_ok()
     assert O32.dtype == torch.float32
-    assert torch.equal(O32.to(torch.bfloat16), O16)
+    R32 = O32.to(torch.bfloat16)
+    assert torch.equal(R32, O16s)
+    starts = np.concatenate([[0], np.cumsum(w.lens)])
+    for s0, L in zip(starts[:-1], w.lens):
+        first = slice(int(s0), int(s0) + min(B, L))
+        assert torch.equal(R32[first], O16[first]), "first query block: P split"
     want = _oracle_O_all(w, orows, W[0].cpu().numpy(), V.cpu())
     _raw_close(O32.cpu().numpy(), want, 2e-2, 1e-2, name)
+    assert_O_close(O16.float().cpu().numpy(), want, "bf16", f"{name} bf16 output")
 
 
 def test_float32_output_full_size_sampled():
