@@ -930,9 +930,11 @@ def main():
             dt = oracle_sample(w, [slabs[i] for i in idx], W_l, V_host, [rows[i] for i in idx], cores)
             return dt, sum(min(w.lens[0], (rows[i] + 1) * w.B) - rows[i] * w.B for i in idx)
 
-        warm = min(args.warmup, 2)
-        for t in range(warm):
-            one(t)
+        # the requested warm-up steps (bounded by ~20 s of wall time)
+        warm, t_warm = 0, time.time()
+        while warm < args.warmup and time.time() - t_warm < 20.0:
+            one(warm)
+            warm += 1
         spent, k, toks = 0.0, 0, 0
         while k < max(args.steps, 1) and (spent < 60.0 or k == 0):
             dt, n = one(warm + k)
