@@ -7,15 +7,15 @@
 // and only those are written -- no second dense matrix is assembled.
 //
 // Kernels (one launch each, all on the caller's stream):
-//   k_meta          per-sequence geometry of the varlen pack (one thread)
+//   k_meta          per-sequence geometry of the varlen pack (one thread); the grid
+//                   clears the selection's look-back flags
 //   k_stats         head-summed mass of every causal block: a streaming reduction
 //                   with 16-byte loads, float32 partials of 8 (bf16) or 4 (f32)
 //                   elements combined in float64, fixed order (deterministic)
 //   k_select        per query block: sort candidates (mass desc, kb asc), walk
-//                   the running float64 sum until it reaches tau * total, write the
-//                   row's kept indices in ascending order to a per-row list
-//   k_scan_compact  row_ptr by exclusive scan of the counts, then copy the per-row
-//                   lists into col_idx
+//                   the running float64 sum until it reaches tau * total; the row's
+//                   offset by a decoupled look-back over the earlier rows' counts,
+//                   then its kept indices in ascending order into col_idx
 //   k_gather        copy each kept block with the causal/length mask applied, one
 //                   (block, sender head) unit per CTA iteration
 #include <cuda_bf16.h>
@@ -49,7 +49,11 @@ __device__ inline int tri_row(int64_t c) {
 
 __global__ void k_meta(const int32_t* cu, const int64_t* off, int nseq, int max_seqlen, int B,
                        int elem_bytes, int64_t* meta, uint32_t* status, int32_t* row_ptr,
-                       int32_t* nnz_out) {
+                       int32_t* nnz_out, unsigned long long* flags, int64_t max_rows) {
+  // the selection's look-back flags start cleared (every thread of the grid)
+  for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < max_rows;
+       r += (int64_t)gridDim.x * blockDim.x)
+    flags[r] = 0ull;
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   int64_t rows = 0, cb = 0;
   uint32_t st = 0;
@@ -63,7 +67,7 @@ __global__ void k_meta(const int32_t* cu, const int64_t* off, int nseq, int max_
     rows += nqb;
     cb += nqb * (nqb + 1) / 2;
   }
-  meta[0] = rows; meta[1] = cb; meta[2] = 0; meta[3] = 0;  // meta[2]: rows selected so far
+  meta[0] = rows; meta[1] = cb; meta[2] = 0; meta[3] = 0;  // meta[2]: selection ticket
   if (rows == 0) {  // no query block at all: an empty BSR
     row_ptr[0] = 0;
     *nnz_out = 0;
@@ -172,17 +176,38 @@ __device__ inline uint64_t order_key(double x) {
   return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
 }
 
-// One CTA per query block (row).  Candidates kb < qb sorted by (mass desc, kb asc);
-// the walk starts from the diagonal block.
+// One CTA per query block (row).  Candidates kb < qb sorted by (mass desc, kb asc); the walk
+// starts from the diagonal block.  The row's place in col_idx comes from a decoupled look-back
+// (single-pass prefix sum): rows are numbered by a ticket taken when the CTA starts (meta[2]),
+// so every earlier row is already running; each row publishes its count (FLAG_AGG), sums the
+// counts or the inclusive prefix (FLAG_PREFIX) of the rows before it, publishes its own
+// inclusive prefix and writes its kept blocks into col_idx / kept_row and its row_ptr entry.
+// The flags were cleared by k_meta.  Waiting for an earlier row's flag is bounded by wait_ns.
+constexpr unsigned long long FLAG_AGG = 1ull << 62, FLAG_PREFIX = 1ull << 63,
+                             FLAG_VALUE = (1ull << 62) - 1;
+__device__ __forceinline__ uint64_t gtime() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 template <int NT>
-__global__ void __launch_bounds__(NT) k_select(const int64_t* __restrict__ meta, int nseq,
+__global__ void __launch_bounds__(NT) k_select(int64_t* __restrict__ meta, int nseq,
                                                const double* __restrict__ mass, double tau,
-                                               int32_t* __restrict__ counts,
-                                               int32_t* __restrict__ kept_local) {
+                                               unsigned long long* __restrict__ flags,
+                                               int32_t* __restrict__ row_ptr,
+                                               int32_t* __restrict__ col_idx,
+                                               int32_t* __restrict__ kept_row,
+                                               int32_t* __restrict__ nnz_out, int64_t capacity,
+                                               uint32_t* status, uint64_t wait_ns) {
   extern __shared__ uint64_t sm[];
   __shared__ int s_nkeep;
-  const int64_t row = blockIdx.x;
-  if (row >= meta[0]) return;
+  __shared__ int64_t s_row, s_base;
+  if (threadIdx.x == 0)
+    s_row = (int64_t)atomicAdd(reinterpret_cast<unsigned long long*>(meta + 2), 1ull);
+  __syncthreads();
+  const int64_t row = s_row;
+  const int64_t R = meta[0];
+  if (row >= R) return;
   const int s = find_seq(meta, nseq, row, 2);
   const int64_t* m = meta + META_HDR + 4 * s;
   const int qb = (int)(row - m[2]);
@@ -232,22 +257,63 @@ __global__ void __launch_bounds__(NT) k_select(const int64_t* __restrict__ meta,
       }
     }
     s_nkeep = nk;
-    counts[row] = nk;
   }
   __syncthreads();
-  // kept flags by key-block index (reusing the key array), then an ordered compaction:
-  // the row's kept indices in ascending order at kept_local[tri ...]
   const int nk = s_nkeep;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // publish this row's count, then find its offset from the rows before it
+  if (threadIdx.x == 0) {
+    const unsigned long long w = FLAG_AGG | (unsigned long long)nk;
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(flags + row), "l"(w) : "memory");
+  }
+  if (warp == 0) {
+    int64_t prefix = 0;
+    int64_t j0 = row - 1;  // lane l reads row j0 - l; rows before 0 count as a prefix of 0
+    const uint64_t t0 = gtime();
+    while (true) {
+      const int64_t j = j0 - lane;
+      unsigned long long f = FLAG_PREFIX;
+      if (j >= 0) asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(f) : "l"(flags + j) : "memory");
+      if (!__all_sync(0xffffffffu, f != 0ull)) {  // an earlier row has not published yet
+        if (gtime() - t0 > wait_ns) {
+          if (lane == 0) atomicOr(status, ST_TIMEOUT);
+          break;
+        }
+        continue;
+      }
+      const uint32_t pre = __ballot_sync(0xffffffffu, (f & FLAG_PREFIX) != 0ull);
+      const int first = pre ? __ffs(pre) - 1 : 31;  // nearest row holding an inclusive prefix
+      int64_t v = lane <= first ? (int64_t)(f & FLAG_VALUE) : 0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      prefix += v;
+      if (pre) break;
+      j0 -= 32;
+    }
+    if (lane == 0) {
+      s_base = prefix;
+      const unsigned long long w = FLAG_PREFIX | (unsigned long long)(prefix + nk);
+      asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(flags + row), "l"(w) : "memory");
+      row_ptr[row] = (int32_t)prefix;
+      if (row == R - 1) {
+        row_ptr[R] = (int32_t)(prefix + nk);
+        *nnz_out = (int32_t)(prefix + nk);
+        if (prefix + nk > capacity) atomicOr(status, ST_CAPACITY);
+      }
+    }
+  }
+  // kept flags by key-block index (reusing the key array), then an ordered compaction into
+  // col_idx[base ...] (ascending key blocks), skipping entries past the capacity
   uint8_t* kept = reinterpret_cast<uint8_t*>(key);
   for (int t = threadIdx.x; t <= n; t += NT) kept[t] = 0;
   __syncthreads();
   for (int t = threadIdx.x; t < nk - 1; t += NT) kept[idx[t]] = 1;
   if (threadIdx.x == 0) kept[qb] = 1;
   __syncthreads();
+  const int64_t base = s_base;
   __shared__ int s_warp[NT / 32];
-  __shared__ int s_base;
-  if (threadIdx.x == 0) s_base = 0;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ int s_cnt;
+  if (threadIdx.x == 0) s_cnt = 0;
   for (int k0 = 0; k0 <= n; k0 += NT) {
     const int kb = k0 + threadIdx.x;
     const bool f = kb <= n && kept[kb];
@@ -255,76 +321,16 @@ __global__ void __launch_bounds__(NT) k_select(const int64_t* __restrict__ meta,
     __syncthreads();
     if (lane == 0) s_warp[warp] = __popc(bal);
     __syncthreads();
-    int before = s_base;
+    int before = s_cnt;
     for (int w = 0; w < warp; ++w) before += s_warp[w];
-    if (f) kept_local[tri + before + __popc(bal & ((1u << lane) - 1u))] = kb;
+    const int64_t e = base + before + __popc(bal & ((1u << lane) - 1u));
+    if (f && e < capacity) {
+      col_idx[e] = kb;
+      kept_row[e] = (int32_t)row;
+    }
     __syncthreads();
     if (threadIdx.x == 0)
-      for (int w = 0; w < NT / 32; ++w) s_base += s_warp[w];
-  }
-}
-
-// One CTA: exclusive scan of the counts into row_ptr (independent loads, so their
-// latencies overlap), then each row's list is copied into col_idx (warp per row).
-constexpr int SCAN_NT = 1024, SCAN_PER = 8;
-__global__ void __launch_bounds__(SCAN_NT) k_scan_compact(
-    const int64_t* __restrict__ meta, int nseq, const int32_t* __restrict__ counts,
-    const int32_t* __restrict__ kept_local, int32_t* __restrict__ row_ptr,
-    int32_t* __restrict__ col_idx, int32_t* __restrict__ kept_row, int32_t* __restrict__ nnz_out,
-    int64_t capacity, uint32_t* status) {
-  __shared__ int64_t part[SCAN_NT];
-  __shared__ int64_t carry;
-  const int64_t R = meta[0];
-  const int t = threadIdx.x;
-  if (t == 0) carry = 0;
-  __syncthreads();
-  for (int64_t base = 0; base < R; base += (int64_t)SCAN_NT * SCAN_PER) {
-    const int64_t r0 = base + (int64_t)t * SCAN_PER;
-    int32_t c[SCAN_PER];
-#pragma unroll
-    for (int k = 0; k < SCAN_PER; ++k) c[k] = r0 + k < R ? counts[r0 + k] : 0;
-    int64_t sum = 0;
-#pragma unroll
-    for (int k = 0; k < SCAN_PER; ++k) sum += c[k];
-    part[t] = sum;
-    __syncthreads();
-    for (int o = 1; o < SCAN_NT; o <<= 1) {  // inclusive Hillis-Steele scan
-      const int64_t v = t >= o ? part[t - o] : 0;
-      __syncthreads();
-      part[t] += v;
-      __syncthreads();
-    }
-    int64_t run = carry + part[t] - sum;
-#pragma unroll
-    for (int k = 0; k < SCAN_PER; ++k)
-      if (r0 + k < R) {
-        row_ptr[r0 + k] = (int32_t)run;
-        run += c[k];
-      }
-    __syncthreads();
-    if (t == SCAN_NT - 1) carry += part[SCAN_NT - 1];
-    __syncthreads();
-  }
-  const int64_t nnz = carry;
-  if (t == 0) {
-    row_ptr[R] = (int32_t)nnz;
-    *nnz_out = (int32_t)nnz;
-    if (nnz > capacity) atomicOr(status, ST_CAPACITY);
-  }
-  __syncthreads();
-  const int warp = t >> 5, lane = t & 31;
-  for (int64_t row = warp; row < R; row += SCAN_NT / 32) {
-    const int s = find_seq(meta, nseq, row, 2);
-    const int64_t* m = meta + META_HDR + 4 * s;
-    const int qb = (int)(row - m[2]);
-    const int32_t* kl = kept_local + m[3] + (int64_t)qb * (qb + 1) / 2;
-    const int64_t n0 = row_ptr[row];
-    const int cnt = counts[row];
-    for (int k = lane; k < cnt; k += 32)
-      if (n0 + k < capacity) {
-        col_idx[n0 + k] = kl[k];
-        kept_row[n0 + k] = (int32_t)row;
-      }
+      for (int w = 0; w < NT / 32; ++w) s_cnt += s_warp[w];
   }
 }
 
@@ -410,8 +416,9 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 cudaError_t launch_meta(const int32_t* cu, const int64_t* off, int nseq, int max_seqlen, int B,
                         int elem_bytes, const CompressWs& ws, uint32_t* status, int32_t* row_ptr,
                         int32_t* nnz_out, cudaStream_t st) {
-  k_meta<<<1, 32, 0, st>>>(cu, off, nseq, max_seqlen, B, elem_bytes, ws.meta, status, row_ptr,
-                           nnz_out);
+  const int grid = (int)std::min<int64_t>(std::max<int64_t>((ws.max_rows + 255) / 256, 1), 1024);
+  k_meta<<<grid, 256, 0, st>>>(cu, off, nseq, max_seqlen, B, elem_bytes, ws.meta, status, row_ptr,
+                               nnz_out, ws.flags, ws.max_rows);
   return cudaGetLastError();
 }
 
@@ -427,10 +434,9 @@ cudaError_t launch_select(const CompressWs& ws, int nseq, int max_seqlen, int B,
                                          (int)smem_sel);
     if (e != cudaSuccess) return e;
   }
-  k_select<128><<<(unsigned)ws.max_rows, 128, smem_sel, st>>>(ws.meta, nseq, mass, tau, ws.counts,
-                                                              ws.kept_local);
-  k_scan_compact<<<1, SCAN_NT, 0, st>>>(ws.meta, nseq, ws.counts, ws.kept_local, row_ptr, col_idx,
-                                        ws.kept_row, nnz_out, capacity, status);
+  k_select<128><<<(unsigned)std::max<int64_t>(ws.max_rows, 1), 128, smem_sel, st>>>(
+      ws.meta, nseq, mass, tau, ws.flags, row_ptr, col_idx, ws.kept_row, nnz_out, capacity, status,
+      wait_limit_ns());
   return cudaGetLastError();
 }
 
@@ -441,15 +447,13 @@ size_t compress_ws_layout(const mf_compress_desc& d, CompressWs* ws, void* base)
   size_t off = 0;
   const size_t o_meta = off; off = align_up(off + sizeof(int64_t) * (META_HDR + 4 * (size_t)d.nseq), 256);
   const size_t o_mass = off; off = align_up(off + sizeof(double) * (size_t)max_cb, 256);
-  const size_t o_kept_local = off; off = align_up(off + sizeof(int32_t) * (size_t)max_cb, 256);
-  const size_t o_counts = off; off = align_up(off + sizeof(int32_t) * (size_t)max_rows, 256);
+  const size_t o_flags = off; off = align_up(off + sizeof(uint64_t) * (size_t)std::max<int64_t>(max_rows, 1), 256);
   const size_t o_kept = off; off = align_up(off + sizeof(int32_t) * (size_t)std::max<int64_t>(d.capacity_blocks, 1), 256);
   if (ws) {
     char* b = static_cast<char*>(base);
     ws->meta = reinterpret_cast<int64_t*>(b + o_meta);
     ws->mass = reinterpret_cast<double*>(b + o_mass);
-    ws->kept_local = reinterpret_cast<int32_t*>(b + o_kept_local);
-    ws->counts = reinterpret_cast<int32_t*>(b + o_counts);
+    ws->flags = reinterpret_cast<unsigned long long*>(b + o_flags);
     ws->kept_row = reinterpret_cast<int32_t*>(b + o_kept);
     ws->max_cb = max_cb;
     ws->max_rows = max_rows;

@@ -28,11 +28,10 @@ constexpr uint64_t DRAIN_NS = 2000000000ull;  // bound of the waits for work alr
 
 // scratch of mf_compress (carved out of the caller's workspace)
 struct CompressWs {
-  int64_t* meta;      // [4 + 4 * nseq]: total rows, total causal blocks, -, -, then per
-                      // sequence (L, nqb, row_base, cb_base)
+  int64_t* meta;      // [4 + 4 * nseq]: total rows, total causal blocks, selection ticket, -,
+                      // then per sequence (L, nqb, row_base, cb_base)
   double* mass;       // [max_cb] head-summed block masses
-  int32_t* kept_local;  // [max_cb] each row's kept key blocks, ascending, at its causal base
-  int32_t* counts;    // [max_rows] kept blocks per row
+  unsigned long long* flags;  // [max_rows] selection look-back: count or prefix per row
   int32_t* kept_row;  // [capacity] BSR row of each kept block
   int64_t max_cb, max_rows;
 };

@@ -43,8 +43,9 @@ def test_workspace_size_bounds(mf):
     small = mf.mf_compress_workspace_size(1, 256, 32, 10)
     big = mf.mf_compress_workspace_size(16, 8192, 64, 100000)
     assert 0 < small < big
-    # per-sequence meta + masses + flags of 128*129/2 blocks per sequence + kept rows
-    assert big >= 16 * (128 * 129 // 2) * 9 + 100000 * 4
+    # per-sequence meta + float64 masses of 128*129/2 blocks per sequence + one 8-byte
+    # look-back flag per query block + kept rows
+    assert big >= 16 * (128 * 129 // 2) * 8 + 16 * 128 * 8 + 100000 * 4
     assert mf.mf_compress_workspace_size(1, 100, 64, 0) % 256 == 0
 
 
