@@ -47,14 +47,12 @@ __device__ inline int tri_row(int64_t c) {
   return q;
 }
 
-__global__ void k_meta(const int32_t* cu, const int64_t* off, int nseq, int max_seqlen, int B,
-                       int elem_bytes, int64_t* meta, uint32_t* status, int32_t* row_ptr,
-                       int32_t* nnz_out, unsigned long long* flags, int64_t max_rows) {
-  // the selection's look-back flags start cleared (every thread of the grid)
-  for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < max_rows;
-       r += (int64_t)gridDim.x * blockDim.x)
-    flags[r] = 0ull;
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+// The varlen pack's geometry: header (total rows, total causal blocks, selection ticket = 0, -)
+// and per sequence (L, nqb, row_base, cb_base), from its cu_seqlens (cu) and map offsets (off,
+// may be null; a(s) = off[s] * elem_bytes must be 16-byte aligned).  One thread; returns the
+// status bits of invalid sequences (which count as empty).
+__device__ uint32_t meta_fill(const int32_t* cu, const int64_t* off, int nseq, int max_seqlen,
+                              int B, int elem_bytes, int64_t* meta) {
   int64_t rows = 0, cb = 0;
   uint32_t st = 0;
   for (int s = 0; s < nseq; ++s) {
@@ -68,7 +66,19 @@ __global__ void k_meta(const int32_t* cu, const int64_t* off, int nseq, int max_
     cb += nqb * (nqb + 1) / 2;
   }
   meta[0] = rows; meta[1] = cb; meta[2] = 0; meta[3] = 0;  // meta[2]: selection ticket
-  if (rows == 0) {  // no query block at all: an empty BSR
+  return st;
+}
+
+__global__ void k_meta(const int32_t* cu, const int64_t* off, int nseq, int max_seqlen, int B,
+                       int elem_bytes, int64_t* meta, uint32_t* status, int32_t* row_ptr,
+                       int32_t* nnz_out, unsigned long long* flags, int64_t max_rows) {
+  // the selection's look-back flags start cleared (every thread of the grid)
+  for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < max_rows;
+       r += (int64_t)gridDim.x * blockDim.x)
+    flags[r] = 0ull;
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  const uint32_t st = meta_fill(cu, off, nseq, max_seqlen, B, elem_bytes, meta);
+  if (meta[0] == 0) {  // no query block at all: an empty BSR
     row_ptr[0] = 0;
     *nnz_out = 0;
   }
@@ -104,15 +114,60 @@ __device__ inline double block_sum_f64(double v, double* red) {
   return t;  // valid in thread 0
 }
 
+// Geometry computed inside k_stats (no k_meta launch) for batches of up to this many sequences
+constexpr int INLINE_META_SEQ = 64;
+struct MetaIn {           // k_stats computes the geometry itself when inline_meta is set
+  const int32_t* cu;
+  int max_seqlen, elem_bytes, inline_meta;
+  int64_t* meta_out;      // written by CTA 0
+  uint32_t* status;
+  int32_t* row_ptr;       // empty batch: row_ptr[0] = 0
+  int32_t* nnz_out;
+  unsigned long long* flags;  // cleared by the grid
+  int64_t max_rows;
+};
+
 // Masses of every causal block.  Item = (sequence, qb, kb) over all sender heads.
 template <typename T, int B, int NT>
 __global__ void __launch_bounds__(NT) k_stats(const T* __restrict__ maps,
                                               const int64_t* __restrict__ seq_off,
-                                              const int64_t* __restrict__ meta, int nseq,
-                                              int h_s, double* __restrict__ mass) {
+                                              const int64_t* __restrict__ meta_g, int nseq,
+                                              int h_s, double* __restrict__ mass, MetaIn mi) {
   constexpr int EPV = Vec<T>::EPV, VPR = B / EPV, VPB = B * VPR;  // vectors per row / per head
   constexpr int U = 4;
   __shared__ double red[NT / 32];
+  __shared__ int64_t s_meta[META_HDR + 4 * INLINE_META_SEQ];
+  __shared__ int32_t s_cu[INLINE_META_SEQ + 1];
+  __shared__ int64_t s_off[INLINE_META_SEQ];
+  const int64_t* meta = meta_g;
+  if (mi.inline_meta) {
+    // the selection's look-back flags start cleared (every thread of the grid)
+    for (int64_t r = (int64_t)blockIdx.x * NT + threadIdx.x; r < mi.max_rows;
+         r += (int64_t)gridDim.x * NT)
+      mi.flags[r] = 0ull;
+    // every CTA computes the geometry into shared memory (warp 0 loads the inputs, thread 0
+    // runs the sums); CTA 0 also publishes it for the later passes
+    if (threadIdx.x < 32) {
+      for (int k = threadIdx.x; k <= nseq; k += 32) s_cu[k] = mi.cu[k];
+      if (seq_off)
+        for (int k = threadIdx.x; k < nseq; k += 32) s_off[k] = seq_off[k];
+      __syncwarp();
+      if (threadIdx.x == 0) {
+        const uint32_t st = meta_fill(s_cu, seq_off ? s_off : nullptr, nseq, mi.max_seqlen, B,
+                                      mi.elem_bytes, s_meta);
+        if (blockIdx.x == 0) {
+          for (int k = 0; k < META_HDR + 4 * nseq; ++k) mi.meta_out[k] = s_meta[k];
+          if (s_meta[0] == 0) {  // no query block at all: an empty BSR
+            mi.row_ptr[0] = 0;
+            *mi.nnz_out = 0;
+          }
+          if (st) atomicOr(mi.status, st);
+        }
+      }
+    }
+    __syncthreads();
+    meta = s_meta;
+  }
   const int64_t total = meta[1];
   const int64_t nv = (int64_t)h_s * VPB;
   for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
@@ -396,8 +451,14 @@ cudaError_t launch_typed(const mf_compress_desc& d, const CompressWs& ws, uint32
   const T* maps = static_cast<const T*>(d.maps);
   double* mass = d.block_mass_out ? d.block_mass_out : ws.mass;
   const int grid_stats = (int)std::min<int64_t>(ws.max_cb, (int64_t)sms * 8);
+  MetaIn mi{};
+  if (d.nseq <= INLINE_META_SEQ) {
+    mi.cu = d.cu_seqlens; mi.max_seqlen = d.max_seqlen; mi.elem_bytes = (int)sizeof(T);
+    mi.inline_meta = 1; mi.meta_out = ws.meta; mi.status = status; mi.row_ptr = d.row_ptr;
+    mi.nnz_out = d.nnz_out; mi.flags = ws.flags; mi.max_rows = ws.max_rows;
+  }
   k_stats<T, B, NT><<<grid_stats, NT, 0, st>>>(maps, d.map_seq_offset, ws.meta, d.nseq, d.h_s,
-                                                mass);
+                                                mass, mi);
   cudaError_t e = launch_select(ws, d.nseq, d.max_seqlen, B, mass, d.tau, d.row_ptr, d.col_idx,
                                 d.nnz_out, d.capacity_blocks, status, st);
   if (e != cudaSuccess) return e;
@@ -467,9 +528,13 @@ cudaError_t launch_compress(const mf_compress_desc& d, const CompressWs& ws, uin
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int elem = d.dtype == MF_F32 ? 4 : 2;
-  cudaError_t e = launch_meta(d.cu_seqlens, d.map_seq_offset, d.nseq, d.max_seqlen, d.B, elem, ws,
-                              status, d.row_ptr, d.nnz_out, st);
-  if (e != cudaSuccess) return e;
+  // the geometry pass: inside k_stats for up to INLINE_META_SEQ sequences, else its own launch
+  // (also when there is no query block at all and k_stats does not run)
+  if (d.nseq > INLINE_META_SEQ || ws.max_cb == 0) {
+    cudaError_t e = launch_meta(d.cu_seqlens, d.map_seq_offset, d.nseq, d.max_seqlen, d.B, elem,
+                                ws, status, d.row_ptr, d.nnz_out, st);
+    if (e != cudaSuccess) return e;
+  }
   if (ws.max_cb == 0) return cudaSuccess;  // no query block (max_seqlen 0): k_meta wrote the empty BSR
   if (d.dtype == MF_F32) {
     if (d.B == 32) return launch_typed<float, 32>(d, ws, status, st, sms);
