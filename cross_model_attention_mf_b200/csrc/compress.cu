@@ -230,6 +230,10 @@ __device__ inline uint64_t order_key(double x) {
   const uint64_t b = (uint64_t)__double_as_longlong(x);
   return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
 }
+// the mass a key was made from (bit for bit; -0 comes back as +0)
+__device__ inline double key_mass(uint64_t k) {
+  return __longlong_as_double((long long)((k >> 63) ? (k & 0x7fffffffffffffffull) : ~k));
+}
 
 // One CTA per query block (row).  Candidates kb < qb sorted by (mass desc, kb asc); the walk
 // starts from the diagonal block.  The row's place in col_idx comes from a decoupled look-back
@@ -296,18 +300,21 @@ __global__ void __launch_bounds__(NT) k_select(int64_t* __restrict__ meta, int n
       __syncthreads();
     }
   if (threadIdx.x == 0) {
+    // the walk reads the candidates' masses back from their sorted keys (independent shared
+    // loads; only the float64 sums form a chain)
+    const double diag = mr[qb];
     double total = 0.0;
-    total += mr[qb];
-    for (int t = 0; t < n; ++t) total += mr[idx[t]];
+    total += diag;
+    for (int t = 0; t < n; ++t) total += key_mass(key[t]);
     const double target = tau * total;
     double S = 0.0;
     int nk = n + 1;
-    S += mr[qb];
+    S += diag;
     if (S >= target) {
       nk = 1;
     } else {
       for (int t = 0; t < n; ++t) {
-        S += mr[idx[t]];
+        S += key_mass(key[t]);
         if (S >= target) { nk = t + 2; break; }
       }
     }
