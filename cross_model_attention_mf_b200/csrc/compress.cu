@@ -51,7 +51,7 @@ __device__ inline int tri_row(int64_t c) {
 // and per sequence (L, nqb, row_base, cb_base), from its cu_seqlens (cu) and map offsets (off,
 // may be null; a(s) = off[s] * elem_bytes must be 16-byte aligned).  One thread; returns the
 // status bits of invalid sequences (which count as empty).
-__device__ uint32_t meta_fill(const int32_t* cu, const int64_t* off, int nseq, int max_seqlen,
+__device__ __noinline__ uint32_t meta_fill(const int32_t* cu, const int64_t* off, int nseq, int max_seqlen,
                               int B, int elem_bytes, int64_t* meta) {
   int64_t rows = 0, cb = 0;
   uint32_t st = 0;
@@ -115,7 +115,11 @@ __device__ inline double block_sum_f64(double v, double* red) {
 }
 
 // Geometry computed inside k_stats (no k_meta launch) for batches of up to this many sequences
+// and blocks of up to 64: measured faster there (Ministral-like pair: -3 us per call); with
+// B = 128 the inlined pass changed k_stats' register allocation and cost ~17 us on the
+// long-context case, so that size keeps the separate launch
 constexpr int INLINE_META_SEQ = 64;
+inline bool inline_meta_for(int nseq, int B) { return nseq <= INLINE_META_SEQ && B <= 64; }
 struct MetaIn {           // k_stats computes the geometry itself when inline_meta is set
   const int32_t* cu;
   int max_seqlen, elem_bytes, inline_meta;
@@ -140,33 +144,36 @@ __global__ void __launch_bounds__(NT) k_stats(const T* __restrict__ maps,
   __shared__ int32_t s_cu[INLINE_META_SEQ + 1];
   __shared__ int64_t s_off[INLINE_META_SEQ];
   const int64_t* meta = meta_g;
-  if (mi.inline_meta) {
-    // the selection's look-back flags start cleared (every thread of the grid)
-    for (int64_t r = (int64_t)blockIdx.x * NT + threadIdx.x; r < mi.max_rows;
-         r += (int64_t)gridDim.x * NT)
-      mi.flags[r] = 0ull;
-    // every CTA computes the geometry into shared memory (warp 0 loads the inputs, thread 0
-    // runs the sums); CTA 0 also publishes it for the later passes
-    if (threadIdx.x < 32) {
-      for (int k = threadIdx.x; k <= nseq; k += 32) s_cu[k] = mi.cu[k];
-      if (seq_off)
-        for (int k = threadIdx.x; k < nseq; k += 32) s_off[k] = seq_off[k];
-      __syncwarp();
-      if (threadIdx.x == 0) {
-        const uint32_t st = meta_fill(s_cu, seq_off ? s_off : nullptr, nseq, mi.max_seqlen, B,
-                                      mi.elem_bytes, s_meta);
-        if (blockIdx.x == 0) {
-          for (int k = 0; k < META_HDR + 4 * nseq; ++k) mi.meta_out[k] = s_meta[k];
-          if (s_meta[0] == 0) {  // no query block at all: an empty BSR
-            mi.row_ptr[0] = 0;
-            *mi.nnz_out = 0;
+  // (compiled for B <= 64 only: see inline_meta_for)
+  if constexpr (B <= 64) {
+    if (mi.inline_meta) {
+      // the selection's look-back flags start cleared (every thread of the grid)
+      for (int64_t r = (int64_t)blockIdx.x * NT + threadIdx.x; r < mi.max_rows;
+           r += (int64_t)gridDim.x * NT)
+        mi.flags[r] = 0ull;
+      // every CTA computes the geometry into shared memory (warp 0 loads the inputs, thread 0
+      // runs the sums); CTA 0 also publishes it for the later passes
+      if (threadIdx.x < 32) {
+        for (int k = threadIdx.x; k <= nseq; k += 32) s_cu[k] = mi.cu[k];
+        if (seq_off)
+          for (int k = threadIdx.x; k < nseq; k += 32) s_off[k] = seq_off[k];
+        __syncwarp();
+        if (threadIdx.x == 0) {
+          const uint32_t st = meta_fill(s_cu, seq_off ? s_off : nullptr, nseq, mi.max_seqlen, B,
+                                        mi.elem_bytes, s_meta);
+          if (blockIdx.x == 0) {
+            for (int k = 0; k < META_HDR + 4 * nseq; ++k) mi.meta_out[k] = s_meta[k];
+            if (s_meta[0] == 0) {  // no query block at all: an empty BSR
+              mi.row_ptr[0] = 0;
+              *mi.nnz_out = 0;
+            }
+            if (st) atomicOr(mi.status, st);
           }
-          if (st) atomicOr(mi.status, st);
         }
       }
+      __syncthreads();
+      meta = s_meta;
     }
-    __syncthreads();
-    meta = s_meta;
   }
   const int64_t total = meta[1];
   const int64_t nv = (int64_t)h_s * VPB;
@@ -459,7 +466,7 @@ cudaError_t launch_typed(const mf_compress_desc& d, const CompressWs& ws, uint32
   double* mass = d.block_mass_out ? d.block_mass_out : ws.mass;
   const int grid_stats = (int)std::min<int64_t>(ws.max_cb, (int64_t)sms * 8);
   MetaIn mi{};
-  if (d.nseq <= INLINE_META_SEQ) {
+  if (inline_meta_for(d.nseq, B)) {
     mi.cu = d.cu_seqlens; mi.max_seqlen = d.max_seqlen; mi.elem_bytes = (int)sizeof(T);
     mi.inline_meta = 1; mi.meta_out = ws.meta; mi.status = status; mi.row_ptr = d.row_ptr;
     mi.nnz_out = d.nnz_out; mi.flags = ws.flags; mi.max_rows = ws.max_rows;
@@ -535,9 +542,9 @@ cudaError_t launch_compress(const mf_compress_desc& d, const CompressWs& ws, uin
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int elem = d.dtype == MF_F32 ? 4 : 2;
-  // the geometry pass: inside k_stats for up to INLINE_META_SEQ sequences, else its own launch
-  // (also when there is no query block at all and k_stats does not run)
-  if (d.nseq > INLINE_META_SEQ || ws.max_cb == 0) {
+  // the geometry pass: inside k_stats where inline_meta_for says so, else its own launch (also
+  // when there is no query block at all and k_stats does not run)
+  if (!inline_meta_for(d.nseq, d.B) || ws.max_cb == 0) {
     cudaError_t e = launch_meta(d.cu_seqlens, d.map_seq_offset, d.nseq, d.max_seqlen, d.B, elem,
                                 ws, status, d.row_ptr, d.nnz_out, st);
     if (e != cudaSuccess) return e;
