@@ -498,15 +498,18 @@ __global__ void __launch_bounds__(NT, 1)
               looked |= 1u << q;
             }
           }
-#pragma unroll
-          for (int q = 0; q < KT / 8; ++q)
-            if (((looked >> q) & 1u) && (pages[q] < 0 || pages[q] >= q_r.n_pages)) {
-              atomicOr(p.status, ST_PAGE);
-              pages[q] = q_r.n_pages;
-            }
           for (int h = 0; h < NG / PH && ok; ++h) {
             if (!(ok = mbar_wait(bar(B_HEMPTY + vs), vph ^ 1, abort_flag, p.status, p.wait_ns))) break;
             TRACE(5, 4);
+            if (h == 0) {
+              // checked after the first wait, so that the lookups' latency overlaps it
+#pragma unroll
+              for (int q = 0; q < KT / 8; ++q)
+                if (((looked >> q) & 1u) && (pages[q] < 0 || pages[q] >= q_r.n_pages)) {
+                  atomicOr(p.status, ST_PAGE);
+                  pages[q] = q_r.n_pages;
+                }
+            }
             mbar_expect_tx(bar(B_HFULL + vs), V_BYTES);
             for (int gl = 0; gl < PH; ++gl) {
               const uint32_t dst = sb + OFF_V + vs * V_BYTES + gl * VGRP_BYTES;
