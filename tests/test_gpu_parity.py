@@ -100,6 +100,19 @@ def test_small_bf16_varlen_tcgen05():
     assert_O_close(O[0].float().cpu().numpy(), O2[0].float().cpu().numpy(), "bf16", "tc vs simt")
 
 
+@pytest.mark.parametrize("nseq", [64, 70])
+def test_many_sequences(nseq):
+    """A batch of short sequences around the 64-sequence limit of the geometry computed inside
+    the statistics kernel (64: inside, 70: the separate geometry pass); ~200 query blocks, so
+    the selection's look-back runs over several 32-row windows.  Every row's kept set, values
+    and O are compared with the oracle."""
+    lens = tuple(64 + (37 * k) % 257 for k in range(nseq))
+    w = synth.Workload(f"many{nseq}", lens, B=64, h_s=16, h_r=16, h_kv=4, d=128, dtype="bf16",
+                       tau=0.95, n_heavy=8, reading=3)
+    assert sum(w.nqb) > 64
+    _full_check(w, expect_path=1)
+
+
 def test_small_bf16_simt_path():
     w = synth.Workload("small_simt", (200, 70), B=64, h_s=32, h_r=32, h_kv=8, d=128,
                        dtype="bf16", tau=0.9, n_heavy=16, reading=3)
