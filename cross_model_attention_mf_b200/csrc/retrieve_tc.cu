@@ -412,8 +412,10 @@ __global__ void __launch_bounds__(NT, 1)
       wt[(base + ((rv + 16) >> 3) * 128 + (rv & 7) * 16) >> 1] = *reinterpret_cast<uint16_t*>(&lo);
     }
   }
-  // the item table: one decode per item instead of one per item and role
-  for (int k = threadIdx.x; k < ITEMS_MAX; k += NT) {
+  // the item table: one decode per item instead of one per item and role; decoded by the last
+  // ITEMS_MAX threads (no W^T work while h_s <= 32), so its chain of loads overlaps W^T's
+  if (threadIdx.x >= NT - ITEMS_MAX) {
+    const int k = threadIdx.x - (NT - ITEMS_MAX);
     const int idx = blockIdx.x + k * gridDim.x;
     if (idx < p.n_items) s_items[k] = decode(p, idx);
   }
