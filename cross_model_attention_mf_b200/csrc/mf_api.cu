@@ -412,7 +412,9 @@ mf_status mf_map_retrieve(const mf_retrieve_desc* desc, void* stream) {
     const mfi::RetrieveLayer L = layer_of(*desc, l);
     if (tc) {
       std::string err;
-      if (!mfi::launch_retrieve_tc(&desc, &L, 1, st, static_cast<cudaStream_t>(stream), &err))
+      // layers after the first start as the previous layer's CTAs exit (different O regions)
+      if (!mfi::launch_retrieve_tc(&desc, &L, 1, st, static_cast<cudaStream_t>(stream), &err,
+                                   l > desc->l_r_begin))
         return fail(MF_ERR_CUDA, "mf_map_retrieve (tcgen05): " + err);
     } else {
       cudaError_t e = mfi::launch_retrieve_simt(*desc, L, st, static_cast<cudaStream_t>(stream));
@@ -456,7 +458,9 @@ mf_status mf_map_retrieve_multi(const mf_retrieve_desc* descs, int n, void* stre
         Ls[k] = layer_of(descs[k0 + k], descs[k0 + k].l_r_begin + j);
       }
       std::string err;
-      if (!mfi::launch_retrieve_tc(ptrs, Ls, cnt, st, static_cast<cudaStream_t>(stream), &err))
+      // launches after the first write other receivers' or layers' O
+      if (!mfi::launch_retrieve_tc(ptrs, Ls, cnt, st, static_cast<cudaStream_t>(stream), &err,
+                                   j > 0 || k0 > 0))
         return fail(MF_ERR_CUDA, "mf_map_retrieve_multi (tcgen05): " + err);
     }
   return MF_OK;

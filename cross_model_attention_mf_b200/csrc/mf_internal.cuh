@@ -78,9 +78,12 @@ cudaError_t launch_retrieve_simt(const mf_retrieve_desc& d, const RetrieveLayer&
 bool tc_supported(const mf_retrieve_desc& d);
 
 // one launch for n (1..4) receivers that share the sender BSR layer and the query / key
-// packing; returns false and fills *err on a host-side failure (tensor-map encoding, launch)
+// packing; returns false and fills *err on a host-side failure (tensor-map encoding, launch).
+// pdl: the launch may start while the previous kernel on the stream still runs (programmatic
+// dependent launch), for launches after the first of one call, which read nothing the earlier
+// launches of that call write
 bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* ls, int n,
-                        uint32_t* status, cudaStream_t st, std::string* err);
+                        uint32_t* status, cudaStream_t st, std::string* err, bool pdl = false);
 
 // prefix-hash block cache
 struct BlockCache;

@@ -337,6 +337,9 @@ __device__ __forceinline__ Item decode(const TcParams& p, int idx) {
 __global__ void __launch_bounds__(NT, 1)
     k_retrieve_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ VMaps tmVs,
                   const __grid_constant__ TcParams p) {
+  // a later launch of the same call (programmatic dependent launch) may take SMs as soon as
+  // this grid's CTAs exit: it reads nothing this grid writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
@@ -930,7 +933,7 @@ bool tc_supported(const mf_retrieve_desc& d) {
 }
 
 bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* ls, int n,
-                        uint32_t* status, cudaStream_t st, std::string* err) {
+                        uint32_t* status, cudaStream_t st, std::string* err, bool pdl) {
   if (n < 1 || n > NRMAX) { *err = "1 to 4 receivers per launch"; return false; }
   const mf_retrieve_desc& d0 = *ds[0];
   const RetrieveLayer& l0 = ls[0];
@@ -998,7 +1001,22 @@ bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* 
   cudaError_t e = cudaFuncSetAttribute(k_retrieve_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SMEM_BYTES);
   if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
-  k_retrieve_tc<<<(unsigned)grid, NT, SMEM_BYTES, st>>>(tmA, vm, p);
+  if (pdl) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k_retrieve_tc, tmA, vm, p);
+    if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
+  } else {
+    k_retrieve_tc<<<(unsigned)grid, NT, SMEM_BYTES, st>>>(tmA, vm, p);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
   return true;
