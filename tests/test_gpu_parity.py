@@ -232,6 +232,35 @@ def test_layouts_bitwise_identical():
     _status_ok()
 
 
+@pytest.mark.parametrize("page_size", [8, 16, 32, 64])
+def test_paged_page_sizes_bitwise(page_size):
+    """Every supported page size (the V slot holds whole pages of both groups of a half tile, a
+    K step of 16 keys spanning two 8-token pages or part of a larger one) gives O bit for bit
+    equal to contiguous V."""
+    w = synth.Workload(f"pg{page_size}", (300, 129, 64), B=64, h_s=32, h_r=32, h_kv=8, d=128,
+                       dtype="bf16", tau=0.95, n_heavy=16, reading=3, page_size=page_size)
+    pack = sdev.fill_maps(sdev.alloc_maps(w), w, 0)
+    bsr = run_compress(w, pack)
+    W = sdev.w_weights(w)
+    V = sdev.v_contiguous(w, 0)
+    whole = _retrieve(w, pack, bsr, W, V)[0]
+    Vp, table = sdev.v_paged(w, V)
+    cu = pack.cu_seqlens
+    paged = mf.mf_map_retrieve([bsr], [0], W, Vp, cu, cu, sdev.qblock_base(w), max(w.lens),
+                               w.h_r, w.h_kv, total_q=w.tokens, paged=(table, w.page_size))[0]
+    _status_ok()
+    assert torch.equal(paged, whole)
+
+
+@pytest.mark.parametrize("h_r,h_kv", [(4, 1), (8, 2), (12, 3)])
+def test_few_kv_heads_tcgen05(h_r, h_kv):
+    """One, two and three KV heads on the tensor-core path (the V copies hold two heads, or one
+    when there is only one) against the oracle."""
+    w = synth.Workload(f"kv{h_kv}", (300, 129), B=64, h_s=16, h_r=h_r, h_kv=h_kv, d=128,
+                       dtype="bf16", tau=0.95, n_heavy=8, reading=3)
+    _full_check(w, expect_path=1)
+
+
 def test_layer_batch_and_layer_map():
     """Three receiver layers over two sender layers in one call equal three single-layer calls."""
     w = synth.Workload("lm", (200,), B=64, h_s=32, h_r=32, h_kv=8, d=128, dtype="bf16", tau=0.9,
