@@ -83,10 +83,10 @@ constexpr int HS = 2;   // half-tile slots: one key tile
 constexpr uint32_t A_BYTES = R * SC * KT * 2;   // 32 KB
 constexpr uint32_t VGRP_BYTES = KT * D * 2;     // 16 KB: one group's V tile
 constexpr uint32_t V_BYTES = PH * VGRP_BYTES;   // 32 KB: V of one half tile
-// A V slot holds the half tile's two groups as [d half (16 KB)][page][group][page rows][128 B]
-// (contiguous V: one 64-row page), so that for paged V one TMA copy (a two-head box) brings a d
-// half of both groups for one page; the P.V descriptors step through it per K step of 16 keys.
-constexpr uint32_t VDH_BYTES = V_BYTES / 2;     // one d half of a slot
+// A V slot holds the half tile's two groups as [page][d half][group][page rows][128 B]
+// (contiguous V: one 64-row page), which is the order in which one TMA box over (64 dims, page
+// rows, 2 kv heads, 2 d halves) lands, so a stage takes one copy per page; the P.V descriptors
+// step through it per K step of 16 keys.
 constexpr uint32_t PT_BYTES = KT * 64 * 2;      // 8 KB: one group's P^T (hi or lo)
 constexpr uint32_t PSLOT_BYTES = 2 * PT_BYTES;  // hi + lo of one group
 constexpr uint32_t OFF_A = 0;
@@ -131,7 +131,6 @@ struct RecvParams {
   const int32_t* block_table;
   int paged, page_size, n_pages, max_pages;
   int total_k;     // V rows (contiguous V): the out-of-range row that reads zeros
-  uint32_t v_tx;   // bytes one half tile's paged V copies bring
   int h_r, h_kv, gq, hcs;
 };
 struct TcParams {
@@ -203,20 +202,20 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
   }
 }
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
-                                            int c0, int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
                                             int c0, int c1, int c2, int c3) {
   asm volatile(
       "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
+                                            int c0, int c1, int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
       : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() {
@@ -483,15 +482,10 @@ __global__ void __launch_bounds__(NT, 1)
               if (!(ok = mbar_wait(bar(B_HEMPTY + vs), vph ^ 1, abort_flag, p.status, p.wait_ns))) break;
               TRACE(5, 4);
               mbar_expect_tx(bar(B_HFULL + vs), V_BYTES);
-              // one copy per group and d half: 64 keys of one kv head (coordinates: dim, kv
-              // head, token); a box over two heads would walk the strides out of order, which
-              // the copy engine serves far more slowly
-              for (int gl = 0; gl < PH; ++gl) {
-                const uint32_t dst = sb + OFF_V + vs * V_BYTES + gl * (KT * 128);
-                const int G = hc * NG + h * PH + gl;
-                tma_load_3d(dst, tmV, bar(B_HFULL + vs), 0, G, row);
-                tma_load_3d(dst + VDH_BYTES, tmV, bar(B_HFULL + vs), 64, G, row);
-              }
+              // one copy: 64 keys of both groups and both d halves (coordinates: dim, token,
+              // kv head, d half; a head past h_kv reads zeros)
+              tma_load_4d(sb + OFF_V + vs * V_BYTES, tmV, bar(B_HFULL + vs), 0, row,
+                          hc * NG + h * PH, 0);
               ++v_issued;
               TRACE(5, 3);
               if (++vs == HS) { vs = 0; vph ^= 1; }
@@ -523,17 +517,16 @@ __global__ void __launch_bounds__(NT, 1)
                   pages[q] = q_r.n_pages;
                 }
             }
-            mbar_expect_tx(bar(B_HFULL + vs), q_r.v_tx);
-            // per page and d half one copy of both groups' rows (coordinates: dim, row in page,
-            // kv head, page)
+            mbar_expect_tx(bar(B_HFULL + vs), V_BYTES);
+            // one copy per page: its rows of both groups and both d halves (coordinates: dim,
+            // row in page, kv head, d half, page)
             const uint32_t dst = sb + OFF_V + vs * V_BYTES;
             const int G = hc * NG + h * PH;
 #pragma unroll
             for (int q = 0; q < KT / 8; ++q) {
               if (q * ps >= KT) break;
-              const uint32_t pq = (uint32_t)(q * 2 * ps * 128);
-              tma_load_4d(dst + pq, tmV, bar(B_HFULL + vs), 0, 0, G, pages[q]);
-              tma_load_4d(dst + VDH_BYTES + pq, tmV, bar(B_HFULL + vs), 64, 0, G, pages[q]);
+              tma_load_5d(dst + (uint32_t)(q * 4 * ps * 128), tmV, bar(B_HFULL + vs), 0, 0, G, 0,
+                          pages[q]);
             }
             ++v_issued;
             TRACE(5, 3);
@@ -609,17 +602,19 @@ __global__ void __launch_bounds__(NT, 1)
       uint32_t vph = 0;
       bool ok = true;
       int T = 0, K = 0;  // tiles and items processed so far
-      // V^T operand: the two d halves VDH_BYTES apart; 8-key groups 1024 bytes apart, or with
-      // 8-token pages the next page of the K step (2 groups x 8 rows x 128 bytes further)
+      // V^T operand: the two d halves of a page 2 x page rows x 128 bytes apart; 8-key groups
+      // 1024 bytes apart, or with 8-token pages the next page (2 d halves x 2 groups x 8 rows x
+      // 128 bytes further)
       const int vps = q_r.paged ? q_r.page_size : KT;  // rows per V page in the slot
-      const uint64_t vdesc0 = smem_desc(sb + OFF_V, VDH_BYTES, vps == 8 ? 2048u : 1024u, 2u);
+      const uint64_t vdesc0 =
+          smem_desc(sb + OFF_V, (uint32_t)(2 * vps * 128), vps == 8 ? 4096u : 1024u, 2u);
       // offset (16-byte units) of group gl's keys [16 k, 16 k + 16) within a d half of the slot:
       // vbase[k] + gl * vgrp, worked out once (the issuing thread sets the MMA rate)
       uint32_t vbase[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int q = (16 * k) / vps, r0 = (16 * k) % vps;
-        vbase[k] = (uint32_t)(q * (2 * vps * 128) + r0 * 128) >> 4;
+        vbase[k] = (uint32_t)(q * (4 * vps * 128) + r0 * 128) >> 4;
       }
       const uint32_t vgrp = (uint32_t)(vps * 128) >> 4;
       const uint64_t pdesc0 = smem_desc(sb + OFF_P, 8192u, 1024u, 2u);
@@ -992,18 +987,19 @@ bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* 
   for (int k = 0; k < n; ++k) {
     const mf_retrieve_desc& d = *ds[k];
     const RetrieveLayer& l = ls[k];
-    if (!d.paged) {  // V [T][h_kv][d]: dims (dim, kv head, token)
-      const uint64_t dims[3] = {(uint64_t)D, (uint64_t)d.h_kv, (uint64_t)std::max<int64_t>(d.total_k, 1)};
-      const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)d.h_kv * D * 2};
-      const uint32_t box[3] = {64, 1, KT};
-      if (!encode(&vm.m[k], l.V, 3, dims, strides, box, err)) return false;
-    } else {  // V [pages][page][h_kv][d]: dims (dim, row in page, kv head, page); two kv heads
-      const uint64_t dims[4] = {(uint64_t)D, (uint64_t)d.page_size, (uint64_t)d.h_kv,
-                                (uint64_t)std::max(d.n_pages, 1)};
-      const uint64_t strides[3] = {(uint64_t)d.h_kv * D * 2, (uint64_t)D * 2,
-                                   (uint64_t)d.page_size * d.h_kv * D * 2};
-      const uint32_t box[4] = {64, (uint32_t)d.page_size, d.h_kv >= 2 ? 2u : 1u, 1};
+    // a box: 64 dims x the rows x 2 kv heads x 2 d halves, landing as [d half][head][row]
+    if (!d.paged) {  // V [T][h_kv][d]: dims (dim in half, token, kv head, d half)
+      const uint64_t dims[4] = {64, (uint64_t)std::max<int64_t>(d.total_k, 1), (uint64_t)d.h_kv, 2};
+      const uint64_t strides[3] = {(uint64_t)d.h_kv * D * 2, (uint64_t)D * 2, 128};
+      const uint32_t box[4] = {64, KT, 2, 2};
       if (!encode(&vm.m[k], l.V, 4, dims, strides, box, err)) return false;
+    } else {  // V [pages][page][h_kv][d]: dims (dim in half, row in page, kv head, d half, page)
+      const uint64_t dims[5] = {64, (uint64_t)d.page_size, (uint64_t)d.h_kv, 2,
+                                (uint64_t)std::max(d.n_pages, 1)};
+      const uint64_t strides[4] = {(uint64_t)d.h_kv * D * 2, (uint64_t)D * 2, 128,
+                                   (uint64_t)d.page_size * d.h_kv * D * 2};
+      const uint32_t box[5] = {64, (uint32_t)d.page_size, 2, 2, 1};
+      if (!encode(&vm.m[k], l.V, 5, dims, strides, box, err)) return false;
     }
     RecvParams& r = p.rv[k];
     r.W = l.W; r.O = l.O;
@@ -1011,9 +1007,6 @@ bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* 
     r.p_split = (d.flags & MF_RETRIEVE_P_SPLIT) ? 1 : 0;
     r.block_table = d.block_table; r.paged = d.paged; r.page_size = d.page_size;
     r.n_pages = d.n_pages; r.max_pages = d.max_pages; r.total_k = (int)d.total_k;
-    // a paged box holds min(2, h_kv) kv heads: with one the slot's second group (padding) is not
-    // loaded; contiguous V loads both groups, a head past h_kv as the fill value
-    r.v_tx = (d.paged && d.h_kv < 2) ? V_BYTES / 2 : V_BYTES;
     r.h_r = d.h_r; r.h_kv = d.h_kv; r.gq = d.h_r / d.h_kv;
     r.hcs = (d.h_kv + NG - 1) / NG;
     p.hh_base[k] = NH;
