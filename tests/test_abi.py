@@ -116,7 +116,7 @@ def test_retrieve_path_selection(mf):
 
 @pytest.mark.parametrize("field,value", [("h_r", 30), ("l_r_end", 2), ("d", 0), ("nseq", 0),
                                          ("W", 0), ("map_dtype", 9), ("l_r_begin", -1),
-                                         ("flags", 8)])
+                                         ("flags", 8), ("V", 4104)])
 def test_retrieve_rejects_bad_descriptor(mf, field, value):
     arr = (mf.BsrDesc * 1)(mf.BsrDesc(4096, 4096, 4096, 100))
     lm = (ctypes.c_int32 * 2)(0, 3)
