@@ -268,6 +268,11 @@ __global__ void __launch_bounds__(NT) k_select(int64_t* __restrict__ meta, int n
   extern __shared__ uint64_t sm[];
   __shared__ int s_nkeep;
   __shared__ int64_t s_row, s_base;
+  // launched as a programmatic dependent of the block-mass pass: wait until that grid has
+  // completed and its writes are visible (returns at once after an ordinary launch); the gather
+  // may then be launched, and waits for this grid in turn
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0)
     s_row = (int64_t)atomicAdd(reinterpret_cast<unsigned long long*>(meta + 2), 1ull);
   __syncthreads();
@@ -414,6 +419,8 @@ __global__ void __launch_bounds__(NT) k_gather(const T* __restrict__ maps,
                                                T* __restrict__ values) {
   constexpr int EPV = Vec<T>::EPV, VPR = B / EPV, VPB = B * VPR;  // vectors per row / per head
   constexpr int U = (VPB + NT - 1) / NT;
+  // launched as a programmatic dependent of the selection: wait for its writes
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t nnz = min((int64_t)*nnz_in, capacity);
   const int64_t units = nnz * h_s;
   for (int64_t u0 = blockIdx.x; u0 < units; u0 += gridDim.x) {
@@ -458,6 +465,20 @@ __global__ void __launch_bounds__(NT) k_gather(const T* __restrict__ maps,
   }
 }
 
+// a launch that may start while the previous kernel on the stream drains (programmatic
+// dependent launch); the kernel waits (griddepcontrol.wait) before reading that kernel's output
+void dependent_launch(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* at, int grid, int block,
+                      size_t smem, cudaStream_t st) {
+  cfg->gridDim = dim3((unsigned)grid);
+  cfg->blockDim = dim3((unsigned)block);
+  cfg->dynamicSmemBytes = smem;
+  cfg->stream = st;
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg->attrs = at;
+  cfg->numAttrs = 1;
+}
+
 template <typename T, int B>
 cudaError_t launch_typed(const mf_compress_desc& d, const CompressWs& ws, uint32_t* status,
                          cudaStream_t st, int sms) {
@@ -478,10 +499,13 @@ cudaError_t launch_typed(const mf_compress_desc& d, const CompressWs& ws, uint32
   if (e != cudaSuccess) return e;
   const int grid_g = (int)std::max<int64_t>(
       1, std::min<int64_t>(std::max<int64_t>(d.capacity_blocks, 1) * d.h_s, (int64_t)sms * 8));
-  k_gather<T, B, NT><<<grid_g, NT, 0, st>>>(maps, d.map_seq_offset, ws.meta, d.nseq, d.h_s,
-                                            d.nnz_out, d.capacity_blocks, d.col_idx, ws.kept_row,
-                                            static_cast<T*>(d.values));
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute at[1];
+  dependent_launch(&cfg, at, grid_g, NT, 0, st);
+  return cudaLaunchKernelEx(&cfg, k_gather<T, B, NT>, maps, d.map_seq_offset,
+                            (const int64_t*)ws.meta, d.nseq, d.h_s, (const int32_t*)d.nnz_out,
+                            d.capacity_blocks, (const int32_t*)d.col_idx,
+                            (const int32_t*)ws.kept_row, static_cast<T*>(d.values));
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -509,10 +533,11 @@ cudaError_t launch_select(const CompressWs& ws, int nseq, int max_seqlen, int B,
                                          (int)smem_sel);
     if (e != cudaSuccess) return e;
   }
-  k_select<128><<<(unsigned)std::max<int64_t>(ws.max_rows, 1), 128, smem_sel, st>>>(
-      ws.meta, nseq, mass, tau, ws.flags, row_ptr, col_idx, ws.kept_row, nnz_out, capacity, status,
-      wait_limit_ns());
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute at[1];
+  dependent_launch(&cfg, at, (int)std::max<int64_t>(ws.max_rows, 1), 128, smem_sel, st);
+  return cudaLaunchKernelEx(&cfg, k_select<128>, ws.meta, nseq, mass, tau, ws.flags, row_ptr,
+                            col_idx, ws.kept_row, nnz_out, capacity, status, wait_limit_ns());
 }
 
 size_t compress_ws_layout(const mf_compress_desc& d, CompressWs* ws, void* base) {

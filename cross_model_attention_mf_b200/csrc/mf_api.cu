@@ -414,7 +414,7 @@ mf_status mf_map_retrieve(const mf_retrieve_desc* desc, void* stream) {
       std::string err;
       // layers after the first start as the previous layer's CTAs exit (different O regions)
       if (!mfi::launch_retrieve_tc(&desc, &L, 1, st, static_cast<cudaStream_t>(stream), &err,
-                                   l > desc->l_r_begin))
+                                   l == desc->l_r_begin))
         return fail(MF_ERR_CUDA, "mf_map_retrieve (tcgen05): " + err);
     } else {
       cudaError_t e = mfi::launch_retrieve_simt(*desc, L, st, static_cast<cudaStream_t>(stream));
@@ -460,7 +460,7 @@ mf_status mf_map_retrieve_multi(const mf_retrieve_desc* descs, int n, void* stre
       std::string err;
       // launches after the first write other receivers' or layers' O
       if (!mfi::launch_retrieve_tc(ptrs, Ls, cnt, st, static_cast<cudaStream_t>(stream), &err,
-                                   j > 0 || k0 > 0))
+                                   j == 0 && k0 == 0))
         return fail(MF_ERR_CUDA, "mf_map_retrieve_multi (tcgen05): " + err);
     }
   return MF_OK;

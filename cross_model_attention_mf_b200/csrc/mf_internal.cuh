@@ -79,11 +79,11 @@ bool tc_supported(const mf_retrieve_desc& d);
 
 // one launch for n (1..4) receivers that share the sender BSR layer and the query / key
 // packing; returns false and fills *err on a host-side failure (tensor-map encoding, launch).
-// pdl: the launch may start while the previous kernel on the stream still runs (programmatic
-// dependent launch), for launches after the first of one call, which read nothing the earlier
-// launches of that call write
+// Every launch may start while the previous kernel on the stream still runs (programmatic
+// dependent launch).  first: the call's first launch, which waits for that kernel before its
+// first global access; later launches of one call read nothing the earlier ones write.
 bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* ls, int n,
-                        uint32_t* status, cudaStream_t st, std::string* err, bool pdl = false);
+                        uint32_t* status, cudaStream_t st, std::string* err, bool first = true);
 
 // prefix-hash block cache
 struct BlockCache;

@@ -150,6 +150,7 @@ struct TcParams {
   uint32_t* status;
   uint64_t wait_ns;  // limit of every pipeline wait
   int stall;         // test: the mixing issuer first waits on B_NEVER
+  int dep_wait;      // the call's first launch: wait for the previous kernel on the stream
 };
 struct VMaps {
   CUtensorMap m[NRMAX];
@@ -341,9 +342,11 @@ __device__ __forceinline__ Item decode(const TcParams& p, int idx) {
 __global__ void __launch_bounds__(NT, 1)
     k_retrieve_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ VMaps tmVs,
                   const __grid_constant__ TcParams p) {
-  // a later launch of the same call (programmatic dependent launch) may take SMs as soon as
-  // this grid's CTAs exit: it reads nothing this grid writes
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // Every launch is a programmatic dependent launch.  A later launch of the same call reads
+  // nothing this grid writes, so it may take SMs as soon as this grid's CTAs exit; the call's
+  // first launch waits for the previous kernel on the stream (below, before its first global
+  // access) and only then lets the later launches start.
+  if (!p.dep_wait) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
@@ -400,6 +403,10 @@ __global__ void __launch_bounds__(NT, 1)
                  "r"(512)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (p.dep_wait) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   }
   // W^T of this CTA's 16 virtual heads, bf16, K-major without swizzle, 32 rows per s:
   // row n < 16 is the hi part of head n, row 16 + n its lo part.  Element (n, s) at
@@ -958,7 +965,7 @@ bool tc_supported(const mf_retrieve_desc& d) {
 }
 
 bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* ls, int n,
-                        uint32_t* status, cudaStream_t st, std::string* err, bool pdl) {
+                        uint32_t* status, cudaStream_t st, std::string* err, bool first) {
   if (n < 1 || n > NRMAX) { *err = "1 to 4 receivers per launch"; return false; }
   const mf_retrieve_desc& d0 = *ds[0];
   const RetrieveLayer& l0 = ls[0];
@@ -983,6 +990,7 @@ bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* 
   p.status = status;
   p.wait_ns = wait_limit_ns();
   p.stall = wait_stall();
+  p.dep_wait = first ? 1 : 0;
   int NH = 0;
   for (int k = 0; k < n; ++k) {
     const mf_retrieve_desc& d = *ds[k];
@@ -1027,22 +1035,18 @@ bool launch_retrieve_tc(const mf_retrieve_desc* const* ds, const RetrieveLayer* 
   cudaError_t e = cudaFuncSetAttribute(k_retrieve_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SMEM_BYTES);
   if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
-  if (pdl) {
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(NT);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
-    cfg.stream = st;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, k_retrieve_tc, tmA, vm, p);
-    if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
-  } else {
-    k_retrieve_tc<<<(unsigned)grid, NT, SMEM_BYTES, st>>>(tmA, vm, p);
-  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(NT);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k_retrieve_tc, tmA, vm, p);
+  if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
   e = cudaGetLastError();
   if (e != cudaSuccess) { *err = cudaGetErrorString(e); return false; }
   return true;
