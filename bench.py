@@ -593,7 +593,7 @@ def _comp_line(w, t, nnz, hbm, causal=None, rows=None):
             "tokens_per_s_layer": w.tokens / t}
 
 
-def run_long_context(mf, dev, hbm, tf, points, reps=3):
+def run_long_context(mf, dev, hbm, tf, points, reps=3, oracle_rows=0):
     """Long-context workload (L = 32768, B = 128, 32 -> 24 / 8 heads) at the given
     (tau, heavy columns, map reading) points: compression of the 68.7 GB dense layer (larger
     than L2 by itself) and retrieval of the compressed layer (L2 flushed before each
@@ -629,6 +629,9 @@ def run_long_context(mf, dev, hbm, tf, points, reps=3):
                     "density": nnz / w.causal_blocks,
                     "compress": _comp_line(w, t_c, nnz, hbm),
                     "retrieve": _ret_line(w, t_r, b, f, hbm, tf, w.tokens)})
+        if oracle_rows > 0 and len(out) == 1:  # the oracle beside the first point
+            out[0]["oracle_cpu"] = oracle_config_sample(w, pack, W[0].cpu().numpy(),
+                                                        V[:w.lens[0]].cpu(), oracle_rows)
         del bsr, ws, W, V, O
     del pack, flush
     torch.cuda.empty_cache()
@@ -636,7 +639,7 @@ def run_long_context(mf, dev, hbm, tf, points, reps=3):
             "points": out, "reps": reps, "l2": "retrieval: L2 flushed before every repetition"}
 
 
-def run_qwen(mf, dev, hbm, tf, reps=3):
+def run_qwen(mf, dev, hbm, tf, reps=3, oracle_rows=0):
     """Qwen-like pair: 40 sender layers compressed one by one (each layer's dense maps, 6 GB,
     generated into one reused buffer; compression timed per layer), then the 36 receiver layers
     retrieved (layer map l_s = round(l_r 39 / 35)): each layer alone, all 36 in one call, and
@@ -658,6 +661,9 @@ def run_qwen(mf, dev, hbm, tf, reps=3):
                                                     w.h_s, w.B, w.tau, b, ws), st, 2, warm=1))
         bsrs.append(b)
         nnzs.append(int(b.nnz.cpu()[0]))
+        if l == 0 and oracle_rows > 0:  # receiver layer 0 reads sender layer 0
+            ocpu = oracle_config_sample(w, pack, sdev.w_weights(w, dev)[0].cpu().numpy(),
+                                        sdev.v_contiguous(w, 0, dev)[:w.lens[0]].cpu(), oracle_rows)
     _status_or_raise(mf, "qwen compress")
     del pack
     torch.cuda.empty_cache()
@@ -714,10 +720,11 @@ def run_qwen(mf, dev, hbm, tf, reps=3):
                                                      layers=w.n_receiver_layers),
             "retrieve_36_layers_graph": _ret_line(w, t_graph, b_all, f_all, hbm, tf, T,
                                                   layers=w.n_receiver_layers),
+            **({"oracle_cpu": ocpu} if oracle_rows > 0 else {}),
             "reps": reps, "l2": "retrieval: L2 flushed before every repetition"}
 
 
-def run_routing(mf, dev, hbm, tf, reps=3):
+def run_routing(mf, dev, hbm, tf, reps=3, oracle_rows=0):
     """Multi-turn routing batch: 16 varlen sequences (1k-8k tokens) compressed in one call, then
     retrieved by chunked prefill (2048-token query chunks against the whole prefix) over a paged
     V (16-token pages, shuffled block table): every chunk step timed, and the sum."""
@@ -734,6 +741,10 @@ def run_routing(mf, dev, hbm, tf, reps=3):
                                         w.B, w.tau, bsr, ws), st, reps, warm=1)
     nnz = int(bsr.nnz.cpu()[0])
     rp = bsr.row_ptr.cpu().numpy()
+    ocpu = None
+    if oracle_rows > 0:
+        ocpu = oracle_config_sample(w, pack, sdev.w_weights(w, dev)[0].cpu().numpy(),
+                                    sdev.v_contiguous(w, 0, dev)[:w.lens[0]].cpu(), oracle_rows)
     del pack
     torch.cuda.empty_cache()
     W = sdev.w_weights(w, dev)
@@ -775,6 +786,7 @@ def run_routing(mf, dev, hbm, tf, reps=3):
             "compress": _comp_line(w, t_c, nnz, hbm),
             "retrieve_per_chunk_step": steps,
             "retrieve_all_steps": _ret_line(w, t_tot, b_tot, f_tot, hbm, tf, w.tokens),
+            **({"oracle_cpu": ocpu} if ocpu is not None else {}),
             "reps": reps, "l2": "retrieval: L2 flushed before every repetition"}
 
 
@@ -878,6 +890,23 @@ def cpu_baseline(w, dev, n_rows):
                       f"block per task), {dt:.2f} s wall"}
 
 
+def oracle_config_sample(w, pack, W_l, V_host, n_rows):
+    """The oracle (compress + retrieve) on n_rows query blocks of a config's first sequence,
+    spread over it, on all host cores: the CPU figure beside that config's GPU figures.  pack
+    holds the config's dense maps on the device; V_host is the first sequence's V rows."""
+    nqb = w.nqb[0]
+    rows = sorted(set(np.linspace(0, nqb - 1, n_rows).astype(int).tolist()))
+    view = pack.seq_view(0, w.h_s, w.B)
+    slabs = [view[:, qb * w.B:(qb + 1) * w.B, :(qb + 1) * w.B].cpu() for qb in rows]
+    cores = host_cores()
+    dt = oracle_sample(w, slabs, W_l, V_host, rows, cores)
+    toks = sum(min(w.lens[0], (qb + 1) * w.B) - qb * w.B for qb in rows)
+    return {"value": toks / dt, "unit": "tokens/s/layer", "cores": cores, "kind": "oracle",
+            "seconds": dt, "sample": f"{len(rows)} of {nqb} query blocks ({toks} tokens) of the "
+                                    f"first sequence (length {w.lens[0]}), compress + retrieve, "
+                                    f"float64 C oracle on {cores} host threads"}
+
+
 # ------------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -887,6 +916,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="ministral_pair")
     ap.add_argument("--reading", type=int, default=1)
+    ap.add_argument("--config-oracle-rows", type=int, default=16,
+                    help="query blocks of each config's first sequence that the oracle is timed on "
+                         "(0: none)")
     ap.add_argument("--cpu-rows", type=int, default=128,
                     help="query blocks of sequence 0 the CPU oracle runs (default: all of them for the Ministral-like pair)")
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -1040,9 +1072,12 @@ def main():
             pts = [tuple(float(x) if i == 0 else int(x) for i, x in enumerate(p.split(":")))
                    for p in args.long_points.split(",") if p]
             line["configs"] = {}
-            for name, fn in (("qwen_pair", lambda: run_qwen(mf_mod(), dev, hbm, tf_burst)),
-                             ("long_context", lambda: run_long_context(mf_mod(), dev, hbm, tf_burst, pts)),
-                             ("routing_batch", lambda: run_routing(mf_mod(), dev, hbm, tf_burst))):
+            orows = 0 if (args.no_cpu or world > 1) else args.config_oracle_rows
+            for name, fn in (("qwen_pair", lambda: run_qwen(mf_mod(), dev, hbm, tf_burst, oracle_rows=orows)),
+                             ("long_context", lambda: run_long_context(mf_mod(), dev, hbm, tf_burst, pts,
+                                                                       oracle_rows=orows)),
+                             ("routing_batch", lambda: run_routing(mf_mod(), dev, hbm, tf_burst,
+                                                                   oracle_rows=orows))):
                 line["configs"][name] = fn()
                 # each workload's figures also go to stderr as soon as they exist
                 print(json.dumps({name: line["configs"][name]}, default=_json_default), file=sys.stderr,
