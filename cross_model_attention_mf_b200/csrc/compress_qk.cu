@@ -24,8 +24,9 @@
 //                         written as bfloat16 values (0 where j > i or i >= L).
 //
 // Roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer + TMEM owner, warps 2-5 one
-// thread per query row (TMEM lane quarter warp % 4).  Two CTAs share an SM, so one CTA's
-// exponentials overlap the other's MMAs.  Every mbarrier wait is bounded: on expiry the CTA
+// thread per query row (TMEM lane quarter warp % 4).  Three CTAs share an SM (a two-stage K
+// ring keeps each within a third of the shared memory), so one CTA's exponentials overlap the
+// others' MMAs.  Every mbarrier wait is bounded: on expiry the CTA
 // records ST_TIMEOUT, every role stops, in-flight copies and MMAs are drained (bounded) and
 // TMEM is freed.
 #include <cuda.h>
@@ -46,7 +47,8 @@ constexpr int QT = 192;                        // 6 warps
 constexpr int QROWS = 128;                     // query rows per item
 constexpr int KB = 64;                         // keys per tile (= block size)
 constexpr int DH = 128;                        // head dim
-constexpr int KS = 4;                          // K ring stages
+constexpr int KS = 2;                          // K ring stages
+constexpr int CTAS_PER_SM = 3;                 // resident CTAs per SM (shared memory, TMEM, threads)
 constexpr uint32_t Q_BYTES = QROWS * DH * 2;   // 32 KB: two 16 KB halves (dims 0-63, 64-127)
 constexpr uint32_t K_BYTES = KB * DH * 2;      // 16 KB: two 8 KB halves
 constexpr uint32_t OFF_Q = 0;
@@ -61,7 +63,8 @@ enum {
   B_COUNT = B_NEVER + 1
 };
 static_assert(B_COUNT * 8 <= 256, "barrier area");
-static_assert(2 * QK_SMEM <= 232448, "two CTAs per SM");
+static_assert(CTAS_PER_SM * QK_SMEM <= 232448, "CTAs per SM");
+static_assert(CTAS_PER_SM * 128 <= 512, "TMEM columns of the resident CTAs");
 // kind::f16, D float32, A and B bf16 K-major, N = 64, M = 128
 constexpr uint32_t IDESC_QK = (1u << 4) | (1u << 7) | (1u << 10) | ((64u >> 3) << 17) |
                               ((128u >> 4) << 24);
@@ -279,7 +282,7 @@ __device__ __forceinline__ bool tiles_next(const QkParams& p, const QItem& it, T
 
 // ------------------------------------------------------------------ stats / gather kernel
 template <bool GATHER>
-__global__ void __launch_bounds__(QT, 2)
+__global__ void __launch_bounds__(QT, CTAS_PER_SM)
     k_qk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
          const __grid_constant__ QkParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -685,7 +688,7 @@ bool launch_compress_qk(const mf_compress_qk_desc& d, const CompressWs& ws, cons
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(p.n_items, 2 * (int64_t)sms));
+  const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(p.n_items, CTAS_PER_SM * (int64_t)sms));
   e = cudaFuncSetAttribute(k_qk<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QK_SMEM);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_qk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QK_SMEM);
