@@ -837,13 +837,15 @@ def synth_chunks(w):
 
 # ------------------------------------------------------------------------ oracle (CPU baseline)
 def _oracle_row(w, qb, slab, W_l, V_host):
-    """Oracle compression + retrieval of one query block (whole rows of sequence 0)."""
+    """Oracle compression + retrieval of one query block (whole rows of sequence 0); True when
+    the row is a near tie (its cumulative-mass boundary within 1e-5 of tau)."""
     import oracle
     m = oracle.row_masses(slab, w.lens[0], w.B, qb)
-    kept, _ = oracle.select(m, qb, w.tau)
+    kept, info = oracle.select(m, qb, w.tau)
     vals = np.stack([oracle.gather_block(slab, w.lens[0], w.B, qb, int(kb)) for kb in kept])
     lo, hi = 0, min(w.lens[0], (qb + 1) * w.B) - qb * w.B
     oracle.retrieve_block(vals, kept, qb, w.B, W_l, V_host, w.h_kv, (lo, hi))
+    return bool(oracle.is_boundary(info, w.tau))
 
 
 def host_cores():
@@ -853,14 +855,18 @@ def host_cores():
         return os.cpu_count() or 1
 
 
-def oracle_sample(w, slabs, W_l, V_host, rows, threads):
+def oracle_sample(w, slabs, W_l, V_host, rows, threads, ties=None):
     """Wall time of the oracle on the sampled query blocks, one block per task on `threads`
-    host threads (the C oracle runs with the GIL released)."""
+    host threads (the C oracle runs with the GIL released); `ties`, a list, receives the number
+    of near-tie rows among them."""
     from concurrent.futures import ThreadPoolExecutor
     t0 = time.perf_counter()
     with ThreadPoolExecutor(max_workers=threads) as pool:
-        list(pool.map(lambda a: _oracle_row(w, a[0], a[1], W_l, V_host), zip(rows, slabs)))
-    return time.perf_counter() - t0
+        near = list(pool.map(lambda a: _oracle_row(w, a[0], a[1], W_l, V_host), zip(rows, slabs)))
+    dt = time.perf_counter() - t0
+    if ties is not None:
+        ties.append(sum(near))
+    return dt
 
 
 def cpu_sample_inputs(w, n_rows, dev):
@@ -882,9 +888,11 @@ def cpu_sample_inputs(w, n_rows, dev):
 def cpu_baseline(w, dev, n_rows):
     rows, slabs, W_l, V_host = cpu_sample_inputs(w, n_rows, dev)
     cores = host_cores()
-    dt = oracle_sample(w, slabs, W_l, V_host, rows, cores)
+    ties = []
+    dt = oracle_sample(w, slabs, W_l, V_host, rows, cores, ties)
     toks = sum(min(w.lens[0], (qb + 1) * w.B) - qb * w.B for qb in rows)
     return {"value": toks / dt, "unit": "tokens/s/layer", "cores": cores, "kind": "oracle",
+            "near_tie_rows": ties[0],
             "sample": f"{len(rows)} of {w.nqb[0]} query blocks ({toks} tokens) of sequence 0, "
                       f"compress + retrieve, float64 C oracle on {cores} host threads (one query "
                       f"block per task), {dt:.2f} s wall"}
@@ -899,10 +907,11 @@ def oracle_config_sample(w, pack, W_l, V_host, n_rows):
     view = pack.seq_view(0, w.h_s, w.B)
     slabs = [view[:, qb * w.B:(qb + 1) * w.B, :(qb + 1) * w.B].cpu() for qb in rows]
     cores = host_cores()
-    dt = oracle_sample(w, slabs, W_l, V_host, rows, cores)
+    ties = []
+    dt = oracle_sample(w, slabs, W_l, V_host, rows, cores, ties)
     toks = sum(min(w.lens[0], (qb + 1) * w.B) - qb * w.B for qb in rows)
     return {"value": toks / dt, "unit": "tokens/s/layer", "cores": cores, "kind": "oracle",
-            "seconds": dt, "sample": f"{len(rows)} of {nqb} query blocks ({toks} tokens) of the "
+            "seconds": dt, "near_tie_rows": ties[0], "sample": f"{len(rows)} of {nqb} query blocks ({toks} tokens) of the "
                                     f"first sequence (length {w.lens[0]}), compress + retrieve, "
                                     f"float64 C oracle on {cores} host threads"}
 
