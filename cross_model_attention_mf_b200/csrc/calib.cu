@@ -165,6 +165,11 @@ __host__ __device__ inline void tile_of(int64_t t, int* i, int* c) {
   *i = 64 * a + (int)(rem / (a + 1));
   *c = (int)(rem % (a + 1));
 }
+// the tile after (i, c) in that order
+__host__ __device__ inline void next_tile(int* i, int* c) {
+  if (*c < (*i >> 6)) ++*c;
+  else { ++*i; *c = 0; }
+}
 inline int64_t tiles_of_length(int L) {
   const int64_t A = L / 64, rest = L - 64 * A;
   return 32 * A * (A + 1) + rest * (A + 1);
@@ -240,9 +245,9 @@ __global__ void __launch_bounds__(GT, 1)
       stage_tiles(st, &ta, &n);
       if (lane == 0) {
         bar_expect(FULL(s), (uint32_t)(n * (p.h_s + p.h_r) * 128));
-        for (int k = 0; k < n; ++k) {
-          int i, c;
-          tile_of(ta + k, &i, &c);
+        int i, c;  // the stage's first tile, then stepped along (no square root per tile)
+        tile_of(ta, &i, &c);
+        for (int k = 0; k < n; ++k, next_tile(&i, &c)) {
           const uint32_t dst = sb + s * G_STAGE_BYTES + k * tile_bytes;
           tma3(dst, &tmX, FULL(s), c * KEYS, 0, i);
           tma3(dst + p.h_s * 128u, &tmY, FULL(s), c * KEYS, 0, i);
@@ -277,9 +282,9 @@ __global__ void __launch_bounds__(GT, 1)
       int n;
       stage_tiles(st, &ta, &n);
       // keys j > i of a diagonal tile do not count: zero them in every feature row
-      for (int k = 0; k < n; ++k) {
-        int i, c;
-        tile_of(ta + k, &i, &c);
+      int i, c;
+      tile_of(ta, &i, &c);
+      for (int k = 0; k < n; ++k, next_tile(&i, &c)) {
         const int r0 = i & 63;
         if (c != (i >> 6) || r0 == 63) continue;
         uint8_t* tb = smem + s * G_STAGE_BYTES + k * tile_bytes;
