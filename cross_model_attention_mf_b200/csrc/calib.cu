@@ -40,8 +40,8 @@ namespace {
 
 constexpr int GT = 192;                      // 6 warps
 constexpr int KEYS = 64;                     // keys per tile (one 128-byte row per head)
-constexpr int G_STAGES = 3;
-constexpr uint32_t G_STAGE_BYTES = 64 * 1024;
+constexpr int G_STAGES = 2;                   // two large stages: each stage costs a fixed
+constexpr uint32_t G_STAGE_BYTES = 96 * 1024;  // hand-off (~0.6 us) beside its tiles' share
 constexpr uint32_t G_PAD_BYTES = 128 * 128;  // rows an M=128 operand may read past the last tile
 constexpr uint32_t G_OFF_BAR = G_STAGES * G_STAGE_BYTES + G_PAD_BYTES;
 constexpr uint32_t G_SMEM = G_OFF_BAR + 256 + 1024;  // + alignment slack
@@ -158,7 +158,7 @@ __device__ __forceinline__ void ld32(uint32_t taddr, uint32_t (&v)[32]) {
 // tile t of a sequence -> (query row i, key chunk c): rows 64a .. 64a+63 have a + 1 tiles
 // each, and 32 a (a + 1) tiles come before row 64a
 __host__ __device__ inline void tile_of(int64_t t, int* i, int* c) {
-  int a = (int)((sqrt(1.0 + (double)t / 8.0) - 1.0) * 0.5);
+  int a = (int)((sqrtf(1.0f + (float)t * 0.125f) - 1.0f) * 0.5f);  // corrected below
   while (32ll * (a + 1) * (a + 2) <= t) ++a;
   while (a > 0 && 32ll * a * (a + 1) > t) --a;
   const int64_t rem = t - 32ll * a * (a + 1);
