@@ -39,3 +39,19 @@ def test_causal_slabs_cover_every_causal_block(name, group):
         need = np.array([(qb + 1) * B for qb in range(nqb)])
         assert (covered >= need[None, :]).all()
         assert total >= base + w.h_s * Lp * Lp
+
+
+def test_oracle_config_sample_on_the_host():
+    """The bench's per-config CPU leg on the tiny workload with maps built by the CPU recipe:
+    the reported tokens, core count and near-tie count are consistent."""
+    import torch
+    from synth import maps as sm
+    w = synth.ALL["tiny"]
+    pack = sdev.fill_maps(sdev.alloc_maps(w, "cpu"), w, 0, use_gpu=False)
+    W = np.asarray(sm.gen_w(1, w.h_r, w.h_s, seed=w.seed))[0]
+    V = torch.as_tensor(sm.gen_v(w.lens[0], w.h_kv, w.d, seed=w.seed))
+    out = bench.oracle_config_sample(w, pack, W, V, n_rows=4)
+    assert out["kind"] == "oracle" and out["cores"] >= 1
+    assert out["near_tie_rows"] == 0  # the tiny workload has no near-tie row
+    assert out["value"] > 0 and out["seconds"] > 0
+    assert "4 of 8 query blocks" in out["sample"]
